@@ -1,0 +1,115 @@
+"""Seeded synthetic workloads for the fused MXFP4 routed-MoE layer.
+
+This module only draws random inputs; it holds none of the layer's arithmetic
+(no quantisation, no softmax, no matmul).  The tests, the smoke check and the
+bench share it, so that the CUDA path and the CPU oracle see the same inputs.
+
+Recipe (per workload, seed 0, fixed draw order x, logits, bias, w1, w2; each
+tensor and each expert has its own generator so sizes do not shift streams):
+  x      ~ N(0, 1) drawn in float32, rounded to bf16 (RNE)        [T, H]
+  logits ~ N(0, 1) float32, plus a per-expert bias folded in      [T, E]
+           'normal': b_e ~ N(0, 0.5)              (mildly uneven loads)
+           'zipf'  : b_e = 2*ln(1/(rank_e + 1)),  rank = seeded permutation
+  w1     ~ N(0, 0.02) float32 per expert                          [E, 2I, H]
+           rows [0, I) are the gate projection, rows [I, 2I) the up projection
+  w2     ~ N(0, 0.02) float32 per expert                          [E, H, I]
+The float32 weights are then quantised to MXFP4 along the reduction dim by the
+caller (the oracle's quantiser in tests, the library's quantiser in the bench;
+the two are checked bit-exact against each other).
+
+Weights are drawn on the device the caller names with torch's Philox-based
+generator; x and logits are always drawn on the CPU.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    T: int
+    H: int
+    I: int
+    E: int
+    top_k: int
+    act: str = "bf16"          # "bf16" (w4a16) or "mxfp8" (w4a8)
+    bias: str = "none"         # "none" | "normal" | "zipf"
+    seed: int = 0
+    description: str = ""
+
+    @property
+    def pairs(self) -> int:
+        return self.T * self.top_k
+
+    def with_tokens(self, T: int) -> "Workload":
+        return dataclasses.replace(self, T=T, name=f"{self.name}[T={T}]")
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", 16, 256, 128, 8, 2, "bf16", "none", 0,
+                     "tiny MoE, w4a16: T=16 H=256 I=128 E=8 top-2"),
+    "decode": Workload("decode", 16, 7168, 2048, 384, 8, "bf16", "none", 0,
+                       "decode-shaped, w4a16: T=16 H=7168 I=2048 E=384 top-8"),
+    "batched_decode": Workload("batched_decode", 256, 7168, 2048, 384, 8, "bf16", "normal", 0,
+                               "batched decode, w4a16: T=256, logits + N(0,0.5) expert bias"),
+    "prefill": Workload("prefill", 8192, 7168, 2048, 384, 8, "bf16", "zipf", 0,
+                        "prefill, w4a16: T=8192, Zipf-like expert bias"),
+    "prefill_w4a8": Workload("prefill_w4a8", 16384, 4096, 1536, 128, 8, "mxfp8", "none", 0,
+                             "prefill, w4a8: T=16384 H=4096 I=1536 E=128 top-8"),
+}
+
+_STREAM = {"x": 1, "logits": 2, "bias": 3, "w1": 4, "w2": 5}
+
+
+def _gen(wl: Workload, stream: str, index: int = 0, device: str = "cpu") -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed((wl.seed * 1_000_003 + _STREAM[stream] * 100_003 + index) & 0x7FFF_FFFF_FFFF_FFFF)
+    return g
+
+
+def draw_x(wl: Workload) -> torch.Tensor:
+    """bf16 [T, H] on the CPU."""
+    g = _gen(wl, "x")
+    return torch.randn(wl.T, wl.H, generator=g, dtype=torch.float32).to(torch.bfloat16)
+
+
+def draw_bias(wl: Workload) -> torch.Tensor:
+    """float32 [E] per-expert logit bias (zeros for 'none')."""
+    g = _gen(wl, "bias")
+    if wl.bias == "none":
+        return torch.zeros(wl.E, dtype=torch.float32)
+    if wl.bias == "normal":
+        return torch.randn(wl.E, generator=g, dtype=torch.float32) * 0.5
+    if wl.bias == "zipf":
+        rank = torch.randperm(wl.E, generator=g)
+        return torch.tensor([2.0 * math.log(1.0 / (int(r) + 1)) for r in rank], dtype=torch.float32)
+    raise ValueError(f"unknown bias kind {wl.bias!r}")
+
+
+def draw_logits(wl: Workload) -> torch.Tensor:
+    """float32 [T, E] on the CPU, the expert bias already folded in."""
+    g = _gen(wl, "logits")
+    base = torch.randn(wl.T, wl.E, generator=g, dtype=torch.float32)
+    return (base + draw_bias(wl)[None, :]).contiguous()
+
+
+def draw_w1_expert(wl: Workload, e: int, device: str = "cpu") -> torch.Tensor:
+    """float32 [2I, H] for expert e (gate rows then up rows)."""
+    g = _gen(wl, "w1", e, device)
+    return torch.randn(2 * wl.I, wl.H, generator=g, dtype=torch.float32, device=device) * 0.02
+
+
+def draw_w2_expert(wl: Workload, e: int, device: str = "cpu") -> torch.Tensor:
+    """float32 [H, I] for expert e."""
+    g = _gen(wl, "w2", e, device)
+    return torch.randn(wl.H, wl.I, generator=g, dtype=torch.float32, device=device) * 0.02
+
+
+def bf16_bits(t: torch.Tensor):
+    """The uint16 bit patterns (numpy) of a bf16 tensor."""
+    import numpy as np
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
