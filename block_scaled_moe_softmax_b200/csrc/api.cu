@@ -1,0 +1,467 @@
+// api.cu -- the C ABI of libmoe_mx.so (declared in include/moe_mx.h): handle
+// and workspace management, host-side validation, tensor-map encoding and the
+// launch sequence of one forward:
+//   route -> scan -> scatter -> gather -> FC1(+SwiGLU) -> FC2 -> combine.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+
+#include "../../include/moe_mx.h"
+#include "kernels.cuh"
+
+using namespace moe_mx;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(MOE_MX_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2-D row-major tensor map: inner dimension `cols` elements, `rows` rows.
+int encode_2d(CUtensorMap *map, CUtensorMapDataType dt, int elem_bytes, const void *ptr, uint64_t cols,
+              uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz)
+{
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc)
+        return fail(MOE_MX_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(MOE_MX_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    return MOE_MX_OK;
+}
+
+bool is_device_ptr(const void *p, int dev)
+{
+    if (!p)
+        return false;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError(); // clear the sticky-free error of an unknown pointer
+        return false;
+    }
+    if (at.type == cudaMemoryTypeManaged)
+        return true;
+    return at.type == cudaMemoryTypeDevice && at.device == dev;
+}
+
+int check_ptr(const void *p, int dev, const char *name)
+{
+    if (!is_device_ptr(p, dev))
+        return fail(MOE_MX_ERR_INVALID_ARG, "%s must be a device pointer on device %d", name, dev);
+    if (reinterpret_cast<uintptr_t>(p) % 16 != 0)
+        return fail(MOE_MX_ERR_INVALID_ARG, "%s must be 16-byte aligned", name);
+    return MOE_MX_OK;
+}
+
+int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+
+int64_t grouped_rows_bound(int E, int64_t pairs)
+{
+    const int64_t hit = pairs < E ? pairs : E;
+    return round_up(pairs + hit * (kBlockRows - 1), kBlockRows);
+}
+
+int env_int(const char *name, int dflt)
+{
+    const char *v = getenv(name);
+    return (v && *v) ? atoi(v) : dflt;
+}
+
+} // namespace
+
+struct moe_mx_handle {
+    int H, I, E, maxT, maxK, dev, num_sms;
+    int64_t max_rows;
+    int swap_rows;
+    unsigned long long timeout_ns;
+    void *ws;
+    int32_t *topk_ids, *chunk_hist, *counts, *pad_offsets, *num_rowblocks, *sorted_pair, *pos_of_pair;
+    float *topk_w;
+    int4 *rowblocks;
+    __nv_bfloat16 *A, *Hbuf, *Y;
+    uint32_t *err;
+    CUtensorMap map_A, map_H;
+    const void *w1_key, *w2_key;
+    CUtensorMap map_w1, map_w2;
+    int last_T, last_k;
+};
+
+extern "C" {
+
+const char *moe_mx_last_error(void) { return g_last_error.c_str(); }
+
+int moe_mx_block_rows(void) { return kBlockRows; }
+
+int64_t moe_mx_max_grouped_rows(const moe_mx_handle *h, int num_tokens, int top_k)
+{
+    if (!h || num_tokens < 0 || top_k < 1)
+        return 0;
+    return grouped_rows_bound(h->E, (int64_t)num_tokens * top_k);
+}
+
+int moe_mx_create(moe_mx_handle **out, int hidden, int inter, int num_experts, int max_tokens, int max_top_k,
+                  int device)
+{
+    g_last_error.clear();
+    if (!out)
+        return fail(MOE_MX_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (hidden < 256 || hidden > 16384 || hidden % 256 != 0)
+        return fail(MOE_MX_ERR_UNSUPPORTED, "hidden=%d must be a multiple of 256 in [256, 16384]", hidden);
+    if (inter < 128 || inter > 8192 || inter % 128 != 0)
+        return fail(MOE_MX_ERR_UNSUPPORTED, "inter=%d must be a multiple of 128 in [128, 8192]", inter);
+    if (num_experts < 1 || num_experts > kMaxExperts)
+        return fail(MOE_MX_ERR_UNSUPPORTED, "num_experts=%d must be in [1, %d]", num_experts, kMaxExperts);
+    if (max_tokens < 1 || max_tokens > 65536)
+        return fail(MOE_MX_ERR_INVALID_ARG, "max_tokens=%d must be in [1, 65536]", max_tokens);
+    if (max_top_k < 1 || max_top_k > num_experts || max_top_k > kMaxTopK)
+        return fail(MOE_MX_ERR_INVALID_ARG, "max_top_k=%d must be in [1, min(E, %d)]", max_top_k, kMaxTopK);
+    int ndev = 0;
+    cudaError_t ce = cudaGetDeviceCount(&ndev);
+    if (ce != cudaSuccess)
+        return cuda_fail(ce, "cudaGetDeviceCount");
+    if (device < 0 || device >= ndev)
+        return fail(MOE_MX_ERR_INVALID_ARG, "device %d out of range (%d devices)", device, ndev);
+    cudaDeviceProp prop;
+    if ((ce = cudaGetDeviceProperties(&prop, device)) != cudaSuccess)
+        return cuda_fail(ce, "cudaGetDeviceProperties");
+    if (prop.major != 10 || prop.minor != 0)
+        return fail(MOE_MX_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", device,
+                    prop.major, prop.minor);
+    int prev = 0;
+    cudaGetDevice(&prev);
+    if ((ce = cudaSetDevice(device)) != cudaSuccess)
+        return cuda_fail(ce, "cudaSetDevice");
+
+    moe_mx_handle *h = new moe_mx_handle();
+    h->H = hidden;
+    h->I = inter;
+    h->E = num_experts;
+    h->maxT = max_tokens;
+    h->maxK = max_top_k;
+    h->dev = device;
+    h->num_sms = prop.multiProcessorCount;
+    const int64_t pairs = (int64_t)max_tokens * max_top_k;
+    h->max_rows = grouped_rows_bound(num_experts, pairs);
+    h->swap_rows = env_int("MOE_MX_SWAP_ROWS", 64);
+    if (h->swap_rows < 0)
+        h->swap_rows = 0;
+    if (h->swap_rows > kBlockRows)
+        h->swap_rows = kBlockRows;
+    h->timeout_ns = (unsigned long long)env_int("MOE_MX_TIMEOUT_MS", 2000) * 1000000ull;
+
+    const int64_t nchunks = (max_tokens + kRouteChunk - 1) / kRouteChunk;
+    struct Part {
+        void **dst;
+        size_t bytes;
+    } parts[] = {
+        {(void **)&h->topk_ids, sizeof(int32_t) * pairs},
+        {(void **)&h->topk_w, sizeof(float) * pairs},
+        {(void **)&h->chunk_hist, sizeof(int32_t) * nchunks * num_experts},
+        {(void **)&h->counts, sizeof(int32_t) * num_experts},
+        {(void **)&h->pad_offsets, sizeof(int32_t) * (num_experts + 1)},
+        {(void **)&h->rowblocks, sizeof(int4) * (h->max_rows / kBlockRows)},
+        {(void **)&h->num_rowblocks, sizeof(int32_t)},
+        {(void **)&h->sorted_pair, sizeof(int32_t) * h->max_rows},
+        {(void **)&h->pos_of_pair, sizeof(int32_t) * pairs},
+        {(void **)&h->err, sizeof(uint32_t)},
+        {(void **)&h->A, sizeof(__nv_bfloat16) * h->max_rows * hidden},
+        {(void **)&h->Hbuf, sizeof(__nv_bfloat16) * h->max_rows * inter},
+        {(void **)&h->Y, sizeof(__nv_bfloat16) * h->max_rows * hidden},
+    };
+    size_t total = 0;
+    for (auto &p : parts)
+        total += round_up((int64_t)p.bytes, 1024);
+    if ((ce = cudaMalloc(&h->ws, total)) != cudaSuccess) {
+        cudaGetLastError();
+        delete h;
+        cudaSetDevice(prev);
+        return fail(MOE_MX_ERR_NO_MEMORY, "cudaMalloc of %zu workspace bytes failed", total);
+    }
+    size_t off = 0;
+    for (auto &p : parts) {
+        *p.dst = static_cast<uint8_t *>(h->ws) + off;
+        off += round_up((int64_t)p.bytes, 1024);
+    }
+    int rc = MOE_MX_OK;
+    if ((ce = cudaMemset(h->ws, 0, total)) != cudaSuccess)
+        rc = cuda_fail(ce, "cudaMemset(workspace)");
+    if (rc == MOE_MX_OK && (ce = fc_gemm_prepare()) != cudaSuccess)
+        rc = cuda_fail(ce, "cudaFuncSetAttribute(fc_gemm)");
+    if (rc == MOE_MX_OK)
+        rc = encode_2d(&h->map_A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h->A, hidden, h->max_rows, 64, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc == MOE_MX_OK)
+        rc = encode_2d(&h->map_H, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h->Hbuf, inter, h->max_rows, 64, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc == MOE_MX_OK && (ce = cudaDeviceSynchronize()) != cudaSuccess)
+        rc = cuda_fail(ce, "cudaDeviceSynchronize(create)");
+    cudaSetDevice(prev);
+    if (rc != MOE_MX_OK) {
+        cudaFree(h->ws);
+        delete h;
+        return rc;
+    }
+    *out = h;
+    return MOE_MX_OK;
+}
+
+int moe_mx_destroy(moe_mx_handle *h)
+{
+    if (!h)
+        return MOE_MX_OK;
+    int prev = 0;
+    cudaGetDevice(&prev);
+    cudaSetDevice(h->dev);
+    cudaDeviceSynchronize();
+    cudaFree(h->ws);
+    cudaSetDevice(prev);
+    delete h;
+    return MOE_MX_OK;
+}
+
+int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, int num_tokens, const uint8_t *w1,
+                   const uint8_t *w1_scale, const uint8_t *w2, const uint8_t *w2_scale, int top_k, int act_dtype,
+                   void *out, void *stream)
+{
+    g_last_error.clear();
+    if (!h)
+        return fail(MOE_MX_ERR_INVALID_ARG, "handle is NULL");
+    if (num_tokens < 0 || num_tokens > h->maxT)
+        return fail(MOE_MX_ERR_INVALID_ARG, "num_tokens=%d must be in [0, %d]", num_tokens, h->maxT);
+    if (top_k < 1 || top_k > h->maxK || top_k > h->E)
+        return fail(MOE_MX_ERR_INVALID_ARG, "top_k=%d must be in [1, min(E=%d, max_top_k=%d)]", top_k, h->E,
+                    h->maxK);
+    if (act_dtype != MOE_MX_ACT_BF16 && act_dtype != MOE_MX_ACT_MXFP8)
+        return fail(MOE_MX_ERR_INVALID_ARG, "act_dtype=%d is not MOE_MX_ACT_BF16 or MOE_MX_ACT_MXFP8", act_dtype);
+    if (num_tokens == 0)
+        return MOE_MX_OK;
+    int rc;
+    if ((rc = check_ptr(x, h->dev, "x")) || (rc = check_ptr(router_logits, h->dev, "router_logits")) ||
+        (rc = check_ptr(w1, h->dev, "w1")) || (rc = check_ptr(w1_scale, h->dev, "w1_scale")) ||
+        (rc = check_ptr(w2, h->dev, "w2")) || (rc = check_ptr(w2_scale, h->dev, "w2_scale")) ||
+        (rc = check_ptr(out, h->dev, "out")))
+        return rc;
+    if (x == out)
+        return fail(MOE_MX_ERR_INVALID_ARG, "out must not alias x");
+
+    const int H = h->H, I = h->I, E = h->E, T = num_tokens, k = top_k;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int prev = 0;
+    cudaGetDevice(&prev);
+    if (prev != h->dev)
+        cudaSetDevice(h->dev);
+
+    if (w1 != h->w1_key) {
+        if ((rc = encode_2d(&h->map_w1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w1, H / 2, (uint64_t)E * 2 * I, 32, 128,
+                            CU_TENSOR_MAP_SWIZZLE_NONE)))
+            goto done;
+        h->w1_key = w1;
+    }
+    if (w2 != h->w2_key) {
+        if ((rc = encode_2d(&h->map_w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w2, I / 2, (uint64_t)E * H, 32, 128,
+                            CU_TENSOR_MAP_SWIZZLE_NONE)))
+            goto done;
+        h->w2_key = w2;
+    }
+    {
+        const int64_t pairs = (int64_t)T * k;
+        const int64_t rows = grouped_rows_bound(E, pairs);
+        cudaError_t ce = cudaMemsetAsync(h->sorted_pair, 0xFF, sizeof(int32_t) * rows, s);
+        if (ce != cudaSuccess) {
+            rc = cuda_fail(ce, "cudaMemsetAsync(sorted_pair)");
+            goto done;
+        }
+        RouteGroupArgs ra{router_logits, T, E, k, h->topk_ids, h->topk_w, h->chunk_hist, h->counts,
+                          h->pad_offsets, h->rowblocks, h->num_rowblocks, h->sorted_pair, h->pos_of_pair};
+        launch_route_and_group(ra, s);
+        launch_gather(static_cast<const __nv_bfloat16 *>(x), (int)pairs, H, k, h->pos_of_pair, h->A,
+                      act_dtype == MOE_MX_ACT_MXFP8, h->num_sms, s);
+
+        FcGemmArgs f1{};
+        f1.rowblocks = h->rowblocks;
+        f1.num_rowblocks = h->num_rowblocks;
+        f1.wscale = w1_scale;
+        f1.out = h->Hbuf;
+        f1.err = h->err;
+        f1.timeout_ns = h->timeout_ns;
+        f1.K = H;
+        f1.R = 2 * I;
+        f1.n_tiles = I / 128;
+        f1.out_ld = I;
+        f1.fc1 = 1;
+        f1.act_mxfp8 = act_dtype == MOE_MX_ACT_MXFP8;
+        f1.swap_rows = h->swap_rows;
+        launch_fc_gemm(f1, h->map_A, h->map_w1, h->num_sms, s);
+
+        FcGemmArgs f2 = f1;
+        f2.wscale = w2_scale;
+        f2.out = h->Y;
+        f2.K = I;
+        f2.R = H;
+        f2.n_tiles = H / 256;
+        f2.out_ld = H;
+        f2.fc1 = 0;
+        f2.act_mxfp8 = 0;
+        launch_fc_gemm(f2, h->map_H, h->map_w2, h->num_sms, s);
+
+        launch_combine(h->Y, T, H, k, h->pos_of_pair, h->topk_w, static_cast<__nv_bfloat16 *>(out), h->num_sms, s);
+        ce = cudaGetLastError();
+        if (ce != cudaSuccess) {
+            rc = cuda_fail(ce, "kernel launch");
+            goto done;
+        }
+        h->last_T = T;
+        h->last_k = k;
+    }
+done:
+    if (prev != h->dev)
+        cudaSetDevice(prev);
+    return rc;
+}
+
+int moe_mx_sync_status(moe_mx_handle *h, void *stream)
+{
+    g_last_error.clear();
+    if (!h)
+        return fail(MOE_MX_ERR_INVALID_ARG, "handle is NULL");
+    cudaError_t ce = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (ce != cudaSuccess)
+        return cuda_fail(ce, "cudaStreamSynchronize");
+    uint32_t word = 0;
+    if ((ce = cudaMemcpy(&word, h->err, sizeof(word), cudaMemcpyDeviceToHost)) != cudaSuccess)
+        return cuda_fail(ce, "cudaMemcpy(error word)");
+    if (word != 0) {
+        cudaMemset(h->err, 0, sizeof(uint32_t));
+        cudaDeviceSynchronize();
+        return fail(MOE_MX_ERR_TIMEOUT, "a device-side wait gave up (error word 0x%x)", word);
+    }
+    return MOE_MX_OK;
+}
+
+int moe_mx_quantize(const float *src, int64_t rows, int64_t K, int fmt, uint8_t *codes, uint8_t *scales,
+                    void *stream)
+{
+    g_last_error.clear();
+    if (rows < 0 || K <= 0 || K % 32 != 0)
+        return fail(MOE_MX_ERR_INVALID_ARG, "rows=%lld K=%lld: K must be a positive multiple of 32",
+                    (long long)rows, (long long)K);
+    if (fmt != MOE_MX_FMT_MXFP4 && fmt != MOE_MX_FMT_MXFP8)
+        return fail(MOE_MX_ERR_INVALID_ARG, "fmt=%d is not MOE_MX_FMT_MXFP4 or MOE_MX_FMT_MXFP8", fmt);
+    if (rows == 0)
+        return MOE_MX_OK;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, src) == cudaSuccess && at.type == cudaMemoryTypeDevice)
+        dev = at.device;
+    else
+        cudaGetLastError();
+    int rc;
+    if ((rc = check_ptr(src, dev, "src")) || (rc = check_ptr(codes, dev, "codes")) ||
+        (rc = check_ptr(scales, dev, "scales")))
+        return rc;
+    int nsm = 148;
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    int prev = 0;
+    cudaGetDevice(&prev);
+    if (prev != dev)
+        cudaSetDevice(dev);
+    launch_mx_quantize(src, rows, K, fmt, codes, scales, nsm, static_cast<cudaStream_t>(stream));
+    cudaError_t ce = cudaGetLastError();
+    if (prev != dev)
+        cudaSetDevice(prev);
+    if (ce != cudaSuccess)
+        return cuda_fail(ce, "mx_quantize launch");
+    return MOE_MX_OK;
+}
+
+int moe_mx_get_routing(const moe_mx_handle *h, int32_t *topk_ids, float *topk_w, int32_t *counts,
+                       int32_t *pad_offsets, int32_t *sorted_pair, void *stream)
+{
+    g_last_error.clear();
+    if (!h)
+        return fail(MOE_MX_ERR_INVALID_ARG, "handle is NULL");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t pairs = (int64_t)h->last_T * h->last_k;
+    struct Copy {
+        void *dst;
+        const void *src;
+        size_t bytes;
+        const char *name;
+    } copies[] = {
+        {topk_ids, h->topk_ids, sizeof(int32_t) * pairs, "topk_ids"},
+        {topk_w, h->topk_w, sizeof(float) * pairs, "topk_w"},
+        {counts, h->counts, sizeof(int32_t) * h->E, "counts"},
+        {pad_offsets, h->pad_offsets, sizeof(int32_t) * (h->E + 1), "pad_offsets"},
+        {sorted_pair, h->sorted_pair, sizeof(int32_t) * grouped_rows_bound(h->E, pairs), "sorted_pair"},
+    };
+    for (auto &c : copies) {
+        if (!c.dst || c.bytes == 0)
+            continue;
+        if (!is_device_ptr(c.dst, h->dev))
+            return fail(MOE_MX_ERR_INVALID_ARG, "%s must be a device pointer on device %d", c.name, h->dev);
+        cudaError_t ce = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyDeviceToDevice, s);
+        if (ce != cudaSuccess)
+            return cuda_fail(ce, "cudaMemcpyAsync(routing state)");
+    }
+    return MOE_MX_OK;
+}
+
+int moe_mx_debug_watchdog(moe_mx_handle *h, int timeout_us, void *stream)
+{
+    g_last_error.clear();
+    if (!h)
+        return fail(MOE_MX_ERR_INVALID_ARG, "handle is NULL");
+    if (timeout_us < 1 || timeout_us > 10000000)
+        return fail(MOE_MX_ERR_INVALID_ARG, "timeout_us=%d must be in [1, 1e7]", timeout_us);
+    launch_watchdog(h->err, (unsigned long long)timeout_us * 1000ull, static_cast<cudaStream_t>(stream));
+    cudaError_t ce = cudaGetLastError();
+    if (ce != cudaSuccess)
+        return cuda_fail(ce, "watchdog launch");
+    return MOE_MX_OK;
+}
+
+} // extern "C"

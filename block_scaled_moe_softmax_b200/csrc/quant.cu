@@ -1,0 +1,92 @@
+// quant.cu -- MX quantisation of float32 rows on the GPU (OCP Microscaling
+// Formats v1.0: per 32-element block, shared scale exponent
+// s = floor(log2(amax)) - emax_elem clamped to [-127, 127], stored as the E8M0
+// byte s + 127; elements rounded to nearest-even onto the element grid,
+// saturating).  Used to prepare MXFP4 weights; the forward's activation
+// quantisation shares mx_quantize32_e4m3.
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace moe_mx {
+
+namespace {
+
+__device__ __forceinline__ uint32_t mx_quantize32_e2m1(const float (&v)[32], uint8_t (&packed)[16])
+{
+    float amax = 0.f;
+    bool finite = true;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const float a = fabsf(v[i]);
+        finite = finite && (a <= 3.402823466e38f);
+        amax = fmaxf(amax, a);
+    }
+    if (!finite) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            packed[i] = 0;
+        return 0xFF;
+    }
+    int s = (amax == 0.f) ? -127 : floor_log2_pos(amax) - 2;
+    s = max(-127, min(127, s));
+    const float inv = exp2_int(-s);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const uint32_t lo = f32_to_e2m1(__fmul_rn(v[2 * i], inv));
+        const uint32_t hi = f32_to_e2m1(__fmul_rn(v[2 * i + 1], inv));
+        packed[i] = (uint8_t)(lo | (hi << 4));
+    }
+    return (uint32_t)(s + 127);
+}
+
+__global__ void __launch_bounds__(256) mx_quantize_kernel(const float *__restrict__ src, long long nblocks, int fmt,
+                                                          uint8_t *__restrict__ codes, uint8_t *__restrict__ scales)
+{
+    for (long long b = blockIdx.x * (long long)blockDim.x + threadIdx.x; b < nblocks;
+         b += (long long)gridDim.x * blockDim.x) {
+        float v[32];
+        const float4 *s4 = reinterpret_cast<const float4 *>(src + b * 32);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float4 f = __ldg(s4 + i);
+            v[4 * i] = f.x;
+            v[4 * i + 1] = f.y;
+            v[4 * i + 2] = f.z;
+            v[4 * i + 3] = f.w;
+        }
+        if (fmt == 0) {
+            uint8_t p[16];
+            scales[b] = (uint8_t)mx_quantize32_e2m1(v, p);
+            uint4 o;
+            uint8_t *ob = reinterpret_cast<uint8_t *>(&o);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                ob[i] = p[i];
+            reinterpret_cast<uint4 *>(codes)[b] = o;
+        } else {
+            uint8_t c[32];
+            scales[b] = (uint8_t)mx_quantize32_e4m3(v, c);
+            uint4 o[2];
+            uint8_t *ob = reinterpret_cast<uint8_t *>(o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                ob[i] = c[i];
+            reinterpret_cast<uint4 *>(codes)[2 * b] = o[0];
+            reinterpret_cast<uint4 *>(codes)[2 * b + 1] = o[1];
+        }
+    }
+}
+
+} // namespace
+
+void launch_mx_quantize(const float *src, int64_t rows, int64_t K, int fmt, uint8_t *codes, uint8_t *scales,
+                        int num_sms, cudaStream_t s)
+{
+    const long long nblocks = (long long)rows * (K / 32);
+    const long long want = (nblocks + 255) / 256;
+    const long long cap = (long long)num_sms * 16;
+    const int grid = (int)(want < cap ? want : cap);
+    mx_quantize_kernel<<<grid > 0 ? grid : 1, 256, 0, s>>>(src, nblocks, fmt, codes, scales);
+}
+
+} // namespace moe_mx

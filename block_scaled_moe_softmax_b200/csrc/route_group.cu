@@ -1,0 +1,304 @@
+// route_group.cu -- top-k softmax routing and grouping of (token, slot) pairs
+// by expert into the padded grouped layout.
+//
+// Routing: softmax over the router logits, top-k with the lowest expert index
+// winning ties, weights renormalised to sum to 1 (TokenSpeed-kernel README,
+// "Public API", moe_route; fusedtok package description, "Operators" and "API
+// stability").  The selection is taken on the float32 logits (softmax is
+// monotone, so it picks the same experts) which keeps the choice free of exp
+// rounding; the k weights are the softmax over the selected logits, which is
+// the renormalised full softmax.
+//
+// Grouping (TokenSpeed-kernel README, "Public API", moe_dispatch): pairs
+// p = t*k + j are counting-sorted by expert, stably (ascending t within an
+// expert), into segments padded to kBlockRows rows; the activation rows are
+// gathered into that order (and, for w4a8, MXFP8-quantised on the way:
+// tokenspeed-situ package description, "Activation precision (w4a16 vs
+// w4a8)").  Every step is deterministic: integer counts only, no float atomics.
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace moe_mx {
+
+// ---------------------------------------------------------------- router
+// One warp per token; each CTA covers kRouteChunk tokens and also writes the
+// per-expert histogram of its chunk (the first level of the counting sort).
+__global__ void __launch_bounds__(kRouteThreads) route_kernel(const float *__restrict__ logits, int T, int E,
+                                                               int k, int32_t *__restrict__ topk_ids,
+                                                               float *__restrict__ topk_w,
+                                                               int32_t *__restrict__ chunk_hist)
+{
+    __shared__ int32_t hist[kMaxExperts];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        hist[e] = 0;
+    __syncthreads();
+
+    const int t_begin = blockIdx.x * kRouteChunk;
+    const int t_end = min(T, t_begin + kRouteChunk);
+    constexpr int kPerLane = kMaxExperts / 32;
+    for (int t = t_begin + warp; t < t_end; t += kRouteThreads / 32) {
+        const float *row = logits + (size_t)t * E;
+        float v[kPerLane];
+        uint32_t taken = 0;
+#pragma unroll
+        for (int i = 0; i < kPerLane; ++i) {
+            const int e = i * 32 + lane;
+            float x = (e < E) ? __ldg(row + e) : -INFINITY;
+            if (x != x) // NaN never outranks a number
+                x = -INFINITY;
+            v[i] = x;
+            if (e >= E)
+                taken |= 1u << i; // out of range: never selectable
+        }
+        float sel_logit[kMaxTopK];
+        int sel_id[kMaxTopK];
+        for (int j = 0; j < k; ++j) {
+            // this lane's best untaken entry (entries are in ascending expert order)
+            float bv = -INFINITY;
+            int bi = 0x7FFFFFFF;
+#pragma unroll
+            for (int i = 0; i < kPerLane; ++i) {
+                const int e = i * 32 + lane;
+                const bool free_ = !((taken >> i) & 1u);
+                if (free_ && (v[i] > bv || (v[i] == bv && e < bi))) {
+                    bv = v[i];
+                    bi = e;
+                }
+            }
+            // warp arg-max with the lowest index winning ties
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
+                const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, off);
+                if (ov > bv || (ov == bv && oi < bi)) {
+                    bv = ov;
+                    bi = oi;
+                }
+            }
+            if ((bi & 31) == lane)
+                taken |= 1u << (bi >> 5);
+            sel_logit[j] = bv;
+            sel_id[j] = bi;
+        }
+        if (lane == 0) {
+            // softmax over the k selected logits == renormalised top-k of the full softmax
+            const float m = sel_logit[0];
+            float u[kMaxTopK];
+            float z = 0.f;
+            for (int j = 0; j < k; ++j) {
+                u[j] = expf(sel_logit[j] - m);
+                z += u[j];
+            }
+            for (int j = 0; j < k; ++j) {
+                topk_ids[(size_t)t * k + j] = sel_id[j];
+                topk_w[(size_t)t * k + j] = u[j] / z;
+                atomicAdd(&hist[sel_id[j]], 1);
+            }
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        chunk_hist[(size_t)blockIdx.x * E + e] = hist[e];
+}
+
+// ---------------------------------------------------------------- scan
+// One CTA: per-expert totals over chunks, padded exclusive scan over experts,
+// per-chunk base rows, the row-block list and the padding markers.
+__global__ void __launch_bounds__(1024) scan_kernel(int E, int nchunks, int32_t *__restrict__ chunk_hist,
+                                                    int32_t *__restrict__ counts, int32_t *__restrict__ pad_offsets,
+                                                    int4 *__restrict__ rowblocks, int32_t *__restrict__ num_rowblocks,
+                                                    int32_t *__restrict__ sorted_pair)
+{
+    __shared__ int32_t s_pad[kMaxExperts];
+    __shared__ int32_t s_warp[32];
+    const int e = threadIdx.x;
+    int total = 0;
+    if (e < E) {
+        for (int c = 0; c < nchunks; ++c) {
+            const int h = chunk_hist[(size_t)c * E + e];
+            chunk_hist[(size_t)c * E + e] = total; // exclusive prefix within the expert
+            total += h;
+        }
+        counts[e] = total;
+    }
+    const int nb = (total + kBlockRows - 1) / kBlockRows;
+    // block-wide exclusive scan of nb (padded rows = nb * kBlockRows)
+    int incl = nb;
+    const int lane = e & 31, warp = e >> 5;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if (lane >= off)
+            incl += y;
+    }
+    if (lane == 31)
+        s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = s_warp[lane];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, w, off);
+            if (lane >= off)
+                w += y;
+        }
+        s_warp[lane] = w;
+    }
+    __syncthreads();
+    const int excl_nb = incl - nb + (warp > 0 ? s_warp[warp - 1] : 0);
+    if (e < E) {
+        s_pad[e] = excl_nb * kBlockRows;
+        pad_offsets[e] = excl_nb * kBlockRows;
+        if (e == E - 1) {
+            pad_offsets[E] = (excl_nb + nb) * kBlockRows;
+            *num_rowblocks = excl_nb + nb;
+        }
+        for (int b = 0; b < nb; ++b)
+            rowblocks[excl_nb + b] =
+                make_int4(e, excl_nb * kBlockRows + b * kBlockRows, min(kBlockRows, total - b * kBlockRows), 0);
+        for (int r = total; r < nb * kBlockRows; ++r)
+            sorted_pair[excl_nb * kBlockRows + r] = -1;
+    }
+    __syncthreads();
+    if (e < E) {
+        const int base = s_pad[e];
+        for (int c = 0; c < nchunks; ++c)
+            chunk_hist[(size_t)c * E + e] += base;
+    }
+}
+
+// ---------------------------------------------------------------- scatter
+// One warp per chunk: walks the chunk's pairs in ascending p and places each
+// at its expert's cursor, so equal experts keep ascending-token order.
+__global__ void __launch_bounds__(32) scatter_kernel(int T, int E, int k, const int32_t *__restrict__ topk_ids,
+                                                     const int32_t *__restrict__ chunk_base,
+                                                     int32_t *__restrict__ sorted_pair,
+                                                     int32_t *__restrict__ pos_of_pair)
+{
+    __shared__ int32_t cursor[kMaxExperts];
+    const int lane = threadIdx.x;
+    for (int e = lane; e < E; e += 32)
+        cursor[e] = chunk_base[(size_t)blockIdx.x * E + e];
+    __syncwarp();
+    const int p_begin = blockIdx.x * kRouteChunk * k;
+    const int p_end = min(T, (blockIdx.x + 1) * kRouteChunk) * k;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int base = p_begin; base < p_end; base += 32) {
+        const int p = base + lane;
+        const bool valid = p < p_end;
+        const int e = valid ? topk_ids[p] : -1 - lane; // invalid lanes never match each other
+        const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+        const int rank = __popc(peers & lt_mask);
+        int row = 0;
+        if (valid)
+            row = cursor[e] + rank;
+        __syncwarp();
+        if (valid && (32 - __clz(peers)) - 1 == lane) // highest lane of the group advances the cursor
+            cursor[e] += __popc(peers);
+        __syncwarp();
+        if (valid) {
+            sorted_pair[row] = p;
+            pos_of_pair[p] = row;
+        }
+    }
+}
+
+// ---------------------------------------------------------------- gather
+// Copy x[t] into grouped row pos_of_pair[p] for every pair p.  One thread per
+// 32 consecutive elements (64 bytes).  With act_mxfp8 the 32 elements (one MX
+// block) are quantised to MXFP8 E4M3 and written back as their exact bf16
+// values, which is what FC1 consumes.
+__global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16 *__restrict__ x, int P, int H, int k,
+                                                     const int32_t *__restrict__ pos_of_pair,
+                                                     __nv_bfloat16 *__restrict__ A, int act_mxfp8)
+{
+    const int blocks_per_row = H / 32;
+    const long long total = (long long)P * blocks_per_row;
+    for (long long g = blockIdx.x * (long long)blockDim.x + threadIdx.x; g < total;
+         g += (long long)gridDim.x * blockDim.x) {
+        const int p = (int)(g / blocks_per_row);
+        const int b = (int)(g % blocks_per_row);
+        const int t = p / k;
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H + (size_t)b * 32);
+        uint4 *dst = reinterpret_cast<uint4 *>(A + (size_t)pos_of_pair[p] * H + (size_t)b * 32);
+        uint4 v[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            v[i] = __ldg(src + i);
+        if (act_mxfp8)
+            mxfp8_roundtrip_bf16x32(v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            dst[i] = v[i];
+    }
+}
+
+// ---------------------------------------------------------------- combine
+// out[t, n] = bf16( sum_{j<k} w[t,j] * Y[pos(t,j), n] ), j ascending, f32.
+// One thread per 8 consecutive outputs (16-byte loads and stores).
+__global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16 *__restrict__ Y, int T, int H, int k,
+                                                      const int32_t *__restrict__ pos_of_pair,
+                                                      const float *__restrict__ topk_w,
+                                                      __nv_bfloat16 *__restrict__ out)
+{
+    const int vec_per_row = H / 8;
+    const long long total = (long long)T * vec_per_row;
+    for (long long g = blockIdx.x * (long long)blockDim.x + threadIdx.x; g < total;
+         g += (long long)gridDim.x * blockDim.x) {
+        const int t = (int)(g / vec_per_row);
+        const int c = (int)(g % vec_per_row);
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            acc[i] = 0.f;
+        for (int j = 0; j < k; ++j) {
+            const float w = __ldg(topk_w + (size_t)t * k + j);
+            const int row = __ldg(pos_of_pair + (size_t)t * k + j);
+            const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(Y + (size_t)row * H) + c);
+            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(h2[i]);
+                acc[2 * i] = fmaf(w, f.x, acc[2 * i]);
+                acc[2 * i + 1] = fmaf(w, f.y, acc[2 * i + 1]);
+            }
+        }
+        uint4 o;
+        __nv_bfloat162 *o2 = reinterpret_cast<__nv_bfloat162 *>(&o);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            o2[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+        reinterpret_cast<uint4 *>(out + (size_t)t * H)[c] = o;
+    }
+}
+
+// ---------------------------------------------------------------- launchers
+void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s)
+{
+    const int nchunks = (a.T + kRouteChunk - 1) / kRouteChunk;
+    route_kernel<<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist);
+    scan_kernel<<<1, 1024, 0, s>>>(a.E, nchunks, a.chunk_hist, a.counts, a.pad_offsets, a.rowblocks,
+                                   a.num_rowblocks, a.sorted_pair);
+    scatter_kernel<<<nchunks, 32, 0, s>>>(a.T, a.E, a.k, a.topk_ids, a.chunk_hist, a.sorted_pair, a.pos_of_pair);
+}
+
+void launch_gather(const __nv_bfloat16 *x, int P, int H, int k, const int32_t *pos_of_pair, __nv_bfloat16 *A,
+                   int act_mxfp8, int num_sms, cudaStream_t s)
+{
+    const long long work = (long long)P * (H / 32);
+    const long long want = (work + 255) / 256;
+    const int grid = (int)(want < (long long)num_sms * 8 ? want : (long long)num_sms * 8);
+    gather_kernel<<<grid > 0 ? grid : 1, 256, 0, s>>>(x, P, H, k, pos_of_pair, A, act_mxfp8);
+}
+
+void launch_combine(const __nv_bfloat16 *Y, int T, int H, int k, const int32_t *pos_of_pair, const float *topk_w,
+                    __nv_bfloat16 *out, int num_sms, cudaStream_t s)
+{
+    const long long work = (long long)T * (H / 8);
+    const long long want = (work + 255) / 256;
+    const int grid = (int)(want < (long long)num_sms * 8 ? want : (long long)num_sms * 8);
+    combine_kernel<<<grid > 0 ? grid : 1, 256, 0, s>>>(Y, T, H, k, pos_of_pair, topk_w, out);
+}
+
+} // namespace moe_mx

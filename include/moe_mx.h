@@ -1,0 +1,201 @@
+/*
+ * moe_mx.h -- C ABI of libmoe_mx.so, a fused routed mixture-of-experts layer
+ * with OCP MXFP4 expert weights for NVIDIA B200 (sm_100a).
+ *
+ * One call, moe_mx_forward, runs the whole layer on one GPU, on the caller's
+ * stream, as hand-written CUDA kernels:
+ *   1. top-k softmax routing (lowest expert index wins ties, weights
+ *      renormalised to sum to 1)
+ *        -- TokenSpeed-kernel README, "Public API" (moe_route); fusedtok
+ *           package description, "Operators" and "API stability";
+ *   2. grouping of the (token, slot) pairs by expert into a padded layout
+ *        -- TokenSpeed-kernel README, "Public API" (moe_dispatch);
+ *           mxfp6-sm120 package description, "Execution model" (indirect
+ *           routing on the grouped path);
+ *   3. FC1 (gate and up projections, MXFP4 weights) with a fused SwiGLU,
+ *      h = silu(gate) * up
+ *        -- tokenspeed-situ package description, intro ("FC1 MXFP4 + ...")
+ *           and "Supported contract"; b12x package description, "What's in
+ *           here" (SwiGLU);
+ *   4. FC2 (MXFP4 weights)
+ *        -- tokenspeed-situ package description, intro (matching FC2);
+ *   5. routing-weighted combine, out[t] = sum_j w[t,j] * y[t,j], j ascending
+ *        -- TokenSpeed-kernel README, "Public API" (moe_combine).
+ * Activations are bf16 (w4a16) or, with MOE_MX_ACT_MXFP8, quantised on the fly
+ * to MXFP8 E4M3 with one E8M0 scale per 32 elements (w4a8); on the w4a8 path
+ * FC1's output is quantised to MXFP8 and dequantised to bf16 before FC2
+ *        -- tokenspeed-situ package description, "Activation precision
+ *           (w4a16 vs w4a8)"; mxfp6-sm120 package description, "Execution
+ *           model".
+ * MX encodings follow the OCP Microscaling Formats (MX) v1.0 specification.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every tensor argument is a plain device pointer to contiguous row-major
+ *   memory owned by the caller, 16-byte aligned; sizes are element counts.
+ *   Host pointers are rejected with MOE_MX_ERR_INVALID_ARG.
+ * - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *   stream).  Entry points only enqueue work on it; none synchronises the host
+ *   (except the explicitly synchronous helpers noted below).
+ * - Return value: MOE_MX_OK (0) or a negative MOE_MX_ERR_* code; the text of
+ *   the last error on the calling host thread is moe_mx_last_error().
+ *   Arguments are validated on the host before any launch: a rejected call
+ *   enqueues nothing.  No entry point traps or aborts the process.
+ * - Layout choices the pages leave open, fixed here:
+ *   * packed FP4: element 2i is the low nibble of byte i, element 2i+1 the
+ *     high nibble;
+ *   * w1's 2I rows per expert are the gate rows [0, I) then the up rows
+ *     [I, 2I);
+ *   * scales are unswizzled row-major [rows, K/32] E8M0 bytes (2^(byte-127)).
+ */
+#ifndef MOE_MX_H
+#define MOE_MX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_MX_API __attribute__((visibility("default")))
+#else
+#define MOE_MX_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define MOE_MX_OK 0
+#define MOE_MX_ERR_INVALID_ARG (-1) /* null/host/misaligned pointer, bad size or enum */
+#define MOE_MX_ERR_UNSUPPORTED (-2) /* device is not sm_100, or a shape outside the supported set */
+#define MOE_MX_ERR_CUDA (-3)        /* a CUDA runtime/driver call failed; text in moe_mx_last_error */
+#define MOE_MX_ERR_TIMEOUT (-4)     /* a bounded device-side wait gave up (see moe_mx_sync_status) */
+#define MOE_MX_ERR_NO_MEMORY (-5)   /* workspace allocation failed in moe_mx_create */
+
+/* Activation precision (act_dtype). */
+#define MOE_MX_ACT_BF16 0  /* w4a16: bf16 activations x MXFP4 weights */
+#define MOE_MX_ACT_MXFP8 1 /* w4a8: activations quantised to MXFP8 E4M3 before FC1 */
+
+/* Element formats for moe_mx_quantize. */
+#define MOE_MX_FMT_MXFP4 0 /* E2M1 codes, two per byte */
+#define MOE_MX_FMT_MXFP8 1 /* E4M3 codes, one per byte */
+
+typedef struct moe_mx_handle moe_mx_handle;
+
+/*
+ * Create a layer handle for fixed dimensions and allocate its workspace on
+ * `device` (the workspace is sized once, for max_tokens tokens and
+ * max_top_k slots; moe_mx_forward never allocates).
+ *   hidden      H, the model dimension: a multiple of 256, 256..16384.
+ *   inter       I, the expert intermediate dimension: a multiple of 128,
+ *               128..8192.
+ *   num_experts E: 1..1024.
+ *   max_tokens  largest num_tokens a forward will be given: 1..65536.
+ *   max_top_k   largest top_k a forward will be given: 1..min(E, 32).
+ *   device      CUDA device ordinal; must be compute capability 10.0.
+ * On success *out receives the handle (caller owns it; free it with
+ * moe_mx_destroy).  Errors: INVALID_ARG, UNSUPPORTED, NO_MEMORY, CUDA.
+ */
+MOE_MX_API int moe_mx_create(moe_mx_handle **out, int hidden, int inter, int num_experts, int max_tokens,
+                  int max_top_k, int device);
+
+/*
+ * Run the layer: out = MoE(x) for num_tokens tokens, enqueued on `stream`.
+ *   x              bf16 [T, H] activations.
+ *   router_logits  float32 [T, E] router logits (any per-expert bias already
+ *                  folded in).
+ *   num_tokens     T: 0..max_tokens (T = 0 returns MOE_MX_OK and enqueues
+ *                  nothing).
+ *   w1             MXFP4 codes  [E, 2I, H/2] bytes (gate rows, then up rows).
+ *   w1_scale       E8M0 scales  [E, 2I, H/32] bytes.
+ *   w2             MXFP4 codes  [E, H, I/2] bytes.
+ *   w2_scale       E8M0 scales  [E, H, I/32] bytes.
+ *   top_k          k: 1..min(E, max_top_k).
+ *   act_dtype      MOE_MX_ACT_BF16 or MOE_MX_ACT_MXFP8.
+ *   out            bf16 [T, H], written (not accumulated); must not alias x.
+ * Only experts that receive at least one token have their weights read.
+ * Dequantised weight values (code value * 2^(scale-127)) must be normal
+ * bf16 numbers, i.e. weight scale bytes in [2, 252]; other scale bytes give
+ * undefined (but finite-time, non-faulting) results.
+ * The call does not synchronise the host, allocates nothing and may be
+ * captured in a CUDA graph.  One forward may be in flight per handle.
+ * Device-side failures (a bounded wait that gave up) surface through
+ * moe_mx_sync_status.  Errors: INVALID_ARG, CUDA.
+ */
+MOE_MX_API int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, int num_tokens,
+                   const uint8_t *w1, const uint8_t *w1_scale, const uint8_t *w2,
+                   const uint8_t *w2_scale, int top_k, int act_dtype, void *out, void *stream);
+
+/* Free the handle and its workspace (waits for the device).  NULL is a no-op. */
+MOE_MX_API int moe_mx_destroy(moe_mx_handle *h);
+
+/* Text of the last error raised on the calling host thread ("" if none). */
+MOE_MX_API const char *moe_mx_last_error(void);
+
+/*
+ * Synchronise `stream` and read the handle's device error word: MOE_MX_OK,
+ * MOE_MX_ERR_TIMEOUT if a kernel's bounded wait gave up since the last call
+ * (the word is then cleared), or MOE_MX_ERR_CUDA for an asynchronous CUDA
+ * error.  Synchronous.
+ */
+MOE_MX_API int moe_mx_sync_status(moe_mx_handle *h, void *stream);
+
+/*
+ * Quantise a float32 matrix src [rows, K] (K a multiple of 32) to MX along K
+ * on the GPU, with the rule the layer's inputs follow: per 32-element block,
+ * scale exponent s = floor(log2(amax)) - emax (emax 2 for E2M1, 8 for E4M3),
+ * clamped to [-127, 127], E8M0 byte s + 127 (all-zero block: byte 0); codes =
+ * round-to-nearest-even of v * 2^-s, saturating at the largest magnitude.
+ * (OCP MX v1.0 specification; tokenspeed-situ package description,
+ * "Activation precision (w4a16 vs w4a8)".)
+ *   fmt MOE_MX_FMT_MXFP4: codes [rows, K/2]; MOE_MX_FMT_MXFP8: codes [rows, K].
+ *   scales [rows, K/32].
+ * A utility for preparing weights; the forward quantises activations with
+ * the same device code.  Errors: INVALID_ARG, CUDA.
+ */
+MOE_MX_API int moe_mx_quantize(const float *src, int64_t rows, int64_t K, int fmt, uint8_t *codes,
+                    uint8_t *scales, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Inspection entry points (tests and diagnostics).  They copy the routing and
+ * grouping state of the most recent forward on `stream` into caller buffers
+ * (device pointers); call them after moe_mx_forward on the same stream.
+ * ------------------------------------------------------------------------- */
+
+/* Rows of the padded grouped layout per expert segment (128). */
+MOE_MX_API int moe_mx_block_rows(void);
+
+/*
+ * Number of rows of the padded grouped layout the most recent forward of T
+ * tokens and top_k slots may occupy at most: T*k + E*(block_rows-1), rounded
+ * up to block_rows.  Host-only arithmetic.
+ */
+MOE_MX_API int64_t moe_mx_max_grouped_rows(const moe_mx_handle *h, int num_tokens, int top_k);
+
+/*
+ * Copy the routing/grouping state of the most recent forward:
+ *   topk_ids    int32 [T, k]   selected experts, descending logit;
+ *   topk_w      float [T, k]   renormalised weights;
+ *   counts      int32 [E]      pairs per expert;
+ *   pad_offsets int32 [E+1]    first grouped row of each expert segment;
+ *                              segment e spans ceil(counts[e]/128)*128 rows;
+ *   sorted_pair int32 [rows]   pair id t*k+j at each grouped row, -1 on
+ *                              padding rows; rows = moe_mx_max_grouped_rows.
+ * Any pointer may be NULL to skip that array.  Errors: INVALID_ARG, CUDA.
+ */
+MOE_MX_API int moe_mx_get_routing(const moe_mx_handle *h, int32_t *topk_ids, float *topk_w, int32_t *counts,
+                       int32_t *pad_offsets, int32_t *sorted_pair, void *stream);
+
+/*
+ * Self-test of the device watchdog: launch one kernel that waits on a device
+ * flag nothing sets, with a wait limit of timeout_us microseconds.  The wait
+ * gives up, the kernel records MOE_MX_ERR_TIMEOUT in the handle's error word
+ * and returns; moe_mx_sync_status then reports it.  Nothing faults or traps.
+ */
+MOE_MX_API int moe_mx_debug_watchdog(moe_mx_handle *h, int timeout_us, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_MX_H */

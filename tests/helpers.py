@@ -65,3 +65,54 @@ def max_abs_over_rms(got, ref):
 # units of the reference RMS), used by every GPU-vs-oracle output comparison.
 TOL_REL_FRO = 5e-3
 TOL_MAX_OVER_RMS = 2e-2
+
+
+# ---------------------------------------------------------------- GPU-side helpers
+def host_inputs(wl, weights=None):
+    """Seeded inputs for workload wl on the host (weights quantised by the oracle on the CPU)."""
+    x = workloads.draw_x(wl)
+    logits = workloads.draw_logits(wl)
+    wq = weights if weights is not None else quantize_weights_cpu(wl)
+    return dict(x=x, xb=workloads.bf16_bits(x), logits=logits, **wq)
+
+
+def to_device(inp, device="cuda"):
+    out = {"x": inp["x"].to(device), "logits": inp["logits"].to(device)}
+    for k in ("w1", "w1s", "w2", "w2s"):
+        out[k] = torch.from_numpy(inp[k]).to(device)
+    return out
+
+
+def oracle_forward(inp, top_k, act_mode, tokens=None):
+    out, ids, w = oracle.moe_forward(inp["xb"], inp["logits"].numpy(), inp["w1"], inp["w1s"], inp["w2"],
+                                     inp["w2s"], top_k, act_mode, tokens=tokens)
+    return oracle.bf16_bits_to_f64(out), ids, w
+
+
+def check_output(got_bf16, ref_f64, tag=""):
+    got = got_bf16.float().cpu().double().numpy()
+    rf = rel_frobenius(got, ref_f64)
+    mx = max_abs_over_rms(got, ref_f64)
+    assert np.all(np.isfinite(got)), f"{tag}: non-finite outputs"
+    assert rf <= TOL_REL_FRO, f"{tag}: relative Frobenius error {rf:.3e} > {TOL_REL_FRO}"
+    assert mx <= TOL_MAX_OVER_RMS, f"{tag}: max|gpu-ref|/RMS(ref) {mx:.3e} > {TOL_MAX_OVER_RMS}"
+    return rf, mx
+
+
+def check_routing(layer, T, k, E, logits_np):
+    """Bit-exact ids/counts/offsets/permutation against the oracle; weights within 2e-6 relative."""
+    ids_g, w_g, counts_g, pad_g, sp_g = [a.cpu().numpy() for a in layer.routing(T, k)]
+    ids_o, w_o = oracle.route(logits_np, k)
+    assert np.array_equal(ids_g, ids_o), "top-k expert ids differ from the oracle"
+    np.testing.assert_allclose(w_g, w_o, rtol=2e-6, atol=0)
+    counts_o, offs_o, sp_o = oracle.group(ids_o, E)
+    assert np.array_equal(counts_g, counts_o), "per-expert counts differ"
+    bm = 128
+    padded = (counts_o + bm - 1) // bm * bm
+    pad_o = np.concatenate([[0], np.cumsum(padded)]).astype(np.int32)
+    assert np.array_equal(pad_g, pad_o), "padded segment offsets differ"
+    for e in range(E):
+        seg = sp_g[pad_o[e]:pad_o[e + 1]]
+        assert np.array_equal(seg[:counts_o[e]], sp_o[offs_o[e]:offs_o[e + 1]]), f"permutation differs at expert {e}"
+        assert np.all(seg[counts_o[e]:] == -1), f"padding rows of expert {e} are not marked -1"
+    return ids_o
