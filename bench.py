@@ -1,0 +1,407 @@
+#!/usr/bin/env python
+"""Benchmark of the fused MXFP4 routed-MoE layer on B200; prints ONE JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode|tiny|batched_decode|prefill|prefill_w4a8]
+
+Workload (default): the decode-shaped layer, w4a16, T=16 tokens, H=7168,
+I=2048, E=384 experts, top-8; synthetic seeded inputs (bf16 x ~ N(0,1),
+float32 logits ~ N(0,1), weights N(0,0.02) quantised to MXFP4 on the GPU by the
+library's quantiser).  One step = one whole forward (routing, grouping, FC1 +
+SwiGLU, FC2, combine) through the C ABI, inputs resident in HBM.  The weights
+(8.98 GB) are far larger than L2 and L2 is additionally flushed (512 MiB write)
+before every timed step; each step is timed with CUDA events on the launching
+stream.
+
+--impl ours (default): the CUDA path.  Reported: tokens/s (value), the same
+metric end to end with host buffers (e2e: pinned H2D of x and logits, forward,
+D2H of the output, all inside the timed step), the roofline of the dominant
+kernel (FC1 grouped GEMM; algorithmic bytes = FP4 codes + E8M0 scales of the
+hit experts' W1 + activation rows read + h rows written, divided by its mean
+event-timed duration, against the measured HBM copy bandwidth), and the CPU
+oracle timed on a bounded token sample on the host cores (cpu_baseline).
+
+--impl reference: the CPU oracle (the only reference this path has), timed on
+the host cores on a bounded token sample of the same workload per step.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs an independent
+replica of the workload (the layer has no exchange step at this scope), timed
+between barriers; value = tokens of all ranks / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_scaled_moe_softmax_b200 import moe_mx, workloads  # noqa: E402
+
+METRIC = "MoE layer tokens/s; % of HBM roofline (decode) / MMA peak (prefill)"
+FLUSH_BYTES = 512 << 20
+KERNELS_PER_FORWARD = 7  # route, scan, scatter, gather, fc1, fc2, combine
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def workload_desc(wl):
+    return (f"{wl.name}: T={wl.T} H={wl.H} I={wl.I} E={wl.E} top-{wl.top_k} "
+            f"{'w4a8' if wl.act == 'mxfp8' else 'w4a16'}, logit bias {wl.bias}")
+
+
+# ------------------------------------------------------------------ inputs
+def make_gpu_weights(wl, dev):
+    """Draw float32 weights per expert on the GPU and quantise them with the library's MX quantiser."""
+    E, H, I = wl.E, wl.H, wl.I
+    w1 = torch.empty(E, 2 * I, H // 2, dtype=torch.uint8, device=dev)
+    w1s = torch.empty(E, 2 * I, H // 32, dtype=torch.uint8, device=dev)
+    w2 = torch.empty(E, H, I // 2, dtype=torch.uint8, device=dev)
+    w2s = torch.empty(E, H, I // 32, dtype=torch.uint8, device=dev)
+    for e in range(E):
+        f1 = workloads.draw_w1_expert(wl, e, device=str(dev))
+        moe_mx.moe_mx_quantize(f1, 2 * I, H, moe_mx.MOE_MX_FMT_MXFP4, w1[e], w1s[e])
+        f2 = workloads.draw_w2_expert(wl, e, device=str(dev))
+        moe_mx.moe_mx_quantize(f2, H, I, moe_mx.MOE_MX_FMT_MXFP4, w2[e], w2s[e])
+    torch.cuda.synchronize(dev)
+    return w1, w1s, w2, w2s
+
+
+def oracle_weights_for(wl, experts, dev):
+    """Oracle-quantised weights (host, numpy) for the given experts; other experts stay zero."""
+    import oracle
+    E, H, I = wl.E, wl.H, wl.I
+    w1 = np.zeros((E, 2 * I, H // 2), np.uint8)
+    w1s = np.zeros((E, 2 * I, H // 32), np.uint8)
+    w2 = np.zeros((E, H, I // 2), np.uint8)
+    w2s = np.zeros((E, H, I // 32), np.uint8)
+    for e in experts:
+        w1[e], w1s[e] = oracle.mx_quantize(workloads.draw_w1_expert(wl, e, device=dev).cpu().numpy(),
+                                           oracle.FMT_E2M1)
+        w2[e], w2s[e] = oracle.mx_quantize(workloads.draw_w2_expert(wl, e, device=dev).cpu().numpy(),
+                                           oracle.FMT_E2M1)
+    return w1, w1s, w2, w2s
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_index):
+        try:
+            props = torch.cuda.get_device_properties(dev_index)
+            self.bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+        except (AttributeError, RuntimeError):
+            self.bus = str(dev_index)
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.bus, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def oracle_time_tokens(wl, xb, logits_np, wq, tokens, nthreads):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.moe_forward(xb, logits_np, *wq, wl.top_k, 1 if wl.act == "mxfp8" else 0, tokens=tokens,
+                       nthreads=nthreads)
+    return time.perf_counter() - t0
+
+
+def cpu_sample_setup(wl, sample_tokens):
+    import oracle
+    logits = workloads.draw_logits(wl)
+    ids, _ = oracle.route(logits.numpy()[sample_tokens], wl.top_k)
+    experts = sorted(set(int(e) for e in ids.reshape(-1)))
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    wq = oracle_weights_for(wl, experts, dev)
+    xb = workloads.bf16_bits(workloads.draw_x(wl))
+    return xb, logits.numpy(), wq, experts
+
+
+def cpu_baseline(wl, cores):
+    """The oracle on a bounded sample (about 10-30 s of CPU work): a few tokens, one thread each."""
+    n_tok = max(1, min(4, cores, wl.T))
+    tokens = list(range(n_tok))
+    xb, logits_np, wq, experts = cpu_sample_setup(wl, tokens)
+    dt = oracle_time_tokens(wl, xb, logits_np, wq, tokens, n_tok)
+    return {"value": n_tok / dt, "unit": "tokens/s", "cores": n_tok, "kind": "oracle",
+            "sample": f"tokens 0..{n_tok - 1} of the {wl.name} workload ({len(experts)} experts hit), "
+                      f"one oracle call, {n_tok} threads, {dt:.1f} s wall"}
+
+
+def run_reference(args, wl):
+    """The oracle as the reference arm: one token of the workload per step; steps run in batches of
+    up to `cores` concurrent steps (one thread each), so K steps take about K/cores token-times."""
+    cores = len(os.sched_getaffinity(0))
+    sample = list(range(min(wl.T, cores)))
+    xb, logits_np, wq, experts = cpu_sample_setup(wl, sample)
+
+    def run_steps(n):
+        done, wall = 0, 0.0
+        while done < n:
+            batch = min(cores, n - done)
+            toks = [sample[(done + i) % len(sample)] for i in range(batch)]
+            wall += oracle_time_tokens(wl, xb, logits_np, wq, toks, batch)
+            done += batch
+        return wall
+
+    run_steps(args.warmup)
+    total = run_steps(args.steps)
+    value = args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 0,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": workload_desc(wl), "tokens_per_step": 1},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": min(cores, args.steps), "kind": "oracle",
+                         "sample": f"one token of {wl.name} per step (tokens 0..{len(sample) - 1} cycled, "
+                                   f"{len(experts)} experts hit), up to {cores} steps concurrently"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ the CUDA path
+def fc1_algorithmic_bytes(wl, counts):
+    hit = int((counts > 0).sum())
+    P = int(counts.sum())
+    w = hit * (2 * wl.I * wl.H // 2 + 2 * wl.I * wl.H // 32)
+    return w + P * wl.H * 2 + P * wl.I * 2, hit
+
+
+def layer_weight_bytes(wl, hit):
+    return hit * (3 * wl.I * wl.H // 2 + 3 * wl.I * wl.H // 32)
+
+
+def traffic_record(kernel_src):
+    """DRAM bytes per FC1 launch from the committed ncu summary, if the kernel source is unchanged."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    h = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
+    if rec.get("kernel_sha") != h:
+        return None
+    return rec.get("fc1_dram_bytes_per_launch")
+
+
+def run_ours(args, wl):
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    hbm_peak, bf16_peak, peak_src = measured_peaks()
+    act = moe_mx.MOE_MX_ACT_MXFP8 if wl.act == "mxfp8" else moe_mx.MOE_MX_ACT_BF16
+
+    log(f"[rank {rank}] generating weights for {workload_desc(wl)}")
+    w1, w1s, w2, w2s = make_gpu_weights(wl, dev)
+    x = workloads.draw_x(wl).to(dev)
+    logits = workloads.draw_logits(wl).to(dev)
+    out = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=dev)
+    layer = moe_mx.MoeMxLayer(wl.H, wl.I, wl.E, wl.T, wl.top_k, device=dev.index)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def fwd():
+        moe_mx.moe_mx_forward(layer.handle, x, logits, wl.T, w1, w1s, w2, w2s, wl.top_k, act, out, stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        fwd()
+    torch.cuda.synchronize()
+    status = layer.sync_status()
+    assert status == moe_mx.MOE_MX_OK, moe_mx.moe_mx_last_error()
+    _, _, counts, _, _ = layer.routing(wl.T, wl.top_k)
+    counts = counts.cpu().numpy()
+    fc1_bytes, hit = fc1_algorithmic_bytes(wl, counts)
+
+    # ---------------- timed region (device-resident inputs)
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    moe_mx.moe_mx_set_stage_timing(layer.handle, True)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    for i in range(args.steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        fwd()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    stage = moe_mx.moe_mx_get_stage_times(layer.handle)
+    moe_mx.moe_mx_set_stage_timing(layer.handle, False)
+    assert layer.sync_status() == moe_mx.MOE_MX_OK, moe_mx.moe_mx_last_error()
+    ms = statistics.mean(step_ms)
+    ms_all = max_over_ranks(ms, world)
+    value = world * wl.T / (ms_all / 1000.0)
+
+    # ---------------- end to end through the public API with host buffers
+    x_h = workloads.draw_x(wl).pin_memory()
+    l_h = workloads.draw_logits(wl).pin_memory()
+    o_h = torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory()
+    x_d = torch.empty_like(x)
+    l_d = torch.empty_like(logits)
+    e2e_steps = max(3, min(args.steps, 200))
+    e2e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(e2e_steps):
+        flush.zero_()
+        e2e_evs[i][0].record(stream)
+        x_d.copy_(x_h, non_blocking=True)
+        l_d.copy_(l_h, non_blocking=True)
+        moe_mx.moe_mx_forward(layer.handle, x_d, l_d, wl.T, w1, w1s, w2, w2s, wl.top_k, act, out, stream)
+        o_h.copy_(out, non_blocking=True)
+        e2e_evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in e2e_evs), world)
+    assert torch.equal(o_h.view(torch.int16), out.cpu().view(torch.int16))
+
+    fc1_ms = stage["fc1"]
+    achieved = fc1_bytes / (fc1_ms / 1000.0) / 1e9
+    layer_bytes = layer_weight_bytes(wl, hit)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_all, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_desc(wl), "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "top_k": wl.top_k,
+                   "act": wl.act, "hit_experts": hit, "global_batch": wl.T * world, "parallelism": f"replicas{world}",
+                   "l2": f"weights {(w1.numel() + w1s.numel() + w2.numel() + w2s.numel()) / 1e9:.2f} GB, "
+                         "a 512 MiB L2 flush before every timed step"},
+        "e2e": {"value": world * wl.T / (e2e_ms / 1000.0), "unit": "tokens/s",
+                "h2d_bytes_per_step": wl.T * wl.H * 2 + wl.T * wl.E * 4, "d2h_bytes_per_step": wl.T * wl.H * 2},
+        "gpu_launches": KERNELS_PER_FORWARD * args.steps,
+        "roofline": {"bound": "hbm", "kernel": "fc_gemm_kernel (FC1 + SwiGLU)", "achieved": achieved,
+                     "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+                     "traffic": traffic_record(os.path.join(ROOT, "block_scaled_moe_softmax_b200", "csrc",
+                                                            "fc_gemm.cu")),
+                     "peak_source": f"{peak_src} HBM copy bandwidth",
+                     "algorithmic_bytes_per_launch": fc1_bytes},
+        "layer_roofline": {"weight_bytes": layer_bytes, "achieved_gbs": layer_bytes / (ms_all / 1000.0) / 1e9,
+                           "frac": layer_bytes / (ms_all / 1000.0) / 1e9 / hbm_peak},
+        "stage_ms": stage,
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        cores = len(os.sched_getaffinity(0))
+        line["cpu_baseline"] = cpu_baseline(wl, cores)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    layer.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(workloads.WORKLOADS), default="decode")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = workloads.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        run_reference(args, wl)
+        return
+    from block_scaled_moe_softmax_b200 import build as lib_build
+    lib_build.build()
+    run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

@@ -120,13 +120,23 @@ struct moe_mx_handle {
     int32_t *topk_ids, *chunk_hist, *counts, *pad_offsets, *num_rowblocks, *sorted_pair, *pos_of_pair;
     float *topk_w;
     int4 *rowblocks;
-    __nv_bfloat16 *A, *Hbuf, *Y;
+    __nv_bfloat16 *A, *Hbuf;
+    float *Y;
     uint32_t *err;
     CUtensorMap map_A, map_H;
     const void *w1_key, *w2_key;
     CUtensorMap map_w1, map_w2;
     int last_T, last_k;
+    // stage timing: a ring of kTimingRing event sets, one set per timed forward
+    cudaEvent_t *ev;
+    bool timing;
+    long long n_timed;
 };
+
+namespace {
+constexpr int kTimingRing = 1024;
+constexpr int kEvPerFwd = MOE_MX_NUM_STAGES + 1;
+} // namespace
 
 extern "C" {
 
@@ -209,7 +219,7 @@ int moe_mx_create(moe_mx_handle **out, int hidden, int inter, int num_experts, i
         {(void **)&h->err, sizeof(uint32_t)},
         {(void **)&h->A, sizeof(__nv_bfloat16) * h->max_rows * hidden},
         {(void **)&h->Hbuf, sizeof(__nv_bfloat16) * h->max_rows * inter},
-        {(void **)&h->Y, sizeof(__nv_bfloat16) * h->max_rows * hidden},
+        {(void **)&h->Y, sizeof(float) * h->max_rows * hidden},
     };
     size_t total = 0;
     for (auto &p : parts)
@@ -256,6 +266,11 @@ int moe_mx_destroy(moe_mx_handle *h)
     cudaGetDevice(&prev);
     cudaSetDevice(h->dev);
     cudaDeviceSynchronize();
+    if (h->timing) {
+        for (int i = 0; i < kTimingRing * kEvPerFwd; ++i)
+            cudaEventDestroy(h->ev[i]);
+        delete[] h->ev;
+    }
     cudaFree(h->ws);
     cudaSetDevice(prev);
     delete h;
@@ -314,9 +329,16 @@ int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, 
             rc = cuda_fail(ce, "cudaMemsetAsync(sorted_pair)");
             goto done;
         }
+        cudaEvent_t *evset = h->timing ? h->ev + (h->n_timed % kTimingRing) * kEvPerFwd : nullptr;
+        auto mark = [&](int i) {
+            if (evset)
+                cudaEventRecord(evset[i], s);
+        };
+        mark(0);
         RouteGroupArgs ra{router_logits, T, E, k, h->topk_ids, h->topk_w, h->chunk_hist, h->counts,
                           h->pad_offsets, h->rowblocks, h->num_rowblocks, h->sorted_pair, h->pos_of_pair};
         launch_route_and_group(ra, s);
+        mark(1);
         launch_gather(static_cast<const __nv_bfloat16 *>(x), (int)pairs, H, k, h->pos_of_pair, h->A,
                       act_dtype == MOE_MX_ACT_MXFP8, h->num_sms, s);
 
@@ -334,7 +356,9 @@ int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, 
         f1.fc1 = 1;
         f1.act_mxfp8 = act_dtype == MOE_MX_ACT_MXFP8;
         f1.swap_rows = h->swap_rows;
+        mark(2);
         launch_fc_gemm(f1, h->map_A, h->map_w1, h->num_sms, s);
+        mark(3);
 
         FcGemmArgs f2 = f1;
         f2.wscale = w2_scale;
@@ -346,15 +370,18 @@ int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, 
         f2.fc1 = 0;
         f2.act_mxfp8 = 0;
         launch_fc_gemm(f2, h->map_H, h->map_w2, h->num_sms, s);
-
+        mark(4);
         launch_combine(h->Y, T, H, k, h->pos_of_pair, h->topk_w, static_cast<__nv_bfloat16 *>(out), h->num_sms, s);
         ce = cudaGetLastError();
         if (ce != cudaSuccess) {
             rc = cuda_fail(ce, "kernel launch");
             goto done;
         }
+        mark(5);
         h->last_T = T;
         h->last_k = k;
+        if (h->timing)
+            ++h->n_timed;
     }
 done:
     if (prev != h->dev)
@@ -447,6 +474,72 @@ int moe_mx_get_routing(const moe_mx_handle *h, int32_t *topk_ids, float *topk_w,
         if (ce != cudaSuccess)
             return cuda_fail(ce, "cudaMemcpyAsync(routing state)");
     }
+    return MOE_MX_OK;
+}
+
+int moe_mx_set_stage_timing(moe_mx_handle *h, int enable)
+{
+    g_last_error.clear();
+    if (!h)
+        return fail(MOE_MX_ERR_INVALID_ARG, "handle is NULL");
+    int prev = 0;
+    cudaGetDevice(&prev);
+    cudaSetDevice(h->dev);
+    if (h->timing) { // disable, or re-enable = reset
+        cudaDeviceSynchronize();
+        for (int i = 0; i < kTimingRing * kEvPerFwd; ++i)
+            cudaEventDestroy(h->ev[i]);
+        delete[] h->ev;
+        h->ev = nullptr;
+        h->timing = false;
+    }
+    int rc = MOE_MX_OK;
+    if (enable) {
+        h->ev = new cudaEvent_t[kTimingRing * kEvPerFwd];
+        for (int i = 0; i < kTimingRing * kEvPerFwd; ++i) {
+            cudaError_t ce = cudaEventCreate(&h->ev[i]);
+            if (ce != cudaSuccess) {
+                for (int j = 0; j < i; ++j)
+                    cudaEventDestroy(h->ev[j]);
+                delete[] h->ev;
+                h->ev = nullptr;
+                rc = cuda_fail(ce, "cudaEventCreate");
+                break;
+            }
+        }
+        if (rc == MOE_MX_OK) {
+            h->timing = true;
+            h->n_timed = 0;
+        }
+    }
+    cudaSetDevice(prev);
+    return rc;
+}
+
+int moe_mx_get_stage_times(moe_mx_handle *h, float *ms)
+{
+    g_last_error.clear();
+    if (!h || !ms)
+        return fail(MOE_MX_ERR_INVALID_ARG, "handle and ms must be non-NULL");
+    if (!h->timing || h->n_timed == 0)
+        return fail(MOE_MX_ERR_INVALID_ARG, "stage timing is not enabled or no timed forward ran yet");
+    const long long n = h->n_timed < kTimingRing ? h->n_timed : kTimingRing;
+    const long long first = h->n_timed - n;
+    cudaError_t ce = cudaEventSynchronize(h->ev[((h->n_timed - 1) % kTimingRing) * kEvPerFwd + MOE_MX_NUM_STAGES]);
+    if (ce != cudaSuccess)
+        return cuda_fail(ce, "cudaEventSynchronize");
+    double acc[MOE_MX_NUM_STAGES] = {0};
+    for (long long f = first; f < h->n_timed; ++f) {
+        cudaEvent_t *set = h->ev + (f % kTimingRing) * kEvPerFwd;
+        for (int i = 0; i < MOE_MX_NUM_STAGES; ++i) {
+            float v = 0.f;
+            if ((ce = cudaEventElapsedTime(&v, set[i], set[i + 1])) != cudaSuccess)
+                return cuda_fail(ce, "cudaEventElapsedTime");
+            acc[i] += v;
+        }
+    }
+    for (int i = 0; i < MOE_MX_NUM_STAGES; ++i)
+        ms[i] = (float)(acc[i] / (double)n);
     return MOE_MX_OK;
 }
 

@@ -21,7 +21,8 @@
 //               K-major layout the tensor core reads.
 //   warp 1      MMA issuer (one thread) + TMEM owner; tcgen05.mma kind::f16,
 //               commits free the stage and publish the accumulator.
-//   warps 6-9   epilogue: tcgen05.ld -> (SwiGLU) -> bf16 stores; the
+//   warps 6-9   epilogue: tcgen05.ld -> FC1: SwiGLU -> bf16 stores,
+//               FC2: f32 stores (the combine rounds once, at the end); the
 //               accumulator is double-buffered in TMEM (2 x 256 columns).
 // Orientation per work unit: a block of more than `swap_rows` rows runs with
 // tokens on the MMA's M side (M = 128, N = 256 weight rows); a smaller block
@@ -311,8 +312,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!swap) {
                 const int rl = 32 * q + lane;
                 const bool valid = rl < rows;
-                __nv_bfloat16 *orow = a.out + (size_t)(blk.y + rl) * a.out_ld;
                 if (a.fc1) {
+                    __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(a.out) + (size_t)(blk.y + rl) * a.out_ld;
                     for (int c = 0; c < 4; ++c) {
                         uint32_t g0[16], g1[16], u0[16], u1[16];
                         tmem_ld16(tb + 32 * c, g0);
@@ -332,19 +333,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                             store_bf16x32(orow + nt * 128 + 32 * c, h);
                     }
                 } else {
-                    for (int c = 0; c < 8; ++c) {
-                        uint32_t y0[16], y1[16];
-                        tmem_ld16(tb + 32 * c, y0);
-                        tmem_ld16(tb + 32 * c + 16, y1);
+                    float *orow = static_cast<float *>(a.out) + (size_t)(blk.y + rl) * a.out_ld + nt * 256;
+                    for (int c = 0; c < 16; ++c) {
+                        uint32_t y0[16];
+                        tmem_ld16(tb + 16 * c, y0);
                         tmem_wait_ld();
-                        float y[32];
+                        if (valid) {
+                            uint4 *d = reinterpret_cast<uint4 *>(orow + 16 * c);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            y[i] = __uint_as_float(y0[i]);
-                            y[16 + i] = __uint_as_float(y1[i]);
+                            for (int i = 0; i < 4; ++i)
+                                d[i] = make_uint4(y0[4 * i], y0[4 * i + 1], y0[4 * i + 2], y0[4 * i + 3]);
                         }
-                        if (valid)
-                            store_bf16x32(orow + nt * 256 + 32 * c, y);
                     }
                 }
             } else {
@@ -360,15 +359,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int n = n0 + j;
                         if (n >= rows)
                             break;
-                        __nv_bfloat16 *orow = a.out + (size_t)(blk.y + n) * a.out_ld;
                         if (a.fc1) {
+                            __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(a.out) + (size_t)(blk.y + n) * a.out_ld;
                             float hv = silu_mul(__uint_as_float(v0[j]), __uint_as_float(v1[j]));
                             if (a.act_mxfp8)
                                 hv = mxfp8_roundtrip_warp(hv);
                             orow[nt * 128 + L] = __float2bfloat16_rn(hv);
                         } else {
-                            orow[nt * 256 + L] = __float2bfloat16_rn(__uint_as_float(v0[j]));
-                            orow[nt * 256 + 128 + L] = __float2bfloat16_rn(__uint_as_float(v1[j]));
+                            float *orow = static_cast<float *>(a.out) + (size_t)(blk.y + n) * a.out_ld;
+                            orow[nt * 256 + L] = __uint_as_float(v0[j]);
+                            orow[nt * 256 + 128 + L] = __uint_as_float(v1[j]);
                         }
                     }
                 }

@@ -34,7 +34,7 @@ struct RouteGroupArgs {
 void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s);
 void launch_gather(const __nv_bfloat16 *x, int P, int H, int k, const int32_t *pos_of_pair, __nv_bfloat16 *A,
                    int act_mxfp8, int num_sms, cudaStream_t s);
-void launch_combine(const __nv_bfloat16 *Y, int T, int H, int k, const int32_t *pos_of_pair, const float *topk_w,
+void launch_combine(const float *Y, int T, int H, int k, const int32_t *pos_of_pair, const float *topk_w,
                     __nv_bfloat16 *out, int num_sms, cudaStream_t s);
 void launch_mx_quantize(const float *src, int64_t rows, int64_t K, int fmt, uint8_t *codes, uint8_t *scales,
                         int num_sms, cudaStream_t s);
@@ -44,7 +44,7 @@ struct FcGemmArgs {
     const int4 *rowblocks;       // {expert, first grouped row, rows, 0}
     const int32_t *num_rowblocks;
     const uint8_t *wscale;       // E8M0 scales of the weight, [E*R, K/32]
-    __nv_bfloat16 *out;          // FC1: Hbuf [rows, I]; FC2: Y [rows, H]
+    void *out;                   // FC1: bf16 Hbuf [rows, I]; FC2: f32 Y [rows, H]
     uint32_t *err;
     unsigned long long timeout_ns;
     int K;                       // reduction length (FC1: H, FC2: I)

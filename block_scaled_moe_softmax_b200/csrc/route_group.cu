@@ -236,8 +236,9 @@ __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16 *__rest
 
 // ---------------------------------------------------------------- combine
 // out[t, n] = bf16( sum_{j<k} w[t,j] * Y[pos(t,j), n] ), j ascending, f32.
-// One thread per 8 consecutive outputs (16-byte loads and stores).
-__global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16 *__restrict__ Y, int T, int H, int k,
+// Y is kept in f32 so the only rounding of the result is the final one.
+// One thread per 8 consecutive outputs (2 x 16-byte loads per slot, one 16-byte store).
+__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ Y, int T, int H, int k,
                                                       const int32_t *__restrict__ pos_of_pair,
                                                       const float *__restrict__ topk_w,
                                                       __nv_bfloat16 *__restrict__ out)
@@ -255,14 +256,16 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16 *__res
         for (int j = 0; j < k; ++j) {
             const float w = __ldg(topk_w + (size_t)t * k + j);
             const int row = __ldg(pos_of_pair + (size_t)t * k + j);
-            const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(Y + (size_t)row * H) + c);
-            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float2 f = __bfloat1622float2(h2[i]);
-                acc[2 * i] = fmaf(w, f.x, acc[2 * i]);
-                acc[2 * i + 1] = fmaf(w, f.y, acc[2 * i + 1]);
-            }
+            const float4 *src = reinterpret_cast<const float4 *>(Y + (size_t)row * H) + 2 * c;
+            const float4 a0 = __ldg(src), a1 = __ldg(src + 1);
+            acc[0] = fmaf(w, a0.x, acc[0]);
+            acc[1] = fmaf(w, a0.y, acc[1]);
+            acc[2] = fmaf(w, a0.z, acc[2]);
+            acc[3] = fmaf(w, a0.w, acc[3]);
+            acc[4] = fmaf(w, a1.x, acc[4]);
+            acc[5] = fmaf(w, a1.y, acc[5]);
+            acc[6] = fmaf(w, a1.z, acc[6]);
+            acc[7] = fmaf(w, a1.w, acc[7]);
         }
         uint4 o;
         __nv_bfloat162 *o2 = reinterpret_cast<__nv_bfloat162 *>(&o);
@@ -292,7 +295,7 @@ void launch_gather(const __nv_bfloat16 *x, int P, int H, int k, const int32_t *p
     gather_kernel<<<grid > 0 ? grid : 1, 256, 0, s>>>(x, P, H, k, pos_of_pair, A, act_mxfp8);
 }
 
-void launch_combine(const __nv_bfloat16 *Y, int T, int H, int k, const int32_t *pos_of_pair, const float *topk_w,
+void launch_combine(const float *Y, int T, int H, int k, const int32_t *pos_of_pair, const float *topk_w,
                     __nv_bfloat16 *out, int num_sms, cudaStream_t s)
 {
     const long long work = (long long)T * (H / 8);

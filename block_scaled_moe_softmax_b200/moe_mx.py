@@ -43,7 +43,10 @@ SIGNATURES = {
     "moe_mx_max_grouped_rows": (_I64, [_P, _I, _I]),
     "moe_mx_get_routing": (_I, [_P, _P, _P, _P, _P, _P, _P]),
     "moe_mx_debug_watchdog": (_I, [_P, _I, _P]),
+    "moe_mx_set_stage_timing": (_I, [_P, _I]),
+    "moe_mx_get_stage_times": (_I, [_P, _P]),
 }
+STAGES = ("route", "gather", "fc1", "fc2", "combine")
 
 _lock = threading.Lock()
 _lib = None
@@ -142,6 +145,16 @@ def moe_mx_get_routing(handle: int, topk_ids=None, topk_w=None, counts=None, pad
 
 def moe_mx_debug_watchdog(handle: int, timeout_us: int, stream=None) -> None:
     _check(load_library().moe_mx_debug_watchdog(handle, timeout_us, _stream(stream)))
+
+
+def moe_mx_set_stage_timing(handle: int, enable: bool) -> None:
+    _check(load_library().moe_mx_set_stage_timing(handle, int(bool(enable))))
+
+
+def moe_mx_get_stage_times(handle: int) -> dict:
+    ms = (ctypes.c_float * len(STAGES))()
+    _check(load_library().moe_mx_get_stage_times(handle, ctypes.cast(ms, ctypes.c_void_p)))
+    return dict(zip(STAGES, [float(v) for v in ms]))
 
 
 # ------------------------------------------------------------------ convenience wrappers

@@ -186,6 +186,31 @@ MOE_MX_API int64_t moe_mx_max_grouped_rows(const moe_mx_handle *h, int num_token
 MOE_MX_API int moe_mx_get_routing(const moe_mx_handle *h, int32_t *topk_ids, float *topk_w, int32_t *counts,
                        int32_t *pad_offsets, int32_t *sorted_pair, void *stream);
 
+/* Stages of one forward, in launch order (indices into moe_mx_get_stage_times). */
+#define MOE_MX_STAGE_ROUTE 0   /* routing, histogram, scan, stable scatter */
+#define MOE_MX_STAGE_GATHER 1  /* gather of activation rows (+ MXFP8 quantisation) */
+#define MOE_MX_STAGE_FC1 2     /* FC1 grouped GEMM with the SwiGLU epilogue */
+#define MOE_MX_STAGE_FC2 3     /* FC2 grouped GEMM */
+#define MOE_MX_STAGE_COMBINE 4 /* weighted combine */
+#define MOE_MX_NUM_STAGES 5
+
+/*
+ * Enable (1) or disable (0) per-stage timing.  Enabling (again) resets the
+ * record.  While enabled, every forward records CUDA events on its stream
+ * between its stages (no host synchronisation; a few microseconds of device
+ * overhead per forward); the events of the last 1024 timed forwards are kept.
+ * Errors: INVALID_ARG, CUDA.
+ */
+MOE_MX_API int moe_mx_set_stage_timing(moe_mx_handle *h, int enable);
+
+/*
+ * Mean per-stage device time, in milliseconds, over the timed forwards kept
+ * (at most the last 1024 since timing was enabled): ms[MOE_MX_NUM_STAGES],
+ * indexed by MOE_MX_STAGE_*.  Waits for the last timed forward's final event.
+ * Errors: INVALID_ARG (timing not enabled or no timed forward yet), CUDA.
+ */
+MOE_MX_API int moe_mx_get_stage_times(moe_mx_handle *h, float *ms);
+
 /*
  * Self-test of the device watchdog: launch one kernel that waits on a device
  * flag nothing sets, with a wait limit of timeout_us microseconds.  The wait
