@@ -53,15 +53,16 @@ EncodeTiledFn get_encode_fn()
     return fn;
 }
 
-// 2-D row-major tensor map: inner dimension `cols` elements, `rows` rows.
-int encode_2d(CUtensorMap *map, CUtensorMapDataType dt, int elem_bytes, const void *ptr, uint64_t cols,
+// 2-D row-major tensor map: inner dimension `cols` elements, `rows` rows,
+// `row_bytes` bytes from one row to the next.
+int encode_2d(CUtensorMap *map, CUtensorMapDataType dt, uint64_t row_bytes, const void *ptr, uint64_t cols,
               uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz)
 {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc)
         return fail(MOE_MX_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
     const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
+    const cuuint64_t strides[1] = {row_bytes};
     const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = enc(map, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr,
@@ -120,10 +121,10 @@ struct moe_mx_handle {
     int32_t *topk_ids, *chunk_hist, *counts, *pad_offsets, *num_rowblocks, *sorted_pair, *pos_of_pair;
     float *topk_w;
     int4 *rowblocks;
-    __nv_bfloat16 *A, *Hbuf;
+    uint8_t *Aq, *Asf, *Hq, *Hsf; // MXFP8 operand planes [2][rows][K] and their scale atoms
     float *Y;
     uint32_t *err;
-    CUtensorMap map_A, map_H;
+    CUtensorMap map_A, map_A16, map_H, map_H16;
     const void *w1_key, *w2_key;
     CUtensorMap map_w1, map_w2;
     int last_T, last_k;
@@ -158,8 +159,8 @@ int moe_mx_create(moe_mx_handle **out, int hidden, int inter, int num_experts, i
     if (!out)
         return fail(MOE_MX_ERR_INVALID_ARG, "out is NULL");
     *out = nullptr;
-    if (hidden < 256 || hidden > 16384 || hidden % 256 != 0)
-        return fail(MOE_MX_ERR_UNSUPPORTED, "hidden=%d must be a multiple of 256 in [256, 16384]", hidden);
+    if (hidden < 128 || hidden > 16384 || hidden % 128 != 0)
+        return fail(MOE_MX_ERR_UNSUPPORTED, "hidden=%d must be a multiple of 128 in [128, 16384]", hidden);
     if (inter < 128 || inter > 8192 || inter % 128 != 0)
         return fail(MOE_MX_ERR_UNSUPPORTED, "inter=%d must be a multiple of 128 in [128, 8192]", inter);
     if (num_experts < 1 || num_experts > kMaxExperts)
@@ -217,8 +218,10 @@ int moe_mx_create(moe_mx_handle **out, int hidden, int inter, int num_experts, i
         {(void **)&h->sorted_pair, sizeof(int32_t) * h->max_rows},
         {(void **)&h->pos_of_pair, sizeof(int32_t) * pairs},
         {(void **)&h->err, sizeof(uint32_t)},
-        {(void **)&h->A, sizeof(__nv_bfloat16) * h->max_rows * hidden},
-        {(void **)&h->Hbuf, sizeof(__nv_bfloat16) * h->max_rows * inter},
+        {(void **)&h->Aq, (size_t)2 * h->max_rows * hidden},
+        {(void **)&h->Asf, (size_t)(h->max_rows / 128) * (hidden / 128) * 1024},
+        {(void **)&h->Hq, (size_t)2 * h->max_rows * inter},
+        {(void **)&h->Hsf, (size_t)(h->max_rows / 128) * (inter / 128) * 1024},
         {(void **)&h->Y, sizeof(float) * h->max_rows * hidden},
     };
     size_t total = 0;
@@ -240,11 +243,19 @@ int moe_mx_create(moe_mx_handle **out, int hidden, int inter, int num_experts, i
         rc = cuda_fail(ce, "cudaMemset(workspace)");
     if (rc == MOE_MX_OK && (ce = fc_gemm_prepare()) != cudaSuccess)
         rc = cuda_fail(ce, "cudaFuncSetAttribute(fc_gemm)");
+    // activation operand planes: [2 terms x rows, K] E4M3 codes, 128 x 128 boxes (16-row boxes for
+    // token-on-N tiles), 128-byte swizzle = the K-major layout the MMA reads
     if (rc == MOE_MX_OK)
-        rc = encode_2d(&h->map_A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h->A, hidden, h->max_rows, 64, 128,
+        rc = encode_2d(&h->map_A, CU_TENSOR_MAP_DATA_TYPE_UINT8, hidden, h->Aq, hidden, 2 * h->max_rows, 128, 128,
                        CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc == MOE_MX_OK)
-        rc = encode_2d(&h->map_H, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h->Hbuf, inter, h->max_rows, 64, 128,
+        rc = encode_2d(&h->map_A16, CU_TENSOR_MAP_DATA_TYPE_UINT8, hidden, h->Aq, hidden, 2 * h->max_rows, 128, 16,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc == MOE_MX_OK)
+        rc = encode_2d(&h->map_H, CU_TENSOR_MAP_DATA_TYPE_UINT8, inter, h->Hq, inter, 2 * h->max_rows, 128, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc == MOE_MX_OK)
+        rc = encode_2d(&h->map_H16, CU_TENSOR_MAP_DATA_TYPE_UINT8, inter, h->Hq, inter, 2 * h->max_rows, 128, 16,
                        CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc == MOE_MX_OK && (ce = cudaDeviceSynchronize()) != cudaSuccess)
         rc = cuda_fail(ce, "cudaDeviceSynchronize(create)");
@@ -301,6 +312,8 @@ int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, 
         return rc;
     if (x == out)
         return fail(MOE_MX_ERR_INVALID_ARG, "out must not alias x");
+    if (reinterpret_cast<uintptr_t>(w1) % 32 != 0 || reinterpret_cast<uintptr_t>(w2) % 32 != 0)
+        return fail(MOE_MX_ERR_INVALID_ARG, "w1 and w2 must be 32-byte aligned");
 
     const int H = h->H, I = h->I, E = h->E, T = num_tokens, k = top_k;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -309,15 +322,17 @@ int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, 
     if (prev != h->dev)
         cudaSetDevice(h->dev);
 
+    // weights: packed E2M1 [rows, K] unpacked by the TMA into 8-bit containers (16 codes per
+    // 16-byte granule), 128-code x 64-row boxes, 128-byte swizzle
     if (w1 != h->w1_key) {
-        if ((rc = encode_2d(&h->map_w1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w1, H / 2, (uint64_t)E * 2 * I, 32, 128,
-                            CU_TENSOR_MAP_SWIZZLE_NONE)))
+        if ((rc = encode_2d(&h->map_w1, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, H / 2, w1, H, (uint64_t)E * 2 * I,
+                            128, 64, CU_TENSOR_MAP_SWIZZLE_128B)))
             goto done;
         h->w1_key = w1;
     }
     if (w2 != h->w2_key) {
-        if ((rc = encode_2d(&h->map_w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w2, I / 2, (uint64_t)E * H, 32, 128,
-                            CU_TENSOR_MAP_SWIZZLE_NONE)))
+        if ((rc = encode_2d(&h->map_w2, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, I / 2, w2, I, (uint64_t)E * H, 128,
+                            64, CU_TENSOR_MAP_SWIZZLE_128B)))
             goto done;
         h->w2_key = w2;
     }
@@ -339,37 +354,44 @@ int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, 
                           h->pad_offsets, h->rowblocks, h->num_rowblocks, h->sorted_pair, h->pos_of_pair};
         launch_route_and_group(ra, s);
         mark(1);
-        launch_gather(static_cast<const __nv_bfloat16 *>(x), (int)pairs, H, k, h->pos_of_pair, h->A,
-                      act_dtype == MOE_MX_ACT_MXFP8, h->num_sms, s);
+        const int mx8 = act_dtype == MOE_MX_ACT_MXFP8;
+        launch_gather(static_cast<const __nv_bfloat16 *>(x), (int)pairs, H, k, h->pos_of_pair, h->Aq, h->Asf,
+                      (int)h->max_rows, mx8, h->num_sms, s);
 
         FcGemmArgs f1{};
         f1.rowblocks = h->rowblocks;
         f1.num_rowblocks = h->num_rowblocks;
         f1.wscale = w1_scale;
-        f1.out = h->Hbuf;
+        f1.act_sf = h->Asf;
+        f1.hq = h->Hq;
+        f1.hsf = h->Hsf;
+        f1.y = h->Y;
         f1.err = h->err;
         f1.timeout_ns = h->timeout_ns;
         f1.K = H;
         f1.R = 2 * I;
-        f1.n_tiles = I / 128;
+        f1.n_tiles = I / 64;
         f1.out_ld = I;
+        f1.act_rows = (int)h->max_rows;
+        f1.hq_rows = (int)h->max_rows;
+        f1.terms = mx8 ? 1 : 2;
         f1.fc1 = 1;
-        f1.act_mxfp8 = act_dtype == MOE_MX_ACT_MXFP8;
+        f1.act_mxfp8 = mx8;
         f1.swap_rows = h->swap_rows;
         mark(2);
-        launch_fc_gemm(f1, h->map_A, h->map_w1, h->num_sms, s);
+        launch_fc_gemm(f1, h->map_A, h->map_A16, h->map_w1, h->num_sms, s);
         mark(3);
 
         FcGemmArgs f2 = f1;
         f2.wscale = w2_scale;
-        f2.out = h->Y;
+        f2.act_sf = h->Hsf;
         f2.K = I;
         f2.R = H;
-        f2.n_tiles = H / 256;
+        f2.n_tiles = H / 128;
         f2.out_ld = H;
         f2.fc1 = 0;
         f2.act_mxfp8 = 0;
-        launch_fc_gemm(f2, h->map_H, h->map_w2, h->num_sms, s);
+        launch_fc_gemm(f2, h->map_H, h->map_H16, h->map_w2, h->num_sms, s);
         mark(4);
         launch_combine(h->Y, T, H, k, h->pos_of_pair, h->topk_w, static_cast<__nv_bfloat16 *>(out), h->num_sms, s);
         ce = cudaGetLastError();

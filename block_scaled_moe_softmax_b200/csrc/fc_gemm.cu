@@ -1,35 +1,39 @@
-// fc_gemm.cu -- persistent grouped GEMM for FC1 (+SwiGLU) and FC2 with MXFP4
-// weights on the 5th-generation tensor cores (tcgen05, accumulators in TMEM).
+// fc_gemm.cu -- persistent grouped GEMM for FC1 (+SwiGLU) and FC2 on the
+// 5th-generation tensor cores, consuming the MXFP4 weights directly.
 //
-// What it computes (tokenspeed-situ package description, intro: "FC1 MXFP4 +
-// <gated activation>" and the matching FC2; b12x package description, "What's
-// in here": "W4A16 ... with inline FP4 weight dequant"): for every row block
-// (an expert's slice of at most 128 grouped rows) and every 256-row tile of
-// that expert's weight,
-//     D[rows, 256] = A[rows, K] . W[256, K]^T,   f32 accumulation,
-// with W decoded from MXFP4 (E2M1 code * 2^(E8M0 - 127)) to bf16 on chip.
-// FC1 tiles pair 128 gate rows with the matching 128 up rows, so the epilogue
-// applies h = silu(gate) * up in registers (and, on the w4a8 path, the MXFP8
-// round trip of h: tokenspeed-situ package description, "Activation precision
-// (w4a16 vs w4a8)").
+// What it computes (tokenspeed-situ package description, intro: FC1 "MXFP4 +
+// <gated activation>" and the matching FC2, and "Activation precision (w4a16
+// vs w4a8)"): for every row block (an expert's slice of at most 128 grouped
+// rows) and every 128-row tile of that expert's weight,
+//     D[rows, 128] = A[rows, K] . W[128, K]^T,   f32 accumulation,
+// with W the E2M1 codes times their E8M0 block scales (OCP MX: one scale per 32
+// elements along K) and A the activation rows as MXFP8 E4M3 with E8M0 block
+// scales.  tcgen05.mma kind::mxf8f6f4.block_scale applies both scales inside
+// the tensor core, so no weight element is ever dequantised by the ALU:
+//   * w4a8: A is the MXFP8-quantised activation (one term);
+//   * w4a16: A is a two-term MXFP8 expansion of the bf16 activation,
+//     x = x1 + x2 (see mx_encode32 in kernels.cuh), accumulated by two MMAs
+//     into the same TMEM accumulator.
+// FC1 tiles hold 64 gate rows followed by the matching 64 up rows, so the
+// epilogue forms h = silu(gate) * up and writes h for FC2 in the same MXFP8
+// form (two terms of h rounded to bf16 for w4a16; the OCP-quantised h for
+// w4a8, whose dequantised value is the bf16 value FC2 consumes).  FC2 writes
+// f32 rows that the combine kernel sums.
 //
 // Per CTA (one per SM, persistent over work units u = (row block, tile)):
-//   warp 0      producer: TMA of the activation tile (128 x 64 bf16, 128-byte
-//               swizzle) and of the FP4 weight tile (256 x 32 bytes), cp.async
-//               of the scale bytes; one mbarrier per stage.
-//   warps 2-5   dequant: FP4 + E8M0 -> bf16 into the 128-byte swizzled
-//               K-major layout the tensor core reads.
-//   warp 1      MMA issuer (one thread) + TMEM owner; tcgen05.mma kind::f16,
-//               commits free the stage and publish the accumulator.
-//   warps 6-9   epilogue: tcgen05.ld -> FC1: SwiGLU -> bf16 stores,
-//               FC2: f32 stores (the combine rounds once, at the end); the
-//               accumulator is double-buffered in TMEM (2 x 256 columns).
-// Orientation per work unit: a block of more than `swap_rows` rows runs with
-// tokens on the MMA's M side (M = 128, N = 256 weight rows); a smaller block
-// (decode) runs weight rows on M (two M = 128 MMAs, gate/up or lower/upper
-// half) and its tokens on N (16..128), so the tensor core does not multiply
-// padding rows.  Every wait is bounded; a wait that gives up records an error
-// word and the CTA drains its own copies and MMAs before freeing TMEM.
+//   warp 0      producer: TMA of the activation codes (128-byte swizzle), TMA
+//               of the E2M1 codes through the 4-bit -> 8-bit-container
+//               unpacking mode, a bulk copy of the activation scale atoms and
+//               cp.async of the weight scale bytes into the same atom layout;
+//   warp 1      MMA issuer (one thread) + TMEM owner: tcgen05.cp moves the
+//               stage's scale atoms to TMEM, then the block-scaled MMAs;
+//   warps 2-5   epilogue (tcgen05.ld); accumulators double-buffered in TMEM.
+// Orientation per work unit: a block of more than `swap_rows` rows puts its
+// tokens on the MMA's M side (M = 128, N = 128 weight rows); a smaller block
+// (decode) puts the weight rows on M and its tokens on N (16..128), so the
+// tensor core does not multiply padding rows.  Every wait is bounded; a wait
+// that gives up records an error word, and the CTA drains its own copies and
+// MMAs before freeing TMEM.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -37,109 +41,133 @@ namespace moe_mx {
 
 namespace {
 
-constexpr int kStages = 3;
-constexpr int kThreads = 320;
-constexpr int kActBytes = 128 * 128;      // 128 rows x 64 bf16
-constexpr int kWbBytes = 256 * 128;       // 256 rows x 64 bf16 (dequantised)
-constexpr int kFp4Bytes = 256 * 32;       // 256 rows x 64 FP4 codes
-constexpr int kSclBytes = 256 * 4;        // 256 rows x one 4-byte scale word
+constexpr int kStages = 4;
+constexpr int kThreads = 192;
+constexpr int kTermBytes = 128 * 128;          // 128 rows x 128 E4M3 codes
+constexpr int kActBytes = 2 * kTermBytes;      // up to two terms
+constexpr int kWBytes = 128 * 128;             // 128 rows x 128 E2M1 codes in 8-bit containers
+constexpr int kWTxBytes = 128 * 128 / 2;       // ... of which the TMA transfers (and counts) the packed 4-bit data
+constexpr int kAsfBytes = 2 * 512;             // one 512-byte scale atom per term
+constexpr int kWsfBytes = 512;
 constexpr int kOffAct = 0;
-constexpr int kOffWb = kOffAct + kStages * kActBytes;
-constexpr int kOffFp4 = kOffWb + kStages * kWbBytes;
-constexpr int kOffScl = kOffFp4 + kStages * kFp4Bytes;
-constexpr int kOffBar = kOffScl + kStages * kSclBytes;
-constexpr int kNumBars = 4 * kStages + 4 + 1;
+constexpr int kOffW = kOffAct + kStages * kActBytes;
+constexpr int kOffAsf = kOffW + kStages * kWBytes;
+constexpr int kOffWsf = kOffAsf + kStages * kAsfBytes;
+constexpr int kOffX = kOffWsf + kStages * kWsfBytes; // epilogue exchange, 64 lanes x 16 columns f32
+constexpr int kXBytes = 64 * 16 * 4;
+constexpr int kOffBar = kOffX + kXBytes;
+constexpr int kNumBars = 2 * kStages + 1 + 4;
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffTmemSlot + 16 + 1024; // + slack for 1024-byte alignment
 constexpr uint32_t kTmemCols = 512;
-constexpr unsigned long long kDrainTimeoutNs = 200000000ull; // 0.2 s for the final drains
+constexpr uint32_t kSfCol = 256; // TMEM columns 256..267 hold the stage's scale factors
+constexpr unsigned long long kDrainTimeoutNs = 200000000ull;
+
+constexpr uint32_t kFmtE4M3 = 0, kFmtE2M1 = 5;
 
 struct Bars {
     uint32_t base;
-    __device__ uint32_t full_tma(int s) const { return base + 8 * s; }
-    __device__ uint32_t full_deq(int s) const { return base + 8 * (kStages + s); }
-    __device__ uint32_t empty(int s) const { return base + 8 * (2 * kStages + s); }
-    __device__ uint32_t mma_done() const { return base + 8 * (3 * kStages); }
-    __device__ uint32_t acc_full(int b) const { return base + 8 * (3 * kStages + 1 + b); }
-    __device__ uint32_t acc_empty(int b) const { return base + 8 * (3 * kStages + 3 + b); }
+    __device__ uint32_t full(int s) const { return base + 8 * s; }
+    __device__ uint32_t empty(int s) const { return base + 8 * (kStages + s); }
+    __device__ uint32_t mma_done() const { return base + 8 * (2 * kStages); }
+    __device__ uint32_t acc_full(int b) const { return base + 8 * (2 * kStages + 1 + b); }
+    __device__ uint32_t acc_empty(int b) const { return base + 8 * (2 * kStages + 3 + b); }
 };
+
+// Instruction descriptor of kind::mxf8f6f4 with E8M0 block scales (one scale
+// per 32 elements): [4,6) B scale byte, [7,10) A format, [10,13) B format,
+// [17,23) N/8, [23] scale format E8M0, [24,29) M/16, [29,31) A scale byte.
+__device__ __forceinline__ uint32_t idesc_mx(uint32_t a_fmt, uint32_t b_fmt, uint32_t M, uint32_t N, uint32_t sf_id)
+{
+    return (sf_id << 4) | (a_fmt << 7) | (b_fmt << 10) | ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24) |
+           (sf_id << 29);
+}
+
+__device__ __forceinline__ void umma_mx(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// Copy one 512-byte scale atom (32 rows x 16 bytes) from shared memory to TMEM
+// columns [col, col+4), replicated into the four 32-lane quarters: lane
+// (32q + r) column (col + j) then holds the four scale bytes (one per 32-element
+// block) of tile row r + 32j.
+__device__ __forceinline__ void tmem_cp_sf_atom(uint32_t taddr, uint32_t saddr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+    d |= (uint64_t)1 << 16;          // leading offset (single 16-byte column)
+    d |= (uint64_t)(128 >> 4) << 32; // next 8-row core matrix: 128 bytes
+    d |= (uint64_t)1 << 46;          // descriptor version
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
+}
+
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// All `count` threads of named barrier `id` agree on v (logical AND).
+__device__ __forceinline__ bool named_bar_all(uint32_t id, uint32_t count, bool v)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
 
 __device__ __forceinline__ float silu_mul(float g, float u)
 {
     return g / (1.0f + expf(-g)) * u;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
-{
-    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t *>(&v);
-}
-
-// Store 32 floats as bf16 (64 contiguous bytes).
-__device__ __forceinline__ void store_bf16x32(__nv_bfloat16 *dst, const float (&v)[32])
-{
-    uint4 *d = reinterpret_cast<uint4 *>(dst);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        d[i] = make_uint4(pack_bf16x2(v[8 * i + 0], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
-                          pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
-}
-
-// MXFP8 round trip of 32 values held by one thread (quantise, then dequantise).
-__device__ __forceinline__ void mxfp8_roundtrip32(float (&v)[32])
-{
-    uint8_t c[32];
-    const uint32_t sb = mx_quantize32_e4m3(v, c);
-    const float scale = (sb == 0xFF) ? __uint_as_float(0x7FC00000u) : exp2_int((int)sb - 127);
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-        v[i] = __fmul_rn(e4m3_to_f32(c[i]), scale);
-}
-
-// MXFP8 round trip of one value per lane, the 32 lanes forming one MX block.
-__device__ __forceinline__ float mxfp8_roundtrip_warp(float v)
-{
-    float amax = fabsf(v);
-    bool finite = amax <= 3.402823466e38f;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-    finite = __all_sync(0xFFFFFFFFu, finite);
-    if (!finite)
-        return __uint_as_float(0x7FC00000u);
-    int s = (amax == 0.f) ? -127 : floor_log2_pos(amax) - 8;
-    s = max(-127, min(127, s));
-    const uint32_t code = f32_to_e4m3(__fmul_rn(v, exp2_int(-s)));
-    return __fmul_rn(e4m3_to_f32(code), exp2_int(s));
-}
-
 } // namespace
 
 __global__ void __launch_bounds__(kThreads, 1)
     fc_gemm_kernel(const FcGemmArgs a, const __grid_constant__ CUtensorMap act_map,
-                   const __grid_constant__ CUtensorMap w_map)
+                   const __grid_constant__ CUtensorMap act_map16, const __grid_constant__ CUtensorMap w_map)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
-    uint8_t *const gsm = smem_raw + (base - raw); // generic pointer to the aligned base
+    uint8_t *const gsm = smem_raw + (base - raw);
     const Bars bars{base + kOffBar};
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(bars.full_tma(s), 1 + 32); // producer's expect_tx + 32 cp.async arrivals
-            mbar_init(bars.full_deq(s), 128);    // every dequant thread
-            mbar_init(bars.empty(s), 1);         // MMA commit
+            mbar_init(bars.full(s), 1 + 32); // producer's expect_tx + 32 cp.async arrivals
+            mbar_init(bars.empty(s), 1);     // MMA commit
         }
         mbar_init(bars.mma_done(), 1);
         for (int b = 0; b < 2; ++b) {
-            mbar_init(bars.acc_full(b), 1);   // MMA commit
-            mbar_init(bars.acc_empty(b), 128); // every epilogue thread
+            mbar_init(bars.acc_full(b), 1);
+            mbar_init(bars.acc_empty(b), 128);
         }
         fence_mbar_init();
         fence_proxy_async_smem();
         prefetch_tensormap(&act_map);
+        prefetch_tensormap(&act_map16);
         prefetch_tensormap(&w_map);
     }
     if (warp == 1) {
@@ -153,8 +181,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int nrb = *a.num_rowblocks;
     const int total_units = nrb * a.n_tiles;
-    const int kst = a.K / 64;
-    const int half_rows = a.fc1 ? a.R / 2 : 0; // FC1: offset of the up rows
+    const int kst = a.K / 128; // K stages of 128 elements (4 scale blocks)
+    const int terms = a.terms; // activation terms per row: 1 (w4a8) or 2 (w4a16)
     const unsigned long long tmo = a.timeout_ns;
 
     if (warp == 0) {
@@ -165,8 +193,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
             const int4 blk = a.rowblocks[u / a.n_tiles];
             const int nt = u % a.n_tiles;
-            const int wrow_a = blk.x * a.R + (a.fc1 ? nt * 128 : nt * 256);
-            const int wrow_b = a.fc1 ? wrow_a + half_rows : wrow_a + 128;
+            const bool swap = blk.z <= a.swap_rows;
+            const int npad = (blk.z + 15) & ~15;
+            // weight rows of this tile, as two 64-row halves: FC1 tile nt = gate rows [64nt, 64nt+64)
+            // then the matching up rows; FC2 tile nt = rows [128nt, 128nt+128)
+            const int wrow_a = blk.x * a.R + (a.fc1 ? nt * 64 : nt * 128);
+            const int wrow_b = a.fc1 ? wrow_a + a.R / 2 : wrow_a + 64;
+            const int rb = blk.y / 128;
+            const uint32_t act_bytes = (uint32_t)terms * (swap ? (uint32_t)npad * 128u : (uint32_t)kTermBytes);
             for (int kk = 0; kk < kst; ++kk, ++g) {
                 const int s = g % kStages;
                 const uint32_t ph = (g / kStages) & 1;
@@ -178,19 +212,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
-                const uint32_t scl = base + kOffScl + s * kSclBytes;
-                for (int r = lane; r < 256; r += 32) {
-                    const int wr = r < 128 ? wrow_a + r : wrow_b + (r - 128);
-                    cp_async_4(scl + 4 * r, a.wscale + (size_t)wr * scl_ld + (kk >> 1) * 4);
+                // weight scale bytes: 4 per row (the 4 blocks of this K stage) into the atom layout
+                const uint32_t wsf = base + kOffWsf + s * kWsfBytes;
+                for (int r = lane; r < 128; r += 32) {
+                    const int wr = r < 64 ? wrow_a + r : wrow_b + (r - 64);
+                    cp_async_4(wsf + sf_atom_offset(r, 0), a.wscale + (size_t)wr * scl_ld + kk * 4);
                 }
-                cp_async_mbar_arrive_noinc(bars.full_tma(s));
+                cp_async_mbar_arrive_noinc(bars.full(s));
                 __syncwarp();
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(bars.full_tma(s), kActBytes + kFp4Bytes);
-                    tma_load_2d(base + kOffAct + s * kActBytes, &act_map, kk * 64, blk.y, bars.full_tma(s));
-                    const uint32_t f = base + kOffFp4 + s * kFp4Bytes;
-                    tma_load_2d(f, &w_map, kk * 32, wrow_a, bars.full_tma(s));
-                    tma_load_2d(f + kFp4Bytes / 2, &w_map, kk * 32, wrow_b, bars.full_tma(s));
+                    mbar_arrive_expect_tx(bars.full(s), act_bytes + kWTxBytes + (uint32_t)terms * 512u);
+                    const uint32_t act = base + kOffAct + s * kActBytes;
+                    for (int t = 0; t < terms; ++t) {
+                        const int row = t * a.act_rows + blk.y;
+                        if (!swap) {
+                            tma_load_2d(act + t * kTermBytes, &act_map, kk * 128, row, bars.full(s));
+                        } else {
+                            for (int r16 = 0; r16 < npad; r16 += 16)
+                                tma_load_2d(act + t * kTermBytes + r16 * 128, &act_map16, kk * 128, row + r16,
+                                            bars.full(s));
+                        }
+                    }
+                    const uint32_t wdst = base + kOffW + s * kWBytes;
+                    tma_load_2d(wdst, &w_map, kk * 128, wrow_a, bars.full(s));
+                    tma_load_2d(wdst + kWBytes / 2, &w_map, kk * 128, wrow_b, bars.full(s));
+                    bulk_copy_g2s(base + kOffAsf + s * kAsfBytes, a.act_sf + ((size_t)rb * kst + kk) * 1024,
+                                  (uint32_t)terms * 512u, bars.full(s));
                 }
                 __syncwarp();
             }
@@ -199,47 +246,50 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             const uint32_t first = g > (uint32_t)kStages ? g - kStages : 0u;
             for (uint32_t q = first; q < g; ++q)
-                mbar_wait_bounded(bars.full_tma(q % kStages), (q / kStages) & 1, nullptr, kDrainTimeoutNs);
+                mbar_wait_bounded(bars.full(q % kStages), (q / kStages) & 1, nullptr, kDrainTimeoutNs);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             uint32_t g = 0, cnt = 0;
             bool ok = true;
+            const uint32_t sf_w = tmem_base + kSfCol;
             for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x, ++cnt) {
                 const int4 blk = a.rowblocks[u / a.n_tiles];
                 const bool swap = blk.z <= a.swap_rows;
                 const uint32_t npad = (uint32_t)((blk.z + 15) & ~15);
-                const uint32_t idesc = swap ? idesc_bf16_f32(128, npad) : idesc_bf16_f32(128, 256);
                 const int buf = cnt & 1;
                 if (!mbar_wait_bounded(bars.acc_empty(buf), ((cnt >> 1) & 1) ^ 1, a.err, tmo)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d = tmem_base + buf * 256;
+                const uint32_t d = tmem_base + buf * 128;
                 for (int kk = 0; kk < kst; ++kk, ++g) {
                     const int s = g % kStages;
                     const uint32_t ph = (g / kStages) & 1;
-                    if (!mbar_wait_bounded(bars.full_tma(s), ph, a.err, tmo) ||
-                        !mbar_wait_bounded(bars.full_deq(s), ph, a.err, tmo)) {
+                    if (!mbar_wait_bounded(bars.full(s), ph, a.err, tmo)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
+                    // scale atoms -> TMEM (in order with the MMAs below and with the previous stage's MMAs)
+                    tmem_cp_sf_atom(sf_w, base + kOffWsf + s * kWsfBytes);
+                    for (int t = 0; t < terms; ++t)
+                        tmem_cp_sf_atom(sf_w + 4 + 4 * t, base + kOffAsf + s * kAsfBytes + 512 * t);
                     const uint32_t act = base + kOffAct + s * kActBytes;
-                    const uint32_t wb = base + kOffWb + s * kWbBytes;
+                    const uint32_t wt = base + kOffW + s * kWBytes;
 #pragma unroll
-                    for (int k16 = 0; k16 < 4; ++k16) {
-                        const uint64_t da = smem_desc_sw128(act + 32 * k16);
-                        const uint64_t dw = smem_desc_sw128(wb + 32 * k16);
-                        const uint32_t acc = (kk | k16) != 0;
-                        if (!swap) {
-                            umma_f16_ss(d, da, dw, idesc, acc);
-                        } else {
-                            const uint64_t dw_hi = smem_desc_sw128(wb + kWbBytes / 2 + 32 * k16);
-                            umma_f16_ss(d, dw, da, idesc, acc);
-                            umma_f16_ss(d + 128, dw_hi, da, idesc, acc);
+                    for (int k32 = 0; k32 < 4; ++k32) {
+                        const uint64_t dw = smem_desc_sw128(wt + 32 * k32);
+                        for (int t = 0; t < terms; ++t) {
+                            const uint64_t da = smem_desc_sw128(act + t * kTermBytes + 32 * k32);
+                            const uint32_t sf_a = sf_w + 4 + 4 * t;
+                            const uint32_t acc = (kk | k32 | t) != 0;
+                            if (!swap)
+                                umma_mx(d, da, dw, idesc_mx(kFmtE4M3, kFmtE2M1, 128, 128, k32), sf_a, sf_w, acc);
+                            else
+                                umma_mx(d, dw, da, idesc_mx(kFmtE2M1, kFmtE4M3, 128, npad, k32), sf_w, sf_a, acc);
                         }
                     }
                     umma_commit(bars.empty(s));
@@ -252,52 +302,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait_bounded(bars.mma_done(), 0, nullptr, kDrainTimeoutNs);
         }
         __syncwarp();
-    } else if (warp >= 2 && warp < 6) {
-        // ------------------------------------------------------------ dequant
-        const int t = threadIdx.x - 64; // 0..127
-        uint32_t g = 0;
-        bool ok = true;
-        for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
-            for (int kk = 0; kk < kst; ++kk, ++g) {
-                const int s = g % kStages;
-                const uint32_t ph = (g / kStages) & 1;
-                if (!mbar_wait_bounded(bars.full_tma(s), ph, a.err, tmo)) {
-                    ok = false;
-                    break;
-                }
-                const uint8_t *fp4 = gsm + kOffFp4 + s * kFp4Bytes;
-                const uint8_t *scl = gsm + kOffScl + s * kSclBytes;
-                uint8_t *wb = gsm + kOffWb + s * kWbBytes;
-                const int sh = (kk & 1) * 16;
-#pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                    const int r = t + 128 * rr;
-                    const uint4 q0 = *reinterpret_cast<const uint4 *>(fp4 + r * 32);
-                    const uint4 q1 = *reinterpret_cast<const uint4 *>(fp4 + r * 32 + 16);
-                    const uint32_t sw = *reinterpret_cast<const uint32_t *>(scl + r * 4);
-                    const uint32_t sb0 = (sw >> sh) & 0xFF, sb1 = (sw >> (sh + 8)) & 0xFF;
-                    const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint32_t wv = words[c];
-                        const uint32_t sb = c < 4 ? sb0 : sb1;
-                        uint32_t o[4];
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const uint32_t byte = (wv >> (8 * j)) & 0xFF;
-                            o[j] = e2m1_bf16_bits(byte & 0xF, sb) | (e2m1_bf16_bits(byte >> 4, sb) << 16);
-                        }
-                        *reinterpret_cast<uint4 *>(wb + r * 128 + ((c ^ (r & 7)) << 4)) =
-                            make_uint4(o[0], o[1], o[2], o[3]);
-                    }
-                }
-                fence_proxy_async_smem();
-                mbar_arrive(bars.full_deq(s));
-            }
-        }
-    } else if (warp >= 6) {
-        // ------------------------------------------------------------ epilogue
+    } else {
+        // ------------------------------------------------------------ epilogue (warps 2..5)
         const int q = warp & 3; // TMEM lane quarter this warp may access
+        float *xch = reinterpret_cast<float *>(gsm + kOffX);
         uint32_t cnt = 0;
         for (int u = blockIdx.x; u < total_units; u += gridDim.x, ++cnt) {
             const int4 blk = a.rowblocks[u / a.n_tiles];
@@ -305,21 +313,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int rows = blk.z;
             const bool swap = rows <= a.swap_rows;
             const int buf = cnt & 1;
-            if (!mbar_wait_bounded(bars.acc_full(buf), (cnt >> 1) & 1, a.err, tmo))
+            // the four epilogue warps leave together or not at all (they share named barrier 1 below)
+            const bool got = mbar_wait_bounded(bars.acc_full(buf), (cnt >> 1) & 1, a.err, tmo);
+            if (!named_bar_all(2, 128, got))
                 break;
             tc_fence_after();
-            const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + buf * 256;
+            const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + buf * 128;
             if (!swap) {
+                // thread = one grouped row; TMEM columns = the tile's 128 weight rows
                 const int rl = 32 * q + lane;
                 const bool valid = rl < rows;
+                const int row = blk.y + rl;
                 if (a.fc1) {
-                    __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(a.out) + (size_t)(blk.y + rl) * a.out_ld;
-                    for (int c = 0; c < 4; ++c) {
+                    // columns 0..63 gate, 64..127 up, for i = nt*64 + c
+                    for (int c32 = 0; c32 < 2; ++c32) {
                         uint32_t g0[16], g1[16], u0[16], u1[16];
-                        tmem_ld16(tb + 32 * c, g0);
-                        tmem_ld16(tb + 32 * c + 16, g1);
-                        tmem_ld16(tb + 128 + 32 * c, u0);
-                        tmem_ld16(tb + 128 + 32 * c + 16, u1);
+                        tmem_ld16(tb + 32 * c32, g0);
+                        tmem_ld16(tb + 32 * c32 + 16, g1);
+                        tmem_ld16(tb + 64 + 32 * c32, u0);
+                        tmem_ld16(tb + 64 + 32 * c32 + 16, u1);
                         tmem_wait_ld();
                         float h[32];
 #pragma unroll
@@ -327,48 +339,58 @@ __global__ void __launch_bounds__(kThreads, 1)
                             h[i] = silu_mul(__uint_as_float(g0[i]), __uint_as_float(u0[i]));
                             h[16 + i] = silu_mul(__uint_as_float(g1[i]), __uint_as_float(u1[i]));
                         }
-                        if (a.act_mxfp8)
-                            mxfp8_roundtrip32(h);
                         if (valid)
-                            store_bf16x32(orow + nt * 128 + 32 * c, h);
+                            store_act_block32(a.hq, a.hsf, a.hq_rows, a.out_ld, row, nt * 64 + 32 * c32, h,
+                                              a.act_mxfp8);
                     }
                 } else {
-                    float *orow = static_cast<float *>(a.out) + (size_t)(blk.y + rl) * a.out_ld + nt * 256;
-                    for (int c = 0; c < 16; ++c) {
+                    float *orow = a.y + (size_t)row * a.out_ld + nt * 128;
+                    for (int c = 0; c < 8; ++c) {
                         uint32_t y0[16];
                         tmem_ld16(tb + 16 * c, y0);
                         tmem_wait_ld();
                         if (valid) {
-                            uint4 *d = reinterpret_cast<uint4 *>(orow + 16 * c);
+                            uint4 *dst = reinterpret_cast<uint4 *>(orow + 16 * c);
 #pragma unroll
                             for (int i = 0; i < 4; ++i)
-                                d[i] = make_uint4(y0[4 * i], y0[4 * i + 1], y0[4 * i + 2], y0[4 * i + 3]);
+                                dst[i] = make_uint4(y0[4 * i], y0[4 * i + 1], y0[4 * i + 2], y0[4 * i + 3]);
                         }
                     }
                 }
             } else {
-                const int L = 32 * q + lane; // weight row within the 128-row half
+                // lane L of the tile = weight row; TMEM columns = tokens
+                const int L = 32 * q + lane;
                 const int npad = (rows + 15) & ~15;
                 for (int n0 = 0; n0 < npad; n0 += 16) {
-                    uint32_t v0[16], v1[16];
-                    tmem_ld16(tb + n0, v0);
-                    tmem_ld16(tb + 128 + n0, v1);
+                    uint32_t v[16];
+                    tmem_ld16(tb + n0, v);
                     tmem_wait_ld();
+                    if (a.fc1) {
+                        // the up rows live in lanes 64..127: hand them to the gate lanes through smem
+                        if (q >= 2) {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int n = n0 + j;
-                        if (n >= rows)
-                            break;
-                        if (a.fc1) {
-                            __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(a.out) + (size_t)(blk.y + n) * a.out_ld;
-                            float hv = silu_mul(__uint_as_float(v0[j]), __uint_as_float(v1[j]));
-                            if (a.act_mxfp8)
-                                hv = mxfp8_roundtrip_warp(hv);
-                            orow[nt * 128 + L] = __float2bfloat16_rn(hv);
-                        } else {
-                            float *orow = static_cast<float *>(a.out) + (size_t)(blk.y + n) * a.out_ld;
-                            orow[nt * 256 + L] = __uint_as_float(v0[j]);
-                            orow[nt * 256 + 128 + L] = __uint_as_float(v1[j]);
+                            for (int j = 0; j < 16; ++j)
+                                xch[(L - 64) * 16 + j] = __uint_as_float(v[j]);
+                        }
+                        named_bar_sync(1, 128);
+                        if (q < 2) {
+                            const int i = nt * 64 + L;
+                            for (int j = 0; j < 16; ++j) {
+                                const int n = n0 + j;
+                                if (n >= rows)
+                                    break;
+                                const float hv = silu_mul(__uint_as_float(v[j]), xch[L * 16 + j]);
+                                store_act_warp32(a.hq, a.hsf, a.hq_rows, a.out_ld, blk.y + n, i, hv, a.act_mxfp8,
+                                                 lane);
+                            }
+                        }
+                        named_bar_sync(1, 128);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int n = n0 + j;
+                            if (n < rows)
+                                a.y[(size_t)(blk.y + n) * a.out_ld + nt * 128 + L] = __uint_as_float(v[j]);
                         }
                     }
                 }
@@ -393,10 +415,10 @@ cudaError_t fc_gemm_prepare()
     return cudaFuncSetAttribute(fc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
 }
 
-void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUtensorMap &w_map, int grid,
-                    cudaStream_t s)
+void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUtensorMap &act_map16,
+                    const CUtensorMap &w_map, int grid, cudaStream_t s)
 {
-    fc_gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(a, act_map, w_map);
+    fc_gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(a, act_map, act_map16, w_map);
 }
 
 // ---------------------------------------------------------------- watchdog self-test

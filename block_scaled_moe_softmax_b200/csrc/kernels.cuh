@@ -32,33 +32,40 @@ struct RouteGroupArgs {
 };
 
 void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s);
-void launch_gather(const __nv_bfloat16 *x, int P, int H, int k, const int32_t *pos_of_pair, __nv_bfloat16 *A,
-                   int act_mxfp8, int num_sms, cudaStream_t s);
+void launch_gather(const __nv_bfloat16 *x, int P, int H, int k, const int32_t *pos_of_pair, uint8_t *aq,
+                   uint8_t *asf, int act_rows, int act_mxfp8, int num_sms, cudaStream_t s);
 void launch_combine(const float *Y, int T, int H, int k, const int32_t *pos_of_pair, const float *topk_w,
                     __nv_bfloat16 *out, int num_sms, cudaStream_t s);
 void launch_mx_quantize(const float *src, int64_t rows, int64_t K, int fmt, uint8_t *codes, uint8_t *scales,
                         int num_sms, cudaStream_t s);
 
-// Grouped FC GEMM (FC1 with SwiGLU, or FC2) over the row-block list.
+// Grouped FC GEMM (FC1 with SwiGLU, or FC2) over the row-block list, on
+// block-scaled MXFP8 x MXFP4 tensor-core MMAs.
 struct FcGemmArgs {
     const int4 *rowblocks;       // {expert, first grouped row, rows, 0}
     const int32_t *num_rowblocks;
-    const uint8_t *wscale;       // E8M0 scales of the weight, [E*R, K/32]
-    void *out;                   // FC1: bf16 Hbuf [rows, I]; FC2: f32 Y [rows, H]
+    const uint8_t *wscale;       // caller's E8M0 weight scales, [E*R, K/32] row-major
+    const uint8_t *act_sf;       // activation scale atoms, [rows/128][K/128][2 terms][512]
+    uint8_t *hq;                 // FC1 output codes, [2 terms][hq_rows][I] (E4M3)
+    uint8_t *hsf;                // FC1 output scale atoms, [hq_rows/128][I/128][2][512]
+    float *y;                    // FC2 output, f32 [rows, H]
     uint32_t *err;
     unsigned long long timeout_ns;
     int K;                       // reduction length (FC1: H, FC2: I)
     int R;                       // weight rows per expert (FC1: 2I, FC2: H)
-    int n_tiles;                 // 256-row weight tiles per expert (FC1: I/128, FC2: H/256)
-    int out_ld;                  // leading dimension of out (FC1: I, FC2: H)
+    int n_tiles;                 // 128-row weight tiles per expert (FC1: I/64, FC2: H/128)
+    int out_ld;                  // leading dimension of the output (FC1: I, FC2: H)
+    int act_rows;                // rows of one activation term plane (offset of term 1)
+    int hq_rows;                 // rows of one FC1 output term plane
+    int terms;                   // activation terms: 2 (w4a16 split) or 1 (w4a8)
     int fc1;                     // 1: gate/up rows + SwiGLU epilogue
-    int act_mxfp8;               // FC1 only: MXFP8 round trip of h before it is stored
+    int act_mxfp8;               // FC1 only: h in OCP MXFP8 (w4a8) instead of the two-term split
     int swap_rows;               // row blocks of at most this many rows (<= 128) put the
                                  // weight rows on the MMA M side and the tokens on N
 };
 
-void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUtensorMap &w_map, int grid,
-                    cudaStream_t s);
+void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUtensorMap &act_map16,
+                    const CUtensorMap &w_map, int grid, cudaStream_t s);
 size_t fc_gemm_smem_bytes();
 cudaError_t fc_gemm_prepare();
 
@@ -93,31 +100,128 @@ __device__ __forceinline__ uint32_t mx_quantize32_e4m3(const float (&v)[32], uin
     return (uint32_t)(s + 127);
 }
 
-// MXFP8 round trip of 32 bf16 values held in four uint4: quantise, then write
-// back the exact dequantised values (E4M3 value * 2^s is representable in bf16).
-__device__ __forceinline__ void mxfp8_roundtrip_bf16x32(uint4 (&v)[4])
+// ---------------------------------------------------------------- activation operand format
+// Activations reach the tensor core as MXFP8 E4M3 codes in [term][row][K]
+// planes plus E8M0 block scales stored in "scale atoms": for every 128 rows x
+// 128 K elements, 512 bytes in which tile row m = m0 + 32*m1 (m0 < 32, m1 < 4)
+// owns bytes m0*16 + m1*4 + kb (kb = 32-element block within the 128), the
+// layout one tcgen05.cp 32x128b.warpx4 moves into TMEM as the MMA expects it.
+__device__ __forceinline__ int sf_atom_offset(int m, int kb)
 {
-    float f[32];
+    return (m & 31) * 16 + (m >> 5) * 4 + kb;
+}
+
+__device__ __forceinline__ size_t sf_atom_byte(int row, int col, int K, int term)
+{
+    return ((size_t)(row >> 7) * (size_t)(K >> 7) + (size_t)(col >> 7)) * 1024 + (size_t)term * 512 +
+           (size_t)sf_atom_offset(row & 127, (col >> 5) & 3);
+}
+
+// E8M0 exponent of a block: floor(log2(amax)) - emax_shift, clamped to [-127, 127]
+// (all-zero block: -127).
+__device__ __forceinline__ int mx_block_exp(float amax, int emax_shift)
+{
+    const int s = (amax == 0.f) ? -127 : floor_log2_pos(amax) - emax_shift;
+    return max(-127, min(127, s));
+}
+
+// Encode 32 values as MXFP8 terms.  act_mxfp8 = 1: the OCP rule (shared
+// exponent floor(log2 amax) - 8, round-to-nearest-even, saturating) -- one term,
+// the w4a8 activation.  act_mxfp8 = 0: an exact two-term expansion of bf16
+// values, v = x1 + x2: x1 takes exponent floor(log2 amax) - 7 (the block max
+// lands in [128, 256), below the E4M3 maximum, so nothing saturates) and keeps
+// the top 4 significant bits of every element; x2 encodes the remainder v - x1,
+// which has at most 4 significant bits, with its own block exponent.  Elements
+// within 2^-13 of the block maximum are represented exactly; smaller ones keep
+// an absolute error below 2^-20 of the block maximum.
+__device__ __forceinline__ void mx_encode32(const float (&v)[32], int act_mxfp8, uint8_t (&c0)[32], uint8_t (&c1)[32],
+                                            uint32_t &s0, uint32_t &s1)
+{
+    float amax = 0.f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&v[i]);
+    for (int i = 0; i < 32; ++i)
+        amax = fmaxf(amax, fabsf(v[i]));
+    const int e0 = mx_block_exp(amax, act_mxfp8 ? 8 : 7);
+    const float inv0 = exp2_int(-e0), sc0 = exp2_int(e0);
+    float r[32];
+    float amax1 = 0.f;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float2 t = __bfloat1622float2(h2[j]);
-            f[8 * i + 2 * j] = t.x;
-            f[8 * i + 2 * j + 1] = t.y;
-        }
+    for (int i = 0; i < 32; ++i) {
+        c0[i] = (uint8_t)f32_to_e4m3(__fmul_rn(v[i], inv0));
+        r[i] = __fsub_rn(v[i], __fmul_rn(e4m3_to_f32(c0[i]), sc0));
+        amax1 = fmaxf(amax1, fabsf(r[i]));
     }
-    uint8_t c[32];
-    const uint32_t sb = mx_quantize32_e4m3(f, c);
-    const float scale = (sb == 0xFF) ? __uint_as_float(0x7FC00000u) : exp2_int((int)sb - 127);
+    s0 = (uint32_t)(e0 + 127);
+    if (act_mxfp8) {
+        s1 = 0;
+        return;
+    }
+    const int e1 = mx_block_exp(amax1, 7);
+    const float inv1 = exp2_int(-e1);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        __nv_bfloat162 *h2 = reinterpret_cast<__nv_bfloat162 *>(&v[i]);
+    for (int i = 0; i < 32; ++i)
+        c1[i] = (uint8_t)f32_to_e4m3(__fmul_rn(r[i], inv1));
+    s1 = (uint32_t)(e1 + 127);
+}
+
+__device__ __forceinline__ void store_codes32(uint8_t *dst, const uint8_t (&c)[32])
+{
+    uint4 w[2];
+    uint8_t *b = reinterpret_cast<uint8_t *>(w);
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-            h2[j] = __floats2bfloat162_rn(__fmul_rn(e4m3_to_f32(c[8 * i + 2 * j]), scale),
-                                          __fmul_rn(e4m3_to_f32(c[8 * i + 2 * j + 1]), scale));
+    for (int i = 0; i < 32; ++i)
+        b[i] = c[i];
+    reinterpret_cast<uint4 *>(dst)[0] = w[0];
+    reinterpret_cast<uint4 *>(dst)[1] = w[1];
+}
+
+// One thread writes the 32-element block [col, col+32) of `row` (values v, f32):
+// rounded to bf16 first unless act_mxfp8, then encoded as above.
+__device__ __forceinline__ void store_act_block32(uint8_t *q, uint8_t *sf, int plane_rows, int K, int row, int col,
+                                                  float (&v)[32], int act_mxfp8)
+{
+    if (!act_mxfp8) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            v[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
+    }
+    uint8_t c0[32], c1[32];
+    uint32_t s0, s1;
+    mx_encode32(v, act_mxfp8, c0, c1, s0, s1);
+    store_codes32(q + (size_t)row * K + col, c0);
+    sf[sf_atom_byte(row, col, K, 0)] = (uint8_t)s0;
+    if (!act_mxfp8) {
+        store_codes32(q + ((size_t)plane_rows + row) * K + col, c1);
+        sf[sf_atom_byte(row, col, K, 1)] = (uint8_t)s1;
+    }
+}
+
+// The 32 lanes of a warp write one 32-element block of `row`, lane l holding
+// element col0 + l (col0 = col rounded down to 32).
+__device__ __forceinline__ void store_act_warp32(uint8_t *q, uint8_t *sf, int plane_rows, int K, int row, int col,
+                                                 float v, int act_mxfp8, int lane)
+{
+    if (!act_mxfp8)
+        v = __bfloat162float(__float2bfloat16_rn(v));
+    float amax = fabsf(v);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+    const int e0 = mx_block_exp(amax, act_mxfp8 ? 8 : 7);
+    const uint32_t c0 = f32_to_e4m3(__fmul_rn(v, exp2_int(-e0)));
+    q[(size_t)row * K + col] = (uint8_t)c0;
+    if (lane == 0)
+        sf[sf_atom_byte(row, col, K, 0)] = (uint8_t)(e0 + 127);
+    if (!act_mxfp8) {
+        const float r = __fsub_rn(v, __fmul_rn(e4m3_to_f32(c0), exp2_int(e0)));
+        float amax1 = fabsf(r);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            amax1 = fmaxf(amax1, __shfl_xor_sync(0xFFFFFFFFu, amax1, off));
+        const int e1 = mx_block_exp(amax1, 7);
+        q[((size_t)plane_rows + row) * K + col] = (uint8_t)f32_to_e4m3(__fmul_rn(r, exp2_int(-e1)));
+        if (lane == 0)
+            sf[sf_atom_byte(row, col, K, 1)] = (uint8_t)(e1 + 127);
     }
 }
 

@@ -12,9 +12,10 @@
 // Grouping (TokenSpeed-kernel README, "Public API", moe_dispatch): pairs
 // p = t*k + j are counting-sorted by expert, stably (ascending t within an
 // expert), into segments padded to kBlockRows rows; the activation rows are
-// gathered into that order (and, for w4a8, MXFP8-quantised on the way:
-// tokenspeed-situ package description, "Activation precision (w4a16 vs
-// w4a8)").  Every step is deterministic: integer counts only, no float atomics.
+// gathered into that order as the MXFP8 operand of the block-scaled FC1 (for
+// w4a8 the OCP MXFP8 quantisation of tokenspeed-situ package description,
+// "Activation precision (w4a16 vs w4a8)"; for w4a16 an exact two-term
+// expansion of the bf16 row).  Every step is deterministic: integer counts only, no float atomics.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -205,13 +206,14 @@ __global__ void __launch_bounds__(32) scatter_kernel(int T, int E, int k, const 
 }
 
 // ---------------------------------------------------------------- gather
-// Copy x[t] into grouped row pos_of_pair[p] for every pair p.  One thread per
-// 32 consecutive elements (64 bytes).  With act_mxfp8 the 32 elements (one MX
-// block) are quantised to MXFP8 E4M3 and written back as their exact bf16
-// values, which is what FC1 consumes.
+// Encode x[t] into grouped row pos_of_pair[p] for every pair p, as the MXFP8
+// operand FC1 consumes (see mx_encode32): the OCP MXFP8 quantisation for w4a8,
+// the exact two-term expansion of the bf16 row for w4a16.  One thread per
+// 32-element block: 64 bytes in, 32 (or 2 x 32) code bytes and 1 (or 2) scale
+// bytes out.
 __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16 *__restrict__ x, int P, int H, int k,
-                                                     const int32_t *__restrict__ pos_of_pair,
-                                                     __nv_bfloat16 *__restrict__ A, int act_mxfp8)
+                                                     const int32_t *__restrict__ pos_of_pair, uint8_t *__restrict__ aq,
+                                                     uint8_t *__restrict__ asf, int act_rows, int act_mxfp8)
 {
     const int blocks_per_row = H / 32;
     const long long total = (long long)P * blocks_per_row;
@@ -221,16 +223,19 @@ __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16 *__rest
         const int b = (int)(g % blocks_per_row);
         const int t = p / k;
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H + (size_t)b * 32);
-        uint4 *dst = reinterpret_cast<uint4 *>(A + (size_t)pos_of_pair[p] * H + (size_t)b * 32);
-        uint4 v[4];
+        float v[32];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            v[i] = __ldg(src + i);
-        if (act_mxfp8)
-            mxfp8_roundtrip_bf16x32(v);
+        for (int i = 0; i < 4; ++i) {
+            const uint4 raw = __ldg(src + i);
+            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            dst[i] = v[i];
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = __bfloat1622float2(h2[j]);
+                v[8 * i + 2 * j] = f.x;
+                v[8 * i + 2 * j + 1] = f.y;
+            }
+        }
+        store_act_block32(aq, asf, act_rows, H, pos_of_pair[p], b * 32, v, act_mxfp8);
     }
 }
 
@@ -286,13 +291,13 @@ void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s)
     scatter_kernel<<<nchunks, 32, 0, s>>>(a.T, a.E, a.k, a.topk_ids, a.chunk_hist, a.sorted_pair, a.pos_of_pair);
 }
 
-void launch_gather(const __nv_bfloat16 *x, int P, int H, int k, const int32_t *pos_of_pair, __nv_bfloat16 *A,
-                   int act_mxfp8, int num_sms, cudaStream_t s)
+void launch_gather(const __nv_bfloat16 *x, int P, int H, int k, const int32_t *pos_of_pair, uint8_t *aq,
+                   uint8_t *asf, int act_rows, int act_mxfp8, int num_sms, cudaStream_t s)
 {
     const long long work = (long long)P * (H / 32);
     const long long want = (work + 255) / 256;
     const int grid = (int)(want < (long long)num_sms * 8 ? want : (long long)num_sms * 8);
-    gather_kernel<<<grid > 0 ? grid : 1, 256, 0, s>>>(x, P, H, k, pos_of_pair, A, act_mxfp8);
+    gather_kernel<<<grid > 0 ? grid : 1, 256, 0, s>>>(x, P, H, k, pos_of_pair, aq, asf, act_rows, act_mxfp8);
 }
 
 void launch_combine(const float *Y, int T, int H, int k, const int32_t *pos_of_pair, const float *topk_w,
