@@ -378,6 +378,7 @@ int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, 
         f1.fc1 = 1;
         f1.act_mxfp8 = mx8;
         f1.swap_rows = h->swap_rows;
+        f1.max_block_rows = T < kBlockRows ? T : kBlockRows; // a block holds one expert's tokens
         mark(2);
         launch_fc_gemm(f1, h->map_A, h->map_A16, h->map_w1, h->num_sms, s);
         mark(3);

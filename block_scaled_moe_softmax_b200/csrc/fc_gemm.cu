@@ -41,31 +41,42 @@ namespace moe_mx {
 
 namespace {
 
-constexpr int kStages = 4;
 constexpr int kThreads = 192;
-constexpr int kTermBytes = 128 * 128;          // 128 rows x 128 E4M3 codes
-constexpr int kActBytes = 2 * kTermBytes;      // up to two terms
+constexpr int kTermRowBytes = 128;             // one activation row of a K stage: 128 E4M3 codes
 constexpr int kWBytes = 128 * 128;             // 128 rows x 128 E2M1 codes in 8-bit containers
 constexpr int kWTxBytes = 128 * 128 / 2;       // ... of which the TMA transfers (and counts) the packed 4-bit data
 constexpr int kAsfBytes = 2 * 512;             // one 512-byte scale atom per term
 constexpr int kWsfBytes = 512;
-constexpr int kOffAct = 0;
-constexpr int kOffW = kOffAct + kStages * kActBytes;
-constexpr int kOffAsf = kOffW + kStages * kWBytes;
-constexpr int kOffWsf = kOffAsf + kStages * kAsfBytes;
-constexpr int kOffX = kOffWsf + kStages * kWsfBytes; // epilogue exchange, 64 lanes x 16 columns f32
-constexpr int kXBytes = 64 * 16 * 4;
-constexpr int kOffBar = kOffX + kXBytes;
-constexpr int kNumBars = 2 * kStages + 1 + 4;
-constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
-constexpr int kSmemBytes = kOffTmemSlot + 16 + 1024; // + slack for 1024-byte alignment
+constexpr int kXBytes = 64 * 16 * 4;           // epilogue exchange, 64 lanes x 16 columns f32
+constexpr int kSmemLimit = 227 * 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCol = 256; // TMEM columns 256..267 hold the stage's scale factors
 constexpr unsigned long long kDrainTimeoutNs = 200000000ull;
 
+// Shared-memory plan for a kernel whose activation tiles hold at most kActRows
+// rows per term: as many pipeline stages as fit (more stages = more bytes in
+// flight per SM, which is what the weight-streaming decode shapes need).
+template <int kActRows> struct Plan {
+    static constexpr int kTermBytes = kActRows * kTermRowBytes;
+    static constexpr int kActBytes = 2 * kTermBytes;
+    static constexpr int kStageBytes = kActBytes + kWBytes + kAsfBytes + kWsfBytes;
+    static constexpr int kStages = (kSmemLimit - 1024 - kXBytes - 256) / kStageBytes;
+    static constexpr int kOffAct = 0;
+    static constexpr int kOffW = kOffAct + kStages * kActBytes;
+    static constexpr int kOffAsf = kOffW + kStages * kWBytes;
+    static constexpr int kOffWsf = kOffAsf + kStages * kAsfBytes;
+    static constexpr int kOffX = kOffWsf + kStages * kWsfBytes;
+    static constexpr int kOffBar = kOffX + kXBytes;
+    static constexpr int kNumBars = 2 * kStages + 1 + 4;
+    static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
+    static constexpr int kSmemBytes = kOffTmemSlot + 16 + 1024; // + slack for 1024-byte alignment
+    static_assert(kSmemBytes <= kSmemLimit, "shared memory plan too large");
+    static_assert(kStages >= 3, "too few pipeline stages");
+};
+
 constexpr uint32_t kFmtE4M3 = 0, kFmtE2M1 = 5;
 
-struct Bars {
+template <int kStages> struct Bars {
     uint32_t base;
     __device__ uint32_t full(int s) const { return base + 8 * s; }
     __device__ uint32_t empty(int s) const { return base + 8 * (kStages + s); }
@@ -73,6 +84,16 @@ struct Bars {
     __device__ uint32_t acc_full(int b) const { return base + 8 * (2 * kStages + 1 + b); }
     __device__ uint32_t acc_empty(int b) const { return base + 8 * (2 * kStages + 3 + b); }
 };
+
+// One lane of a converged warp is elected (tcgen05 and TMA instructions are
+// issued once per warp while the whole warp runs the loop, so their operands
+// stay warp-uniform).
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t p = 0;
+    asm volatile("{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.b32 %0, 1, 0, P;\n\t}" : "=r"(p));
+    return p != 0;
+}
 
 // Instruction descriptor of kind::mxf8f6f4 with E8M0 block scales (one scale
 // per 32 elements): [4,6) B scale byte, [7,10) A format, [10,13) B format,
@@ -143,15 +164,21 @@ __device__ __forceinline__ float silu_mul(float g, float u)
 
 } // namespace
 
+template <int kActRows>
 __global__ void __launch_bounds__(kThreads, 1)
     fc_gemm_kernel(const FcGemmArgs a, const __grid_constant__ CUtensorMap act_map,
                    const __grid_constant__ CUtensorMap act_map16, const __grid_constant__ CUtensorMap w_map)
 {
+    using P = Plan<kActRows>;
+    constexpr int kStages = P::kStages;
+    constexpr int kTermBytes = P::kTermBytes, kActBytes = P::kActBytes;
+    constexpr int kOffAct = P::kOffAct, kOffW = P::kOffW, kOffAsf = P::kOffAsf, kOffWsf = P::kOffWsf;
+    constexpr int kOffX = P::kOffX, kOffBar = P::kOffBar, kOffTmemSlot = P::kOffTmemSlot;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *const gsm = smem_raw + (base - raw);
-    const Bars bars{base + kOffBar};
+    const Bars<kStages> bars{base + kOffBar};
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -186,14 +213,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const unsigned long long tmo = a.timeout_ns;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ producer
+        // ------------------------------------------------------------ producer (whole warp)
         uint32_t g = 0;
         bool ok = true;
         const int scl_ld = a.K / 32;
         for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
             const int4 blk = a.rowblocks[u / a.n_tiles];
             const int nt = u % a.n_tiles;
-            const bool swap = blk.z <= a.swap_rows;
+            const bool swap = kActRows < 128 || blk.z <= a.swap_rows;
             const int npad = (blk.z + 15) & ~15;
             // weight rows of this tile, as two 64-row halves: FC1 tile nt = gate rows [64nt, 64nt+64)
             // then the matching up rows; FC2 tile nt = rows [128nt, 128nt+128)
@@ -204,11 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < kst; ++kk, ++g) {
                 const int s = g % kStages;
                 const uint32_t ph = (g / kStages) & 1;
-                bool w = true;
-                if (lane == 0)
-                    w = mbar_wait_bounded(bars.empty(s), ph ^ 1, a.err, tmo);
-                w = __shfl_sync(0xFFFFFFFFu, w, 0);
-                if (!w) {
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.empty(s), ph ^ 1, a.err, tmo))) {
                     ok = false;
                     break;
                 }
@@ -220,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 cp_async_mbar_arrive_noinc(bars.full(s));
                 __syncwarp();
-                if (lane == 0) {
+                if (elect_one()) {
                     mbar_arrive_expect_tx(bars.full(s), act_bytes + kWTxBytes + (uint32_t)terms * 512u);
                     const uint32_t act = base + kOffAct + s * kActBytes;
                     for (int t = 0; t < terms; ++t) {
@@ -243,65 +266,71 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         // drain: every stage issued must have landed before the CTA may exit
-        if (lane == 0) {
-            const uint32_t first = g > (uint32_t)kStages ? g - kStages : 0u;
-            for (uint32_t q = first; q < g; ++q)
-                mbar_wait_bounded(bars.full(q % kStages), (q / kStages) & 1, nullptr, kDrainTimeoutNs);
-        }
+        const uint32_t first = g > (uint32_t)kStages ? g - kStages : 0u;
+        for (uint32_t q = first; q < g; ++q)
+            mbar_wait_bounded(bars.full(q % kStages), (q / kStages) & 1, nullptr, kDrainTimeoutNs);
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            uint32_t g = 0, cnt = 0;
-            bool ok = true;
-            const uint32_t sf_w = tmem_base + kSfCol;
-            for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x, ++cnt) {
-                const int4 blk = a.rowblocks[u / a.n_tiles];
-                const bool swap = blk.z <= a.swap_rows;
-                const uint32_t npad = (uint32_t)((blk.z + 15) & ~15);
-                const int buf = cnt & 1;
-                if (!mbar_wait_bounded(bars.acc_empty(buf), ((cnt >> 1) & 1) ^ 1, a.err, tmo)) {
+        // ------------------------------------------------------------ MMA issuer (whole warp, one lane issues)
+        uint32_t g = 0, cnt = 0;
+        bool ok = true;
+        const uint32_t sf_w = tmem_base + kSfCol;
+        for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x, ++cnt) {
+            const int4 blk = a.rowblocks[u / a.n_tiles];
+            const bool swap = kActRows < 128 || blk.z <= a.swap_rows;
+            const uint32_t npad = (uint32_t)((blk.z + 15) & ~15);
+            const uint32_t idesc0 = swap ? idesc_mx(kFmtE2M1, kFmtE4M3, 128, npad, 0)
+                                         : idesc_mx(kFmtE4M3, kFmtE2M1, 128, 128, 0);
+            const int buf = cnt & 1;
+            if (!__all_sync(0xFFFFFFFFu,
+                            mbar_wait_bounded(bars.acc_empty(buf), ((cnt >> 1) & 1) ^ 1, a.err, tmo))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d = tmem_base + buf * 128;
+            for (int kk = 0; kk < kst; ++kk, ++g) {
+                const int s = g % kStages;
+                const uint32_t ph = (g / kStages) & 1;
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.full(s), ph, a.err, tmo))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d = tmem_base + buf * 128;
-                for (int kk = 0; kk < kst; ++kk, ++g) {
-                    const int s = g % kStages;
-                    const uint32_t ph = (g / kStages) & 1;
-                    if (!mbar_wait_bounded(bars.full(s), ph, a.err, tmo)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
+                const uint32_t act = base + kOffAct + s * kActBytes;
+                const uint32_t wt = base + kOffW + s * kWBytes;
+                if (elect_one()) {
                     // scale atoms -> TMEM (in order with the MMAs below and with the previous stage's MMAs)
                     tmem_cp_sf_atom(sf_w, base + kOffWsf + s * kWsfBytes);
                     for (int t = 0; t < terms; ++t)
                         tmem_cp_sf_atom(sf_w + 4 + 4 * t, base + kOffAsf + s * kAsfBytes + 512 * t);
-                    const uint32_t act = base + kOffAct + s * kActBytes;
-                    const uint32_t wt = base + kOffW + s * kWBytes;
 #pragma unroll
                     for (int k32 = 0; k32 < 4; ++k32) {
                         const uint64_t dw = smem_desc_sw128(wt + 32 * k32);
+                        // the scale-factor byte of this 32-element block sits in both sf-id fields
+                        const uint32_t idesc = idesc0 | ((uint32_t)k32 << 4) | ((uint32_t)k32 << 29);
                         for (int t = 0; t < terms; ++t) {
                             const uint64_t da = smem_desc_sw128(act + t * kTermBytes + 32 * k32);
                             const uint32_t sf_a = sf_w + 4 + 4 * t;
                             const uint32_t acc = (kk | k32 | t) != 0;
                             if (!swap)
-                                umma_mx(d, da, dw, idesc_mx(kFmtE4M3, kFmtE2M1, 128, 128, k32), sf_a, sf_w, acc);
+                                umma_mx(d, da, dw, idesc, sf_a, sf_w, acc);
                             else
-                                umma_mx(d, dw, da, idesc_mx(kFmtE2M1, kFmtE4M3, 128, npad, k32), sf_w, sf_a, acc);
+                                umma_mx(d, dw, da, idesc, sf_w, sf_a, acc);
                         }
                     }
                     umma_commit(bars.empty(s));
                 }
-                if (ok)
-                    umma_commit(bars.acc_full(buf));
+                __syncwarp();
             }
-            // all MMAs must have completed before TMEM is released
-            umma_commit(bars.mma_done());
-            mbar_wait_bounded(bars.mma_done(), 0, nullptr, kDrainTimeoutNs);
+            if (ok && elect_one())
+                umma_commit(bars.acc_full(buf));
+            __syncwarp();
         }
+        // all MMAs must have completed before TMEM is released
+        if (elect_one())
+            umma_commit(bars.mma_done());
         __syncwarp();
+        mbar_wait_bounded(bars.mma_done(), 0, nullptr, kDrainTimeoutNs);
     } else {
         // ------------------------------------------------------------ epilogue (warps 2..5)
         const int q = warp & 3; // TMEM lane quarter this warp may access
@@ -311,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int4 blk = a.rowblocks[u / a.n_tiles];
             const int nt = u % a.n_tiles;
             const int rows = blk.z;
-            const bool swap = rows <= a.swap_rows;
+            const bool swap = kActRows < 128 || rows <= a.swap_rows;
             const int buf = cnt & 1;
             // the four epilogue warps leave together or not at all (they share named barrier 1 below)
             const bool got = mbar_wait_bounded(bars.acc_full(buf), (cnt >> 1) & 1, a.err, tmo);
@@ -408,17 +437,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-size_t fc_gemm_smem_bytes() { return (size_t)kSmemBytes; }
+size_t fc_gemm_smem_bytes(int act_rows) { return act_rows <= 32 ? Plan<32>::kSmemBytes : Plan<128>::kSmemBytes; }
+
+int fc_gemm_stages(int act_rows) { return act_rows <= 32 ? Plan<32>::kStages : Plan<128>::kStages; }
 
 cudaError_t fc_gemm_prepare()
 {
-    return cudaFuncSetAttribute(fc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(fc_gemm_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Plan<32>::kSmemBytes);
+    if (e != cudaSuccess)
+        return e;
+    return cudaFuncSetAttribute(fc_gemm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Plan<128>::kSmemBytes);
 }
 
 void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUtensorMap &act_map16,
                     const CUtensorMap &w_map, int grid, cudaStream_t s)
 {
-    fc_gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(a, act_map, act_map16, w_map);
+    // At most 32 tokens: every row block has at most 32 rows and runs with its tokens on N,
+    // so the activation tiles shrink and the pipeline gets more stages.
+    if (a.max_block_rows <= 32)
+        fc_gemm_kernel<32><<<grid, kThreads, Plan<32>::kSmemBytes, s>>>(a, act_map, act_map16, w_map);
+    else
+        fc_gemm_kernel<128><<<grid, kThreads, Plan<128>::kSmemBytes, s>>>(a, act_map, act_map16, w_map);
 }
 
 // ---------------------------------------------------------------- watchdog self-test

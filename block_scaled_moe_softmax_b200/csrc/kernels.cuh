@@ -62,11 +62,13 @@ struct FcGemmArgs {
     int act_mxfp8;               // FC1 only: h in OCP MXFP8 (w4a8) instead of the two-term split
     int swap_rows;               // row blocks of at most this many rows (<= 128) put the
                                  // weight rows on the MMA M side and the tokens on N
+    int max_block_rows;          // upper bound on any row block's rows (min(tokens, 128))
 };
 
 void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUtensorMap &act_map16,
                     const CUtensorMap &w_map, int grid, cudaStream_t s);
-size_t fc_gemm_smem_bytes();
+size_t fc_gemm_smem_bytes(int act_rows);
+int fc_gemm_stages(int act_rows);
 cudaError_t fc_gemm_prepare();
 
 void launch_watchdog(uint32_t *err, unsigned long long timeout_ns, cudaStream_t s);

@@ -65,22 +65,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 constexpr uint32_t kErrTimeout = 1u;
 
 // Wait for phase `parity` of an mbarrier to complete, for at most timeout_ns
-// of wall time.  With a non-null global error word `err`, the wait also gives
-// up early once another thread has flagged an error, and a wait that runs out
-// of time records kErrTimeout there.  Returns false when the wait gave up.
+// of wall time (measured on the SM cycle counter, taken as 1 cycle per ns: at
+// clocks above 1 GHz the limit only gets longer).  With a non-null global error
+// word `err`, a wait that has already lasted 100 us also gives up once another
+// thread has flagged an error, and a wait that runs out of time records
+// kErrTimeout there.  Healthy waits never touch global memory.  Returns false
+// when the wait gave up.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint32_t *err,
                                                   uint64_t timeout_ns)
 {
     if (mbar_try_wait(bar, parity))
         return true;
-    const uint64_t t0 = global_timer_ns();
+    const long long t0 = clock64();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity))
             return true;
-        if ((it & 63) == 0) {
-            if (err != nullptr && *(volatile uint32_t *)err != 0)
+        if ((it & 255) == 0) {
+            const unsigned long long dt = (unsigned long long)(clock64() - t0);
+            if (dt > 100000ull && err != nullptr && *(volatile uint32_t *)err != 0)
                 return false;
-            if (global_timer_ns() - t0 > timeout_ns) {
+            if (dt > timeout_ns) {
                 if (err != nullptr)
                     atomicOr(err, kErrTimeout);
                 return false;

@@ -58,6 +58,9 @@ WORKLOADS = {
                                "batched decode, w4a16: T=256, logits + N(0,0.5) expert bias"),
     "prefill": Workload("prefill", 8192, 7168, 2048, 384, 8, "bf16", "zipf", 0,
                         "prefill, w4a16: T=8192, Zipf-like expert bias"),
+    # the decode shape with 64 experts: a capture-sized case (about 1.5 GB of weights) for profiling
+    "decode_e64": Workload("decode_e64", 16, 7168, 2048, 64, 8, "bf16", "none", 0,
+                           "decode-shaped, w4a16, 64 experts (profiling case)"),
     "prefill_w4a8": Workload("prefill_w4a8", 16384, 4096, 1536, 128, 8, "mxfp8", "none", 0,
                              "prefill, w4a8: T=16384 H=4096 I=1536 E=128 top-8"),
 }
