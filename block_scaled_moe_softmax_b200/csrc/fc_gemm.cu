@@ -41,7 +41,6 @@ namespace moe_mx {
 
 namespace {
 
-constexpr int kThreads = 192;
 constexpr int kTermRowBytes = 128;             // one activation row of a K stage: 128 E4M3 codes
 constexpr int kWBytes = 128 * 128;             // 128 rows x 128 E2M1 codes in 8-bit containers
 constexpr int kWTxBytes = 128 * 128 / 2;       // ... of which the TMA transfers (and counts) the packed 4-bit data
@@ -57,6 +56,13 @@ constexpr unsigned long long kDrainTimeoutNs = 200000000ull;
 // rows per term: as many pipeline stages as fit (more stages = more bytes in
 // flight per SM, which is what the weight-streaming decode shapes need).
 template <int kActRows> struct Plan {
+    // Small batches (activation tiles of at most 32 rows) split the per-stage issue work
+    // over two producer warps (alternate stages) and two MMA warps (one activation term
+    // each, into separate accumulators summed by the epilogue): each TMA / tcgen05
+    // instruction occupies its issuing warp for tens of cycles.
+    static constexpr int kProd = kActRows < 128 ? 2 : 1;
+    static constexpr int kMma = kActRows < 128 ? 2 : 1;
+    static constexpr int kThreads = 32 * (2 + 4 + (kProd - 1) + (kMma - 1));
     static constexpr int kTermBytes = kActRows * kTermRowBytes;
     static constexpr int kActBytes = 2 * kTermBytes;
     static constexpr int kStageBytes = kActBytes + kWBytes + kAsfBytes + kWsfBytes;
@@ -164,8 +170,199 @@ __device__ __forceinline__ float silu_mul(float g, float u)
 
 } // namespace
 
+
+// Per-CTA state the warp roles share (all values are CTA-uniform).
+struct Ctx {
+    uint32_t base;        // shared-memory base (1024-byte aligned, shared window)
+    uint32_t tmem_base;
+    int total_units, kst, terms, n_mma;
+    unsigned long long tmo;
+};
+
+// Producer role, one of kProd warps (PI is a compile-time role index so that every
+// operand of the TMA issue stays warp-uniform).
+template <int kActRows, int PI>
+__device__ __forceinline__ void producer_role(const FcGemmArgs &a, const Ctx &c, const CUtensorMap *act_map,
+                                              const CUtensorMap *act_map16, const CUtensorMap *w_map, int lane)
+{
+    using P = Plan<kActRows>;
+    constexpr int kStages = P::kStages, kProd = P::kProd;
+    constexpr int kTermBytes = P::kTermBytes, kActBytes = P::kActBytes;
+    constexpr int kOffAct = P::kOffAct, kOffW = P::kOffW, kOffAsf = P::kOffAsf, kOffWsf = P::kOffWsf;
+    const Bars<kStages> bars{c.base + P::kOffBar};
+    const uint32_t base = c.base;
+    const int total_units = c.total_units, kst = c.kst, terms = c.terms;
+    const unsigned long long tmo = c.tmo;
+    uint32_t g = 0;
+    bool ok = true;
+    const int scl_ld = a.K / 32;
+    for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
+        const int4 blk = a.rowblocks[u / a.n_tiles];
+        const int nt = u % a.n_tiles;
+        const bool swap = kActRows < 128 || blk.z <= a.swap_rows;
+        const int npad = (blk.z + 15) & ~15;
+        // weight rows of this tile, as two 64-row halves: FC1 tile nt = gate rows [64nt, 64nt+64)
+        // then the matching up rows; FC2 tile nt = rows [128nt, 128nt+128)
+        const int wrow_a = blk.x * a.R + (a.fc1 ? nt * 64 : nt * 128);
+        const int wrow_b = a.fc1 ? wrow_a + a.R / 2 : wrow_a + 64;
+        const int rb = blk.y / 128;
+        const uint32_t act_bytes = (uint32_t)terms * (swap ? (uint32_t)npad * 128u : (uint32_t)kTermBytes);
+        for (int kk = 0; kk < kst; ++kk, ++g) {
+            if ((int)(g % kProd) != PI)
+                continue; // the other producer warp fills this stage
+            const int s = g % kStages;
+            const uint32_t ph = (g / kStages) & 1;
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.empty(s), ph ^ 1, a.err, tmo))) {
+                ok = false;
+                break;
+            }
+            // weight scale bytes: 4 per row (the 4 blocks of this K stage) into the atom layout
+            const uint32_t wsf = base + kOffWsf + s * kWsfBytes;
+            for (int r = lane; r < 128; r += 32) {
+                const int wr = r < 64 ? wrow_a + r : wrow_b + (r - 64);
+                cp_async_4(wsf + sf_atom_offset(r, 0), a.wscale + (size_t)wr * scl_ld + kk * 4);
+            }
+            cp_async_mbar_arrive_noinc(bars.full(s));
+            __syncwarp();
+            // every operand below is computed by the whole (converged) warp; then one elected lane
+            // issues the stage's copies back to back
+            const uint32_t full_s = bars.full(s);
+            const uint32_t act = base + kOffAct + s * kActBytes;
+            const uint32_t wdst = base + kOffW + s * kWBytes;
+            const int kx = kk * 128;
+            const uint8_t *asf_src = a.act_sf + ((size_t)rb * kst + kk) * 1024;
+            const uint32_t asf_dst = base + kOffAsf + s * kAsfBytes;
+            const uint32_t tx = act_bytes + kWTxBytes + (uint32_t)terms * 512u;
+            const int row0 = blk.y, row1 = a.act_rows + blk.y;
+            if (elect_one()) {
+                mbar_arrive_expect_tx(full_s, tx);
+                if (!swap) {
+                    tma_load_2d(act, act_map, kx, row0, full_s);
+                    if (terms > 1)
+                        tma_load_2d(act + kTermBytes, act_map, kx, row1, full_s);
+                } else {
+                    for (int r16 = 0; r16 < npad; r16 += 16) {
+                        tma_load_2d(act + r16 * 128, act_map16, kx, row0 + r16, full_s);
+                        if (terms > 1)
+                            tma_load_2d(act + kTermBytes + r16 * 128, act_map16, kx, row1 + r16, full_s);
+                    }
+                }
+                tma_load_2d(wdst, w_map, kx, wrow_a, full_s);
+                tma_load_2d(wdst + kWBytes / 2, w_map, kx, wrow_b, full_s);
+                bulk_copy_g2s(asf_dst, asf_src, (uint32_t)terms * 512u, full_s);
+            }
+            __syncwarp();
+        }
+    }
+    // drain: every stage issued must have landed before the CTA may exit
+    const uint32_t first = g > (uint32_t)kStages ? g - kStages : 0u;
+    for (uint32_t q = first; q < g; ++q)
+        if ((int)(q % kProd) == PI)
+            mbar_wait_bounded(bars.full(q % kStages), (q / kStages) & 1, nullptr, kDrainTimeoutNs);
+}
+
+// MMA role, one of kMma warps; MI (compile-time) selects the activation terms
+// (t % kMma == MI), the accumulator and the scale-factor columns of this warp.
+template <int kActRows, int MI>
+__device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
+{
+    using P = Plan<kActRows>;
+    constexpr int kStages = P::kStages, kMma = P::kMma;
+    constexpr int kTermBytes = P::kTermBytes, kActBytes = P::kActBytes;
+    constexpr int kOffAct = P::kOffAct, kOffW = P::kOffW, kOffAsf = P::kOffAsf, kOffWsf = P::kOffWsf;
+    const Bars<kStages> bars{c.base + P::kOffBar};
+    const uint32_t base = c.base, tmem_base = c.tmem_base;
+    const int total_units = c.total_units, kst = c.kst, terms = c.terms;
+    const unsigned long long tmo = c.tmo;
+    // ------------------------------------------------------------ MMA issuer (whole warp, one lane issues)
+    uint32_t g = 0, cnt = 0;
+    bool ok = true;
+    // this warp's scale-factor columns: weights at +0, its activation terms at +4, +8
+    const uint32_t sf_w = tmem_base + kSfCol + 16u * (uint32_t)MI;
+    for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x, ++cnt) {
+        const int4 blk = a.rowblocks[u / a.n_tiles];
+        const bool swap = kActRows < 128 || blk.z <= a.swap_rows;
+        const uint32_t npad = (uint32_t)((blk.z + 15) & ~15);
+        const uint32_t idesc0 = swap ? idesc_mx(kFmtE2M1, kFmtE4M3, 128, npad, 0)
+                                     : idesc_mx(kFmtE4M3, kFmtE2M1, 128, 128, 0);
+        const int buf = cnt & 1;
+        if (!__all_sync(0xFFFFFFFFu,
+                        mbar_wait_bounded(bars.acc_empty(buf), ((cnt >> 1) & 1) ^ 1, a.err, tmo))) {
+            ok = false;
+            break;
+        }
+        tc_fence_after();
+        // accumulator: one per buffer, or (split) one per buffer and MMA warp, 64 columns apart
+        const uint32_t d = tmem_base + buf * 128 + (kMma > 1 ? 64u * (uint32_t)MI : 0u);
+        for (int kk = 0; kk < kst; ++kk, ++g) {
+            const int s = g % kStages;
+            const uint32_t ph = (g / kStages) & 1;
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.full(s), ph, a.err, tmo))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            // Every operand is computed by the whole (converged) warp first; then one elected lane
+            // issues the stage's scale copies, MMAs and commit back to back (measured: an elect /
+            // reconverge around each instruction costs more than the instruction itself).
+            const uint32_t act = base + kOffAct + s * kActBytes;
+            const uint32_t wt = base + kOffW + s * kWBytes;
+            const uint32_t wsf_s = base + kOffWsf + s * kWsfBytes;
+            const uint32_t asf_s = base + kOffAsf + s * kAsfBytes;
+            uint64_t opa[4][2], opb[4][2];
+            uint32_t idesc[4];
+#pragma unroll
+            for (int k32 = 0; k32 < 4; ++k32) {
+                // the scale-factor byte of this 32-element block sits in both sf-id fields
+                idesc[k32] = idesc0 | ((uint32_t)k32 << 4) | ((uint32_t)k32 << 29);
+                const uint64_t dw = smem_desc_sw128(wt + 32 * k32);
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    const uint64_t da = smem_desc_sw128(act + t * kTermBytes + 32 * k32);
+                    opa[k32][t] = swap ? dw : da;
+                    opb[k32][t] = swap ? da : dw;
+                }
+            }
+            uint32_t sfa[2], sfb[2];
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                sfa[t] = swap ? sf_w : sf_w + 4 + 4 * t;
+                sfb[t] = swap ? sf_w + 4 + 4 * t : sf_w;
+            }
+            const bool t0 = (0 % kMma) == MI, t1 = terms > 1 && (1 % kMma) == MI;
+            const uint32_t empty_s = bars.empty(s);
+            if (elect_one()) {
+                // scale atoms -> TMEM (in order with the MMAs below and with the previous stage's MMAs)
+                tmem_cp_sf_atom(sf_w, wsf_s);
+                if (t0)
+                    tmem_cp_sf_atom(sf_w + 4, asf_s);
+                if (t1)
+                    tmem_cp_sf_atom(sf_w + 8, asf_s + 512);
+#pragma unroll
+                for (int k32 = 0; k32 < 4; ++k32) {
+                    if (t0)
+                        umma_mx(d, opa[k32][0], opb[k32][0], idesc[k32], sfa[0], sfb[0], (kk | k32) != 0);
+                    if (t1)
+                        umma_mx(d, opa[k32][1], opb[k32][1], idesc[k32], sfa[1], sfb[1],
+                                (kMma > 1) ? (kk | k32) != 0 : 1u);
+                }
+                umma_commit(empty_s);
+            }
+            __syncwarp();
+        }
+        if (ok && elect_one())
+            umma_commit(bars.acc_full(buf));
+        __syncwarp();
+    }
+    // all MMAs must have completed before TMEM is released
+    if (elect_one())
+        umma_commit(bars.mma_done());
+    __syncwarp();
+    mbar_wait_bounded(bars.mma_done(), 0, nullptr, kDrainTimeoutNs);
+}
+
 template <int kActRows>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Plan<kActRows>::kThreads, 1)
     fc_gemm_kernel(const FcGemmArgs a, const __grid_constant__ CUtensorMap act_map,
                    const __grid_constant__ CUtensorMap act_map16, const __grid_constant__ CUtensorMap w_map)
 {
@@ -174,21 +371,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kTermBytes = P::kTermBytes, kActBytes = P::kActBytes;
     constexpr int kOffAct = P::kOffAct, kOffW = P::kOffW, kOffAsf = P::kOffAsf, kOffWsf = P::kOffWsf;
     constexpr int kOffX = P::kOffX, kOffBar = P::kOffBar, kOffTmemSlot = P::kOffTmemSlot;
+    constexpr int kProd = P::kProd, kMma = P::kMma;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *const gsm = smem_raw + (base - raw);
     const Bars<kStages> bars{base + kOffBar};
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // warp roles: 0 producer 0, 1 MMA 0 (+ TMEM owner), 2..5 epilogue, 6 producer 1, 7 MMA 1
+    const int n_mma = kMma < a.terms ? kMma : a.terms; // MMA warps with work (one term each when split)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(bars.full(s), 1 + 32); // producer's expect_tx + 32 cp.async arrivals
-            mbar_init(bars.empty(s), 1);     // MMA commit
+            mbar_init(bars.full(s), 1 + 32);  // producer's expect_tx + 32 cp.async arrivals
+            mbar_init(bars.empty(s), n_mma);  // one commit per MMA warp
         }
-        mbar_init(bars.mma_done(), 1);
+        mbar_init(bars.mma_done(), n_mma);
         for (int b = 0; b < 2; ++b) {
-            mbar_init(bars.acc_full(b), 1);
+            mbar_init(bars.acc_full(b), n_mma);
             mbar_init(bars.acc_empty(b), 128);
         }
         fence_mbar_init();
@@ -212,126 +412,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int terms = a.terms; // activation terms per row: 1 (w4a8) or 2 (w4a16)
     const unsigned long long tmo = a.timeout_ns;
 
+    const Ctx ctx{base, tmem_base, total_units, kst, terms, n_mma, tmo};
     if (warp == 0) {
-        // ------------------------------------------------------------ producer (whole warp)
-        uint32_t g = 0;
-        bool ok = true;
-        const int scl_ld = a.K / 32;
-        for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
-            const int4 blk = a.rowblocks[u / a.n_tiles];
-            const int nt = u % a.n_tiles;
-            const bool swap = kActRows < 128 || blk.z <= a.swap_rows;
-            const int npad = (blk.z + 15) & ~15;
-            // weight rows of this tile, as two 64-row halves: FC1 tile nt = gate rows [64nt, 64nt+64)
-            // then the matching up rows; FC2 tile nt = rows [128nt, 128nt+128)
-            const int wrow_a = blk.x * a.R + (a.fc1 ? nt * 64 : nt * 128);
-            const int wrow_b = a.fc1 ? wrow_a + a.R / 2 : wrow_a + 64;
-            const int rb = blk.y / 128;
-            const uint32_t act_bytes = (uint32_t)terms * (swap ? (uint32_t)npad * 128u : (uint32_t)kTermBytes);
-            for (int kk = 0; kk < kst; ++kk, ++g) {
-                const int s = g % kStages;
-                const uint32_t ph = (g / kStages) & 1;
-                if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.empty(s), ph ^ 1, a.err, tmo))) {
-                    ok = false;
-                    break;
-                }
-                // weight scale bytes: 4 per row (the 4 blocks of this K stage) into the atom layout
-                const uint32_t wsf = base + kOffWsf + s * kWsfBytes;
-                for (int r = lane; r < 128; r += 32) {
-                    const int wr = r < 64 ? wrow_a + r : wrow_b + (r - 64);
-                    cp_async_4(wsf + sf_atom_offset(r, 0), a.wscale + (size_t)wr * scl_ld + kk * 4);
-                }
-                cp_async_mbar_arrive_noinc(bars.full(s));
-                __syncwarp();
-                if (elect_one()) {
-                    mbar_arrive_expect_tx(bars.full(s), act_bytes + kWTxBytes + (uint32_t)terms * 512u);
-                    const uint32_t act = base + kOffAct + s * kActBytes;
-                    for (int t = 0; t < terms; ++t) {
-                        const int row = t * a.act_rows + blk.y;
-                        if (!swap) {
-                            tma_load_2d(act + t * kTermBytes, &act_map, kk * 128, row, bars.full(s));
-                        } else {
-                            for (int r16 = 0; r16 < npad; r16 += 16)
-                                tma_load_2d(act + t * kTermBytes + r16 * 128, &act_map16, kk * 128, row + r16,
-                                            bars.full(s));
-                        }
-                    }
-                    const uint32_t wdst = base + kOffW + s * kWBytes;
-                    tma_load_2d(wdst, &w_map, kk * 128, wrow_a, bars.full(s));
-                    tma_load_2d(wdst + kWBytes / 2, &w_map, kk * 128, wrow_b, bars.full(s));
-                    bulk_copy_g2s(base + kOffAsf + s * kAsfBytes, a.act_sf + ((size_t)rb * kst + kk) * 1024,
-                                  (uint32_t)terms * 512u, bars.full(s));
-                }
-                __syncwarp();
-            }
-        }
-        // drain: every stage issued must have landed before the CTA may exit
-        const uint32_t first = g > (uint32_t)kStages ? g - kStages : 0u;
-        for (uint32_t q = first; q < g; ++q)
-            mbar_wait_bounded(bars.full(q % kStages), (q / kStages) & 1, nullptr, kDrainTimeoutNs);
+        producer_role<kActRows, 0>(a, ctx, &act_map, &act_map16, &w_map, lane);
+    } else if (kProd > 1 && warp == 6) {
+        producer_role<kActRows, (kProd > 1 ? 1 : 0)>(a, ctx, &act_map, &act_map16, &w_map, lane);
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer (whole warp, one lane issues)
-        uint32_t g = 0, cnt = 0;
-        bool ok = true;
-        const uint32_t sf_w = tmem_base + kSfCol;
-        for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x, ++cnt) {
-            const int4 blk = a.rowblocks[u / a.n_tiles];
-            const bool swap = kActRows < 128 || blk.z <= a.swap_rows;
-            const uint32_t npad = (uint32_t)((blk.z + 15) & ~15);
-            const uint32_t idesc0 = swap ? idesc_mx(kFmtE2M1, kFmtE4M3, 128, npad, 0)
-                                         : idesc_mx(kFmtE4M3, kFmtE2M1, 128, 128, 0);
-            const int buf = cnt & 1;
-            if (!__all_sync(0xFFFFFFFFu,
-                            mbar_wait_bounded(bars.acc_empty(buf), ((cnt >> 1) & 1) ^ 1, a.err, tmo))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const uint32_t d = tmem_base + buf * 128;
-            for (int kk = 0; kk < kst; ++kk, ++g) {
-                const int s = g % kStages;
-                const uint32_t ph = (g / kStages) & 1;
-                if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.full(s), ph, a.err, tmo))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t act = base + kOffAct + s * kActBytes;
-                const uint32_t wt = base + kOffW + s * kWBytes;
-                if (elect_one()) {
-                    // scale atoms -> TMEM (in order with the MMAs below and with the previous stage's MMAs)
-                    tmem_cp_sf_atom(sf_w, base + kOffWsf + s * kWsfBytes);
-                    for (int t = 0; t < terms; ++t)
-                        tmem_cp_sf_atom(sf_w + 4 + 4 * t, base + kOffAsf + s * kAsfBytes + 512 * t);
-#pragma unroll
-                    for (int k32 = 0; k32 < 4; ++k32) {
-                        const uint64_t dw = smem_desc_sw128(wt + 32 * k32);
-                        // the scale-factor byte of this 32-element block sits in both sf-id fields
-                        const uint32_t idesc = idesc0 | ((uint32_t)k32 << 4) | ((uint32_t)k32 << 29);
-                        for (int t = 0; t < terms; ++t) {
-                            const uint64_t da = smem_desc_sw128(act + t * kTermBytes + 32 * k32);
-                            const uint32_t sf_a = sf_w + 4 + 4 * t;
-                            const uint32_t acc = (kk | k32 | t) != 0;
-                            if (!swap)
-                                umma_mx(d, da, dw, idesc, sf_a, sf_w, acc);
-                            else
-                                umma_mx(d, dw, da, idesc, sf_w, sf_a, acc);
-                        }
-                    }
-                    umma_commit(bars.empty(s));
-                }
-                __syncwarp();
-            }
-            if (ok && elect_one())
-                umma_commit(bars.acc_full(buf));
-            __syncwarp();
-        }
-        // all MMAs must have completed before TMEM is released
-        if (elect_one())
-            umma_commit(bars.mma_done());
-        __syncwarp();
-        mbar_wait_bounded(bars.mma_done(), 0, nullptr, kDrainTimeoutNs);
-    } else {
+        mma_role<kActRows, 0>(a, ctx);
+    } else if (kMma > 1 && warp == 5 + kProd) {
+        if (n_mma > 1)
+            mma_role<kActRows, (kMma > 1 ? 1 : 0)>(a, ctx);
+    } else if (warp >= 2 && warp < 6) {
         // ------------------------------------------------------------ epilogue (warps 2..5)
         const int q = warp & 3; // TMEM lane quarter this warp may access
         float *xch = reinterpret_cast<float *>(gsm + kOffX);
@@ -393,6 +484,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int n0 = 0; n0 < npad; n0 += 16) {
                     uint32_t v[16];
                     tmem_ld16(tb + n0, v);
+                    if (kMma > 1 && terms > 1) {
+                        // split accumulation: add the second MMA warp's partial sums
+                        uint32_t v1[16];
+                        tmem_ld16(tb + 64 + n0, v1);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(v1[j]));
+                    }
                     tmem_wait_ld();
                     if (a.fc1) {
                         // the up rows live in lanes 64..127: hand them to the gate lanes through smem
@@ -457,9 +557,9 @@ void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUten
     // At most 32 tokens: every row block has at most 32 rows and runs with its tokens on N,
     // so the activation tiles shrink and the pipeline gets more stages.
     if (a.max_block_rows <= 32)
-        fc_gemm_kernel<32><<<grid, kThreads, Plan<32>::kSmemBytes, s>>>(a, act_map, act_map16, w_map);
+        fc_gemm_kernel<32><<<grid, Plan<32>::kThreads, Plan<32>::kSmemBytes, s>>>(a, act_map, act_map16, w_map);
     else
-        fc_gemm_kernel<128><<<grid, kThreads, Plan<128>::kSmemBytes, s>>>(a, act_map, act_map16, w_map);
+        fc_gemm_kernel<128><<<grid, Plan<128>::kThreads, Plan<128>::kSmemBytes, s>>>(a, act_map, act_map16, w_map);
 }
 
 // ---------------------------------------------------------------- watchdog self-test
