@@ -61,6 +61,9 @@ WORKLOADS = {
     # the decode shape with 64 experts: a capture-sized case (about 1.5 GB of weights) for profiling
     "decode_e64": Workload("decode_e64", 16, 7168, 2048, 64, 8, "bf16", "none", 0,
                            "decode-shaped, w4a16, 64 experts (profiling case)"),
+    # a prefill shape with 64 experts and 2048 tokens: a capture-sized case for profiling
+    "prefill_e64": Workload("prefill_e64", 2048, 7168, 2048, 64, 8, "bf16", "none", 0,
+                            "prefill-shaped, w4a16, 64 experts, 2048 tokens (profiling case)"),
     "prefill_w4a8": Workload("prefill_w4a8", 16384, 4096, 1536, 128, 8, "mxfp8", "none", 0,
                              "prefill, w4a8: T=16384 H=4096 I=1536 E=128 top-8"),
 }

@@ -55,7 +55,7 @@ def test_host_validation_without_gpu(lib):
     assert lib.moe_mx_quantize(None, 4, 48, 0, None, None, None) == moe_mx.MOE_MX_ERR_INVALID_ARG
     assert lib.moe_mx_quantize(None, 4, 64, 7, None, None, None) == moe_mx.MOE_MX_ERR_INVALID_ARG
     h = ctypes.c_void_p()
-    assert lib.moe_mx_create(ctypes.byref(h), 384, 128, 8, 16, 2, 0) == moe_mx.MOE_MX_ERR_UNSUPPORTED
+    assert lib.moe_mx_create(ctypes.byref(h), 200, 128, 8, 16, 2, 0) == moe_mx.MOE_MX_ERR_UNSUPPORTED
     assert lib.moe_mx_create(ctypes.byref(h), 256, 100, 8, 16, 2, 0) == moe_mx.MOE_MX_ERR_UNSUPPORTED
     assert lib.moe_mx_create(ctypes.byref(h), 256, 128, 8, 16, 9, 0) == moe_mx.MOE_MX_ERR_INVALID_ARG
     assert lib.moe_mx_create(ctypes.byref(h), 256, 128, 2000, 16, 2, 0) == moe_mx.MOE_MX_ERR_UNSUPPORTED
