@@ -79,7 +79,7 @@ def _load():
         lib.oracle_route.restype = None
         lib.oracle_group.argtypes = [i32, i32, i32, P, P, P, P]
         lib.oracle_group.restype = None
-        lib.oracle_moe_forward.argtypes = [i32] * 6 + [P] * 6 + [P, i32, P, P, P, i32]
+        lib.oracle_moe_forward.argtypes = [i32] * 6 + [P] * 6 + [P, i32, P, P, P, P, i32]
         lib.oracle_moe_forward.restype = i32
         _lib = lib
         return lib
@@ -174,13 +174,14 @@ def group(ids: np.ndarray, E: int):
 # ---------------------------------------------------------------- the layer
 def moe_forward(x_bf16_bits: np.ndarray, logits: np.ndarray, w1: np.ndarray, w1s: np.ndarray,
                 w2: np.ndarray, w2s: np.ndarray, top_k: int, act_mode: int = ACT_BF16,
-                tokens=None, nthreads: int | None = None):
+                tokens=None, nthreads: int | None = None, exact: bool = False):
     """Evaluate the layer per token.
 
     x_bf16_bits: uint16 [T, H] (bf16 bit patterns); logits f32 [T, E];
     w1 u8 [E, 2I, H/2], w1s u8 [E, 2I, H/32]; w2 u8 [E, H, I/2], w2s u8 [E, H, I/32].
     tokens: optional list of token indices to evaluate (default: all).
-    Returns (out bf16 bits uint16 [n, H], ids i32 [n, k], w f32 [n, k]).
+    Returns (out bf16 bits uint16 [n, H], ids i32 [n, k], w f32 [n, k]), plus, with
+    exact=True, the float64 output before its final bf16 rounding as a fourth item.
     """
     x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
     logits = np.ascontiguousarray(logits, dtype=np.float32)
@@ -200,12 +201,15 @@ def moe_forward(x_bf16_bits: np.ndarray, logits: np.ndarray, w1: np.ndarray, w1s
     out = np.empty((n, H), dtype=np.uint16)
     ids = np.empty((n, top_k), dtype=np.int32)
     w = np.empty((n, top_k), dtype=np.float32)
+    out_exact = np.empty((n, H), dtype=np.float64) if exact else None
     rc = _load().oracle_moe_forward(
         T, H, I, E, top_k, act_mode, _ptr(x), _ptr(logits), _ptr(w1), _ptr(w1s), _ptr(w2), _ptr(w2s),
         _ptr(tok_arr) if tok_arr is not None else None, n, _ptr(out), _ptr(ids), _ptr(w),
-        nthreads or default_threads())
+        _ptr(out_exact) if exact else None, nthreads or default_threads())
     if rc != 0:
         raise ValueError("oracle_moe_forward rejected its arguments")
+    if exact:
+        return out, ids, w, out_exact
     return out, ids, w
 
 

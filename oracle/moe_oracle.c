@@ -373,6 +373,7 @@ typedef struct {
     const uint8_t *w1, *w1s, *w2, *w2s;
     const int32_t *tokens;
     uint16_t *out;
+    double *out_exact;
     int32_t *ids_out;
     float *w_out;
     int64_t i0, i1;
@@ -452,8 +453,11 @@ static void forward_token(const fwd_job *jb, int64_t slot)
             acc[n] += (double)w[j] * y;
         }
     }
-    for (int n = 0; n < H; ++n)
+    for (int n = 0; n < H; ++n) {
         jb->out[slot * H + n] = double_to_bf16_bits(acc[n]);
+        if (jb->out_exact)
+            jb->out_exact[slot * H + n] = acc[n];
+    }
     free(a);
     free(h);
     free(acc);
@@ -471,6 +475,8 @@ static void *forward_worker(void *arg)
  * Evaluate the layer for n_eval tokens.  tokens == NULL evaluates tokens
  * 0..n_eval-1; otherwise tokens[i] names the token whose output goes to row i
  * of out (bf16 bits, [n_eval, H]) and of ids_out/w_out ([n_eval, k], optional).
+ * out_exact (optional, [n_eval, H]) receives the combined output before its
+ * final rounding to bf16 (the exact value a rounded result is measured against).
  * act_mode 0 = bf16 activations (w4a16), 1 = MXFP8 activations (w4a8).
  * Layouts: x bf16 [T,H]; logits f32 [T,E]; w1 codes [E,2I,H/2] (gate rows
  * [0,I), up rows [I,2I)), w1s [E,2I,H/32]; w2 codes [E,H,I/2], w2s [E,H,I/32].
@@ -479,7 +485,7 @@ static void *forward_worker(void *arg)
 int oracle_moe_forward(int T, int H, int I, int E, int k, int act_mode, const uint16_t *x,
                        const float *logits, const uint8_t *w1, const uint8_t *w1s, const uint8_t *w2,
                        const uint8_t *w2s, const int32_t *tokens, int n_eval, uint16_t *out,
-                       int32_t *ids_out, float *w_out, int nthreads)
+                       int32_t *ids_out, float *w_out, double *out_exact, int nthreads)
 {
     if (T < 0 || H <= 0 || I <= 0 || H % 32 || I % 32 || E < 1 || E > 1024 || k < 1 || k > E ||
         (act_mode != 0 && act_mode != 1) || n_eval < 0 || !out)
@@ -498,7 +504,7 @@ int oracle_moe_forward(int T, int H, int I, int E, int k, int act_mode, const ui
     pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
     fwd_job *jobs = (fwd_job *)malloc(sizeof(fwd_job) * (size_t)nthreads);
     for (int i = 0; i < nthreads; ++i) {
-        jobs[i] = (fwd_job){T, H, I, E, k, act_mode, x, logits, w1, w1s, w2, w2s, tokens, out, ids_out,
+        jobs[i] = (fwd_job){T, H, I, E, k, act_mode, x, logits, w1, w1s, w2, w2s, tokens, out, out_exact, ids_out,
                             w_out, (int64_t)n_eval * i / nthreads, (int64_t)n_eval * (i + 1) / nthreads};
         pthread_create(&th[i], NULL, forward_worker, &jobs[i]);
     }

@@ -84,9 +84,12 @@ def to_device(inp, device="cuda"):
 
 
 def oracle_forward(inp, top_k, act_mode, tokens=None):
-    out, ids, w = oracle.moe_forward(inp["xb"], inp["logits"].numpy(), inp["w1"], inp["w1s"], inp["w2"],
-                                     inp["w2s"], top_k, act_mode, tokens=tokens)
-    return oracle.bf16_bits_to_f64(out), ids, w
+    """The oracle's output for GPU comparisons: the exact (float64) combined value before
+    the final bf16 rounding -- a bf16 result is measured against the value it rounds, not
+    against a second, independent rounding of it -- plus the ids and weights."""
+    _, ids, w, exact = oracle.moe_forward(inp["xb"], inp["logits"].numpy(), inp["w1"], inp["w1s"], inp["w2"],
+                                          inp["w2s"], top_k, act_mode, tokens=tokens, exact=True)
+    return exact, ids, w
 
 
 def check_output(got_bf16, ref_f64, tag=""):

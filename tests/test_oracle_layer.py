@@ -161,3 +161,12 @@ def test_w4a8_on_grid_inputs():
     assert helpers.rel_frobenius(a8, a16) < 0.05
     ref8 = _reference_layer(xg, logits, wq, 1, 1)
     assert helpers.rel_frobenius(a8, ref8) < 5e-3
+
+
+def test_exact_output_rounds_to_the_bf16_output():
+    wl = workloads.WORKLOADS["tiny"]
+    xb, xf, logits, wq = _inputs(wl)
+    out, _, _, exact = oracle.moe_forward(xb, logits, wq["w1"], wq["w1s"], wq["w2"], wq["w2s"], wl.top_k, 0,
+                                          exact=True)
+    rounded = np.array([oracle.round_bf16(v) for v in exact.reshape(-1)]).reshape(exact.shape)
+    assert np.array_equal(rounded, oracle.bf16_bits_to_f64(out))
