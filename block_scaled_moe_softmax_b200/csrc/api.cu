@@ -9,6 +9,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "../../include/moe_mx.h"
@@ -577,6 +578,127 @@ int moe_mx_debug_watchdog(moe_mx_handle *h, int timeout_us, void *stream)
     cudaError_t ce = cudaGetLastError();
     if (ce != cudaSuccess)
         return cuda_fail(ce, "watchdog launch");
+    return MOE_MX_OK;
+}
+
+// ---------------------------------------------------------------- routing without allocation
+// moe_mx_route_group_noalloc serves callers that cannot allocate device memory
+// at the point of the call and keep no handle: a framework op whose device
+// memory all comes from the framework's own pool (a cudaMalloc there bypasses
+// the pool's accounting and can synchronise the device, stalling every other
+// stream), or code that routes once per step from a context where no create /
+// destroy lifetime exists.  Its only scratch -- the per-chunk expert
+// histograms and the row-block list the grouping kernels write -- lives in the
+// file-scope device array below, one copy per device, of fixed size.
+
+} // extern "C"
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20; // 1 MiB per device
+
+// Nothing in it needs to start at zero: every word a call reads is written
+// earlier in the same call (route_kernel writes each chunk's full histogram row
+// before scan_kernel reads it).  All calls on one device share it.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mu;
+void *g_scratch_addr[kMaxScratchDevices]; // per device ordinal, looked up on first use
+
+// Address of this device's copy of the scratch array.  The first lookup on a
+// device may load the library's device code there.
+int scratch_address(int dev, void **addr)
+{
+    if (dev < 0 || dev >= kMaxScratchDevices)
+        return fail(MOE_MX_ERR_UNSUPPORTED, "device %d is beyond the %d devices the scratch table covers", dev,
+                    kMaxScratchDevices);
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void *p = nullptr;
+        cudaError_t ce = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (ce != cudaSuccess)
+            return cuda_fail(ce, "cudaGetSymbolAddress(scratch)");
+        g_scratch_addr[dev] = p;
+    }
+    *addr = g_scratch_addr[dev];
+    return MOE_MX_OK;
+}
+
+} // namespace
+
+extern "C" {
+
+int moe_mx_route_group_noalloc(const float *router_logits, int num_tokens, int num_experts, int top_k,
+                               int32_t *topk_ids, float *topk_w, int32_t *counts, int32_t *pad_offsets,
+                               int32_t *sorted_pair, int32_t *pos_of_pair, void *stream)
+{
+    g_last_error.clear();
+    const int T = num_tokens, E = num_experts, k = top_k;
+    if (T < 0)
+        return fail(MOE_MX_ERR_INVALID_ARG, "num_tokens=%d must be >= 0", T);
+    if (E < 1 || E > kMaxExperts)
+        return fail(MOE_MX_ERR_UNSUPPORTED, "num_experts=%d must be in [1, %d]", E, kMaxExperts);
+    if (k < 1 || k > E || k > kMaxTopK)
+        return fail(MOE_MX_ERR_INVALID_ARG, "top_k=%d must be in [1, min(num_experts, %d)]", k, kMaxTopK);
+    const int64_t pairs = (int64_t)T * k;
+    if (pairs > INT32_MAX / 2)
+        return fail(MOE_MX_ERR_UNSUPPORTED, "num_tokens * top_k = %lld is too large", (long long)pairs);
+    // scratch plan: [num_rowblocks | pad to 256 B][rowblocks int4 x blocks][chunk histograms int32 x chunks x E]
+    auto scratch_bytes = [&](int64_t tokens) {
+        const int64_t nchunks = (tokens + kRouteChunk - 1) / kRouteChunk;
+        const int64_t nblocks = grouped_rows_bound(E, tokens * k) / kBlockRows;
+        return round_up(256 + 16 * nblocks, 256) + 4 * nchunks * E;
+    };
+    const int64_t off_rowblocks = 256;
+    const int64_t off_hist = round_up(off_rowblocks + 16 * (grouped_rows_bound(E, pairs) / kBlockRows), 256);
+    if (scratch_bytes(T) > (int64_t)kNoAllocScratchBytes) {
+        int64_t lo = 0, hi = T; // largest token count that fits, for the message
+        while (lo < hi) {
+            const int64_t mid = (lo + hi + 1) / 2;
+            if (scratch_bytes(mid) <= (int64_t)kNoAllocScratchBytes)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        return fail(MOE_MX_ERR_UNSUPPORTED,
+                    "num_tokens=%d, num_experts=%d, top_k=%d need %lld bytes of routing scratch; the static "
+                    "scratch holds %lld bytes (at most %lld tokens at this expert count and top_k)",
+                    T, E, k, (long long)scratch_bytes(T), (long long)kNoAllocScratchBytes, (long long)lo);
+    }
+    if (T == 0)
+        return MOE_MX_OK;
+    int dev = 0;
+    cudaError_t ce = cudaGetDevice(&dev);
+    if (ce != cudaSuccess)
+        return cuda_fail(ce, "cudaGetDevice");
+    int rc;
+    if ((rc = check_ptr(router_logits, dev, "router_logits")) || (rc = check_ptr(topk_ids, dev, "topk_ids")) ||
+        (rc = check_ptr(topk_w, dev, "topk_w")) || (rc = check_ptr(counts, dev, "counts")) ||
+        (rc = check_ptr(pad_offsets, dev, "pad_offsets")) || (rc = check_ptr(sorted_pair, dev, "sorted_pair")) ||
+        (rc = check_ptr(pos_of_pair, dev, "pos_of_pair")))
+        return rc;
+    void *scratch = nullptr;
+    if ((rc = scratch_address(dev, &scratch)))
+        return rc;
+    unsigned char *base = static_cast<unsigned char *>(scratch);
+    RouteGroupArgs ra{router_logits,
+                      T,
+                      E,
+                      k,
+                      topk_ids,
+                      topk_w,
+                      reinterpret_cast<int32_t *>(base + off_hist),
+                      counts,
+                      pad_offsets,
+                      reinterpret_cast<int4 *>(base + off_rowblocks),
+                      reinterpret_cast<int32_t *>(base),
+                      sorted_pair,
+                      pos_of_pair};
+    launch_route_and_group(ra, static_cast<cudaStream_t>(stream));
+    ce = cudaGetLastError();
+    if (ce != cudaSuccess)
+        return cuda_fail(ce, "routing launch");
     return MOE_MX_OK;
 }
 

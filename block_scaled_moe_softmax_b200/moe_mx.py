@@ -45,6 +45,7 @@ SIGNATURES = {
     "moe_mx_debug_watchdog": (_I, [_P, _I, _P]),
     "moe_mx_set_stage_timing": (_I, [_P, _I]),
     "moe_mx_get_stage_times": (_I, [_P, _P]),
+    "moe_mx_route_group_noalloc": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
 }
 STAGES = ("route", "gather", "fc1", "fc2", "combine")
 
@@ -141,6 +142,14 @@ def moe_mx_get_routing(handle: int, topk_ids=None, topk_w=None, counts=None, pad
                        stream=None) -> None:
     _check(load_library().moe_mx_get_routing(handle, _ptr(topk_ids), _ptr(topk_w), _ptr(counts),
                                              _ptr(pad_offsets), _ptr(sorted_pair), _stream(stream)))
+
+
+def moe_mx_route_group_noalloc(router_logits, num_tokens: int, num_experts: int, top_k: int, topk_ids, topk_w,
+                               counts, pad_offsets, sorted_pair, pos_of_pair, stream=None) -> None:
+    """Routing + grouping into caller buffers, with no handle and no device allocation (see the header)."""
+    _check(load_library().moe_mx_route_group_noalloc(
+        _ptr(router_logits), num_tokens, num_experts, top_k, _ptr(topk_ids), _ptr(topk_w), _ptr(counts),
+        _ptr(pad_offsets), _ptr(sorted_pair), _ptr(pos_of_pair), _stream(stream)))
 
 
 def moe_mx_debug_watchdog(handle: int, timeout_us: int, stream=None) -> None:

@@ -219,6 +219,53 @@ MOE_MX_API int moe_mx_get_stage_times(moe_mx_handle *h, float *ms);
  */
 MOE_MX_API int moe_mx_debug_watchdog(moe_mx_handle *h, int timeout_us, void *stream);
 
+/*
+ * Routing and grouping without a handle and without allocating: the router
+ * (softmax, top-k with the lowest expert index winning ties, renormalised
+ * weights) and the stable grouping by expert into 128-row padded segments --
+ * the same kernels and results as the first stage of moe_mx_forward
+ * (TokenSpeed-kernel README, "Public API": moe_route and moe_dispatch).  The
+ * pages have no counterpart of this entry point; it exists for callers that
+ * cannot allocate device memory at the point of the call and hold no handle
+ * (for example an op whose device memory must all come from its framework's
+ * own pool, where a cudaMalloc would bypass the pool and can synchronise the
+ * device).
+ *
+ * It allocates nothing (no cudaMalloc / cudaFree, no allocating library call).
+ * Its scratch (per-chunk expert histograms, the row-block list) is a static
+ * device array of 1 MiB, one per device; nothing in it needs to start at zero.
+ * A call needs 4*E*ceil(T/64) bytes of histograms plus 16 bytes per 128-row
+ * block of the grouped layout (plus 256-byte alignment): at E = 384, top-8
+ * that allows about 41,000 tokens.  Larger shapes are rejected with
+ * MOE_MX_ERR_UNSUPPORTED and a message giving the limit.
+ *
+ * The first call on a device looks up that device's scratch address
+ * (cudaGetSymbolAddress), which may load the library's device code there: make
+ * that first call outside any stream capture (e.g. at setup).  All calls on one
+ * device share the scratch: calls whose executions overlap (unordered streams,
+ * several host threads) race on it and corrupt each other's results; order
+ * them (one stream, or events).
+ *
+ * All pointers are device memory of the current device, 16-byte aligned,
+ * owned by the caller, and are only read / written on `stream`:
+ *   router_logits float [T, E]    input;
+ *   topk_ids      int32 [T, k]    selected experts, descending logit;
+ *   topk_w        float [T, k]    renormalised weights;
+ *   counts        int32 [E]       pairs per expert;
+ *   pad_offsets   int32 [E+1]     first grouped row of each expert segment;
+ *   sorted_pair   int32 [rows]    pair id t*k+j at each grouped row, -1 on
+ *                                 padding rows; rows = T*k + min(T*k, E)*127
+ *                                 rounded up to 128 (capacity), of which the
+ *                                 first pad_offsets[E] are written;
+ *   pos_of_pair   int32 [T*k]     grouped row of each pair.
+ * num_tokens = 0 is a no-op.  Errors: INVALID_ARG (bad sizes, host or
+ * misaligned pointers), UNSUPPORTED (num_experts > 1024, scratch too small),
+ * CUDA (lookup or launch failure; text in moe_mx_last_error).
+ */
+MOE_MX_API int moe_mx_route_group_noalloc(const float *router_logits, int num_tokens, int num_experts, int top_k,
+                                          int32_t *topk_ids, float *topk_w, int32_t *counts, int32_t *pad_offsets,
+                                          int32_t *sorted_pair, int32_t *pos_of_pair, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
