@@ -56,22 +56,41 @@ EncodeTiledFn get_encode_fn()
 
 // 2-D row-major tensor map: inner dimension `cols` elements, `rows` rows,
 // `row_bytes` bytes from one row to the next.
-int encode_2d(CUtensorMap *map, CUtensorMapDataType dt, uint64_t row_bytes, const void *ptr, uint64_t cols,
-              uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz)
+// Tensor map of `rank` dimensions (innermost first): dims in elements, strides in bytes of
+// dimensions 1..rank-1, box in elements; 128-byte swizzle.
+int encode_nd(CUtensorMap *map, CUtensorMapDataType dt, int rank, const void *ptr, const cuuint64_t *dims,
+              const cuuint64_t *strides, const cuuint32_t *box)
 {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc)
         return fail(MOE_MX_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = enc(map, dt, rank, const_cast<void *>(ptr), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(MOE_MX_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d, rank %d)", (int)r, rank);
+    return MOE_MX_OK;
+}
+
+// 2-D row-major map: `cols` elements per row, `rows` rows, `row_bytes` from one row to the next.
+int encode_2d(CUtensorMap *map, CUtensorMapDataType dt, uint64_t row_bytes, const void *ptr, uint64_t cols,
+              uint64_t rows, uint32_t box_cols, uint32_t box_rows)
+{
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {row_bytes};
     const cuuint32_t box[2] = {box_cols, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = enc(map, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS)
-        return fail(MOE_MX_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
-    return MOE_MX_OK;
+    return encode_nd(map, dt, 2, ptr, dims, strides, box);
+}
+
+// The activation operand as [2 term planes][plane_rows][K] E4M3 codes: boxes of 128 codes x
+// box_rows rows x `terms` planes, so one copy brings both terms of a row range.
+int encode_act(CUtensorMap *map, const void *ptr, uint64_t K, uint64_t plane_rows, uint32_t box_rows, uint32_t terms)
+{
+    const cuuint64_t dims[3] = {K, plane_rows, 2};
+    const cuuint64_t strides[2] = {K, plane_rows * K};
+    const cuuint32_t box[3] = {128, box_rows, terms};
+    return encode_nd(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, ptr, dims, strides, box);
 }
 
 bool is_device_ptr(const void *p, int dev)
@@ -117,15 +136,20 @@ struct moe_mx_handle {
     int H, I, E, maxT, maxK, dev, num_sms;
     int64_t max_rows;
     int swap_rows;
+    int tile_rows; // 0: by token count; else 16, 32, 64 or 128 (MOE_MX_TILE_ROWS)
+    int scale_layout; // MOE_MX_SCALES_ROW_MAJOR or MOE_MX_SCALES_TILED
     unsigned long long timeout_ns;
     void *ws;
     int32_t *topk_ids, *chunk_hist, *counts, *pad_offsets, *num_rowblocks, *sorted_pair, *pos_of_pair;
+    int32_t *unit_counters;
     float *topk_w;
     int4 *rowblocks;
     uint8_t *Aq, *Asf, *Hq, *Hsf; // MXFP8 operand planes [2][rows][K] and their scale atoms
     float *Y;
     uint32_t *err;
-    CUtensorMap map_A, map_A16, map_H, map_H16;
+    // activation operands: [terms - 1] 128-row boxes; [terms - 1][kT2 16/32/64] boxes for tokens
+    // on N; 16-row single-plane boxes
+    CUtensorMap map_A[2], map_Asw[2][3], map_A16, map_H[2], map_Hsw[2][3], map_H16;
     const void *w1_key, *w2_key;
     CUtensorMap map_w1, map_w2;
     int last_T, last_k;
@@ -197,6 +221,10 @@ int moe_mx_create(moe_mx_handle **out, int hidden, int inter, int num_experts, i
     h->num_sms = prop.multiProcessorCount;
     const int64_t pairs = (int64_t)max_tokens * max_top_k;
     h->max_rows = grouped_rows_bound(num_experts, pairs);
+    h->scale_layout = MOE_MX_SCALES_ROW_MAJOR;
+    h->tile_rows = env_int("MOE_MX_TILE_ROWS", 0);
+    if (h->tile_rows != 16 && h->tile_rows != 32 && h->tile_rows != 64 && h->tile_rows != kBlockRows)
+        h->tile_rows = 0;
     h->swap_rows = env_int("MOE_MX_SWAP_ROWS", 64);
     if (h->swap_rows < 0)
         h->swap_rows = 0;
@@ -214,8 +242,9 @@ int moe_mx_create(moe_mx_handle **out, int hidden, int inter, int num_experts, i
         {(void **)&h->chunk_hist, sizeof(int32_t) * nchunks * num_experts},
         {(void **)&h->counts, sizeof(int32_t) * num_experts},
         {(void **)&h->pad_offsets, sizeof(int32_t) * (num_experts + 1)},
-        {(void **)&h->rowblocks, sizeof(int4) * (h->max_rows / kBlockRows)},
+        {(void **)&h->rowblocks, sizeof(int4) * (h->max_rows / 16)}, // work blocks: >= 16 padded rows each
         {(void **)&h->num_rowblocks, sizeof(int32_t)},
+        {(void **)&h->unit_counters, 2 * sizeof(int32_t)}, // FC1, FC2 work-unit counters
         {(void **)&h->sorted_pair, sizeof(int32_t) * h->max_rows},
         {(void **)&h->pos_of_pair, sizeof(int32_t) * pairs},
         {(void **)&h->err, sizeof(uint32_t)},
@@ -244,20 +273,23 @@ int moe_mx_create(moe_mx_handle **out, int hidden, int inter, int num_experts, i
         rc = cuda_fail(ce, "cudaMemset(workspace)");
     if (rc == MOE_MX_OK && (ce = fc_gemm_prepare()) != cudaSuccess)
         rc = cuda_fail(ce, "cudaFuncSetAttribute(fc_gemm)");
-    // activation operand planes: [2 terms x rows, K] E4M3 codes, 128 x 128 boxes (16-row boxes for
-    // token-on-N tiles), 128-byte swizzle = the K-major layout the MMA reads
+    // activation operand planes: [2 terms x rows, K] E4M3 codes (128-byte swizzle = the K-major
+    // layout the MMA reads): boxes over both planes of 128 rows (tokens on M) or of 16, 32 or 64
+    // rows (tokens on N), and 16-row single-plane boxes
+    for (int t = 1; t <= 2 && rc == MOE_MX_OK; ++t) {
+        rc = encode_act(&h->map_A[t - 1], h->Aq, hidden, h->max_rows, 128, t);
+        for (int i = 0; i < 3 && rc == MOE_MX_OK; ++i)
+            rc = encode_act(&h->map_Asw[t - 1][i], h->Aq, hidden, h->max_rows, 16u << i, t);
+    }
+    for (int t = 1; t <= 2 && rc == MOE_MX_OK; ++t) {
+        rc = encode_act(&h->map_H[t - 1], h->Hq, inter, h->max_rows, 128, t);
+        for (int i = 0; i < 3 && rc == MOE_MX_OK; ++i)
+            rc = encode_act(&h->map_Hsw[t - 1][i], h->Hq, inter, h->max_rows, 16u << i, t);
+    }
     if (rc == MOE_MX_OK)
-        rc = encode_2d(&h->map_A, CU_TENSOR_MAP_DATA_TYPE_UINT8, hidden, h->Aq, hidden, 2 * h->max_rows, 128, 128,
-                       CU_TENSOR_MAP_SWIZZLE_128B);
+        rc = encode_2d(&h->map_A16, CU_TENSOR_MAP_DATA_TYPE_UINT8, hidden, h->Aq, hidden, 2 * h->max_rows, 128, 16);
     if (rc == MOE_MX_OK)
-        rc = encode_2d(&h->map_A16, CU_TENSOR_MAP_DATA_TYPE_UINT8, hidden, h->Aq, hidden, 2 * h->max_rows, 128, 16,
-                       CU_TENSOR_MAP_SWIZZLE_128B);
-    if (rc == MOE_MX_OK)
-        rc = encode_2d(&h->map_H, CU_TENSOR_MAP_DATA_TYPE_UINT8, inter, h->Hq, inter, 2 * h->max_rows, 128, 128,
-                       CU_TENSOR_MAP_SWIZZLE_128B);
-    if (rc == MOE_MX_OK)
-        rc = encode_2d(&h->map_H16, CU_TENSOR_MAP_DATA_TYPE_UINT8, inter, h->Hq, inter, 2 * h->max_rows, 128, 16,
-                       CU_TENSOR_MAP_SWIZZLE_128B);
+        rc = encode_2d(&h->map_H16, CU_TENSOR_MAP_DATA_TYPE_UINT8, inter, h->Hq, inter, 2 * h->max_rows, 128, 16);
     if (rc == MOE_MX_OK && (ce = cudaDeviceSynchronize()) != cudaSuccess)
         rc = cuda_fail(ce, "cudaDeviceSynchronize(create)");
     cudaSetDevice(prev);
@@ -324,16 +356,19 @@ int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, 
         cudaSetDevice(h->dev);
 
     // weights: packed E2M1 [rows, K] unpacked by the TMA into 8-bit containers (16 codes per
-    // 16-byte granule), 128-code x 64-row boxes, 128-byte swizzle
+    // 16-byte granule), 128-byte swizzle.  W1 as [2E halves][I rows][H] so that one box of
+    // 128 codes x 64 rows x 2 halves brings a gate slice and its up slice; W2 in 128-row boxes.
     if (w1 != h->w1_key) {
-        if ((rc = encode_2d(&h->map_w1, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, H / 2, w1, H, (uint64_t)E * 2 * I,
-                            128, 64, CU_TENSOR_MAP_SWIZZLE_128B)))
+        const cuuint64_t dims[3] = {(cuuint64_t)H, (cuuint64_t)I, (cuuint64_t)2 * E};
+        const cuuint64_t strides[2] = {(cuuint64_t)H / 2, (cuuint64_t)I * (H / 2)};
+        const cuuint32_t box[3] = {128, 64, 2};
+        if ((rc = encode_nd(&h->map_w1, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, w1, dims, strides, box)))
             goto done;
         h->w1_key = w1;
     }
     if (w2 != h->w2_key) {
         if ((rc = encode_2d(&h->map_w2, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, I / 2, w2, I, (uint64_t)E * H, 128,
-                            64, CU_TENSOR_MAP_SWIZZLE_128B)))
+                            128)))
             goto done;
         h->w2_key = w2;
     }
@@ -341,8 +376,10 @@ int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, 
         const int64_t pairs = (int64_t)T * k;
         const int64_t rows = grouped_rows_bound(E, pairs);
         cudaError_t ce = cudaMemsetAsync(h->sorted_pair, 0xFF, sizeof(int32_t) * rows, s);
+        if (ce == cudaSuccess)
+            ce = cudaMemsetAsync(h->unit_counters, 0, 2 * sizeof(int32_t), s);
         if (ce != cudaSuccess) {
-            rc = cuda_fail(ce, "cudaMemsetAsync(sorted_pair)");
+            rc = cuda_fail(ce, "cudaMemsetAsync(workspace)");
             goto done;
         }
         cudaEvent_t *evset = h->timing ? h->ev + (h->n_timed % kTimingRing) * kEvPerFwd : nullptr;
@@ -351,8 +388,18 @@ int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, 
                 cudaEventRecord(evset[i], s);
         };
         mark(0);
+        // activation tile rows per term of the GEMM variant; the segments are split into work
+        // blocks of at most that many rows (a segment holds one expert's tokens, so at 16 or 32
+        // tokens nothing is split).  Up to a few hundred tokens 64-row blocks, all of which run
+        // with their tokens on N, beat 128-row blocks: more pipeline stages fit.
+        const int tile_rows = h->tile_rows > 0 ? h->tile_rows
+                              : T <= 16        ? 16
+                              : T <= 32        ? 32
+                              : T <= 512       ? 64
+                                               : kBlockRows;
         RouteGroupArgs ra{router_logits, T, E, k, h->topk_ids, h->topk_w, h->chunk_hist, h->counts,
-                          h->pad_offsets, h->rowblocks, h->num_rowblocks, h->sorted_pair, h->pos_of_pair};
+                          h->pad_offsets, h->rowblocks, h->num_rowblocks, h->sorted_pair, h->pos_of_pair,
+                          tile_rows};
         launch_route_and_group(ra, s);
         mark(1);
         const int mx8 = act_dtype == MOE_MX_ACT_MXFP8;
@@ -363,6 +410,8 @@ int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, 
         f1.rowblocks = h->rowblocks;
         f1.num_rowblocks = h->num_rowblocks;
         f1.wscale = w1_scale;
+        f1.wsf_tiled = h->scale_layout == MOE_MX_SCALES_TILED;
+        f1.unit_counter = h->unit_counters;
         f1.act_sf = h->Asf;
         f1.hq = h->Hq;
         f1.hsf = h->Hsf;
@@ -379,13 +428,16 @@ int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, 
         f1.fc1 = 1;
         f1.act_mxfp8 = mx8;
         f1.swap_rows = h->swap_rows;
-        f1.max_block_rows = T < kBlockRows ? T : kBlockRows; // a block holds one expert's tokens
+        f1.max_block_rows = tile_rows;
         mark(2);
-        launch_fc_gemm(f1, h->map_A, h->map_A16, h->map_w1, h->num_sms, s);
+        const int sw_idx = tile_rows <= 16 ? 0 : tile_rows <= 32 ? 1 : 2; // box rows min(tile rows, 64)
+        launch_fc_gemm(f1, h->map_A[f1.terms - 1], h->map_Asw[f1.terms - 1][sw_idx], h->map_A16, h->map_w1, h->num_sms,
+                       s);
         mark(3);
 
         FcGemmArgs f2 = f1;
         f2.wscale = w2_scale;
+        f2.unit_counter = h->unit_counters + 1;
         f2.act_sf = h->Hsf;
         f2.K = I;
         f2.R = H;
@@ -393,7 +445,9 @@ int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, 
         f2.out_ld = H;
         f2.fc1 = 0;
         f2.act_mxfp8 = 0;
-        launch_fc_gemm(f2, h->map_H, h->map_H16, h->map_w2, h->num_sms, s);
+        // the maps' plane count must equal the copy's terms: the stage barrier expects exactly those bytes
+        launch_fc_gemm(f2, h->map_H[f2.terms - 1], h->map_Hsw[f2.terms - 1][sw_idx], h->map_H16, h->map_w2,
+                       h->num_sms, s);
         mark(4);
         launch_combine(h->Y, T, H, k, h->pos_of_pair, h->topk_w, static_cast<__nv_bfloat16 *>(out), h->num_sms, s);
         ce = cudaGetLastError();
@@ -498,6 +552,46 @@ int moe_mx_get_routing(const moe_mx_handle *h, int32_t *topk_ids, float *topk_w,
         if (ce != cudaSuccess)
             return cuda_fail(ce, "cudaMemcpyAsync(routing state)");
     }
+    return MOE_MX_OK;
+}
+
+int moe_mx_set_scale_layout(moe_mx_handle *h, int layout)
+{
+    g_last_error.clear();
+    if (!h)
+        return fail(MOE_MX_ERR_INVALID_ARG, "handle is NULL");
+    if (layout != MOE_MX_SCALES_ROW_MAJOR && layout != MOE_MX_SCALES_TILED)
+        return fail(MOE_MX_ERR_INVALID_ARG, "layout=%d is not MOE_MX_SCALES_ROW_MAJOR or MOE_MX_SCALES_TILED", layout);
+    h->scale_layout = layout;
+    return MOE_MX_OK;
+}
+
+int moe_mx_prepare_scales(const moe_mx_handle *h, int which, const uint8_t *src, uint8_t *dst, void *stream)
+{
+    g_last_error.clear();
+    if (!h)
+        return fail(MOE_MX_ERR_INVALID_ARG, "handle is NULL");
+    if (which != MOE_MX_W1 && which != MOE_MX_W2)
+        return fail(MOE_MX_ERR_INVALID_ARG, "which=%d is not MOE_MX_W1 or MOE_MX_W2", which);
+    int rc;
+    if ((rc = check_ptr(src, h->dev, "src")) || (rc = check_ptr(dst, h->dev, "dst")))
+        return rc;
+    const int fc1 = which == MOE_MX_W1;
+    const int R = fc1 ? 2 * h->I : h->H, K = fc1 ? h->H : h->I;
+    const size_t bytes = (size_t)h->E * R * (K / 32);
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(src), a1 = reinterpret_cast<uintptr_t>(dst);
+    if (a0 < a1 + bytes && a1 < a0 + bytes)
+        return fail(MOE_MX_ERR_INVALID_ARG, "src and dst must not overlap");
+    int prev = 0;
+    cudaGetDevice(&prev);
+    if (prev != h->dev)
+        cudaSetDevice(h->dev);
+    launch_tile_scales(src, dst, h->E, R, K, fc1, h->num_sms, static_cast<cudaStream_t>(stream));
+    cudaError_t ce = cudaGetLastError();
+    if (prev != h->dev)
+        cudaSetDevice(prev);
+    if (ce != cudaSuccess)
+        return cuda_fail(ce, "scale tiling launch");
     return MOE_MX_OK;
 }
 
@@ -642,8 +736,9 @@ int moe_mx_route_group_noalloc(const float *router_logits, int num_tokens, int n
     if (k < 1 || k > E || k > kMaxTopK)
         return fail(MOE_MX_ERR_INVALID_ARG, "top_k=%d must be in [1, min(num_experts, %d)]", k, kMaxTopK);
     const int64_t pairs = (int64_t)T * k;
-    if (pairs > INT32_MAX / 2)
-        return fail(MOE_MX_ERR_UNSUPPORTED, "num_tokens * top_k = %lld is too large", (long long)pairs);
+    if (pairs > (int64_t)65536 * kMaxTopK)
+        return fail(MOE_MX_ERR_UNSUPPORTED, "num_tokens * top_k = %lld exceeds %lld", (long long)pairs,
+                    (long long)65536 * kMaxTopK);
     // scratch plan: [num_rowblocks | pad to 256 B][rowblocks int4 x blocks][chunk histograms int32 x chunks x E]
     auto scratch_bytes = [&](int64_t tokens) {
         const int64_t nchunks = (tokens + kRouteChunk - 1) / kRouteChunk;
@@ -694,7 +789,8 @@ int moe_mx_route_group_noalloc(const float *router_logits, int num_tokens, int n
                       reinterpret_cast<int4 *>(base + off_rowblocks),
                       reinterpret_cast<int32_t *>(base),
                       sorted_pair,
-                      pos_of_pair};
+                      pos_of_pair,
+                      kBlockRows};
     launch_route_and_group(ra, static_cast<cudaStream_t>(stream));
     ce = cudaGetLastError();
     if (ce != cudaSuccess)

@@ -20,20 +20,31 @@
 // w4a8, whose dequantised value is the bf16 value FC2 consumes).  FC2 writes
 // f32 rows that the combine kernel sums.
 //
-// Per CTA (one per SM, persistent over work units u = (row block, tile)):
-//   warp 0      producer: TMA of the activation codes (128-byte swizzle), TMA
-//               of the E2M1 codes through the 4-bit -> 8-bit-container
-//               unpacking mode, a bulk copy of the activation scale atoms and
-//               cp.async of the weight scale bytes into the same atom layout;
-//   warp 1      MMA issuer (one thread) + TMEM owner: tcgen05.cp moves the
-//               stage's scale atoms to TMEM, then the block-scaled MMAs;
-//   warps 2-5   epilogue (tcgen05.ld); accumulators double-buffered in TMEM.
+// Per CTA (one per SM, persistent; work units u = (row block, weight tile) handed
+// out at run time through a global counter):
+//   producers   2 to 4 warps, taking pipeline stages round robin: TMA of the
+//               weight tile (E2M1 codes unpacked to 8-bit containers; for FC1
+//               the gate and up halves in one 3-D box), TMA of both activation
+//               term planes in one 3-D box, the stage's weight scale atom (one
+//               bulk copy in the tiled layout, else 4-byte copies) and the
+//               activation scale atom (bulk copy, or 4-byte copies laid out for
+//               N when the tokens sit on N);
+//   MMA         1 or 2 warps (alternate stages, own accumulators): tcgen05.cp of
+//               the stage's scale atoms to TMEM, then the block-scaled MMAs; one
+//               warp owns the TMEM allocation;
+//   epilogue    4 warps (tcgen05.ld); accumulators double-buffered in TMEM;
+//   scheduler   1 warp: claims work units and publishes them (with their row
+//               block) in a small shared-memory ring every other warp reads.
 // Orientation per work unit: a block of more than `swap_rows` rows puts its
 // tokens on the MMA's M side (M = 128, N = 128 weight rows); a smaller block
 // (decode) puts the weight rows on M and its tokens on N (16..128), so the
-// tensor core does not multiply padding rows.  Every wait is bounded; a wait
-// that gives up records an error word, and the CTA drains its own copies and
-// MMAs before freeing TMEM.
+// tensor core does not multiply padding rows.  With the tokens on N, the two
+// w4a16 terms sit side by side on N as well (term 2 from column kT2 on), so one
+// MMA per 32-element K block covers both: an M = 128 block-scaled MMA occupies
+// the tensor pipe about as long for N = 16 as for N = 128 (measured), so this
+// halves the pipe time of the weight-streaming shapes.  Every wait is bounded;
+// a wait that gives up records an error word, and the CTA drains its own copies
+// and MMAs before freeing TMEM.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -51,31 +62,53 @@ constexpr int kSmemLimit = 227 * 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCol = 256; // TMEM columns 256..267 hold the stage's scale factors
 constexpr unsigned long long kDrainTimeoutNs = 200000000ull;
+// Work units are handed out at run time (a global counter): SMs do not all stream at the same
+// rate (measured: up to 25 % apart on the same work), so a fixed round-robin share leaves the
+// kernel waiting on the slowest.  A scheduler warp takes the CTA's next units from the counter
+// and publishes them through a ring of kRing slots in shared memory; a slot is refilled once
+// every reading warp has taken it, which keeps the claims a few units ahead of the work.
+constexpr int kRing = 4;
 
 // Shared-memory plan for a kernel whose activation tiles hold at most kActRows
 // rows per term: as many pipeline stages as fit (more stages = more bytes in
 // flight per SM, which is what the weight-streaming decode shapes need).
-template <int kActRows> struct Plan {
-    // Small batches (activation tiles of at most 32 rows) split the per-stage issue work
-    // over two producer warps (alternate stages) and two MMA warps (one activation term
-    // each, into separate accumulators summed by the epilogue): each TMA / tcgen05
-    // instruction occupies its issuing warp for tens of cycles.
-    static constexpr int kProd = kActRows < 128 ? 2 : 1;
-    static constexpr int kMma = kActRows < 128 ? 2 : 1;
-    static constexpr int kThreads = 32 * (2 + 4 + (kProd - 1) + (kMma - 1));
+template <int kActRows, int kMmaW> struct Plan {
+    // first N row of the second activation term when both terms share one MMA (tokens on N)
+    static constexpr int kT2 = kActRows < 64 ? kActRows : 64;
     static constexpr int kTermBytes = kActRows * kTermRowBytes;
     static constexpr int kActBytes = 2 * kTermBytes;
     static constexpr int kStageBytes = kActBytes + kWBytes + kAsfBytes + kWsfBytes;
     static constexpr int kStages = (kSmemLimit - 1024 - kXBytes - 256) / kStageBytes;
+    // The per-stage copy issue is split over several producer warps (groups of two stages
+    // round robin): each TMA instruction and each warp-wide 4-byte scale copy occupies its
+    // issuing warp for about a hundred cycles (measured: the cost is per warp, not per SM).
+    // A producer's consecutive stages are kProd apart; its parity waits on a slot's "empty"
+    // barrier are only sound while it cannot get two rounds ahead of that slot, which holds
+    // when kProd <= kStages.
+    static constexpr int kProdWant = kActRows < 128 ? 4 : 2;
+    static constexpr int kProd = kProdWant <= kStages ? kProdWant : kStages;
+    static_assert(kProd >= 1 && kProd <= kStages, "producer warps vs pipeline stages");
+    // With at most 32 tokens per block (N <= 64) two MMA warps may take alternate stages,
+    // each into its own accumulator (the epilogue adds them): one thread issues a block-scaled
+    // MMA about every 64 cycles, and the second warp hides the per-stage wait and bookkeeping.
+    // (Measured: a gain for FC1's long units, a loss for FC2's short ones; the launch chooses.)
+    // (Each MMA warp waits on the stages of its own parity only, and kStages is even, so its
+    // parity waits on "full" barriers are never two phases ahead either.)
+    static constexpr int kMma = kMmaW;
+    static_assert(kMma == 1 || kStages % 2 == 0, "alternating MMA warps need an even stage count");
+    static_assert(kMma == 1 || kActRows <= 32, "two accumulators per buffer need N <= 64");
+    // warps: producer 0, MMA 0, 4 epilogue, producers 1.., MMA 1 (if any), the scheduler
+    static constexpr int kThreads = 32 * (2 + 4 + (kProd - 1) + (kMma - 1) + 1);
     static constexpr int kOffAct = 0;
     static constexpr int kOffW = kOffAct + kStages * kActBytes;
     static constexpr int kOffAsf = kOffW + kStages * kWBytes;
     static constexpr int kOffWsf = kOffAsf + kStages * kAsfBytes;
     static constexpr int kOffX = kOffWsf + kStages * kWsfBytes;
     static constexpr int kOffBar = kOffX + kXBytes;
-    static constexpr int kNumBars = 2 * kStages + 1 + 4;
+    static constexpr int kNumBars = 2 * kStages + 1 + 4 + 2 * kRing;
     static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
-    static constexpr int kSmemBytes = kOffTmemSlot + 16 + 1024; // + slack for 1024-byte alignment
+    static constexpr int kOffUnits = kOffTmemSlot + 16;                 // the work-unit ring
+    static constexpr int kSmemBytes = kOffUnits + 16 * kRing + 1024;   // + slack for 1024-byte alignment
     static_assert(kSmemBytes <= kSmemLimit, "shared memory plan too large");
     static_assert(kStages >= 3, "too few pipeline stages");
 };
@@ -89,6 +122,47 @@ template <int kStages> struct Bars {
     __device__ uint32_t mma_done() const { return base + 8 * (2 * kStages); }
     __device__ uint32_t acc_full(int b) const { return base + 8 * (2 * kStages + 1 + b); }
     __device__ uint32_t acc_empty(int b) const { return base + 8 * (2 * kStages + 3 + b); }
+    __device__ uint32_t ring_full(int i) const { return base + 8 * (2 * kStages + 5 + i); }
+    __device__ uint32_t ring_empty(int i) const { return base + 8 * (2 * kStages + 5 + kRing + i); }
+};
+
+// Readers of the work-unit ring: every producer and MMA warp and each of the 4 epilogue warps
+// reads every slot, then releases it.
+// A slot holds the unit's row block {expert, first grouped row, rows} and, in .w, the unit
+// index (-1: no more work), so that no reader has to fetch the row block from global memory.
+template <int kStages> struct UnitRing {
+    Bars<kStages> bars;
+    volatile int *slots; // kRing x 4 ints
+    // The CTA's i-th work unit (.w = -1: no more work, or a wait gave up).  Whole warp.
+    __device__ int4 take(uint32_t i, uint32_t *err, unsigned long long tmo, int lane) const
+    {
+        const int r = (int)(i % kRing);
+        int4 v = make_int4(0, 0, 0, -1);
+        if (__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.ring_full(r), (i / kRing) & 1, err, tmo)))
+            v = make_int4(slots[4 * r], slots[4 * r + 1], slots[4 * r + 2], slots[4 * r + 3]);
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(bars.ring_empty(r));
+        return v;
+    }
+    // Scheduler (one lane): publish the CTA's j-th unit; false once the work is exhausted.
+    __device__ bool fill(uint32_t j, const FcGemmArgs &a, int total_units, unsigned long long tmo) const
+    {
+        const int r = (int)(j % kRing);
+        const bool got = mbar_wait_bounded(bars.ring_empty(r), ((j / kRing) & 1) ^ 1, a.err, tmo);
+        int u = got ? atomicAdd(a.unit_counter, 1) : -1;
+        int4 blk = make_int4(0, 0, 0, 0);
+        if (u >= total_units)
+            u = -1;
+        if (u >= 0)
+            blk = a.rowblocks[u / a.n_tiles];
+        slots[4 * r] = blk.x;
+        slots[4 * r + 1] = blk.y;
+        slots[4 * r + 2] = blk.z;
+        slots[4 * r + 3] = u;
+        mbar_arrive(bars.ring_full(r)); // release: the slot writes are seen by every reader's acquire
+        return u >= 0;
+    }
 };
 
 // One lane of a converged warp is elected (tcgen05 and TMA instructions are
@@ -174,117 +248,172 @@ __device__ __forceinline__ float silu_mul(float g, float u)
 // Per-CTA state the warp roles share (all values are CTA-uniform).
 struct Ctx {
     uint32_t base;        // shared-memory base (1024-byte aligned, shared window)
+    volatile int *units;  // the work-unit ring (generic pointer to shared memory)
     uint32_t tmem_base;
-    int total_units, kst, terms, n_mma;
+    int total_units, kst, terms;
     unsigned long long tmo;
 };
 
-// Producer role, one of kProd warps (PI is a compile-time role index so that every
-// operand of the TMA issue stays warp-uniform).
-template <int kActRows, int PI>
+// Producer role, one of kProd warps taking stages g with g % kProd == PI (PI is a
+// compile-time role index so that every operand of the TMA issue stays warp-uniform).
+// Consecutive stages come from different warps at nearly the same time, so the two 64-byte
+// halves of a weight row's 128-byte line are requested close together.
+template <int kActRows, int kMmaW, int PI>
 __device__ __forceinline__ void producer_role(const FcGemmArgs &a, const Ctx &c, const CUtensorMap *act_map,
-                                              const CUtensorMap *act_map16, const CUtensorMap *w_map, int lane)
+                                              const CUtensorMap *act_map_sw, const CUtensorMap *act_map16,
+                                              const CUtensorMap *w_map, int lane)
 {
-    using P = Plan<kActRows>;
+    using P = Plan<kActRows, kMmaW>;
     constexpr int kStages = P::kStages, kProd = P::kProd;
     constexpr int kTermBytes = P::kTermBytes, kActBytes = P::kActBytes;
     constexpr int kOffAct = P::kOffAct, kOffW = P::kOffW, kOffAsf = P::kOffAsf, kOffWsf = P::kOffWsf;
     const Bars<kStages> bars{c.base + P::kOffBar};
     const uint32_t base = c.base;
-    const int total_units = c.total_units, kst = c.kst, terms = c.terms;
+    const int kst = c.kst, terms = c.terms;
     const unsigned long long tmo = c.tmo;
     uint32_t g = 0;
     bool ok = true;
     const int scl_ld = a.K / 32;
-    for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
-        const int4 blk = a.rowblocks[u / a.n_tiles];
-        const int nt = u % a.n_tiles;
+    const UnitRing<kStages> ring{bars, c.units};
+    for (uint32_t i = 0; ok; ++i) {
+        const int4 blk = ring.take(i, a.err, tmo, lane);
+        if (blk.w < 0)
+            break;
+        const int nt = blk.w % a.n_tiles;
         const bool swap = kActRows < 128 || blk.z <= a.swap_rows;
         const int npad = (blk.z + 15) & ~15;
+        const bool comb = swap && terms > 1 && npad <= P::kT2; // both terms on N of one MMA
         // weight rows of this tile, as two 64-row halves: FC1 tile nt = gate rows [64nt, 64nt+64)
         // then the matching up rows; FC2 tile nt = rows [128nt, 128nt+128)
         const int wrow_a = blk.x * a.R + (a.fc1 ? nt * 64 : nt * 128);
         const int wrow_b = a.fc1 ? wrow_a + a.R / 2 : wrow_a + 64;
-        const int rb = blk.y / 128;
-        const uint32_t act_bytes = (uint32_t)terms * (swap ? (uint32_t)npad * 128u : (uint32_t)kTermBytes);
+        const int rb = blk.y / 128, o = blk.y & 127;
+        // tokens on N: one box of kT2 rows per term plane covers the block (both terms, one copy),
+        // else (blocks beyond kT2 rows) 16-row boxes per term, term 2 kTermBytes further on
+        const bool sw3 = swap && npad <= P::kT2;
+        const uint32_t act_bytes =
+            (uint32_t)terms * (!swap ? (uint32_t)kTermBytes : sw3 ? (uint32_t)P::kT2 * 128u : (uint32_t)npad * 128u);
+        // activation scales: one bulk copy of the two 128-row atoms (tokens on M), or 4-byte copies
+        // of this block's rows into a stage atom laid out for N (tokens on N); weight scales: one
+        // bulk copy (tiled layout) or 4-byte copies (row-major)
+        const uint32_t tx = act_bytes + kWTxBytes + (swap ? 0u : (uint32_t)terms * 512u) + (a.wsf_tiled ? 512u : 0u);
+        const uint8_t *wsf_tile = a.wscale + ((size_t)blk.x * a.n_tiles + nt) * (size_t)kst * 512;
         for (int kk = 0; kk < kst; ++kk, ++g) {
             if ((int)(g % kProd) != PI)
-                continue; // the other producer warp fills this stage
+                continue; // another producer warp fills this stage
             const int s = g % kStages;
-            const uint32_t ph = (g / kStages) & 1;
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.empty(s), ph ^ 1, a.err, tmo))) {
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.empty(s), ((g / kStages) & 1) ^ 1, a.err, tmo))) {
                 ok = false;
                 break;
             }
-            // weight scale bytes: 4 per row (the 4 blocks of this K stage) into the atom layout
-            const uint32_t wsf = base + kOffWsf + s * kWsfBytes;
-            for (int r = lane; r < 128; r += 32) {
-                const int wr = r < 64 ? wrow_a + r : wrow_b + (r - 64);
-                cp_async_4(wsf + sf_atom_offset(r, 0), a.wscale + (size_t)wr * scl_ld + kk * 4);
-            }
-            cp_async_mbar_arrive_noinc(bars.full(s));
-            __syncwarp();
-            // every operand below is computed by the whole (converged) warp; then one elected lane
-            // issues the stage's copies back to back
+            // Every operand is computed by the whole (converged) warp; one elected lane issues the
+            // stage's bulk copies (the weight tile first: it is the long pole, from DRAM), then the
+            // whole warp issues the 4-byte scale copies, if any.
             const uint32_t full_s = bars.full(s);
             const uint32_t act = base + kOffAct + s * kActBytes;
             const uint32_t wdst = base + kOffW + s * kWBytes;
-            const int kx = kk * 128;
-            const uint8_t *asf_src = a.act_sf + ((size_t)rb * kst + kk) * 1024;
+            const uint32_t wsf = base + kOffWsf + s * kWsfBytes;
             const uint32_t asf_dst = base + kOffAsf + s * kAsfBytes;
-            const uint32_t tx = act_bytes + kWTxBytes + (uint32_t)terms * 512u;
-            const int row0 = blk.y, row1 = a.act_rows + blk.y;
+            const uint8_t *asf_src = a.act_sf + ((size_t)rb * kst + kk) * 1024;
+            const int kx = kk * 128;
             if (elect_one()) {
                 mbar_arrive_expect_tx(full_s, tx);
+                // FC1: gate and up halves of the 64-row slice in one box; FC2: one 128-row box
+                if (a.fc1)
+                    tma_load_3d(wdst, w_map, kx, nt * 64, 2 * blk.x, full_s);
+                else
+                    tma_load_2d(wdst, w_map, kx, wrow_a, full_s);
+                if (a.wsf_tiled)
+                    bulk_copy_g2s(wsf, wsf_tile + (size_t)kk * 512, 512u, full_s);
                 if (!swap) {
-                    tma_load_2d(act, act_map, kx, row0, full_s);
-                    if (terms > 1)
-                        tma_load_2d(act + kTermBytes, act_map, kx, row1, full_s);
+                    tma_load_3d(act, act_map, kx, blk.y, 0, full_s); // [terms][128 rows][128]
+                    bulk_copy_g2s(asf_dst, asf_src, (uint32_t)terms * 512u, full_s);
+                } else if (sw3) {
+                    tma_load_3d(act, act_map_sw, kx, blk.y, 0, full_s); // [terms][kT2 rows][128]
                 } else {
                     for (int r16 = 0; r16 < npad; r16 += 16) {
-                        tma_load_2d(act + r16 * 128, act_map16, kx, row0 + r16, full_s);
+                        tma_load_2d(act + r16 * 128, act_map16, kx, blk.y + r16, full_s);
                         if (terms > 1)
-                            tma_load_2d(act + kTermBytes + r16 * 128, act_map16, kx, row1 + r16, full_s);
+                            tma_load_2d(act + kTermBytes + r16 * 128, act_map16, kx, a.act_rows + blk.y + r16, full_s);
                     }
                 }
-                tma_load_2d(wdst, w_map, kx, wrow_a, full_s);
-                tma_load_2d(wdst + kWBytes / 2, w_map, kx, wrow_b, full_s);
-                bulk_copy_g2s(asf_dst, asf_src, (uint32_t)terms * 512u, full_s);
             }
+            __syncwarp();
+            if (!a.wsf_tiled) // weight scale bytes: 4 per row (the stage's 4 blocks) into the atom layout
+                for (int r = lane; r < 128; r += 32) {
+                    const int wr = r < 64 ? wrow_a + r : wrow_b + (r - 64);
+                    cp_async_4(wsf + sf_atom_offset(r, 0), a.wscale + (size_t)wr * scl_ld + kk * 4);
+                }
+            if (swap) {
+                // row j of term t: from row o + j of the term's 128-row atom to N row t * kT2 + j of
+                // one atom (both terms on N) or to row j of the term's own atom
+                for (int j = lane; j < npad; j += 32)
+                    for (int t = 0; t < terms; ++t)
+                        cp_async_4(comb ? asf_dst + sf_atom_offset(t * P::kT2 + j, 0)
+                                        : asf_dst + 512u * t + sf_atom_offset(j, 0),
+                                   asf_src + 512 * t + sf_atom_offset(o + j, 0));
+            }
+            cp_async_mbar_arrive_noinc(full_s);
             __syncwarp();
         }
     }
-    // drain: every stage issued must have landed before the CTA may exit
+    // drain: every stage this warp issued must have landed before the CTA may exit
     const uint32_t first = g > (uint32_t)kStages ? g - kStages : 0u;
     for (uint32_t q = first; q < g; ++q)
         if ((int)(q % kProd) == PI)
             mbar_wait_bounded(bars.full(q % kStages), (q / kStages) & 1, nullptr, kDrainTimeoutNs);
 }
 
-// MMA role, one of kMma warps; MI (compile-time) selects the activation terms
-// (t % kMma == MI), the accumulator and the scale-factor columns of this warp.
-template <int kActRows, int MI>
+// Scheduler role (one warp, one lane works): takes the CTA's work units from the launch's
+// counter and publishes them kLook units ahead of the first reader, off the producers' path
+// (the counter is a global atomic: a round trip of about a microsecond per unit).
+template <int kActRows, int kMmaW>
+__device__ __forceinline__ void scheduler_role(const FcGemmArgs &a, const Ctx &c, int lane)
+{
+    using P = Plan<kActRows, kMmaW>;
+    const UnitRing<P::kStages> ring{Bars<P::kStages>{c.base + P::kOffBar}, c.units};
+    if (lane == 0)
+        for (uint32_t j = 0; ring.fill(j, a, c.total_units, c.tmo); ++j) {
+        }
+    __syncwarp();
+}
+
+// MMA role: warp 1 (MI = 0) and, with kMma = 2, warp 7 (MI = 1), taking stages g with
+// g % kMma == MI.  The whole warp runs the loop, one elected lane issues.
+template <int kActRows, int kMmaW, int MI>
 __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
 {
-    using P = Plan<kActRows>;
+    using P = Plan<kActRows, kMmaW>;
     constexpr int kStages = P::kStages, kMma = P::kMma;
     constexpr int kTermBytes = P::kTermBytes, kActBytes = P::kActBytes;
     constexpr int kOffAct = P::kOffAct, kOffW = P::kOffW, kOffAsf = P::kOffAsf, kOffWsf = P::kOffWsf;
     const Bars<kStages> bars{c.base + P::kOffBar};
     const uint32_t base = c.base, tmem_base = c.tmem_base;
-    const int total_units = c.total_units, kst = c.kst, terms = c.terms;
+    const int kst = c.kst, terms = c.terms;
     const unsigned long long tmo = c.tmo;
-    // ------------------------------------------------------------ MMA issuer (whole warp, one lane issues)
     uint32_t g = 0, cnt = 0;
     bool ok = true;
-    // this warp's scale-factor columns: weights at +0, its activation terms at +4, +8
+    // this warp's scale-factor columns: the weight atom at +0, the activation atoms at +4 and +8
     const uint32_t sf_w = tmem_base + kSfCol + 16u * (uint32_t)MI;
-    for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x, ++cnt) {
-        const int4 blk = a.rowblocks[u / a.n_tiles];
+    const UnitRing<kStages> ring{bars, c.units};
+    const int lane = threadIdx.x & 31;
+    for (; ok; ++cnt) {
+        const int4 blk = ring.take(cnt, a.err, tmo, lane);
+        if (blk.w < 0)
+            break;
         const bool swap = kActRows < 128 || blk.z <= a.swap_rows;
         const uint32_t npad = (uint32_t)((blk.z + 15) & ~15);
-        const uint32_t idesc0 = swap ? idesc_mx(kFmtE2M1, kFmtE4M3, 128, npad, 0)
+        const bool comb = swap && terms > 1 && npad <= (uint32_t)P::kT2;
+        // MMAs per 32-element K block: one (both terms on N, or a single term) or one per term
+        const bool t1 = !comb && terms > 1;
+        const uint32_t idesc0 = swap ? idesc_mx(kFmtE2M1, kFmtE4M3, 128, comb ? P::kT2 + npad : npad, 0)
                                      : idesc_mx(kFmtE4M3, kFmtE2M1, 128, 128, 0);
+        uint32_t sfa[2], sfb[2];
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            sfa[t] = swap ? sf_w : sf_w + 4 + 4 * t;
+            sfb[t] = swap ? sf_w + 4 + 4 * t : sf_w;
+        }
         const int buf = cnt & 1;
         if (!__all_sync(0xFFFFFFFFu,
                         mbar_wait_bounded(bars.acc_empty(buf), ((cnt >> 1) & 1) ^ 1, a.err, tmo))) {
@@ -292,29 +421,28 @@ __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
             break;
         }
         tc_fence_after();
-        // accumulator: one per buffer, or (split) one per buffer and MMA warp, 64 columns apart
+        // accumulator: one per buffer, or one per buffer and MMA warp (64 columns apart)
         const uint32_t d = tmem_base + buf * 128 + (kMma > 1 ? 64u * (uint32_t)MI : 0u);
+        bool first = true; // this warp's first stage of the unit initialises its accumulator
         for (int kk = 0; kk < kst; ++kk, ++g) {
+            if (kMma > 1 && (int)(g % kMma) != MI)
+                continue; // the other MMA warp takes this stage
             const int s = g % kStages;
             const uint32_t ph = (g / kStages) & 1;
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.full(s), ph, a.err, tmo))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            // Every operand is computed by the whole (converged) warp first; then one elected lane
-            // issues the stage's scale copies, MMAs and commit back to back (measured: an elect /
+            // The stage's operands are computed by the whole warp before the wait; then one elected
+            // lane issues the scale copies, MMAs and commit back to back (measured: an elect /
             // reconverge around each instruction costs more than the instruction itself).
             const uint32_t act = base + kOffAct + s * kActBytes;
             const uint32_t wt = base + kOffW + s * kWBytes;
             const uint32_t wsf_s = base + kOffWsf + s * kWsfBytes;
             const uint32_t asf_s = base + kOffAsf + s * kAsfBytes;
             uint64_t opa[4][2], opb[4][2];
-            uint32_t idesc[4];
+            uint32_t idesc[4], accf[4];
 #pragma unroll
             for (int k32 = 0; k32 < 4; ++k32) {
                 // the scale-factor byte of this 32-element block sits in both sf-id fields
                 idesc[k32] = idesc0 | ((uint32_t)k32 << 4) | ((uint32_t)k32 << 29);
+                accf[k32] = (first && k32 == 0) ? 0u : 1u;
                 const uint64_t dw = smem_desc_sw128(wt + 32 * k32);
 #pragma unroll
                 for (int t = 0; t < 2; ++t) {
@@ -323,32 +451,28 @@ __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
                     opb[k32][t] = swap ? da : dw;
                 }
             }
-            uint32_t sfa[2], sfb[2];
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                sfa[t] = swap ? sf_w : sf_w + 4 + 4 * t;
-                sfb[t] = swap ? sf_w + 4 + 4 * t : sf_w;
-            }
-            const bool t0 = (0 % kMma) == MI, t1 = terms > 1 && (1 % kMma) == MI;
             const uint32_t empty_s = bars.empty(s);
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.full(s), ph, a.err, tmo))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
             if (elect_one()) {
                 // scale atoms -> TMEM (in order with the MMAs below and with the previous stage's MMAs)
                 tmem_cp_sf_atom(sf_w, wsf_s);
-                if (t0)
-                    tmem_cp_sf_atom(sf_w + 4, asf_s);
+                tmem_cp_sf_atom(sf_w + 4, asf_s);
                 if (t1)
                     tmem_cp_sf_atom(sf_w + 8, asf_s + 512);
 #pragma unroll
                 for (int k32 = 0; k32 < 4; ++k32) {
-                    if (t0)
-                        umma_mx(d, opa[k32][0], opb[k32][0], idesc[k32], sfa[0], sfb[0], (kk | k32) != 0);
+                    umma_mx(d, opa[k32][0], opb[k32][0], idesc[k32], sfa[0], sfb[0], accf[k32]);
                     if (t1)
-                        umma_mx(d, opa[k32][1], opb[k32][1], idesc[k32], sfa[1], sfb[1],
-                                (kMma > 1) ? (kk | k32) != 0 : 1u);
+                        umma_mx(d, opa[k32][1], opb[k32][1], idesc[k32], sfa[1], sfb[1], 1u);
                 }
                 umma_commit(empty_s);
             }
             __syncwarp();
+            first = false;
         }
         if (ok && elect_one())
             umma_commit(bars.acc_full(buf));
@@ -361,15 +485,14 @@ __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
     mbar_wait_bounded(bars.mma_done(), 0, nullptr, kDrainTimeoutNs);
 }
 
-template <int kActRows>
-__global__ void __launch_bounds__(Plan<kActRows>::kThreads, 1)
+template <int kActRows, int kMmaW>
+__global__ void __launch_bounds__(Plan<kActRows, kMmaW>::kThreads, 1)
     fc_gemm_kernel(const FcGemmArgs a, const __grid_constant__ CUtensorMap act_map,
-                   const __grid_constant__ CUtensorMap act_map16, const __grid_constant__ CUtensorMap w_map)
+                   const __grid_constant__ CUtensorMap act_map_sw, const __grid_constant__ CUtensorMap act_map16,
+                   const __grid_constant__ CUtensorMap w_map)
 {
-    using P = Plan<kActRows>;
+    using P = Plan<kActRows, kMmaW>;
     constexpr int kStages = P::kStages;
-    constexpr int kTermBytes = P::kTermBytes, kActBytes = P::kActBytes;
-    constexpr int kOffAct = P::kOffAct, kOffW = P::kOffW, kOffAsf = P::kOffAsf, kOffWsf = P::kOffWsf;
     constexpr int kOffX = P::kOffX, kOffBar = P::kOffBar, kOffTmemSlot = P::kOffTmemSlot;
     constexpr int kProd = P::kProd, kMma = P::kMma;
     extern __shared__ uint8_t smem_raw[];
@@ -379,21 +502,25 @@ __global__ void __launch_bounds__(Plan<kActRows>::kThreads, 1)
     const Bars<kStages> bars{base + kOffBar};
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // warp roles: 0 producer 0, 1 MMA 0 (+ TMEM owner), 2..5 epilogue, 6 producer 1, 7 MMA 1
-    const int n_mma = kMma < a.terms ? kMma : a.terms; // MMA warps with work (one term each when split)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bars.full(s), 1 + 32);  // producer's expect_tx + 32 cp.async arrivals
-            mbar_init(bars.empty(s), n_mma);  // one commit per MMA warp
+            mbar_init(bars.empty(s), 1);      // the commit of the MMA warp that took the stage
         }
-        mbar_init(bars.mma_done(), n_mma);
+        mbar_init(bars.mma_done(), kMma);
         for (int b = 0; b < 2; ++b) {
-            mbar_init(bars.acc_full(b), n_mma);
+            mbar_init(bars.acc_full(b), kMma); // every MMA warp commits every unit
             mbar_init(bars.acc_empty(b), 128);
+        }
+        for (int r = 0; r < kRing; ++r) {
+            mbar_init(bars.ring_full(r), 1);                  // the scheduler's publish
+            mbar_init(bars.ring_empty(r), kProd + kMma + 4);  // one release per reading warp
         }
         fence_mbar_init();
         fence_proxy_async_smem();
         prefetch_tensormap(&act_map);
+        prefetch_tensormap(&act_map_sw);
         prefetch_tensormap(&act_map16);
         prefetch_tensormap(&w_map);
     }
@@ -412,24 +539,34 @@ __global__ void __launch_bounds__(Plan<kActRows>::kThreads, 1)
     const int terms = a.terms; // activation terms per row: 1 (w4a8) or 2 (w4a16)
     const unsigned long long tmo = a.timeout_ns;
 
-    const Ctx ctx{base, tmem_base, total_units, kst, terms, n_mma, tmo};
+    const Ctx ctx{base, reinterpret_cast<volatile int *>(gsm + P::kOffUnits), tmem_base, total_units, kst, terms, tmo};
     if (warp == 0) {
-        producer_role<kActRows, 0>(a, ctx, &act_map, &act_map16, &w_map, lane);
-    } else if (kProd > 1 && warp == 6) {
-        producer_role<kActRows, (kProd > 1 ? 1 : 0)>(a, ctx, &act_map, &act_map16, &w_map, lane);
+        producer_role<kActRows, kMmaW, 0>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
+    } else if (warp >= 6 && warp < 5 + kProd) {
+        // further producer warps (compile-time role index: every TMA operand stays warp-uniform)
+        if (warp == 6)
+            producer_role<kActRows, kMmaW, 1 % kProd>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
+        else if (warp == 7)
+            producer_role<kActRows, kMmaW, 2 % kProd>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
+        else if (warp == 8)
+            producer_role<kActRows, kMmaW, 3 % kProd>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
     } else if (warp == 1) {
-        mma_role<kActRows, 0>(a, ctx);
+        mma_role<kActRows, kMmaW, 0>(a, ctx);
     } else if (kMma > 1 && warp == 5 + kProd) {
-        if (n_mma > 1)
-            mma_role<kActRows, (kMma > 1 ? 1 : 0)>(a, ctx);
+        mma_role<kActRows, kMmaW, (kMma > 1 ? 1 : 0)>(a, ctx);
+    } else if (warp == P::kThreads / 32 - 1) {
+        scheduler_role<kActRows, kMmaW>(a, ctx, lane);
     } else if (warp >= 2 && warp < 6) {
         // ------------------------------------------------------------ epilogue (warps 2..5)
         const int q = warp & 3; // TMEM lane quarter this warp may access
         float *xch = reinterpret_cast<float *>(gsm + kOffX);
-        uint32_t cnt = 0;
-        for (int u = blockIdx.x; u < total_units; u += gridDim.x, ++cnt) {
-            const int4 blk = a.rowblocks[u / a.n_tiles];
-            const int nt = u % a.n_tiles;
+        const UnitRing<kStages> ring{bars, reinterpret_cast<volatile int *>(gsm + P::kOffUnits)};
+        for (uint32_t cnt = 0;; ++cnt) {
+            const int4 blk = ring.take(cnt, a.err, tmo, lane);
+            // the four epilogue warps leave together (they share named barriers below)
+            if (!named_bar_all(2, 128, blk.w >= 0))
+                break;
+            const int nt = blk.w % a.n_tiles;
             const int rows = blk.z;
             const bool swap = kActRows < 128 || rows <= a.swap_rows;
             const int buf = cnt & 1;
@@ -481,25 +618,35 @@ __global__ void __launch_bounds__(Plan<kActRows>::kThreads, 1)
                 // lane L of the tile = weight row; TMEM columns = tokens
                 const int L = 32 * q + lane;
                 const int npad = (rows + 15) & ~15;
+                const bool comb = terms > 1 && npad <= P::kT2;
+                // partial sums: per MMA warp with stages in this unit (with one K stage only the
+                // warp that took it), and per term when both terms sit side by side on N
+                const uint32_t g0 = cnt * (uint32_t)kst;
+                const bool acc0 = kMma == 1 || kst > 1 || (g0 & 1) == 0;
+                const bool acc1 = kMma > 1 && (kst > 1 || (g0 & 1) == 1);
                 for (int n0 = 0; n0 < npad; n0 += 16) {
-                    uint32_t v[16];
-                    tmem_ld16(tb + n0, v);
-                    if (kMma > 1 && terms > 1) {
-                        // split accumulation: add the second MMA warp's partial sums
-                        uint32_t v1[16];
-                        tmem_ld16(tb + 64 + n0, v1);
-                        tmem_wait_ld();
+                    float v[16];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(v1[j]));
+                    for (int j = 0; j < 16; ++j)
+                        v[j] = 0.f;
+                    for (int w = 0; w < kMma; ++w) {
+                        if (!(w == 0 ? acc0 : acc1))
+                            continue;
+                        for (int t = 0; t < (comb ? 2 : 1); ++t) {
+                            uint32_t r[16];
+                            tmem_ld16(tb + 64 * w + (t ? P::kT2 : 0) + n0, r);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                v[j] += __uint_as_float(r[j]);
+                        }
                     }
-                    tmem_wait_ld();
                     if (a.fc1) {
                         // the up rows live in lanes 64..127: hand them to the gate lanes through smem
                         if (q >= 2) {
 #pragma unroll
                             for (int j = 0; j < 16; ++j)
-                                xch[(L - 64) * 16 + j] = __uint_as_float(v[j]);
+                                xch[(L - 64) * 16 + j] = v[j];
                         }
                         named_bar_sync(1, 128);
                         if (q < 2) {
@@ -508,7 +655,7 @@ __global__ void __launch_bounds__(Plan<kActRows>::kThreads, 1)
                                 const int n = n0 + j;
                                 if (n >= rows)
                                     break;
-                                const float hv = silu_mul(__uint_as_float(v[j]), xch[L * 16 + j]);
+                                const float hv = silu_mul(v[j], xch[L * 16 + j]);
                                 store_act_warp32(a.hq, a.hsf, a.hq_rows, a.out_ld, blk.y + n, i, hv, a.act_mxfp8,
                                                  lane);
                             }
@@ -519,7 +666,7 @@ __global__ void __launch_bounds__(Plan<kActRows>::kThreads, 1)
                         for (int j = 0; j < 16; ++j) {
                             const int n = n0 + j;
                             if (n < rows)
-                                a.y[(size_t)(blk.y + n) * a.out_ld + nt * 128 + L] = __uint_as_float(v[j]);
+                                a.y[(size_t)(blk.y + n) * a.out_ld + nt * 128 + L] = v[j];
                         }
                     }
                 }
@@ -537,29 +684,51 @@ __global__ void __launch_bounds__(Plan<kActRows>::kThreads, 1)
     }
 }
 
-size_t fc_gemm_smem_bytes(int act_rows) { return act_rows <= 32 ? Plan<32>::kSmemBytes : Plan<128>::kSmemBytes; }
-
-int fc_gemm_stages(int act_rows) { return act_rows <= 32 ? Plan<32>::kStages : Plan<128>::kStages; }
+template <int kActRows, int kMmaW> static cudaError_t prepare_one()
+{
+    return cudaFuncSetAttribute(fc_gemm_kernel<kActRows, kMmaW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Plan<kActRows, kMmaW>::kSmemBytes);
+}
 
 cudaError_t fc_gemm_prepare()
 {
-    cudaError_t e = cudaFuncSetAttribute(fc_gemm_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Plan<32>::kSmemBytes);
-    if (e != cudaSuccess)
+    cudaError_t e;
+    if ((e = prepare_one<16, 1>()) != cudaSuccess || (e = prepare_one<16, 2>()) != cudaSuccess ||
+        (e = prepare_one<32, 1>()) != cudaSuccess || (e = prepare_one<32, 2>()) != cudaSuccess ||
+        (e = prepare_one<64, 1>()) != cudaSuccess)
         return e;
-    return cudaFuncSetAttribute(fc_gemm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                Plan<128>::kSmemBytes);
+    return prepare_one<128, 1>();
 }
 
-void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUtensorMap &act_map16,
-                    const CUtensorMap &w_map, int grid, cudaStream_t s)
+template <int kActRows, int kMmaW>
+static void launch_one(const FcGemmArgs &a, const CUtensorMap &act_map, const CUtensorMap &act_map_sw,
+                       const CUtensorMap &act_map16, const CUtensorMap &w_map, int grid, cudaStream_t s)
 {
-    // At most 32 tokens: every row block has at most 32 rows and runs with its tokens on N,
-    // so the activation tiles shrink and the pipeline gets more stages.
-    if (a.max_block_rows <= 32)
-        fc_gemm_kernel<32><<<grid, Plan<32>::kThreads, Plan<32>::kSmemBytes, s>>>(a, act_map, act_map16, w_map);
-    else
-        fc_gemm_kernel<128><<<grid, Plan<128>::kThreads, Plan<128>::kSmemBytes, s>>>(a, act_map, act_map16, w_map);
+    fc_gemm_kernel<kActRows, kMmaW><<<grid, Plan<kActRows, kMmaW>::kThreads, Plan<kActRows, kMmaW>::kSmemBytes, s>>>(
+        a, act_map, act_map_sw, act_map16, w_map);
+}
+
+void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUtensorMap &act_map_sw,
+                    const CUtensorMap &act_map16, const CUtensorMap &w_map, int grid, cudaStream_t s)
+{
+    // Row blocks of at most 16 / 32 / 64 rows run with their tokens on N; smaller activation
+    // tiles leave room for more pipeline stages (bytes in flight) in the weight-streaming shapes.
+    // Two MMA warps for FC1's small-batch variants (long units), one for FC2 (measured).
+    if (a.max_block_rows <= 16) {
+        if (a.fc1)
+            launch_one<16, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+        else
+            launch_one<16, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+    } else if (a.max_block_rows <= 32) {
+        if (a.fc1)
+            launch_one<32, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+        else
+            launch_one<32, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+    } else if (a.max_block_rows <= 64) {
+        launch_one<64, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+    } else {
+        launch_one<128, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+    }
 }
 
 // ---------------------------------------------------------------- watchdog self-test

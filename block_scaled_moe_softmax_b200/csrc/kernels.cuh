@@ -29,6 +29,7 @@ struct RouteGroupArgs {
     int32_t *num_rowblocks;
     int32_t *sorted_pair;
     int32_t *pos_of_pair;
+    int split_rows; // rows per work block of the row-block list: 16, 32, 64 or kBlockRows
 };
 
 void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s);
@@ -44,12 +45,14 @@ void launch_mx_quantize(const float *src, int64_t rows, int64_t K, int fmt, uint
 struct FcGemmArgs {
     const int4 *rowblocks;       // {expert, first grouped row, rows, 0}
     const int32_t *num_rowblocks;
-    const uint8_t *wscale;       // caller's E8M0 weight scales, [E*R, K/32] row-major
+    const uint8_t *wscale;       // caller's E8M0 weight scales: [E*R, K/32] row-major, or (wsf_tiled)
+                                 // [E][n_tiles][K/128][512] scale atoms (moe_mx_prepare_scales)
     const uint8_t *act_sf;       // activation scale atoms, [rows/128][K/128][2 terms][512]
     uint8_t *hq;                 // FC1 output codes, [2 terms][hq_rows][I] (E4M3)
     uint8_t *hsf;                // FC1 output scale atoms, [hq_rows/128][I/128][2][512]
     float *y;                    // FC2 output, f32 [rows, H]
     uint32_t *err;
+    int *unit_counter;           // work-unit counter of this launch, zero before it starts
     unsigned long long timeout_ns;
     int K;                       // reduction length (FC1: H, FC2: I)
     int R;                       // weight rows per expert (FC1: 2I, FC2: H)
@@ -62,14 +65,25 @@ struct FcGemmArgs {
     int act_mxfp8;               // FC1 only: h in OCP MXFP8 (w4a8) instead of the two-term split
     int swap_rows;               // row blocks of at most this many rows (<= 128) put the
                                  // weight rows on the MMA M side and the tokens on N
-    int max_block_rows;          // upper bound on any row block's rows (min(tokens, 128))
+    int wsf_tiled;               // 1: wscale is in the tiled atom layout (one bulk copy per stage)
+    int max_block_rows;          // upper bound on any row block's rows: 16, 32, 64 or 128; selects
+                                 // the kernel variant (activation tile rows per term)
 };
 
-void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUtensorMap &act_map16,
-                    const CUtensorMap &w_map, int grid, cudaStream_t s);
-size_t fc_gemm_smem_bytes(int act_rows);
-int fc_gemm_stages(int act_rows);
+// Tensor maps: act_map = both term planes, 128-row boxes ([terms][128][128] codes, tokens
+// on M); act_map_sw = both term planes, boxes of min(max_block_rows, 64) rows (tokens on N);
+// act_map16 = 16-row boxes of one plane (tokens on N, blocks beyond that); w_map = FC1: the
+// gate and up halves of a 64-row weight slice in one box, FC2: 128-row boxes.
+void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUtensorMap &act_map_sw,
+                    const CUtensorMap &act_map16, const CUtensorMap &w_map, int grid, cudaStream_t s);
 cudaError_t fc_gemm_prepare();
+
+// Rearrange row-major E8M0 weight scales [E][R][K/32] into the tiled atom layout the GEMM reads:
+// for expert e, 128-row weight tile nt and K stage kk (128 elements), one 512-byte atom at
+// ((e * n_tiles + nt) * (K/128) + kk) * 512 whose byte sf_atom_offset(m, kb) is the scale of tile
+// row m and 32-element block kb.  Tile rows: FC1 (fc1 = 1) gate rows [64 nt, 64 nt + 64) then
+// the matching up rows I + [64 nt, 64 nt + 64) (R = 2I); FC2 rows [128 nt, 128 nt + 128).
+void launch_tile_scales(const uint8_t *src, uint8_t *dst, int E, int R, int K, int fc1, int num_sms, cudaStream_t s);
 
 void launch_watchdog(uint32_t *err, unsigned long long timeout_ns, cudaStream_t s);
 

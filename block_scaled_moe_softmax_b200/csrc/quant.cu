@@ -89,4 +89,33 @@ void launch_mx_quantize(const float *src, int64_t rows, int64_t K, int fmt, uint
     mx_quantize_kernel<<<grid > 0 ? grid : 1, 256, 0, s>>>(src, nblocks, fmt, codes, scales);
 }
 
+// ---------------------------------------------------------------- scale tiling
+// One thread per (atom, tile row): 4 scale bytes (the 4 blocks of one K stage) in, 4 out.
+__global__ void __launch_bounds__(256) tile_scales_kernel(const uint8_t *__restrict__ src, uint8_t *__restrict__ dst,
+                                                          long long n_items, int R, int K, int fc1)
+{
+    const int kst = K / 128, ld = K / 32;
+    const int n_tiles = R / 128; // FC1: I/64 tiles of 64 gate + 64 up rows (R = 2I); FC2: H/128
+    for (long long it = blockIdx.x * (long long)blockDim.x + threadIdx.x; it < n_items;
+         it += (long long)gridDim.x * blockDim.x) {
+        const int m = (int)(it & 127);
+        const long long atom = it >> 7; // ((e * n_tiles + nt) * kst + kk)
+        const int kk = (int)(atom % kst);
+        const long long et = atom / kst;
+        const int nt = (int)(et % n_tiles);
+        const long long e = et / n_tiles;
+        const int row = fc1 ? (m < 64 ? nt * 64 + m : R / 2 + nt * 64 + (m - 64)) : nt * 128 + m;
+        const uint32_t v = *reinterpret_cast<const uint32_t *>(src + (e * R + row) * (long long)ld + kk * 4);
+        *reinterpret_cast<uint32_t *>(dst + atom * 512 + sf_atom_offset(m, 0)) = v;
+    }
+}
+
+void launch_tile_scales(const uint8_t *src, uint8_t *dst, int E, int R, int K, int fc1, int num_sms, cudaStream_t s)
+{
+    const long long n_items = (long long)E * (R / 128) * (K / 128) * 128;
+    const long long want = (n_items + 255) / 256;
+    const int grid = (int)(want < (long long)num_sms * 16 ? want : (long long)num_sms * 16);
+    tile_scales_kernel<<<grid > 0 ? grid : 1, 256, 0, s>>>(src, dst, n_items, R, K, fc1);
+}
+
 } // namespace moe_mx

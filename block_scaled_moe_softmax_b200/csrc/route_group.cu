@@ -105,14 +105,17 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float *__res
 
 // ---------------------------------------------------------------- scan
 // One CTA: per-expert totals over chunks, padded exclusive scan over experts,
-// per-chunk base rows, the row-block list and the padding markers.
-__global__ void __launch_bounds__(1024) scan_kernel(int E, int nchunks, int32_t *__restrict__ chunk_hist,
+// per-chunk base rows, the row-block list and the padding markers.  Segments
+// are padded to kBlockRows rows; the row-block list (the GEMMs' work list)
+// splits each segment into blocks of at most `split` rows (16, 32, 64 or
+// kBlockRows).
+__global__ void __launch_bounds__(1024) scan_kernel(int E, int nchunks, int split, int32_t *__restrict__ chunk_hist,
                                                     int32_t *__restrict__ counts, int32_t *__restrict__ pad_offsets,
                                                     int4 *__restrict__ rowblocks, int32_t *__restrict__ num_rowblocks,
                                                     int32_t *__restrict__ sorted_pair)
 {
     __shared__ int32_t s_pad[kMaxExperts];
-    __shared__ int32_t s_warp[32];
+    __shared__ unsigned long long s_warp[32];
     const int e = threadIdx.x;
     int total = 0;
     if (e < E) {
@@ -123,13 +126,15 @@ __global__ void __launch_bounds__(1024) scan_kernel(int E, int nchunks, int32_t 
         }
         counts[e] = total;
     }
-    const int nb = (total + kBlockRows - 1) / kBlockRows;
-    // block-wide exclusive scan of nb (padded rows = nb * kBlockRows)
-    int incl = nb;
+    const int nb = (total + kBlockRows - 1) / kBlockRows; // padded segment: nb * kBlockRows rows
+    const int nw = (total + split - 1) / split;            // work blocks of the segment
+    // one block-wide exclusive scan of both counts, packed in 32-bit halves
+    const unsigned long long mine = ((unsigned long long)nb << 32) | (unsigned)nw;
+    unsigned long long incl = mine;
     const int lane = e & 31, warp = e >> 5;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        const unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
         if (lane >= off)
             incl += y;
     }
@@ -137,27 +142,27 @@ __global__ void __launch_bounds__(1024) scan_kernel(int E, int nchunks, int32_t 
         s_warp[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        int w = s_warp[lane];
+        unsigned long long w = s_warp[lane];
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
-            const int y = __shfl_up_sync(0xFFFFFFFFu, w, off);
+            const unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, w, off);
             if (lane >= off)
                 w += y;
         }
         s_warp[lane] = w;
     }
     __syncthreads();
-    const int excl_nb = incl - nb + (warp > 0 ? s_warp[warp - 1] : 0);
+    const unsigned long long excl = incl - mine + (warp > 0 ? s_warp[warp - 1] : 0ull);
+    const int excl_nb = (int)(excl >> 32), excl_nw = (int)(excl & 0xFFFFFFFFull);
     if (e < E) {
         s_pad[e] = excl_nb * kBlockRows;
         pad_offsets[e] = excl_nb * kBlockRows;
         if (e == E - 1) {
             pad_offsets[E] = (excl_nb + nb) * kBlockRows;
-            *num_rowblocks = excl_nb + nb;
+            *num_rowblocks = excl_nw + nw;
         }
-        for (int b = 0; b < nb; ++b)
-            rowblocks[excl_nb + b] =
-                make_int4(e, excl_nb * kBlockRows + b * kBlockRows, min(kBlockRows, total - b * kBlockRows), 0);
+        for (int b = 0; b < nw; ++b)
+            rowblocks[excl_nw + b] = make_int4(e, excl_nb * kBlockRows + b * split, min(split, total - b * split), 0);
         for (int r = total; r < nb * kBlockRows; ++r)
             sorted_pair[excl_nb * kBlockRows + r] = -1;
     }
@@ -286,7 +291,7 @@ void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s)
 {
     const int nchunks = (a.T + kRouteChunk - 1) / kRouteChunk;
     route_kernel<<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist);
-    scan_kernel<<<1, 1024, 0, s>>>(a.E, nchunks, a.chunk_hist, a.counts, a.pad_offsets, a.rowblocks,
+    scan_kernel<<<1, 1024, 0, s>>>(a.E, nchunks, a.split_rows, a.chunk_hist, a.counts, a.pad_offsets, a.rowblocks,
                                    a.num_rowblocks, a.sorted_pair);
     scatter_kernel<<<nchunks, 32, 0, s>>>(a.T, a.E, a.k, a.topk_ids, a.chunk_hist, a.sorted_pair, a.pos_of_pair);
 }

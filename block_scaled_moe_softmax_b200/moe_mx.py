@@ -29,6 +29,10 @@ MOE_MX_ACT_BF16 = 0
 MOE_MX_ACT_MXFP8 = 1
 MOE_MX_FMT_MXFP4 = 0
 MOE_MX_FMT_MXFP8 = 1
+MOE_MX_SCALES_ROW_MAJOR = 0
+MOE_MX_SCALES_TILED = 1
+MOE_MX_W1 = 0
+MOE_MX_W2 = 1
 
 # Every symbol include/moe_mx.h declares: name -> (restype, argtypes)
 _P, _I, _I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
@@ -46,6 +50,8 @@ SIGNATURES = {
     "moe_mx_set_stage_timing": (_I, [_P, _I]),
     "moe_mx_get_stage_times": (_I, [_P, _P]),
     "moe_mx_route_group_noalloc": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_mx_prepare_scales": (_I, [_P, _I, _P, _P, _P]),
+    "moe_mx_set_scale_layout": (_I, [_P, _I]),
 }
 STAGES = ("route", "gather", "fc1", "fc2", "combine")
 
@@ -152,6 +158,15 @@ def moe_mx_route_group_noalloc(router_logits, num_tokens: int, num_experts: int,
         _ptr(pad_offsets), _ptr(sorted_pair), _ptr(pos_of_pair), _stream(stream)))
 
 
+def moe_mx_prepare_scales(handle: int, which: int, src, dst, stream=None) -> None:
+    """Rearrange one row-major E8M0 weight-scale tensor into the tiled layout (see the header)."""
+    _check(load_library().moe_mx_prepare_scales(handle, which, _ptr(src), _ptr(dst), _stream(stream)))
+
+
+def moe_mx_set_scale_layout(handle: int, layout: int) -> None:
+    _check(load_library().moe_mx_set_scale_layout(handle, layout))
+
+
 def moe_mx_debug_watchdog(handle: int, timeout_us: int, stream=None) -> None:
     _check(load_library().moe_mx_debug_watchdog(handle, timeout_us, _stream(stream)))
 
@@ -183,6 +198,14 @@ class MoeMxLayer:
             out = torch.empty(T, self.H, dtype=torch.bfloat16, device=x.device)
         moe_mx_forward(self.handle, x, router_logits, T, w1, w1_scale, w2, w2_scale, top_k, act_dtype, out, stream)
         return out
+
+    def prepare_scales(self, w1_scale: torch.Tensor, w2_scale: torch.Tensor, stream=None):
+        """Tiled copies of both weight-scale tensors; later forwards of this layer read that layout."""
+        t1, t2 = torch.empty_like(w1_scale), torch.empty_like(w2_scale)
+        moe_mx_prepare_scales(self.handle, MOE_MX_W1, w1_scale, t1, stream)
+        moe_mx_prepare_scales(self.handle, MOE_MX_W2, w2_scale, t2, stream)
+        moe_mx_set_scale_layout(self.handle, MOE_MX_SCALES_TILED)
+        return t1, t2
 
     def routing(self, T: int, top_k: int, stream=None):
         """The routing/grouping state of the most recent forward (device tensors)."""

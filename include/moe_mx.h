@@ -80,6 +80,14 @@ extern "C" {
 #define MOE_MX_FMT_MXFP4 0 /* E2M1 codes, two per byte */
 #define MOE_MX_FMT_MXFP8 1 /* E4M3 codes, one per byte */
 
+/* Layouts of the E8M0 weight scales moe_mx_forward reads (moe_mx_set_scale_layout). */
+#define MOE_MX_SCALES_ROW_MAJOR 0 /* [E, rows, K/32] as the quantiser writes them (default) */
+#define MOE_MX_SCALES_TILED 1     /* rearranged by moe_mx_prepare_scales */
+
+/* Which expert weight a scale tensor belongs to (moe_mx_prepare_scales). */
+#define MOE_MX_W1 0 /* [E, 2I, H/32]: gate rows then up rows */
+#define MOE_MX_W2 1 /* [E, H, I/32] */
+
 typedef struct moe_mx_handle moe_mx_handle;
 
 /*
@@ -210,6 +218,33 @@ MOE_MX_API int moe_mx_set_stage_timing(moe_mx_handle *h, int enable);
  * Errors: INVALID_ARG (timing not enabled or no timed forward yet), CUDA.
  */
 MOE_MX_API int moe_mx_get_stage_times(moe_mx_handle *h, float *ms);
+
+/*
+ * Weight preparation.  The pages leave tensor preparation to the adapter that owns
+ * the weights (TokenSpeed SiTU package description, "Runtime API"); this library
+ * offers one such step for the E8M0 weight scales.  The GEMM reads, per 128-row
+ * weight tile and 128-element K stage, the 4 scale bytes of each of the 128 rows;
+ * in the row-major layout those are 128 scattered 4-byte pieces, in the tiled
+ * layout one contiguous 512-byte block (one copy instead of 128).
+ *
+ * moe_mx_prepare_scales writes the tiled layout of one scale tensor: src is the
+ * row-major tensor (which = MOE_MX_W1: [E, 2I, H/32]; MOE_MX_W2: [E, H, I/32]),
+ * dst a caller-owned device buffer of the same size; both device pointers on the
+ * handle's device, 16-byte aligned, not overlapping.  Asynchronous on `stream`;
+ * the codes (w1, w2) are not touched and stay row-major.  Layout of dst: for
+ * expert e, weight tile nt and K stage kk, 512 bytes at ((e * n_tiles + nt) *
+ * (K/128) + kk) * 512, byte (m % 32) * 16 + (m / 32) * 4 + b = the scale of tile
+ * row m, 32-element block b of the stage; W1 tiles (n_tiles = I/64) hold gate
+ * rows 64 nt .. 64 nt + 63 then up rows I + 64 nt .. I + 64 nt + 63, W2 tiles
+ * (n_tiles = H/128) rows 128 nt .. 128 nt + 127.  Errors: INVALID_ARG, CUDA.
+ *
+ * moe_mx_set_scale_layout selects which layout the handle's later forwards read
+ * from w1_scale and w2_scale (both tensors in the same layout).  Host-only.
+ * Errors: INVALID_ARG.
+ */
+MOE_MX_API int moe_mx_prepare_scales(const moe_mx_handle *h, int which, const uint8_t *src, uint8_t *dst,
+                                     void *stream);
+MOE_MX_API int moe_mx_set_scale_layout(moe_mx_handle *h, int layout);
 
 /*
  * Self-test of the device watchdog: launch one kernel that waits on a device

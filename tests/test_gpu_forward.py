@@ -4,8 +4,11 @@ Inputs are the seeded synthetic workloads; weights are quantised by the
 oracle's quantiser.  Routing ids, counts, offsets and the permutation must match
 bit-exactly; outputs must meet the layer's tolerance (relative Frobenius error
 <= 5e-3 and max |gpu - ref| <= 2e-2 * RMS(ref)).  Shapes here span several
-GEMM tiles, ragged row blocks and both MMA orientations (tokens on M, or
-weight rows on M with the tokens on N), forced through MOE_MX_SWAP_ROWS.
+GEMM tiles, ragged row blocks, every kernel variant (activation tiles of 16,
+32, 64 or 128 rows per term, forced through MOE_MX_TILE_ROWS: below 128 the
+expert segments are split into work blocks of that many rows) and both MMA
+orientations of the 128-row variant (tokens on M, or weight rows on M with the
+tokens on N), forced through MOE_MX_SWAP_ROWS.
 """
 import numpy as np
 import pytest
@@ -33,9 +36,11 @@ SHAPES = {
 }
 
 
-def _run(wl, act_mode, monkeypatch, swap_rows=None, inp=None):
+def _run(wl, act_mode, monkeypatch, swap_rows=None, inp=None, tile_rows=None):
     if swap_rows is not None:
         monkeypatch.setenv("MOE_MX_SWAP_ROWS", str(swap_rows))
+    if tile_rows is not None:
+        monkeypatch.setenv("MOE_MX_TILE_ROWS", str(tile_rows))
     inp = inp or helpers.host_inputs(wl)
     d = helpers.to_device(inp)
     layer = moe_mx.MoeMxLayer(wl.H, wl.I, wl.E, max(wl.T, 1), wl.top_k)
@@ -44,15 +49,53 @@ def _run(wl, act_mode, monkeypatch, swap_rows=None, inp=None):
     return layer, inp, out
 
 
+# (tile rows, swap rows): the 128-row variant in both orientations and mixed, each smaller
+# variant (always tokens on N), and the automatic choice by token count
+VARIANTS = {
+    "t128_tokens_on_M": (128, 0), "t128_weights_on_M": (128, 128), "t128_mixed": (128, 64),
+    "t64": (64, None), "t32": (32, None), "t16": (16, None), "auto": (None, None),
+}
+
+
 @pytest.mark.parametrize("name", list(SHAPES))
 @pytest.mark.parametrize("act_mode", [0, 1], ids=["w4a16", "w4a8"])
-@pytest.mark.parametrize("swap_rows", [0, 128, 64], ids=["tokens_on_M", "weights_on_M", "mixed"])
-def test_forward_matches_oracle(name, act_mode, swap_rows, monkeypatch):
+@pytest.mark.parametrize("variant", list(VARIANTS))
+def test_forward_matches_oracle(name, act_mode, variant, monkeypatch):
     wl = SHAPES[name]
-    layer, inp, out = _run(wl, act_mode, monkeypatch, swap_rows)
+    tile_rows, swap_rows = VARIANTS[variant]
+    layer, inp, out = _run(wl, act_mode, monkeypatch, swap_rows, tile_rows=tile_rows)
     helpers.check_routing(layer, wl.T, wl.top_k, wl.E, inp["logits"].numpy())
     ref, _, _ = helpers.oracle_forward(inp, wl.top_k, act_mode)
-    helpers.check_output(out, ref, f"{name}/{act_mode}/{swap_rows}")
+    helpers.check_output(out, ref, f"{name}/{act_mode}/{variant}")
+    layer.close()
+
+
+@pytest.mark.parametrize("name", ["multi", "single_expert"])
+@pytest.mark.parametrize("act_mode", [0, 1], ids=["w4a16", "w4a8"])
+@pytest.mark.parametrize("variant", list(VARIANTS))
+def test_tiled_scales_match_row_major(name, act_mode, variant, monkeypatch):
+    """The tiled weight-scale layout (moe_mx_prepare_scales) gives bit-identical outputs."""
+    wl = SHAPES[name]
+    tile_rows, swap_rows = VARIANTS[variant]
+    layer, inp, out_rm = _run(wl, act_mode, monkeypatch, swap_rows, tile_rows=tile_rows)
+    d = helpers.to_device(inp)
+    t1, t2 = layer.prepare_scales(d["w1s"], d["w2s"])
+    out_t = layer.forward(d["x"], d["logits"], d["w1"], t1, d["w2"], t2, wl.top_k, act_mode)
+    assert layer.sync_status() == moe_mx.MOE_MX_OK, moe_mx.moe_mx_last_error()
+    assert torch.equal(out_t.view(torch.int16), out_rm.view(torch.int16))
+    layer.close()
+
+
+def test_prepare_scales_rejects_bad_arguments():
+    wl = SHAPES["tiny"]
+    layer = moe_mx.MoeMxLayer(wl.H, wl.I, wl.E, wl.T, wl.top_k)
+    src = torch.zeros(wl.E, 2 * wl.I, wl.H // 32, dtype=torch.uint8, device="cuda")
+    with pytest.raises(moe_mx.MoeMxError):
+        moe_mx.moe_mx_prepare_scales(layer.handle, 7, src, torch.empty_like(src))
+    with pytest.raises(moe_mx.MoeMxError):
+        moe_mx.moe_mx_prepare_scales(layer.handle, moe_mx.MOE_MX_W1, src, src)  # overlapping
+    with pytest.raises(moe_mx.MoeMxError):
+        moe_mx.moe_mx_set_scale_layout(layer.handle, 5)
     layer.close()
 
 

@@ -12,7 +12,8 @@ Weights are drawn per expert on the GPU (float32, N(0, 0.02)), copied to the
 host and quantised by the ORACLE's quantiser; the library's GPU quantiser is
 run on the same float32 tensors and must agree bit-exactly (a full-size pin of
 moe_mx_quantize).  The decode, batched-decode and prefill workloads share one
-weight set (same H, I, E and seed).
+weight set (same H, I, E and seed).  Each workload is also run with the weight
+scales in the tiled layout (moe_mx_prepare_scales) and must give the same bits.
 """
 import numpy as np
 import pytest
@@ -89,4 +90,9 @@ def test_full_size_forward(name):
     ref, ids_o, _ = helpers.oracle_forward(inp, wl.top_k, act, tokens=toks)
     assert np.array_equal(ids_o, ids[toks])
     helpers.check_output(out[toks], ref, f"{name} sampled tokens {toks}")
+    # the tiled weight-scale layout (the one bench.py times) gives the same bits for all tokens
+    t1, t2 = layer.prepare_scales(dev["w1s"], dev["w2s"])
+    out_t = layer.forward(x.cuda(), logits.cuda(), dev["w1"], t1, dev["w2"], t2, wl.top_k, act)
+    assert layer.sync_status() == moe_mx.MOE_MX_OK, moe_mx.moe_mx_last_error()
+    assert torch.equal(out_t.view(torch.int16), out.view(torch.int16))
     layer.close()
