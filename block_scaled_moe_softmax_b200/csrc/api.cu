@@ -374,14 +374,7 @@ int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, 
     }
     {
         const int64_t pairs = (int64_t)T * k;
-        const int64_t rows = grouped_rows_bound(E, pairs);
-        cudaError_t ce = cudaMemsetAsync(h->sorted_pair, 0xFF, sizeof(int32_t) * rows, s);
-        if (ce == cudaSuccess)
-            ce = cudaMemsetAsync(h->unit_counters, 0, 2 * sizeof(int32_t), s);
-        if (ce != cudaSuccess) {
-            rc = cuda_fail(ce, "cudaMemsetAsync(workspace)");
-            goto done;
-        }
+        cudaError_t ce;
         cudaEvent_t *evset = h->timing ? h->ev + (h->n_timed % kTimingRing) * kEvPerFwd : nullptr;
         auto mark = [&](int i) {
             if (evset)
@@ -399,7 +392,7 @@ int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, 
                                                : kBlockRows;
         RouteGroupArgs ra{router_logits, T, E, k, h->topk_ids, h->topk_w, h->chunk_hist, h->counts,
                           h->pad_offsets, h->rowblocks, h->num_rowblocks, h->sorted_pair, h->pos_of_pair,
-                          tile_rows};
+                          tile_rows, h->unit_counters};
         launch_route_and_group(ra, s);
         mark(1);
         const int mx8 = act_dtype == MOE_MX_ACT_MXFP8;

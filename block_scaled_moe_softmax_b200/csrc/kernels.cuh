@@ -16,6 +16,7 @@ constexpr int kMaxTopK = 32;
 constexpr int kBlockRows = 128;   // grouped-layout segment granularity = GEMM row block
 constexpr int kRouteChunk = 64;   // tokens per router CTA (= per histogram chunk)
 constexpr int kRouteThreads = 512;
+constexpr int kSmallRouteTokens = 64; // at most this many tokens: routing and grouping in one CTA
 
 struct RouteGroupArgs {
     const float *logits;
@@ -30,6 +31,7 @@ struct RouteGroupArgs {
     int32_t *sorted_pair;
     int32_t *pos_of_pair;
     int split_rows; // rows per work block of the row-block list: 16, 32, 64 or kBlockRows
+    int32_t *unit_counters; // optional: the GEMMs' 2 work-unit counters, zeroed here
 };
 
 void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s);

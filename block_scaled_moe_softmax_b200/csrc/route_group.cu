@@ -22,6 +22,73 @@
 namespace moe_mx {
 
 // ---------------------------------------------------------------- router
+// Route one token (whole warp): the k experts in descending logit order, the lowest index
+// first among equal logits, and their weights = the softmax over the selected logits.  Lane 0
+// writes ids and weights and adds the selections to the block's expert histogram.
+__device__ __forceinline__ void route_token(const float *__restrict__ row, int E, int k, int t, int lane,
+                                            int32_t *__restrict__ topk_ids, float *__restrict__ topk_w,
+                                            int32_t *hist)
+{
+    constexpr int kPerLane = kMaxExperts / 32;
+    float v[kPerLane];
+    uint32_t taken = 0;
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i) {
+        const int e = i * 32 + lane;
+        float x = (e < E) ? __ldg(row + e) : -INFINITY;
+        if (x != x) // NaN never outranks a number
+            x = -INFINITY;
+        v[i] = x;
+        if (e >= E)
+            taken |= 1u << i; // out of range: never selectable
+    }
+    float sel_logit[kMaxTopK];
+    int sel_id[kMaxTopK];
+    for (int j = 0; j < k; ++j) {
+        // this lane's best untaken entry (entries are in ascending expert order)
+        float bv = -INFINITY;
+        int bi = 0x7FFFFFFF;
+#pragma unroll
+        for (int i = 0; i < kPerLane; ++i) {
+            const int e = i * 32 + lane;
+            const bool free_ = !((taken >> i) & 1u);
+            if (free_ && (v[i] > bv || (v[i] == bv && e < bi))) {
+                bv = v[i];
+                bi = e;
+            }
+        }
+        // warp arg-max with the lowest index winning ties
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
+            const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, off);
+            if (ov > bv || (ov == bv && oi < bi)) {
+                bv = ov;
+                bi = oi;
+            }
+        }
+        if ((bi & 31) == lane)
+            taken |= 1u << (bi >> 5);
+        sel_logit[j] = bv;
+        sel_id[j] = bi;
+    }
+    if (lane == 0) {
+        // softmax over the k selected logits == renormalised top-k of the full softmax
+        const float m = sel_logit[0];
+        float u[kMaxTopK];
+        float z = 0.f;
+        for (int j = 0; j < k; ++j) {
+            u[j] = expf(sel_logit[j] - m);
+            z += u[j];
+        }
+        for (int j = 0; j < k; ++j) {
+            topk_ids[(size_t)t * k + j] = sel_id[j];
+            topk_w[(size_t)t * k + j] = u[j] / z;
+            atomicAdd(&hist[sel_id[j]], 1);
+        }
+    }
+}
+
 // One warp per token; each CTA covers kRouteChunk tokens and also writes the
 // per-expert histogram of its chunk (the first level of the counting sort).
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float *__restrict__ logits, int T, int E,
@@ -34,98 +101,27 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float *__res
     for (int e = threadIdx.x; e < E; e += blockDim.x)
         hist[e] = 0;
     __syncthreads();
-
     const int t_begin = blockIdx.x * kRouteChunk;
     const int t_end = min(T, t_begin + kRouteChunk);
-    constexpr int kPerLane = kMaxExperts / 32;
-    for (int t = t_begin + warp; t < t_end; t += kRouteThreads / 32) {
-        const float *row = logits + (size_t)t * E;
-        float v[kPerLane];
-        uint32_t taken = 0;
-#pragma unroll
-        for (int i = 0; i < kPerLane; ++i) {
-            const int e = i * 32 + lane;
-            float x = (e < E) ? __ldg(row + e) : -INFINITY;
-            if (x != x) // NaN never outranks a number
-                x = -INFINITY;
-            v[i] = x;
-            if (e >= E)
-                taken |= 1u << i; // out of range: never selectable
-        }
-        float sel_logit[kMaxTopK];
-        int sel_id[kMaxTopK];
-        for (int j = 0; j < k; ++j) {
-            // this lane's best untaken entry (entries are in ascending expert order)
-            float bv = -INFINITY;
-            int bi = 0x7FFFFFFF;
-#pragma unroll
-            for (int i = 0; i < kPerLane; ++i) {
-                const int e = i * 32 + lane;
-                const bool free_ = !((taken >> i) & 1u);
-                if (free_ && (v[i] > bv || (v[i] == bv && e < bi))) {
-                    bv = v[i];
-                    bi = e;
-                }
-            }
-            // warp arg-max with the lowest index winning ties
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
-                const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, off);
-                if (ov > bv || (ov == bv && oi < bi)) {
-                    bv = ov;
-                    bi = oi;
-                }
-            }
-            if ((bi & 31) == lane)
-                taken |= 1u << (bi >> 5);
-            sel_logit[j] = bv;
-            sel_id[j] = bi;
-        }
-        if (lane == 0) {
-            // softmax over the k selected logits == renormalised top-k of the full softmax
-            const float m = sel_logit[0];
-            float u[kMaxTopK];
-            float z = 0.f;
-            for (int j = 0; j < k; ++j) {
-                u[j] = expf(sel_logit[j] - m);
-                z += u[j];
-            }
-            for (int j = 0; j < k; ++j) {
-                topk_ids[(size_t)t * k + j] = sel_id[j];
-                topk_w[(size_t)t * k + j] = u[j] / z;
-                atomicAdd(&hist[sel_id[j]], 1);
-            }
-        }
-    }
+    for (int t = t_begin + warp; t < t_end; t += kRouteThreads / 32)
+        route_token(logits + (size_t)t * E, E, k, t, lane, topk_ids, topk_w, hist);
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x)
         chunk_hist[(size_t)blockIdx.x * E + e] = hist[e];
 }
 
 // ---------------------------------------------------------------- scan
-// One CTA: per-expert totals over chunks, padded exclusive scan over experts,
-// per-chunk base rows, the row-block list and the padding markers.  Segments
-// are padded to kBlockRows rows; the row-block list (the GEMMs' work list)
-// splits each segment into blocks of at most `split` rows (16, 32, 64 or
-// kBlockRows).
-__global__ void __launch_bounds__(1024) scan_kernel(int E, int nchunks, int split, int32_t *__restrict__ chunk_hist,
-                                                    int32_t *__restrict__ counts, int32_t *__restrict__ pad_offsets,
-                                                    int4 *__restrict__ rowblocks, int32_t *__restrict__ num_rowblocks,
-                                                    int32_t *__restrict__ sorted_pair)
+// Padded exclusive scan over the experts, for one CTA of 1024 threads (all threads call;
+// thread e < E holds its expert's pair count `total`): writes counts, pad_offsets, the
+// row-block list and the padding markers, and returns expert e's first grouped row.
+// Segments are padded to kBlockRows rows; the row-block list (the GEMMs' work list) splits
+// each segment into blocks of at most `split` rows (16, 32, 64 or kBlockRows).
+__device__ __forceinline__ int scan_experts(int E, int split, int total, int32_t *__restrict__ counts,
+                                            int32_t *__restrict__ pad_offsets, int4 *__restrict__ rowblocks,
+                                            int32_t *__restrict__ num_rowblocks, int32_t *__restrict__ sorted_pair,
+                                            unsigned long long *s_warp)
 {
-    __shared__ int32_t s_pad[kMaxExperts];
-    __shared__ unsigned long long s_warp[32];
     const int e = threadIdx.x;
-    int total = 0;
-    if (e < E) {
-        for (int c = 0; c < nchunks; ++c) {
-            const int h = chunk_hist[(size_t)c * E + e];
-            chunk_hist[(size_t)c * E + e] = total; // exclusive prefix within the expert
-            total += h;
-        }
-        counts[e] = total;
-    }
     const int nb = (total + kBlockRows - 1) / kBlockRows; // padded segment: nb * kBlockRows rows
     const int nw = (total + split - 1) / split;            // work blocks of the segment
     // one block-wide exclusive scan of both counts, packed in 32-bit halves
@@ -155,7 +151,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(int E, int nchunks, int spli
     const unsigned long long excl = incl - mine + (warp > 0 ? s_warp[warp - 1] : 0ull);
     const int excl_nb = (int)(excl >> 32), excl_nw = (int)(excl & 0xFFFFFFFFull);
     if (e < E) {
-        s_pad[e] = excl_nb * kBlockRows;
+        counts[e] = total;
         pad_offsets[e] = excl_nb * kBlockRows;
         if (e == E - 1) {
             pad_offsets[E] = (excl_nb + nb) * kBlockRows;
@@ -166,29 +162,40 @@ __global__ void __launch_bounds__(1024) scan_kernel(int E, int nchunks, int spli
         for (int r = total; r < nb * kBlockRows; ++r)
             sorted_pair[excl_nb * kBlockRows + r] = -1;
     }
-    __syncthreads();
-    if (e < E) {
-        const int base = s_pad[e];
-        for (int c = 0; c < nchunks; ++c)
-            chunk_hist[(size_t)c * E + e] += base;
-    }
+    return excl_nb * kBlockRows;
 }
 
-// ---------------------------------------------------------------- scatter
-// One warp per chunk: walks the chunk's pairs in ascending p and places each
-// at its expert's cursor, so equal experts keep ascending-token order.
-__global__ void __launch_bounds__(32) scatter_kernel(int T, int E, int k, const int32_t *__restrict__ topk_ids,
-                                                     const int32_t *__restrict__ chunk_base,
-                                                     int32_t *__restrict__ sorted_pair,
-                                                     int32_t *__restrict__ pos_of_pair)
+// One CTA: per-expert totals over the chunk histograms, the scan, and per-chunk base rows
+// for the scatter; also zeroes the GEMMs' work-unit counters (optional).
+__global__ void __launch_bounds__(1024) scan_kernel(int E, int nchunks, int split, int32_t *__restrict__ chunk_hist,
+                                                    int32_t *__restrict__ counts, int32_t *__restrict__ pad_offsets,
+                                                    int4 *__restrict__ rowblocks, int32_t *__restrict__ num_rowblocks,
+                                                    int32_t *__restrict__ sorted_pair, int32_t *__restrict__ unit_counters)
 {
-    __shared__ int32_t cursor[kMaxExperts];
-    const int lane = threadIdx.x;
-    for (int e = lane; e < E; e += 32)
-        cursor[e] = chunk_base[(size_t)blockIdx.x * E + e];
-    __syncwarp();
-    const int p_begin = blockIdx.x * kRouteChunk * k;
-    const int p_end = min(T, (blockIdx.x + 1) * kRouteChunk) * k;
+    __shared__ unsigned long long s_warp[32];
+    const int e = threadIdx.x;
+    if (unit_counters && e < 2) // the GEMMs' work-unit counters start at zero
+        unit_counters[e] = 0;
+    int total = 0;
+    if (e < E) {
+        for (int c = 0; c < nchunks; ++c) {
+            const int h = chunk_hist[(size_t)c * E + e];
+            chunk_hist[(size_t)c * E + e] = total; // exclusive prefix within the expert
+            total += h;
+        }
+    }
+    const int base = scan_experts(E, split, total, counts, pad_offsets, rowblocks, num_rowblocks, sorted_pair, s_warp);
+    if (e < E)
+        for (int c = 0; c < nchunks; ++c)
+            chunk_hist[(size_t)c * E + e] += base;
+}
+
+// Stable placement of pairs [p_begin, p_end) by one warp: each pair goes to its expert's
+// cursor, pairs in ascending p (so equal experts keep ascending-token order).
+__device__ __forceinline__ void scatter_pairs(int p_begin, int p_end, const int32_t *__restrict__ topk_ids,
+                                              int32_t *cursor, int32_t *__restrict__ sorted_pair,
+                                              int32_t *__restrict__ pos_of_pair, int lane)
+{
     const unsigned lt_mask = (1u << lane) - 1u;
     for (int base = p_begin; base < p_end; base += 32) {
         const int p = base + lane;
@@ -208,6 +215,51 @@ __global__ void __launch_bounds__(32) scatter_kernel(int T, int E, int k, const 
             pos_of_pair[p] = row;
         }
     }
+}
+
+// Routing and grouping of a small batch (T <= kSmallRouteTokens) in one CTA: routes, the
+// expert histogram, the scan, the row-block list and the stable scatter, with no global
+// round trip between the steps.  Also zeroes the GEMMs' work-unit counters.
+__global__ void __launch_bounds__(1024) route_group_small_kernel(const RouteGroupArgs a)
+{
+    __shared__ int32_t hist[kMaxExperts]; // counts, then cursors
+    __shared__ unsigned long long s_warp[32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x)
+        hist[e] = 0;
+    if (a.unit_counters && threadIdx.x < 2)
+        a.unit_counters[threadIdx.x] = 0;
+    __syncthreads();
+    for (int t = warp; t < a.T; t += 32)
+        route_token(a.logits + (size_t)t * a.E, a.E, a.k, t, lane, a.topk_ids, a.topk_w, hist);
+    __syncthreads(); // also makes lane 0's id writes visible to the whole CTA
+    const int e = threadIdx.x;
+    const int total = e < a.E ? hist[e] : 0;
+    const int base = scan_experts(a.E, a.split_rows, total, a.counts, a.pad_offsets, a.rowblocks, a.num_rowblocks,
+                                  a.sorted_pair, s_warp);
+    if (e < a.E)
+        hist[e] = base;
+    __syncthreads();
+    if (warp == 0)
+        scatter_pairs(0, a.T * a.k, a.topk_ids, hist, a.sorted_pair, a.pos_of_pair, lane);
+}
+
+// ---------------------------------------------------------------- scatter
+// One warp per chunk: places the chunk's pairs at their experts' cursors (the chunk's base
+// rows from the scan), in ascending p.
+__global__ void __launch_bounds__(32) scatter_kernel(int T, int E, int k, const int32_t *__restrict__ topk_ids,
+                                                     const int32_t *__restrict__ chunk_base,
+                                                     int32_t *__restrict__ sorted_pair,
+                                                     int32_t *__restrict__ pos_of_pair)
+{
+    __shared__ int32_t cursor[kMaxExperts];
+    const int lane = threadIdx.x;
+    for (int e = lane; e < E; e += 32)
+        cursor[e] = chunk_base[(size_t)blockIdx.x * E + e];
+    __syncwarp();
+    const int p_begin = blockIdx.x * kRouteChunk * k;
+    const int p_end = min(T, (blockIdx.x + 1) * kRouteChunk) * k;
+    scatter_pairs(p_begin, p_end, topk_ids, cursor, sorted_pair, pos_of_pair, lane);
 }
 
 // ---------------------------------------------------------------- gather
@@ -289,10 +341,14 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
 // ---------------------------------------------------------------- launchers
 void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s)
 {
+    if (a.T <= kSmallRouteTokens) {
+        route_group_small_kernel<<<1, 1024, 0, s>>>(a);
+        return;
+    }
     const int nchunks = (a.T + kRouteChunk - 1) / kRouteChunk;
     route_kernel<<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist);
     scan_kernel<<<1, 1024, 0, s>>>(a.E, nchunks, a.split_rows, a.chunk_hist, a.counts, a.pad_offsets, a.rowblocks,
-                                   a.num_rowblocks, a.sorted_pair);
+                                   a.num_rowblocks, a.sorted_pair, a.unit_counters);
     scatter_kernel<<<nchunks, 32, 0, s>>>(a.T, a.E, a.k, a.topk_ids, a.chunk_hist, a.sorted_pair, a.pos_of_pair);
 }
 

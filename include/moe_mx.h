@@ -188,7 +188,8 @@ MOE_MX_API int64_t moe_mx_max_grouped_rows(const moe_mx_handle *h, int num_token
  *   pad_offsets int32 [E+1]    first grouped row of each expert segment;
  *                              segment e spans ceil(counts[e]/128)*128 rows;
  *   sorted_pair int32 [rows]   pair id t*k+j at each grouped row, -1 on
- *                              padding rows; rows = moe_mx_max_grouped_rows.
+ *                              padding rows; rows = moe_mx_max_grouped_rows
+ *                              (entries past pad_offsets[E] are unspecified).
  * Any pointer may be NULL to skip that array.  Errors: INVALID_ARG, CUDA.
  */
 MOE_MX_API int moe_mx_get_routing(const moe_mx_handle *h, int32_t *topk_ids, float *topk_w, int32_t *counts,
