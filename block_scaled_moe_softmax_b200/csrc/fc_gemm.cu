@@ -395,6 +395,9 @@ __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
     bool ok = true;
     // this warp's scale-factor columns: the weight atom at +0, the activation atoms at +4 and +8
     const uint32_t sf_w = tmem_base + kSfCol + 16u * (uint32_t)MI;
+    // descriptors of stage slot 0, K block 0 (term 1 of the activations, and the weights)
+    const uint64_t dact0 = smem_desc_sw128(base + kOffAct), dw0 = smem_desc_sw128(base + kOffW);
+    static_assert(P::kSmemBytes + 1024 < (1 << 18), "descriptor start field arithmetic needs addresses < 2^18");
     const UnitRing<kStages> ring{bars, c.units};
     const int lane = threadIdx.x & 31;
     for (; ok; ++cnt) {
@@ -432,10 +435,12 @@ __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
             // The stage's operands are computed by the whole warp before the wait; then one elected
             // lane issues the scale copies, MMAs and commit back to back (measured: an elect /
             // reconverge around each instruction costs more than the instruction itself).
-            const uint32_t act = base + kOffAct + s * kActBytes;
-            const uint32_t wt = base + kOffW + s * kWBytes;
             const uint32_t wsf_s = base + kOffWsf + s * kWsfBytes;
             const uint32_t asf_s = base + kOffAsf + s * kAsfBytes;
+            // descriptors are affine in the address: the start field is address / 16 in the low
+            // 14 bits, and every shared-memory address here stays below 2^18
+            const uint64_t ds_act = dact0 + (uint64_t)((s * kActBytes) >> 4);
+            const uint64_t ds_w = dw0 + (uint64_t)((s * kWBytes) >> 4);
             uint64_t opa[4][2], opb[4][2];
             uint32_t idesc[4], accf[4];
 #pragma unroll
@@ -443,10 +448,10 @@ __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
                 // the scale-factor byte of this 32-element block sits in both sf-id fields
                 idesc[k32] = idesc0 | ((uint32_t)k32 << 4) | ((uint32_t)k32 << 29);
                 accf[k32] = (first && k32 == 0) ? 0u : 1u;
-                const uint64_t dw = smem_desc_sw128(wt + 32 * k32);
+                const uint64_t dw = ds_w + 2u * k32; // +32 bytes per 32-element K block
 #pragma unroll
                 for (int t = 0; t < 2; ++t) {
-                    const uint64_t da = smem_desc_sw128(act + t * kTermBytes + 32 * k32);
+                    const uint64_t da = ds_act + (uint64_t)((t * kTermBytes) >> 4) + 2u * k32;
                     opa[k32][t] = swap ? dw : da;
                     opb[k32][t] = swap ? da : dw;
                 }
