@@ -52,7 +52,10 @@ from block_scaled_moe_softmax_b200 import moe_mx, workloads  # noqa: E402
 
 METRIC = "MoE layer tokens/s; % of HBM roofline (decode) / MMA peak (prefill)"
 FLUSH_BYTES = 512 << 20
-KERNELS_PER_FORWARD = 7  # route, scan, scatter, gather, fc1, fc2, combine
+def kernels_per_forward(T):
+    """Kernel launches of one forward: routing+grouping (one kernel up to 64 tokens, else route,
+    scan and scatter), gather, FC1, FC2, combine."""
+    return (1 if T <= 64 else 3) + 4
 
 
 def log(*a):
@@ -422,7 +425,7 @@ def run_ours(args, wl):
                    "weight_scales": "tiled layout (moe_mx_prepare_scales, once before timing)"},
         "e2e": {"value": world * wl.T / (e2e_ms / 1000.0), "unit": "tokens/s",
                 "h2d_bytes_per_step": wl.T * wl.H * 2 + wl.T * wl.E * 4, "d2h_bytes_per_step": wl.T * wl.H * 2},
-        "gpu_launches": KERNELS_PER_FORWARD * args.steps,
+        "gpu_launches": kernels_per_forward(wl.T) * args.steps,
         "roofline": roofline,
         "layer_roofline": layer_roofline,
         "stage_ms": stage,

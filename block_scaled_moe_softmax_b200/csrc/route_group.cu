@@ -25,11 +25,11 @@ namespace moe_mx {
 // Route one token (whole warp): the k experts in descending logit order, the lowest index
 // first among equal logits, and their weights = the softmax over the selected logits.  Lane 0
 // writes ids and weights and adds the selections to the block's expert histogram.
+template <int kPerLane> // experts per lane: E <= 32 * kPerLane
 __device__ __forceinline__ void route_token(const float *__restrict__ row, int E, int k, int t, int lane,
                                             int32_t *__restrict__ topk_ids, float *__restrict__ topk_w,
                                             int32_t *hist)
 {
-    constexpr int kPerLane = kMaxExperts / 32;
     float v[kPerLane];
     uint32_t taken = 0;
 #pragma unroll
@@ -91,6 +91,7 @@ __device__ __forceinline__ void route_token(const float *__restrict__ row, int E
 
 // One warp per token; each CTA covers kRouteChunk tokens and also writes the
 // per-expert histogram of its chunk (the first level of the counting sort).
+template <int kPerLane>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float *__restrict__ logits, int T, int E,
                                                                int k, int32_t *__restrict__ topk_ids,
                                                                float *__restrict__ topk_w,
@@ -104,7 +105,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float *__res
     const int t_begin = blockIdx.x * kRouteChunk;
     const int t_end = min(T, t_begin + kRouteChunk);
     for (int t = t_begin + warp; t < t_end; t += kRouteThreads / 32)
-        route_token(logits + (size_t)t * E, E, k, t, lane, topk_ids, topk_w, hist);
+        route_token<kPerLane>(logits + (size_t)t * E, E, k, t, lane, topk_ids, topk_w, hist);
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x)
         chunk_hist[(size_t)blockIdx.x * E + e] = hist[e];
@@ -220,6 +221,7 @@ __device__ __forceinline__ void scatter_pairs(int p_begin, int p_end, const int3
 // Routing and grouping of a small batch (T <= kSmallRouteTokens) in one CTA: routes, the
 // expert histogram, the scan, the row-block list and the stable scatter, with no global
 // round trip between the steps.  Also zeroes the GEMMs' work-unit counters.
+template <int kPerLane>
 __global__ void __launch_bounds__(1024) route_group_small_kernel(const RouteGroupArgs a)
 {
     __shared__ int32_t hist[kMaxExperts]; // counts, then cursors
@@ -231,7 +233,7 @@ __global__ void __launch_bounds__(1024) route_group_small_kernel(const RouteGrou
         a.unit_counters[threadIdx.x] = 0;
     __syncthreads();
     for (int t = warp; t < a.T; t += 32)
-        route_token(a.logits + (size_t)t * a.E, a.E, a.k, t, lane, a.topk_ids, a.topk_w, hist);
+        route_token<kPerLane>(a.logits + (size_t)t * a.E, a.E, a.k, t, lane, a.topk_ids, a.topk_w, hist);
     __syncthreads(); // also makes lane 0's id writes visible to the whole CTA
     const int e = threadIdx.x;
     const int total = e < a.E ? hist[e] : 0;
@@ -263,22 +265,27 @@ __global__ void __launch_bounds__(32) scatter_kernel(int T, int E, int k, const 
 }
 
 // ---------------------------------------------------------------- gather
-// Encode x[t] into grouped row pos_of_pair[p] for every pair p, as the MXFP8
-// operand FC1 consumes (see mx_encode32): the OCP MXFP8 quantisation for w4a8,
-// the exact two-term expansion of the bf16 row for w4a16.  One thread per
-// 32-element block: 64 bytes in, 32 (or 2 x 32) code bytes and 1 (or 2) scale
-// bytes out.
-__global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16 *__restrict__ x, int P, int H, int k,
-                                                     const int32_t *__restrict__ pos_of_pair, uint8_t *__restrict__ aq,
-                                                     uint8_t *__restrict__ asf, int act_rows, int act_mxfp8)
+// Encode each token's row once as the MXFP8 operand FC1 consumes (see mx_encode32): the OCP
+// MXFP8 quantisation for w4a8, the exact two-term expansion of the bf16 row for w4a16; and
+// write it to the grouped row of `group` of the token's k pairs (group = k: each block is read
+// and encoded once; group = 1 for small batches, which need the parallelism more).  One thread
+// per (token, 32-element block, pair group): 64 bytes in, group x (32 or 2 x 32) code bytes and
+// group x (1 or 2) scale bytes out.
+__global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H, int k,
+                                                     int group, const int32_t *__restrict__ pos_of_pair,
+                                                     uint8_t *__restrict__ aq, uint8_t *__restrict__ asf, int act_rows,
+                                                     int act_mxfp8)
 {
-    const int blocks_per_row = H / 32;
-    const long long total = (long long)P * blocks_per_row;
+    const int blocks_per_row = H / 32, groups = k / group;
+    const long long total = (long long)T * blocks_per_row * groups;
     for (long long g = blockIdx.x * (long long)blockDim.x + threadIdx.x; g < total;
          g += (long long)gridDim.x * blockDim.x) {
-        const int p = (int)(g / blocks_per_row);
-        const int b = (int)(g % blocks_per_row);
-        const int t = p / k;
+        // consecutive threads take consecutive blocks of one row: coalesced loads and stores
+        const long long per_group = (long long)T * blocks_per_row;
+        const int jg = (int)(g / per_group);
+        const long long tb = g % per_group;
+        const int t = (int)(tb / blocks_per_row);
+        const int b = (int)(tb % blocks_per_row);
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H + (size_t)b * 32);
         float v[32];
 #pragma unroll
@@ -292,7 +299,18 @@ __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16 *__rest
                 v[8 * i + 2 * j + 1] = f.y;
             }
         }
-        store_act_block32(aq, asf, act_rows, H, pos_of_pair[p], b * 32, v, act_mxfp8);
+        uint8_t c0[32], c1[32];
+        uint32_t s0, s1;
+        mx_encode32(v, act_mxfp8, c0, c1, s0, s1); // the values are bf16 already: no rounding step
+        for (int j = jg * group; j < (jg + 1) * group; ++j) {
+            const int row = pos_of_pair[(size_t)t * k + j];
+            store_codes32(aq + (size_t)row * H + b * 32, c0);
+            asf[sf_atom_byte(row, b * 32, H, 0)] = (uint8_t)s0;
+            if (!act_mxfp8) {
+                store_codes32(aq + ((size_t)act_rows + row) * H + b * 32, c1);
+                asf[sf_atom_byte(row, b * 32, H, 1)] = (uint8_t)s1;
+            }
+        }
     }
 }
 
@@ -341,12 +359,23 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
 // ---------------------------------------------------------------- launchers
 void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s)
 {
+    // the top-k scan visits 32 * kPerLane candidates per token: size it to the expert count
     if (a.T <= kSmallRouteTokens) {
-        route_group_small_kernel<<<1, 1024, 0, s>>>(a);
+        if (a.E <= 256)
+            route_group_small_kernel<8><<<1, 1024, 0, s>>>(a);
+        else if (a.E <= 512)
+            route_group_small_kernel<16><<<1, 1024, 0, s>>>(a);
+        else
+            route_group_small_kernel<32><<<1, 1024, 0, s>>>(a);
         return;
     }
     const int nchunks = (a.T + kRouteChunk - 1) / kRouteChunk;
-    route_kernel<<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist);
+    if (a.E <= 256)
+        route_kernel<8><<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist);
+    else if (a.E <= 512)
+        route_kernel<16><<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist);
+    else
+        route_kernel<32><<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist);
     scan_kernel<<<1, 1024, 0, s>>>(a.E, nchunks, a.split_rows, a.chunk_hist, a.counts, a.pad_offsets, a.rowblocks,
                                    a.num_rowblocks, a.sorted_pair, a.unit_counters);
     scatter_kernel<<<nchunks, 32, 0, s>>>(a.T, a.E, a.k, a.topk_ids, a.chunk_hist, a.sorted_pair, a.pos_of_pair);
@@ -355,10 +384,14 @@ void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s)
 void launch_gather(const __nv_bfloat16 *x, int P, int H, int k, const int32_t *pos_of_pair, uint8_t *aq,
                    uint8_t *asf, int act_rows, int act_mxfp8, int num_sms, cudaStream_t s)
 {
-    const long long work = (long long)P * (H / 32);
+    // encode each block once per token when that still fills the GPU, else once per pair
+    const long long token_blocks = (long long)(P / k) * (H / 32);
+    const int group = token_blocks >= (long long)num_sms * 1024 ? k : 1;
+    const long long work = token_blocks * (k / group);
     const long long want = (work + 255) / 256;
     const int grid = (int)(want < (long long)num_sms * 8 ? want : (long long)num_sms * 8);
-    gather_kernel<<<grid > 0 ? grid : 1, 256, 0, s>>>(x, P, H, k, pos_of_pair, aq, asf, act_rows, act_mxfp8);
+    gather_kernel<<<grid > 0 ? grid : 1, 256, 0, s>>>(x, P / k, H, k, group, pos_of_pair, aq, asf, act_rows,
+                                                      act_mxfp8);
 }
 
 void launch_combine(const float *Y, int T, int H, int k, const int32_t *pos_of_pair, const float *topk_w,
