@@ -72,12 +72,16 @@ constexpr int kRing = 4;
 // Shared-memory plan for a kernel whose activation tiles hold at most kActRows
 // rows per term: as many pipeline stages as fit (more stages = more bytes in
 // flight per SM, which is what the weight-streaming decode shapes need).
-template <int kActRows, int kMmaW> struct Plan {
+template <int kActRows, int kMmaW, int kWTiles> struct Plan {
     // first N row of the second activation term when both terms share one MMA (tokens on N)
     static constexpr int kT2 = kActRows < 64 ? kActRows : 64;
     static constexpr int kTermBytes = kActRows * kTermRowBytes;
     static constexpr int kActBytes = 2 * kTermBytes;
-    static constexpr int kStageBytes = kActBytes + kWBytes + kAsfBytes + kWsfBytes;
+    // weight tiles per work unit (1, or 2 adjacent 128-row tiles against one activation block:
+    // twice the weight bytes per stage for the same per-stage bookkeeping and activation copy)
+    static constexpr int kWT = kWTiles;
+    static constexpr int kWStage = kWT * kWBytes, kWsfStage = kWT * kWsfBytes;
+    static constexpr int kStageBytes = kActBytes + kWStage + kAsfBytes + kWsfStage;
     static constexpr int kStages = (kSmemLimit - 1024 - kXBytes - 256) / kStageBytes;
     // The per-stage copy issue is split over several producer warps (groups of two stages
     // round robin): each TMA instruction and each warp-wide 4-byte scale copy occupies its
@@ -97,13 +101,14 @@ template <int kActRows, int kMmaW> struct Plan {
     static constexpr int kMma = kMmaW;
     static_assert(kMma == 1 || kStages % 2 == 0, "alternating MMA warps need an even stage count");
     static_assert(kMma == 1 || kActRows <= 32, "two accumulators per buffer need N <= 64");
+    static_assert(kWT == 1 || (kWT == 2 && kMma == 1 && kActRows <= 32), "two weight tiles: one MMA warp, N <= 64");
     // warps: producer 0, MMA 0, 4 epilogue, producers 1.., MMA 1 (if any), the scheduler
     static constexpr int kThreads = 32 * (2 + 4 + (kProd - 1) + (kMma - 1) + 1);
     static constexpr int kOffAct = 0;
     static constexpr int kOffW = kOffAct + kStages * kActBytes;
-    static constexpr int kOffAsf = kOffW + kStages * kWBytes;
+    static constexpr int kOffAsf = kOffW + kStages * kWStage;
     static constexpr int kOffWsf = kOffAsf + kStages * kAsfBytes;
-    static constexpr int kOffX = kOffWsf + kStages * kWsfBytes;
+    static constexpr int kOffX = kOffWsf + kStages * kWsfStage;
     static constexpr int kOffBar = kOffX + kXBytes;
     static constexpr int kNumBars = 2 * kStages + 1 + 4 + 2 * kRing;
     static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
@@ -146,7 +151,7 @@ template <int kStages> struct UnitRing {
         return v;
     }
     // Scheduler (one lane): publish the CTA's j-th unit; false once the work is exhausted.
-    __device__ bool fill(uint32_t j, const FcGemmArgs &a, int total_units, unsigned long long tmo) const
+    __device__ bool fill(uint32_t j, const FcGemmArgs &a, int total_units, int n_groups, unsigned long long tmo) const
     {
         const int r = (int)(j % kRing);
         const bool got = mbar_wait_bounded(bars.ring_empty(r), ((j / kRing) & 1) ^ 1, a.err, tmo);
@@ -155,7 +160,7 @@ template <int kStages> struct UnitRing {
         if (u >= total_units)
             u = -1;
         if (u >= 0)
-            blk = a.rowblocks[u / a.n_tiles];
+            blk = a.rowblocks[u / n_groups];
         slots[4 * r] = blk.x;
         slots[4 * r + 1] = blk.y;
         slots[4 * r + 2] = blk.z;
@@ -250,7 +255,7 @@ struct Ctx {
     uint32_t base;        // shared-memory base (1024-byte aligned, shared window)
     volatile int *units;  // the work-unit ring (generic pointer to shared memory)
     uint32_t tmem_base;
-    int total_units, kst, terms;
+    int total_units, n_groups, kst, terms; // n_groups: work units per row block (tile groups)
     unsigned long long tmo;
 };
 
@@ -258,13 +263,13 @@ struct Ctx {
 // compile-time role index so that every operand of the TMA issue stays warp-uniform).
 // Consecutive stages come from different warps at nearly the same time, so the two 64-byte
 // halves of a weight row's 128-byte line are requested close together.
-template <int kActRows, int kMmaW, int PI>
+template <int kActRows, int kMmaW, int kWTiles, int PI>
 __device__ __forceinline__ void producer_role(const FcGemmArgs &a, const Ctx &c, const CUtensorMap *act_map,
                                               const CUtensorMap *act_map_sw, const CUtensorMap *act_map16,
                                               const CUtensorMap *w_map, int lane)
 {
-    using P = Plan<kActRows, kMmaW>;
-    constexpr int kStages = P::kStages, kProd = P::kProd;
+    using P = Plan<kActRows, kMmaW, kWTiles>;
+    constexpr int kStages = P::kStages, kProd = P::kProd, kWT = P::kWT;
     constexpr int kTermBytes = P::kTermBytes, kActBytes = P::kActBytes;
     constexpr int kOffAct = P::kOffAct, kOffW = P::kOffW, kOffAsf = P::kOffAsf, kOffWsf = P::kOffWsf;
     const Bars<kStages> bars{c.base + P::kOffBar};
@@ -279,14 +284,10 @@ __device__ __forceinline__ void producer_role(const FcGemmArgs &a, const Ctx &c,
         const int4 blk = ring.take(i, a.err, tmo, lane);
         if (blk.w < 0)
             break;
-        const int nt = blk.w % a.n_tiles;
+        const int nt0 = (blk.w % c.n_groups) * kWT; // the unit's first weight tile
         const bool swap = kActRows < 128 || blk.z <= a.swap_rows;
         const int npad = (blk.z + 15) & ~15;
         const bool comb = swap && terms > 1 && npad <= P::kT2; // both terms on N of one MMA
-        // weight rows of this tile, as two 64-row halves: FC1 tile nt = gate rows [64nt, 64nt+64)
-        // then the matching up rows; FC2 tile nt = rows [128nt, 128nt+128)
-        const int wrow_a = blk.x * a.R + (a.fc1 ? nt * 64 : nt * 128);
-        const int wrow_b = a.fc1 ? wrow_a + a.R / 2 : wrow_a + 64;
         const int rb = blk.y / 128, o = blk.y & 127;
         // tokens on N: one box of kT2 rows per term plane covers the block (both terms, one copy),
         // else (blocks beyond kT2 rows) 16-row boxes per term, term 2 kTermBytes further on
@@ -296,8 +297,10 @@ __device__ __forceinline__ void producer_role(const FcGemmArgs &a, const Ctx &c,
         // activation scales: one bulk copy of the two 128-row atoms (tokens on M), or 4-byte copies
         // of this block's rows into a stage atom laid out for N (tokens on N); weight scales: one
         // bulk copy (tiled layout) or 4-byte copies (row-major)
-        const uint32_t tx = act_bytes + kWTxBytes + (swap ? 0u : (uint32_t)terms * 512u) + (a.wsf_tiled ? 512u : 0u);
-        const uint8_t *wsf_tile = a.wscale + ((size_t)blk.x * a.n_tiles + nt) * (size_t)kst * 512;
+        const uint32_t tx = act_bytes + kWT * kWTxBytes + (swap ? 0u : (uint32_t)terms * 512u) +
+                            (a.wsf_tiled ? kWT * 512u : 0u);
+        // tiled weight scales: the first tile's atoms, one per K stage, then the next tile's
+        const uint8_t *wsf_tile = a.wscale + ((size_t)blk.x * a.n_tiles + nt0) * (size_t)kst * 512;
         for (int kk = 0; kk < kst; ++kk, ++g) {
             if ((int)(g % kProd) != PI)
                 continue; // another producer warp fills this stage
@@ -311,20 +314,24 @@ __device__ __forceinline__ void producer_role(const FcGemmArgs &a, const Ctx &c,
             // whole warp issues the 4-byte scale copies, if any.
             const uint32_t full_s = bars.full(s);
             const uint32_t act = base + kOffAct + s * kActBytes;
-            const uint32_t wdst = base + kOffW + s * kWBytes;
-            const uint32_t wsf = base + kOffWsf + s * kWsfBytes;
+            const uint32_t wdst = base + kOffW + s * P::kWStage;
+            const uint32_t wsf = base + kOffWsf + s * P::kWsfStage;
             const uint32_t asf_dst = base + kOffAsf + s * kAsfBytes;
             const uint8_t *asf_src = a.act_sf + ((size_t)rb * kst + kk) * 1024;
             const int kx = kk * 128;
             if (elect_one()) {
                 mbar_arrive_expect_tx(full_s, tx);
-                // FC1: gate and up halves of the 64-row slice in one box; FC2: one 128-row box
-                if (a.fc1)
-                    tma_load_3d(wdst, w_map, kx, nt * 64, 2 * blk.x, full_s);
-                else
-                    tma_load_2d(wdst, w_map, kx, wrow_a, full_s);
-                if (a.wsf_tiled)
-                    bulk_copy_g2s(wsf, wsf_tile + (size_t)kk * 512, 512u, full_s);
+                // per weight tile nt: FC1 = gate rows [64 nt, 64 nt + 64) and the matching up rows, one
+                // 3-D box; FC2 = rows [128 nt, 128 nt + 128), one box
+                for (int wt = 0; wt < kWT; ++wt) {
+                    const int nt = nt0 + wt;
+                    if (a.fc1)
+                        tma_load_3d(wdst + wt * kWBytes, w_map, kx, nt * 64, 2 * blk.x, full_s);
+                    else
+                        tma_load_2d(wdst + wt * kWBytes, w_map, kx, blk.x * a.R + nt * 128, full_s);
+                    if (a.wsf_tiled)
+                        bulk_copy_g2s(wsf + wt * kWsfBytes, wsf_tile + ((size_t)wt * kst + kk) * 512, 512u, full_s);
+                }
                 if (!swap) {
                     tma_load_3d(act, act_map, kx, blk.y, 0, full_s); // [terms][128 rows][128]
                     bulk_copy_g2s(asf_dst, asf_src, (uint32_t)terms * 512u, full_s);
@@ -340,9 +347,15 @@ __device__ __forceinline__ void producer_role(const FcGemmArgs &a, const Ctx &c,
             }
             __syncwarp();
             if (!a.wsf_tiled) // weight scale bytes: 4 per row (the stage's 4 blocks) into the atom layout
-                for (int r = lane; r < 128; r += 32) {
-                    const int wr = r < 64 ? wrow_a + r : wrow_b + (r - 64);
-                    cp_async_4(wsf + sf_atom_offset(r, 0), a.wscale + (size_t)wr * scl_ld + kk * 4);
+                for (int wt = 0; wt < kWT; ++wt) {
+                    const int nt = nt0 + wt;
+                    // tile rows as two 64-row halves: FC1 gate rows then the matching up rows
+                    const int wrow_a = blk.x * a.R + (a.fc1 ? nt * 64 : nt * 128);
+                    const int wrow_b = a.fc1 ? wrow_a + a.R / 2 : wrow_a + 64;
+                    for (int r = lane; r < 128; r += 32) {
+                        const int wr = r < 64 ? wrow_a + r : wrow_b + (r - 64);
+                        cp_async_4(wsf + wt * kWsfBytes + sf_atom_offset(r, 0), a.wscale + (size_t)wr * scl_ld + kk * 4);
+                    }
                 }
             if (swap) {
                 // row j of term t: from row o + j of the term's 128-row atom to N row t * kT2 + j of
@@ -367,24 +380,24 @@ __device__ __forceinline__ void producer_role(const FcGemmArgs &a, const Ctx &c,
 // Scheduler role (one warp, one lane works): takes the CTA's work units from the launch's
 // counter and publishes them kLook units ahead of the first reader, off the producers' path
 // (the counter is a global atomic: a round trip of about a microsecond per unit).
-template <int kActRows, int kMmaW>
+template <int kActRows, int kMmaW, int kWTiles>
 __device__ __forceinline__ void scheduler_role(const FcGemmArgs &a, const Ctx &c, int lane)
 {
-    using P = Plan<kActRows, kMmaW>;
+    using P = Plan<kActRows, kMmaW, kWTiles>;
     const UnitRing<P::kStages> ring{Bars<P::kStages>{c.base + P::kOffBar}, c.units};
     if (lane == 0)
-        for (uint32_t j = 0; ring.fill(j, a, c.total_units, c.tmo); ++j) {
+        for (uint32_t j = 0; ring.fill(j, a, c.total_units, c.n_groups, c.tmo); ++j) {
         }
     __syncwarp();
 }
 
 // MMA role: warp 1 (MI = 0) and, with kMma = 2, warp 7 (MI = 1), taking stages g with
 // g % kMma == MI.  The whole warp runs the loop, one elected lane issues.
-template <int kActRows, int kMmaW, int MI>
+template <int kActRows, int kMmaW, int kWTiles, int MI>
 __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
 {
-    using P = Plan<kActRows, kMmaW>;
-    constexpr int kStages = P::kStages, kMma = P::kMma;
+    using P = Plan<kActRows, kMmaW, kWTiles>;
+    constexpr int kStages = P::kStages, kMma = P::kMma, kWT = P::kWT;
     constexpr int kTermBytes = P::kTermBytes, kActBytes = P::kActBytes;
     constexpr int kOffAct = P::kOffAct, kOffW = P::kOffW, kOffAsf = P::kOffAsf, kOffWsf = P::kOffWsf;
     const Bars<kStages> bars{c.base + P::kOffBar};
@@ -393,8 +406,10 @@ __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
     const unsigned long long tmo = c.tmo;
     uint32_t g = 0, cnt = 0;
     bool ok = true;
-    // this warp's scale-factor columns: the weight atom at +0, the activation atoms at +4 and +8
+    // this warp's scale-factor columns: the weight atoms at +0 (and +4 for a second tile), then
+    // the activation atoms (one per term)
     const uint32_t sf_w = tmem_base + kSfCol + 16u * (uint32_t)MI;
+    const uint32_t sf_act = sf_w + 4u * kWT;
     // descriptors of stage slot 0, K block 0 (term 1 of the activations, and the weights)
     const uint64_t dact0 = smem_desc_sw128(base + kOffAct), dw0 = smem_desc_sw128(base + kOffW);
     static_assert(P::kSmemBytes + 1024 < (1 << 18), "descriptor start field arithmetic needs addresses < 2^18");
@@ -411,12 +426,16 @@ __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
         const bool t1 = !comb && terms > 1;
         const uint32_t idesc0 = swap ? idesc_mx(kFmtE2M1, kFmtE4M3, 128, comb ? P::kT2 + npad : npad, 0)
                                      : idesc_mx(kFmtE4M3, kFmtE2M1, 128, 128, 0);
-        uint32_t sfa[2], sfb[2];
+        // scale columns of each MMA: tokens on N -> A = weight tile wt, B = activation term t;
+        // tokens on M (one weight tile) -> A = activation term t, B = the weight tile
+        uint32_t sfa[kWT][2], sfb[kWT][2];
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            sfa[t] = swap ? sf_w : sf_w + 4 + 4 * t;
-            sfb[t] = swap ? sf_w + 4 + 4 * t : sf_w;
-        }
+        for (int wt = 0; wt < kWT; ++wt)
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                sfa[wt][t] = swap ? sf_w + 4 * wt : sf_act + 4 * t;
+                sfb[wt][t] = swap ? sf_act + 4 * t : sf_w + 4 * wt;
+            }
         const int buf = cnt & 1;
         if (!__all_sync(0xFFFFFFFFu,
                         mbar_wait_bounded(bars.acc_empty(buf), ((cnt >> 1) & 1) ^ 1, a.err, tmo))) {
@@ -424,7 +443,8 @@ __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
             break;
         }
         tc_fence_after();
-        // accumulator: one per buffer, or one per buffer and MMA warp (64 columns apart)
+        // accumulator: one per buffer, or (64 columns apart) one per buffer and MMA warp or per
+        // buffer and weight tile
         const uint32_t d = tmem_base + buf * 128 + (kMma > 1 ? 64u * (uint32_t)MI : 0u);
         bool first = true; // this warp's first stage of the unit initialises its accumulator
         for (int kk = 0; kk < kst; ++kk, ++g) {
@@ -435,25 +455,28 @@ __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
             // The stage's operands are computed by the whole warp before the wait; then one elected
             // lane issues the scale copies, MMAs and commit back to back (measured: an elect /
             // reconverge around each instruction costs more than the instruction itself).
-            const uint32_t wsf_s = base + kOffWsf + s * kWsfBytes;
+            const uint32_t wsf_s = base + kOffWsf + s * P::kWsfStage;
             const uint32_t asf_s = base + kOffAsf + s * kAsfBytes;
             // descriptors are affine in the address: the start field is address / 16 in the low
             // 14 bits, and every shared-memory address here stays below 2^18
             const uint64_t ds_act = dact0 + (uint64_t)((s * kActBytes) >> 4);
-            const uint64_t ds_w = dw0 + (uint64_t)((s * kWBytes) >> 4);
-            uint64_t opa[4][2], opb[4][2];
+            const uint64_t ds_w = dw0 + (uint64_t)((s * P::kWStage) >> 4);
+            uint64_t opa[4][kWT][2], opb[4][kWT][2];
             uint32_t idesc[4], accf[4];
 #pragma unroll
             for (int k32 = 0; k32 < 4; ++k32) {
                 // the scale-factor byte of this 32-element block sits in both sf-id fields
                 idesc[k32] = idesc0 | ((uint32_t)k32 << 4) | ((uint32_t)k32 << 29);
                 accf[k32] = (first && k32 == 0) ? 0u : 1u;
-                const uint64_t dw = ds_w + 2u * k32; // +32 bytes per 32-element K block
 #pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    const uint64_t da = ds_act + (uint64_t)((t * kTermBytes) >> 4) + 2u * k32;
-                    opa[k32][t] = swap ? dw : da;
-                    opb[k32][t] = swap ? da : dw;
+                for (int wt = 0; wt < kWT; ++wt) {
+                    const uint64_t dw = ds_w + (uint64_t)((wt * kWBytes) >> 4) + 2u * k32; // +32 bytes per K block
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        const uint64_t da = ds_act + (uint64_t)((t * kTermBytes) >> 4) + 2u * k32;
+                        opa[k32][wt][t] = swap ? dw : da;
+                        opb[k32][wt][t] = swap ? da : dw;
+                    }
                 }
             }
             const uint32_t empty_s = bars.empty(s);
@@ -464,16 +487,22 @@ __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
             tc_fence_after();
             if (elect_one()) {
                 // scale atoms -> TMEM (in order with the MMAs below and with the previous stage's MMAs)
-                tmem_cp_sf_atom(sf_w, wsf_s);
-                tmem_cp_sf_atom(sf_w + 4, asf_s);
-                if (t1)
-                    tmem_cp_sf_atom(sf_w + 8, asf_s + 512);
 #pragma unroll
-                for (int k32 = 0; k32 < 4; ++k32) {
-                    umma_mx(d, opa[k32][0], opb[k32][0], idesc[k32], sfa[0], sfb[0], accf[k32]);
-                    if (t1)
-                        umma_mx(d, opa[k32][1], opb[k32][1], idesc[k32], sfa[1], sfb[1], 1u);
-                }
+                for (int wt = 0; wt < kWT; ++wt)
+                    tmem_cp_sf_atom(sf_w + 4 * wt, wsf_s + wt * kWsfBytes);
+                tmem_cp_sf_atom(sf_act, asf_s);
+                if (t1)
+                    tmem_cp_sf_atom(sf_act + 4, asf_s + 512);
+#pragma unroll
+                for (int k32 = 0; k32 < 4; ++k32)
+#pragma unroll
+                    for (int wt = 0; wt < kWT; ++wt) {
+                        umma_mx(d + 64u * wt, opa[k32][wt][0], opb[k32][wt][0], idesc[k32], sfa[wt][0], sfb[wt][0],
+                                accf[k32]);
+                        if (t1)
+                            umma_mx(d + 64u * wt, opa[k32][wt][1], opb[k32][wt][1], idesc[k32], sfa[wt][1],
+                                    sfb[wt][1], 1u);
+                    }
                 umma_commit(empty_s);
             }
             __syncwarp();
@@ -490,13 +519,13 @@ __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
     mbar_wait_bounded(bars.mma_done(), 0, nullptr, kDrainTimeoutNs);
 }
 
-template <int kActRows, int kMmaW>
-__global__ void __launch_bounds__(Plan<kActRows, kMmaW>::kThreads, 1)
+template <int kActRows, int kMmaW, int kWTiles>
+__global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles>::kThreads, 1)
     fc_gemm_kernel(const FcGemmArgs a, const __grid_constant__ CUtensorMap act_map,
                    const __grid_constant__ CUtensorMap act_map_sw, const __grid_constant__ CUtensorMap act_map16,
                    const __grid_constant__ CUtensorMap w_map)
 {
-    using P = Plan<kActRows, kMmaW>;
+    using P = Plan<kActRows, kMmaW, kWTiles>;
     constexpr int kStages = P::kStages;
     constexpr int kOffX = P::kOffX, kOffBar = P::kOffBar, kOffTmemSlot = P::kOffTmemSlot;
     constexpr int kProd = P::kProd, kMma = P::kMma;
@@ -539,28 +568,30 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW>::kThreads, 1)
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(gsm + kOffTmemSlot);
 
     const int nrb = *a.num_rowblocks;
-    const int total_units = nrb * a.n_tiles;
+    const int n_groups = a.n_tiles / P::kWT; // the launch guarantees n_tiles % kWT == 0
+    const int total_units = nrb * n_groups;
     const int kst = a.K / 128; // K stages of 128 elements (4 scale blocks)
     const int terms = a.terms; // activation terms per row: 1 (w4a8) or 2 (w4a16)
     const unsigned long long tmo = a.timeout_ns;
 
-    const Ctx ctx{base, reinterpret_cast<volatile int *>(gsm + P::kOffUnits), tmem_base, total_units, kst, terms, tmo};
+    const Ctx ctx{base, reinterpret_cast<volatile int *>(gsm + P::kOffUnits), tmem_base, total_units, n_groups, kst, terms,
+                  tmo};
     if (warp == 0) {
-        producer_role<kActRows, kMmaW, 0>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
+        producer_role<kActRows, kMmaW, kWTiles, 0>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
     } else if (warp >= 6 && warp < 5 + kProd) {
         // further producer warps (compile-time role index: every TMA operand stays warp-uniform)
         if (warp == 6)
-            producer_role<kActRows, kMmaW, 1 % kProd>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
+            producer_role<kActRows, kMmaW, kWTiles, 1 % kProd>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
         else if (warp == 7)
-            producer_role<kActRows, kMmaW, 2 % kProd>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
+            producer_role<kActRows, kMmaW, kWTiles, 2 % kProd>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
         else if (warp == 8)
-            producer_role<kActRows, kMmaW, 3 % kProd>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
+            producer_role<kActRows, kMmaW, kWTiles, 3 % kProd>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
     } else if (warp == 1) {
-        mma_role<kActRows, kMmaW, 0>(a, ctx);
+        mma_role<kActRows, kMmaW, kWTiles, 0>(a, ctx);
     } else if (kMma > 1 && warp == 5 + kProd) {
-        mma_role<kActRows, kMmaW, (kMma > 1 ? 1 : 0)>(a, ctx);
+        mma_role<kActRows, kMmaW, kWTiles, (kMma > 1 ? 1 : 0)>(a, ctx);
     } else if (warp == P::kThreads / 32 - 1) {
-        scheduler_role<kActRows, kMmaW>(a, ctx, lane);
+        scheduler_role<kActRows, kMmaW, kWTiles>(a, ctx, lane);
     } else if (warp >= 2 && warp < 6) {
         // ------------------------------------------------------------ epilogue (warps 2..5)
         const int q = warp & 3; // TMEM lane quarter this warp may access
@@ -571,7 +602,7 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW>::kThreads, 1)
             // the four epilogue warps leave together (they share named barriers below)
             if (!named_bar_all(2, 128, blk.w >= 0))
                 break;
-            const int nt = blk.w % a.n_tiles;
+            const int nt0 = (blk.w % n_groups) * P::kWT; // the unit's first weight tile
             const int rows = blk.z;
             const bool swap = kActRows < 128 || rows <= a.swap_rows;
             const int buf = cnt & 1;
@@ -582,7 +613,8 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW>::kThreads, 1)
             tc_fence_after();
             const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + buf * 128;
             if (!swap) {
-                // thread = one grouped row; TMEM columns = the tile's 128 weight rows
+                // thread = one grouped row; TMEM columns = the tile's 128 weight rows (one tile)
+                const int nt = nt0;
                 const int rl = 32 * q + lane;
                 const bool valid = rl < rows;
                 const int row = blk.y + rl;
@@ -629,7 +661,9 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW>::kThreads, 1)
                 const uint32_t g0 = cnt * (uint32_t)kst;
                 const bool acc0 = kMma == 1 || kst > 1 || (g0 & 1) == 0;
                 const bool acc1 = kMma > 1 && (kst > 1 || (g0 & 1) == 1);
+                for (int wt = 0; wt < P::kWT; ++wt) // each weight tile of the unit (64 columns apart)
                 for (int n0 = 0; n0 < npad; n0 += 16) {
+                    const int nt = nt0 + wt;
                     float v[16];
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
@@ -639,7 +673,7 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW>::kThreads, 1)
                             continue;
                         for (int t = 0; t < (comb ? 2 : 1); ++t) {
                             uint32_t r[16];
-                            tmem_ld16(tb + 64 * w + (t ? P::kT2 : 0) + n0, r);
+                            tmem_ld16(tb + 64 * (w + wt) + (t ? P::kT2 : 0) + n0, r);
                             tmem_wait_ld();
 #pragma unroll
                             for (int j = 0; j < 16; ++j)
@@ -689,27 +723,28 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW>::kThreads, 1)
     }
 }
 
-template <int kActRows, int kMmaW> static cudaError_t prepare_one()
+template <int kActRows, int kMmaW, int kWTiles> static cudaError_t prepare_one()
 {
-    return cudaFuncSetAttribute(fc_gemm_kernel<kActRows, kMmaW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                Plan<kActRows, kMmaW>::kSmemBytes);
+    return cudaFuncSetAttribute(fc_gemm_kernel<kActRows, kMmaW, kWTiles>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Plan<kActRows, kMmaW, kWTiles>::kSmemBytes);
 }
 
 cudaError_t fc_gemm_prepare()
 {
     cudaError_t e;
-    if ((e = prepare_one<16, 1>()) != cudaSuccess || (e = prepare_one<16, 2>()) != cudaSuccess ||
-        (e = prepare_one<32, 1>()) != cudaSuccess || (e = prepare_one<32, 2>()) != cudaSuccess ||
-        (e = prepare_one<64, 1>()) != cudaSuccess)
+    if ((e = prepare_one<16, 1, 1>()) != cudaSuccess || (e = prepare_one<16, 2, 1>()) != cudaSuccess ||
+        (e = prepare_one<16, 1, 2>()) != cudaSuccess || (e = prepare_one<32, 1, 1>()) != cudaSuccess ||
+        (e = prepare_one<32, 2, 1>()) != cudaSuccess || (e = prepare_one<32, 1, 2>()) != cudaSuccess ||
+        (e = prepare_one<64, 1, 1>()) != cudaSuccess)
         return e;
-    return prepare_one<128, 1>();
+    return prepare_one<128, 1, 1>();
 }
 
-template <int kActRows, int kMmaW>
+template <int kActRows, int kMmaW, int kWTiles>
 static void launch_one(const FcGemmArgs &a, const CUtensorMap &act_map, const CUtensorMap &act_map_sw,
                        const CUtensorMap &act_map16, const CUtensorMap &w_map, int grid, cudaStream_t s)
 {
-    fc_gemm_kernel<kActRows, kMmaW><<<grid, Plan<kActRows, kMmaW>::kThreads, Plan<kActRows, kMmaW>::kSmemBytes, s>>>(
+    fc_gemm_kernel<kActRows, kMmaW, kWTiles><<<grid, Plan<kActRows, kMmaW, kWTiles>::kThreads, Plan<kActRows, kMmaW, kWTiles>::kSmemBytes, s>>>(
         a, act_map, act_map_sw, act_map16, w_map);
 }
 
@@ -718,21 +753,28 @@ void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUten
 {
     // Row blocks of at most 16 / 32 / 64 rows run with their tokens on N; smaller activation
     // tiles leave room for more pipeline stages (bytes in flight) in the weight-streaming shapes.
-    // Two MMA warps for FC1's small-batch variants (long units), one for FC2 (measured).
+    // Small batches (tokens on N): FC1 with two MMA warps on alternate stages; FC2 (short
+    // units) with one MMA warp and two weight tiles per work unit when the tiles pair up.
+    // Each choice measured fastest on the decode shapes.
+    const bool wt2 = !a.fc1 && a.n_tiles % 2 == 0;
     if (a.max_block_rows <= 16) {
         if (a.fc1)
-            launch_one<16, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+            launch_one<16, 2, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+        else if (wt2)
+            launch_one<16, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
         else
-            launch_one<16, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+            launch_one<16, 1, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
     } else if (a.max_block_rows <= 32) {
         if (a.fc1)
-            launch_one<32, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+            launch_one<32, 2, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+        else if (wt2)
+            launch_one<32, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
         else
-            launch_one<32, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+            launch_one<32, 1, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
     } else if (a.max_block_rows <= 64) {
-        launch_one<64, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+        launch_one<64, 1, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
     } else {
-        launch_one<128, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+        launch_one<128, 1, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
     }
 }
 
