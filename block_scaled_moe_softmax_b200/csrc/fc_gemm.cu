@@ -72,11 +72,15 @@ constexpr int kRing = 4;
 // Shared-memory plan for a kernel whose activation tiles hold at most kActRows
 // rows per term: as many pipeline stages as fit (more stages = more bytes in
 // flight per SM, which is what the weight-streaming decode shapes need).
-template <int kActRows, int kMmaW, int kWTiles> struct Plan {
+template <int kActRows, int kMmaW, int kWTiles, int kTm> struct Plan {
     // first N row of the second activation term when both terms share one MMA (tokens on N)
     static constexpr int kT2 = kActRows < 64 ? kActRows : 64;
     static constexpr int kTermBytes = kActRows * kTermRowBytes;
-    static constexpr int kActBytes = 2 * kTermBytes;
+    // activation term planes a stage holds: 2 (the w4a16 split; any launch), or 1 for the
+    // variant that only takes single-term launches (w4a8 FC1), whose smaller stages leave room
+    // for more of them
+    static_assert(kTm == 1 || kTm == 2, "activation terms per stage");
+    static constexpr int kActBytes = kTm * kTermBytes;
     // weight tiles per work unit (1, or 2 adjacent 128-row tiles against one activation block:
     // twice the weight bytes per stage for the same per-stage bookkeeping and activation copy)
     static constexpr int kWT = kWTiles;
@@ -263,12 +267,12 @@ struct Ctx {
 // compile-time role index so that every operand of the TMA issue stays warp-uniform).
 // Consecutive stages come from different warps at nearly the same time, so the two 64-byte
 // halves of a weight row's 128-byte line are requested close together.
-template <int kActRows, int kMmaW, int kWTiles, int PI>
+template <int kActRows, int kMmaW, int kWTiles, int kTm, int PI>
 __device__ __forceinline__ void producer_role(const FcGemmArgs &a, const Ctx &c, const CUtensorMap *act_map,
                                               const CUtensorMap *act_map_sw, const CUtensorMap *act_map16,
                                               const CUtensorMap *w_map, int lane)
 {
-    using P = Plan<kActRows, kMmaW, kWTiles>;
+    using P = Plan<kActRows, kMmaW, kWTiles, kTm>;
     constexpr int kStages = P::kStages, kProd = P::kProd, kWT = P::kWT;
     constexpr int kTermBytes = P::kTermBytes, kActBytes = P::kActBytes;
     constexpr int kOffAct = P::kOffAct, kOffW = P::kOffW, kOffAsf = P::kOffAsf, kOffWsf = P::kOffWsf;
@@ -380,10 +384,10 @@ __device__ __forceinline__ void producer_role(const FcGemmArgs &a, const Ctx &c,
 // Scheduler role (one warp, one lane works): takes the CTA's work units from the launch's
 // counter and publishes them kLook units ahead of the first reader, off the producers' path
 // (the counter is a global atomic: a round trip of about a microsecond per unit).
-template <int kActRows, int kMmaW, int kWTiles>
+template <int kActRows, int kMmaW, int kWTiles, int kTm>
 __device__ __forceinline__ void scheduler_role(const FcGemmArgs &a, const Ctx &c, int lane)
 {
-    using P = Plan<kActRows, kMmaW, kWTiles>;
+    using P = Plan<kActRows, kMmaW, kWTiles, kTm>;
     const UnitRing<P::kStages> ring{Bars<P::kStages>{c.base + P::kOffBar}, c.units};
     if (lane == 0)
         for (uint32_t j = 0; ring.fill(j, a, c.total_units, c.n_groups, c.tmo); ++j) {
@@ -393,10 +397,10 @@ __device__ __forceinline__ void scheduler_role(const FcGemmArgs &a, const Ctx &c
 
 // MMA role: warp 1 (MI = 0) and, with kMma = 2, warp 7 (MI = 1), taking stages g with
 // g % kMma == MI.  The whole warp runs the loop, one elected lane issues.
-template <int kActRows, int kMmaW, int kWTiles, int MI>
+template <int kActRows, int kMmaW, int kWTiles, int kTm, int MI>
 __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
 {
-    using P = Plan<kActRows, kMmaW, kWTiles>;
+    using P = Plan<kActRows, kMmaW, kWTiles, kTm>;
     constexpr int kStages = P::kStages, kMma = P::kMma, kWT = P::kWT;
     constexpr int kTermBytes = P::kTermBytes, kActBytes = P::kActBytes;
     constexpr int kOffAct = P::kOffAct, kOffW = P::kOffW, kOffAsf = P::kOffAsf, kOffWsf = P::kOffWsf;
@@ -519,13 +523,13 @@ __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
     mbar_wait_bounded(bars.mma_done(), 0, nullptr, kDrainTimeoutNs);
 }
 
-template <int kActRows, int kMmaW, int kWTiles>
-__global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles>::kThreads, 1)
+template <int kActRows, int kMmaW, int kWTiles, int kTm>
+__global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads, 1)
     fc_gemm_kernel(const FcGemmArgs a, const __grid_constant__ CUtensorMap act_map,
                    const __grid_constant__ CUtensorMap act_map_sw, const __grid_constant__ CUtensorMap act_map16,
                    const __grid_constant__ CUtensorMap w_map)
 {
-    using P = Plan<kActRows, kMmaW, kWTiles>;
+    using P = Plan<kActRows, kMmaW, kWTiles, kTm>;
     constexpr int kStages = P::kStages;
     constexpr int kOffX = P::kOffX, kOffBar = P::kOffBar, kOffTmemSlot = P::kOffTmemSlot;
     constexpr int kProd = P::kProd, kMma = P::kMma;
@@ -571,27 +575,27 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles>::kThreads, 1)
     const int n_groups = a.n_tiles / P::kWT; // the launch guarantees n_tiles % kWT == 0
     const int total_units = nrb * n_groups;
     const int kst = a.K / 128; // K stages of 128 elements (4 scale blocks)
-    const int terms = a.terms; // activation terms per row: 1 (w4a8) or 2 (w4a16)
+    const int terms = kTm == 1 ? 1 : a.terms; // activation terms per row: 1 (w4a8) or 2 (w4a16)
     const unsigned long long tmo = a.timeout_ns;
 
     const Ctx ctx{base, reinterpret_cast<volatile int *>(gsm + P::kOffUnits), tmem_base, total_units, n_groups, kst, terms,
                   tmo};
     if (warp == 0) {
-        producer_role<kActRows, kMmaW, kWTiles, 0>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
+        producer_role<kActRows, kMmaW, kWTiles, kTm, 0>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
     } else if (warp >= 6 && warp < 5 + kProd) {
         // further producer warps (compile-time role index: every TMA operand stays warp-uniform)
         if (warp == 6)
-            producer_role<kActRows, kMmaW, kWTiles, 1 % kProd>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
+            producer_role<kActRows, kMmaW, kWTiles, kTm, 1 % kProd>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
         else if (warp == 7)
-            producer_role<kActRows, kMmaW, kWTiles, 2 % kProd>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
+            producer_role<kActRows, kMmaW, kWTiles, kTm, 2 % kProd>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
         else if (warp == 8)
-            producer_role<kActRows, kMmaW, kWTiles, 3 % kProd>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
+            producer_role<kActRows, kMmaW, kWTiles, kTm, 3 % kProd>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
     } else if (warp == 1) {
-        mma_role<kActRows, kMmaW, kWTiles, 0>(a, ctx);
+        mma_role<kActRows, kMmaW, kWTiles, kTm, 0>(a, ctx);
     } else if (kMma > 1 && warp == 5 + kProd) {
-        mma_role<kActRows, kMmaW, kWTiles, (kMma > 1 ? 1 : 0)>(a, ctx);
+        mma_role<kActRows, kMmaW, kWTiles, kTm, (kMma > 1 ? 1 : 0)>(a, ctx);
     } else if (warp == P::kThreads / 32 - 1) {
-        scheduler_role<kActRows, kMmaW, kWTiles>(a, ctx, lane);
+        scheduler_role<kActRows, kMmaW, kWTiles, kTm>(a, ctx, lane);
     } else if (warp >= 2 && warp < 6) {
         // ------------------------------------------------------------ epilogue (warps 2..5)
         const int q = warp & 3; // TMEM lane quarter this warp may access
@@ -723,28 +727,28 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles>::kThreads, 1)
     }
 }
 
-template <int kActRows, int kMmaW, int kWTiles> static cudaError_t prepare_one()
+template <int kActRows, int kMmaW, int kWTiles, int kTm> static cudaError_t prepare_one()
 {
-    return cudaFuncSetAttribute(fc_gemm_kernel<kActRows, kMmaW, kWTiles>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                Plan<kActRows, kMmaW, kWTiles>::kSmemBytes);
+    return cudaFuncSetAttribute(fc_gemm_kernel<kActRows, kMmaW, kWTiles, kTm>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Plan<kActRows, kMmaW, kWTiles, kTm>::kSmemBytes);
 }
 
 cudaError_t fc_gemm_prepare()
 {
     cudaError_t e;
-    if ((e = prepare_one<16, 1, 1>()) != cudaSuccess || (e = prepare_one<16, 2, 1>()) != cudaSuccess ||
-        (e = prepare_one<16, 1, 2>()) != cudaSuccess || (e = prepare_one<32, 1, 1>()) != cudaSuccess ||
-        (e = prepare_one<32, 2, 1>()) != cudaSuccess || (e = prepare_one<32, 1, 2>()) != cudaSuccess ||
-        (e = prepare_one<64, 1, 1>()) != cudaSuccess)
+    if ((e = prepare_one<16, 1, 1, 2>()) != cudaSuccess || (e = prepare_one<16, 2, 1, 2>()) != cudaSuccess ||
+        (e = prepare_one<16, 1, 2, 2>()) != cudaSuccess || (e = prepare_one<32, 1, 1, 2>()) != cudaSuccess ||
+        (e = prepare_one<32, 2, 1, 2>()) != cudaSuccess || (e = prepare_one<32, 1, 2, 2>()) != cudaSuccess ||
+        (e = prepare_one<64, 1, 1, 2>()) != cudaSuccess || (e = prepare_one<128, 1, 1, 2>()) != cudaSuccess)
         return e;
-    return prepare_one<128, 1, 1>();
+    return prepare_one<128, 1, 1, 1>();
 }
 
-template <int kActRows, int kMmaW, int kWTiles>
+template <int kActRows, int kMmaW, int kWTiles, int kTm>
 static void launch_one(const FcGemmArgs &a, const CUtensorMap &act_map, const CUtensorMap &act_map_sw,
                        const CUtensorMap &act_map16, const CUtensorMap &w_map, int grid, cudaStream_t s)
 {
-    fc_gemm_kernel<kActRows, kMmaW, kWTiles><<<grid, Plan<kActRows, kMmaW, kWTiles>::kThreads, Plan<kActRows, kMmaW, kWTiles>::kSmemBytes, s>>>(
+    fc_gemm_kernel<kActRows, kMmaW, kWTiles, kTm><<<grid, Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads, Plan<kActRows, kMmaW, kWTiles, kTm>::kSmemBytes, s>>>(
         a, act_map, act_map_sw, act_map16, w_map);
 }
 
@@ -759,22 +763,26 @@ void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUten
     const bool wt2 = !a.fc1 && a.n_tiles % 2 == 0;
     if (a.max_block_rows <= 16) {
         if (a.fc1)
-            launch_one<16, 2, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+            launch_one<16, 2, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
         else if (wt2)
-            launch_one<16, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+            launch_one<16, 1, 2, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
         else
-            launch_one<16, 1, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+            launch_one<16, 1, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
     } else if (a.max_block_rows <= 32) {
         if (a.fc1)
-            launch_one<32, 2, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+            launch_one<32, 2, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
         else if (wt2)
-            launch_one<32, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+            launch_one<32, 1, 2, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
         else
-            launch_one<32, 1, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+            launch_one<32, 1, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
     } else if (a.max_block_rows <= 64) {
-        launch_one<64, 1, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+        launch_one<64, 1, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+    } else if (a.terms == 1) {
+        // single-term activations (w4a8 FC1): the smaller stages leave room for 6 of them
+        // instead of 4, i.e. more bytes in flight per SM
+        launch_one<128, 1, 1, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
     } else {
-        launch_one<128, 1, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+        launch_one<128, 1, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
     }
 }
 

@@ -15,7 +15,7 @@ constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 32;
 constexpr int kBlockRows = 128;   // grouped-layout segment granularity = GEMM row block
 constexpr int kRouteChunk = 64;   // tokens per router CTA (= per histogram chunk)
-constexpr int kRouteThreads = 512;
+constexpr int kRouteThreads = 1024; // 32 warps: two tokens of a 64-token chunk per warp
 constexpr int kSmallRouteTokens = 64; // at most this many tokens: routing and grouping in one CTA
 
 struct RouteGroupArgs {

@@ -23,8 +23,8 @@ namespace moe_mx {
 
 // ---------------------------------------------------------------- router
 // Route one token (whole warp): the k experts in descending logit order, the lowest index
-// first among equal logits, and their weights = the softmax over the selected logits.  Lane 0
-// writes ids and weights and adds the selections to the block's expert histogram.
+// first among equal logits, and their weights = the softmax over the selected logits.  Lane j
+// (j < k) writes the j-th id and weight and adds it to the block's expert histogram.
 template <int kPerLane> // experts per lane: E <= 32 * kPerLane
 __device__ __forceinline__ void route_token(const float *__restrict__ row, int E, int k, int t, int lane,
                                             int32_t *__restrict__ topk_ids, float *__restrict__ topk_w,
@@ -42,8 +42,9 @@ __device__ __forceinline__ void route_token(const float *__restrict__ row, int E
         if (e >= E)
             taken |= 1u << i; // out of range: never selectable
     }
-    float sel_logit[kMaxTopK];
-    int sel_id[kMaxTopK];
+    // selection j ends up in lane j (k <= 32), so the weights and the writes are lane-parallel
+    float my_logit = -INFINITY;
+    int my_id = 0;
     for (int j = 0; j < k; ++j) {
         // this lane's best untaken entry (entries are in ascending expert order)
         float bv = -INFINITY;
@@ -69,23 +70,23 @@ __device__ __forceinline__ void route_token(const float *__restrict__ row, int E
         }
         if ((bi & 31) == lane)
             taken |= 1u << (bi >> 5);
-        sel_logit[j] = bv;
-        sel_id[j] = bi;
+        if (lane == j) {
+            my_logit = bv;
+            my_id = bi;
+        }
     }
-    if (lane == 0) {
-        // softmax over the k selected logits == renormalised top-k of the full softmax
-        const float m = sel_logit[0];
-        float u[kMaxTopK];
-        float z = 0.f;
-        for (int j = 0; j < k; ++j) {
-            u[j] = expf(sel_logit[j] - m);
-            z += u[j];
-        }
-        for (int j = 0; j < k; ++j) {
-            topk_ids[(size_t)t * k + j] = sel_id[j];
-            topk_w[(size_t)t * k + j] = u[j] / z;
-            atomicAdd(&hist[sel_id[j]], 1);
-        }
+    // softmax over the k selected logits == renormalised top-k of the full softmax; the
+    // butterfly sum leaves the same z in every lane (each step adds a commutative pair)
+    const float m = __shfl_sync(0xFFFFFFFFu, my_logit, 0);
+    const float u = lane < k ? expf(my_logit - m) : 0.f;
+    float z = u;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        z += __shfl_xor_sync(0xFFFFFFFFu, z, off);
+    if (lane < k) {
+        topk_ids[(size_t)t * k + lane] = my_id;
+        topk_w[(size_t)t * k + lane] = u / z;
+        atomicAdd(&hist[my_id], 1);
     }
 }
 
@@ -151,6 +152,7 @@ __device__ __forceinline__ int scan_experts(int E, int split, int total, int32_t
     __syncthreads();
     const unsigned long long excl = incl - mine + (warp > 0 ? s_warp[warp - 1] : 0ull);
     const int excl_nb = (int)(excl >> 32), excl_nw = (int)(excl & 0xFFFFFFFFull);
+    __shared__ int2 s_pad[kMaxExperts]; // per expert: first padding row, padding rows
     if (e < E) {
         counts[e] = total;
         pad_offsets[e] = excl_nb * kBlockRows;
@@ -160,8 +162,15 @@ __device__ __forceinline__ int scan_experts(int E, int split, int total, int32_t
         }
         for (int b = 0; b < nw; ++b)
             rowblocks[excl_nw + b] = make_int4(e, excl_nb * kBlockRows + b * split, min(split, total - b * split), 0);
-        for (int r = total; r < nb * kBlockRows; ++r)
-            sorted_pair[excl_nb * kBlockRows + r] = -1;
+        s_pad[e] = make_int2(excl_nb * kBlockRows + total, nb * kBlockRows - total);
+    }
+    __syncthreads();
+    // padding markers, one warp per expert: consecutive lanes write consecutive rows (one thread
+    // per expert writing its own padding would issue a separate memory transaction per row)
+    for (int x = warp; x < E; x += (int)(blockDim.x >> 5)) {
+        const int2 pd = s_pad[x];
+        for (int r = lane; r < pd.y; r += 32)
+            sorted_pair[pd.x + r] = -1;
     }
     return excl_nb * kBlockRows;
 }
@@ -179,10 +188,20 @@ __global__ void __launch_bounds__(1024) scan_kernel(int E, int nchunks, int spli
         unit_counters[e] = 0;
     int total = 0;
     if (e < E) {
-        for (int c = 0; c < nchunks; ++c) {
-            const int h = chunk_hist[(size_t)c * E + e];
-            chunk_hist[(size_t)c * E + e] = total; // exclusive prefix within the expert
-            total += h;
+        // exclusive prefix within the expert over the chunks; the loads go out in groups of
+        // kBatch so that their latencies overlap
+        constexpr int kBatch = 16;
+        for (int c0 = 0; c0 < nchunks; c0 += kBatch) {
+            int h[kBatch];
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i)
+                h[i] = c0 + i < nchunks ? chunk_hist[(size_t)(c0 + i) * E + e] : 0;
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) {
+                if (c0 + i < nchunks)
+                    chunk_hist[(size_t)(c0 + i) * E + e] = total;
+                total += h[i];
+            }
         }
     }
     const int base = scan_experts(E, split, total, counts, pad_offsets, rowblocks, num_rowblocks, sorted_pair, s_warp);
