@@ -16,6 +16,9 @@ function states the passage of the pages it follows in the C source:
 * FC1 -> SwiGLU -> FC2 -> weighted combine with MXFP4 weights
   (tokenspeed-situ description, intro, "Supported contract", "Activation
   precision (w4a16 vs w4a8)"; mxfp6-sm120 description, "Execution model");
+* the same layer with the routing given (precomputed top-k, global expert ids)
+  for one contiguous local expert shard, whose partial outputs add up to the
+  layer (tokenspeed-situ description, "Supported contract");
 * MX codecs per the OCP Microscaling Formats v1.0 specification.
 
 Parity pins (what ties this oracle to something other than itself) are in
@@ -81,6 +84,8 @@ def _load():
         lib.oracle_group.restype = None
         lib.oracle_moe_forward.argtypes = [i32] * 6 + [P] * 6 + [P, i32, P, P, P, P, i32]
         lib.oracle_moe_forward.restype = i32
+        lib.oracle_moe_forward_routed.argtypes = [i32] * 6 + [P, P, P, i32] + [P] * 4 + [P, i32, P, P, P, P, i32]
+        lib.oracle_moe_forward_routed.restype = i32
         _lib = lib
         return lib
 
@@ -211,6 +216,43 @@ def moe_forward(x_bf16_bits: np.ndarray, logits: np.ndarray, w1: np.ndarray, w1s
     if exact:
         return out, ids, w, out_exact
     return out, ids, w
+
+
+def moe_forward_routed(x_bf16_bits: np.ndarray, topk_ids: np.ndarray, topk_w: np.ndarray, local_offset: int,
+                       w1: np.ndarray, w1s: np.ndarray, w2: np.ndarray, w2s: np.ndarray,
+                       act_mode: int = ACT_BF16, tokens=None, nthreads: int | None = None):
+    """Evaluate the layer per token with the routing given (precomputed top-k, global ids).
+
+    topk_ids i32 [T, k] global expert ids, topk_w f32 [T, k]; the weights w1..w2s hold the
+    local shard of E experts, global ids [local_offset, local_offset + E).  Pairs outside the
+    shard contribute nothing (the result is the shard's partial output).
+    Returns (out bf16 bits uint16 [n, H], exact float64 [n, H], local ids i32 [n, k] (-1: not local)).
+    """
+    x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+    ids = np.ascontiguousarray(topk_ids, dtype=np.int32)
+    tw = np.ascontiguousarray(topk_w, dtype=np.float32)
+    T, H = x.shape
+    k = ids.shape[1]
+    E = w1.shape[0]
+    I = w2.shape[2] * 2
+    for a in (w1, w1s, w2, w2s):
+        assert a.dtype == np.uint8 and a.flags["C_CONTIGUOUS"]
+    assert ids.shape == (T, k) and tw.shape == (T, k)
+    assert w1.shape == (E, 2 * I, H // 2) and w1s.shape == (E, 2 * I, H // 32)
+    assert w2.shape == (E, H, I // 2) and w2s.shape == (E, H, I // 32)
+    tok_arr = None if tokens is None else np.ascontiguousarray(tokens, dtype=np.int32)
+    n = T if tok_arr is None else int(tok_arr.shape[0])
+    out = np.empty((n, H), dtype=np.uint16)
+    out_exact = np.empty((n, H), dtype=np.float64)
+    ids_loc = np.empty((n, k), dtype=np.int32)
+    w_out = np.empty((n, k), dtype=np.float32)
+    rc = _load().oracle_moe_forward_routed(
+        T, H, I, E, k, act_mode, _ptr(x), _ptr(ids), _ptr(tw), int(local_offset), _ptr(w1), _ptr(w1s), _ptr(w2),
+        _ptr(w2s), _ptr(tok_arr) if tok_arr is not None else None, n, _ptr(out), _ptr(ids_loc), _ptr(w_out),
+        _ptr(out_exact), nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_moe_forward_routed rejected its arguments")
+    return out, out_exact, ids_loc
 
 
 def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:

@@ -369,7 +369,10 @@ void oracle_group(int T, int k, int E, const int32_t *ids, int32_t *counts, int3
 typedef struct {
     int T, H, I, E, k, act_mode;
     const uint16_t *x;
-    const float *logits;
+    const float *logits;        /* router logits [T,E], or NULL when the routing is given: */
+    const int32_t *given_ids;   /* [T,k] global expert ids (routed form), */
+    const float *given_w;       /* [T,k] their weights, */
+    int local_offset;           /* and the first global id of the local experts [0,E) */
     const uint8_t *w1, *w1s, *w2, *w2s;
     const int32_t *tokens;
     uint16_t *out;
@@ -407,7 +410,18 @@ static void forward_token(const fwd_job *jb, int64_t slot)
     const int t = jb->tokens ? jb->tokens[slot] : (int)slot;
     int32_t ids[1024];
     float w[1024];
-    oracle_route(jb->logits + (int64_t)t * E, E, k, ids, w);
+    if (jb->logits) {
+        oracle_route(jb->logits + (int64_t)t * E, E, k, ids, w);
+    } else {
+        /* routed form: global ids; only the experts of the local shard [offset, offset + E)
+         * contribute, so the result is this shard's partial output */
+        for (int j = 0; j < k; ++j) {
+            const int64_t g = jb->given_ids[(int64_t)t * k + j];
+            const int64_t off = ORACLE_PLANT_MISTAKE == 10 ? 0 : jb->local_offset; /* plant: offset ignored */
+            ids[j] = (g >= off && g < off + E) ? (int32_t)(g - off) : -1;
+            w[j] = jb->given_w[(int64_t)t * k + j];
+        }
+    }
     if (jb->ids_out)
         memcpy(jb->ids_out + slot * k, ids, sizeof(int32_t) * (size_t)k);
     if (jb->w_out)
@@ -423,6 +437,8 @@ static void forward_token(const fwd_job *jb, int64_t slot)
 
     for (int j = 0; j < k - (ORACLE_PLANT_MISTAKE == 7); ++j) { /* plant: last slot dropped */
         const int64_t e = ids[j];
+        if (e < 0)
+            continue; /* routed form: an expert outside the local shard */
         const int64_t r1 = e * 2 * I; /* first W1 row of expert e */
         for (int i = 0; i < I; ++i) {
             double g = 0.0, u = 0.0;
@@ -482,12 +498,12 @@ static void *forward_worker(void *arg)
  * [0,I), up rows [I,2I)), w1s [E,2I,H/32]; w2 codes [E,H,I/2], w2s [E,H,I/32].
  * Returns 0, or -1 on bad arguments.
  */
-int oracle_moe_forward(int T, int H, int I, int E, int k, int act_mode, const uint16_t *x,
-                       const float *logits, const uint8_t *w1, const uint8_t *w1s, const uint8_t *w2,
-                       const uint8_t *w2s, const int32_t *tokens, int n_eval, uint16_t *out,
-                       int32_t *ids_out, float *w_out, double *out_exact, int nthreads)
+static int run_forward(int T, int H, int I, int E, int k, int act_mode, const uint16_t *x, const float *logits,
+                       const int32_t *given_ids, const float *given_w, int local_offset, const uint8_t *w1,
+                       const uint8_t *w1s, const uint8_t *w2, const uint8_t *w2s, const int32_t *tokens, int n_eval,
+                       uint16_t *out, int32_t *ids_out, float *w_out, double *out_exact, int nthreads)
 {
-    if (T < 0 || H <= 0 || I <= 0 || H % 32 || I % 32 || E < 1 || E > 1024 || k < 1 || k > E ||
+    if (T < 0 || H <= 0 || I <= 0 || H % 32 || I % 32 || E < 1 || E > 1024 || k < 1 || k > 1024 || (logits && k > E) ||
         (act_mode != 0 && act_mode != 1) || n_eval < 0 || !out)
         return -1;
     if (n_eval == 0)
@@ -504,8 +520,9 @@ int oracle_moe_forward(int T, int H, int I, int E, int k, int act_mode, const ui
     pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
     fwd_job *jobs = (fwd_job *)malloc(sizeof(fwd_job) * (size_t)nthreads);
     for (int i = 0; i < nthreads; ++i) {
-        jobs[i] = (fwd_job){T, H, I, E, k, act_mode, x, logits, w1, w1s, w2, w2s, tokens, out, out_exact, ids_out,
-                            w_out, (int64_t)n_eval * i / nthreads, (int64_t)n_eval * (i + 1) / nthreads};
+        jobs[i] = (fwd_job){T, H, I, E, k, act_mode, x, logits, given_ids, given_w, local_offset, w1, w1s, w2, w2s,
+                            tokens, out, out_exact, ids_out, w_out, (int64_t)n_eval * i / nthreads,
+                            (int64_t)n_eval * (i + 1) / nthreads};
         pthread_create(&th[i], NULL, forward_worker, &jobs[i]);
     }
     for (int i = 0; i < nthreads; ++i)
@@ -513,4 +530,39 @@ int oracle_moe_forward(int T, int H, int I, int E, int k, int act_mode, const ui
     free(th);
     free(jobs);
     return 0;
+}
+
+int oracle_moe_forward(int T, int H, int I, int E, int k, int act_mode, const uint16_t *x,
+                       const float *logits, const uint8_t *w1, const uint8_t *w1s, const uint8_t *w2,
+                       const uint8_t *w2s, const int32_t *tokens, int n_eval, uint16_t *out,
+                       int32_t *ids_out, float *w_out, double *out_exact, int nthreads)
+{
+    if (!logits)
+        return -1;
+    return run_forward(T, H, I, E, k, act_mode, x, logits, NULL, NULL, 0, w1, w1s, w2, w2s, tokens, n_eval, out,
+                       ids_out, w_out, out_exact, nthreads);
+}
+
+/*
+ * The layer with the routing given instead of the router logits (precomputed,
+ * unpacked top-k: global expert ids and their weights), for the local expert
+ * shard [local_offset, local_offset + E) whose weights w1..w2s hold [E, ...].
+ * Pairs routed to experts outside the shard contribute nothing, so the output
+ * is the shard's partial sum; the partial outputs of all shards add up to the
+ * whole layer.  [tokenspeed-situ package description, "Supported contract":
+ * precomputed top-k routing, global expert ids, contiguous local expert shards
+ * with a local expert offset, partial outputs that the caller all-reduces]
+ * ids_out receives the local ids (-1: not in the shard), w_out the weights.
+ * Returns 0, or -1 on bad arguments.
+ */
+int oracle_moe_forward_routed(int T, int H, int I, int E, int k, int act_mode, const uint16_t *x,
+                              const int32_t *topk_ids, const float *topk_w, int local_offset, const uint8_t *w1,
+                              const uint8_t *w1s, const uint8_t *w2, const uint8_t *w2s, const int32_t *tokens,
+                              int n_eval, uint16_t *out, int32_t *ids_out, float *w_out, double *out_exact,
+                              int nthreads)
+{
+    if (!topk_ids || !topk_w || k > 1024)
+        return -1;
+    return run_forward(T, H, I, E, k, act_mode, x, NULL, topk_ids, topk_w, local_offset, w1, w1s, w2, w2s, tokens,
+                       n_eval, out, ids_out, w_out, out_exact, nthreads);
 }

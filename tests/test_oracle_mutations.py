@@ -24,6 +24,7 @@ PLANTS = [
     (7, "last routed slot dropped", "tests/test_oracle_layer.py"),
     (8, "weights not renormalised", "tests/test_oracle_routing.py"),
     (9, "grouping not stable", "tests/test_oracle_routing.py"),
+    (10, "given routing: local expert offset ignored", "tests/test_oracle_routed.py"),
 ]
 
 
