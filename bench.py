@@ -73,8 +73,13 @@ def measured_peaks():
 
 
 def workload_desc(wl):
+    if wl.routing == "given":
+        route = (f"precomputed top-k over {wl.experts_global or wl.E} experts, local shard "
+                 f"[{wl.local_offset}, {wl.local_offset + wl.E})")
+    else:
+        route = f"logit bias {wl.bias}"
     return (f"{wl.name}: T={wl.T} H={wl.H} I={wl.I} E={wl.E} top-{wl.top_k} "
-            f"{'w4a8' if wl.act == 'mxfp8' else 'w4a16'}, logit bias {wl.bias}")
+            f"{'w4a8' if wl.act == 'mxfp8' else 'w4a16'}, {route}")
 
 
 # ------------------------------------------------------------------ inputs
@@ -191,31 +196,44 @@ def max_over_ranks(v, world):
 
 
 # ------------------------------------------------------------------ CPU oracle timing
-def oracle_time_tokens(wl, xb, logits_np, wq, tokens, nthreads):
+def oracle_time_tokens(wl, xb, route_np, wq, tokens, nthreads):
     import oracle
+    act = 1 if wl.act == "mxfp8" else 0
     t0 = time.perf_counter()
-    oracle.moe_forward(xb, logits_np, *wq, wl.top_k, 1 if wl.act == "mxfp8" else 0, tokens=tokens,
-                       nthreads=nthreads)
+    if wl.routing == "given":
+        ids, w = route_np
+        oracle.moe_forward_routed(xb, ids, w, wl.local_offset, *wq, act, tokens=tokens, nthreads=nthreads)
+    else:
+        oracle.moe_forward(xb, route_np, *wq, wl.top_k, act, tokens=tokens, nthreads=nthreads)
     return time.perf_counter() - t0
 
 
 def cpu_sample_setup(wl, sample_tokens):
+    """Host inputs for the oracle on a token sample: x, the routing input (logits, or given ids
+    and weights), oracle-quantised weights of the experts the sample reaches, those experts."""
     import oracle
-    logits = workloads.draw_logits(wl)
-    ids, _ = oracle.route(logits.numpy()[sample_tokens], wl.top_k)
-    experts = sorted(set(int(e) for e in ids.reshape(-1)))
+    if wl.routing == "given":
+        ids, w = (a.numpy() for a in workloads.draw_topk(wl))
+        loc = ids[sample_tokens] - wl.local_offset
+        experts = sorted(set(int(e) for e in loc.reshape(-1) if 0 <= e < wl.E))
+        route_np = (ids, w)
+    else:
+        logits = workloads.draw_logits(wl)
+        ids, _ = oracle.route(logits.numpy()[sample_tokens], wl.top_k)
+        experts = sorted(set(int(e) for e in ids.reshape(-1)))
+        route_np = logits.numpy()
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     wq = oracle_weights_for(wl, experts, dev)
     xb = workloads.bf16_bits(workloads.draw_x(wl))
-    return xb, logits.numpy(), wq, experts
+    return xb, route_np, wq, experts
 
 
 def cpu_baseline(wl, cores):
     """The oracle on a bounded sample (about 10-30 s of CPU work): a few tokens, one thread each."""
     n_tok = max(1, min(4, cores, wl.T))
     tokens = list(range(n_tok))
-    xb, logits_np, wq, experts = cpu_sample_setup(wl, tokens)
-    dt = oracle_time_tokens(wl, xb, logits_np, wq, tokens, n_tok)
+    xb, route_np, wq, experts = cpu_sample_setup(wl, tokens)
+    dt = oracle_time_tokens(wl, xb, route_np, wq, tokens, n_tok)
     return {"value": n_tok / dt, "unit": "tokens/s", "cores": n_tok, "kind": "oracle",
             "sample": f"tokens 0..{n_tok - 1} of the {wl.name} workload ({len(experts)} experts hit), "
                       f"one oracle call, {n_tok} threads, {dt:.1f} s wall"}
@@ -226,14 +244,14 @@ def run_reference(args, wl):
     up to `cores` concurrent steps (one thread each), so K steps take about K/cores token-times."""
     cores = len(os.sched_getaffinity(0))
     sample = list(range(min(wl.T, cores)))
-    xb, logits_np, wq, experts = cpu_sample_setup(wl, sample)
+    xb, route_np, wq, experts = cpu_sample_setup(wl, sample)
 
     def run_steps(n):
         done, wall = 0, 0.0
         while done < n:
             batch = min(cores, n - done)
             toks = [sample[(done + i) % len(sample)] for i in range(batch)]
-            wall += oracle_time_tokens(wl, xb, logits_np, wq, toks, batch)
+            wall += oracle_time_tokens(wl, xb, route_np, wq, toks, batch)
             done += batch
         return wall
 
@@ -312,7 +330,10 @@ def run_ours(args, wl):
     log(f"[rank {rank}] generating weights for {workload_desc(wl)}")
     w1, w1s, w2, w2s = make_gpu_weights(wl, dev)
     x = workloads.draw_x(wl).to(dev)
-    logits = workloads.draw_logits(wl).to(dev)
+    given = wl.routing == "given"
+    # the routing input: router logits, or the given top-k (global ids and weights)
+    route_host = workloads.draw_topk(wl) if given else (workloads.draw_logits(wl),)
+    route_in = tuple(a.to(dev) for a in route_host)
     out = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=dev)
     layer = moe_mx.MoeMxLayer(wl.H, wl.I, wl.E, wl.T, wl.top_k, device=dev.index)
     # weight preparation, once, like the quantisation: the E8M0 scales in the tiled layout
@@ -321,8 +342,15 @@ def run_ours(args, wl):
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
+    def forward(xin, rin):
+        if given:
+            moe_mx.moe_mx_forward_routed(layer.handle, xin, rin[0], rin[1], wl.T, wl.top_k, wl.local_offset, w1, w1s,
+                                         w2, w2s, act, out, moe_mx.MOE_MX_OUT_BF16, stream)
+        else:
+            moe_mx.moe_mx_forward(layer.handle, xin, rin[0], wl.T, w1, w1s, w2, w2s, wl.top_k, act, out, stream)
+
     def fwd():
-        moe_mx.moe_mx_forward(layer.handle, x, logits, wl.T, w1, w1s, w2, w2s, wl.top_k, act, out, stream)
+        forward(x, route_in)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -361,10 +389,10 @@ def run_ours(args, wl):
 
     # ---------------- end to end through the public API with host buffers
     x_h = workloads.draw_x(wl).pin_memory()
-    l_h = workloads.draw_logits(wl).pin_memory()
+    r_h = tuple(a.pin_memory() for a in route_host)
     o_h = torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory()
     x_d = torch.empty_like(x)
-    l_d = torch.empty_like(logits)
+    r_d = tuple(torch.empty_like(a) for a in route_in)
     e2e_steps = max(3, min(args.steps, 200))
     e2e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
     barrier(world)
@@ -373,8 +401,9 @@ def run_ours(args, wl):
         flush.zero_()
         e2e_evs[i][0].record(stream)
         x_d.copy_(x_h, non_blocking=True)
-        l_d.copy_(l_h, non_blocking=True)
-        moe_mx.moe_mx_forward(layer.handle, x_d, l_d, wl.T, w1, w1s, w2, w2s, wl.top_k, act, out, stream)
+        for dst, src in zip(r_d, r_h):
+            dst.copy_(src, non_blocking=True)
+        forward(x_d, r_d)
         o_h.copy_(out, non_blocking=True)
         e2e_evs[i][1].record(stream)
     torch.cuda.synchronize()
@@ -424,7 +453,8 @@ def run_ours(args, wl):
                          "a 512 MiB L2 flush before every timed step",
                    "weight_scales": "tiled layout (moe_mx_prepare_scales, once before timing)"},
         "e2e": {"value": world * wl.T / (e2e_ms / 1000.0), "unit": "tokens/s",
-                "h2d_bytes_per_step": wl.T * wl.H * 2 + wl.T * wl.E * 4, "d2h_bytes_per_step": wl.T * wl.H * 2},
+                "h2d_bytes_per_step": wl.T * wl.H * 2 + sum(a.numel() * a.element_size() for a in route_host),
+                "d2h_bytes_per_step": wl.T * wl.H * 2},
         "gpu_launches": kernels_per_forward(wl.T) * args.steps,
         "roofline": roofline,
         "layer_roofline": layer_roofline,

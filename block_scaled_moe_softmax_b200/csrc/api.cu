@@ -192,8 +192,8 @@ int moe_mx_create(moe_mx_handle **out, int hidden, int inter, int num_experts, i
         return fail(MOE_MX_ERR_UNSUPPORTED, "num_experts=%d must be in [1, %d]", num_experts, kMaxExperts);
     if (max_tokens < 1 || max_tokens > 65536)
         return fail(MOE_MX_ERR_INVALID_ARG, "max_tokens=%d must be in [1, 65536]", max_tokens);
-    if (max_top_k < 1 || max_top_k > num_experts || max_top_k > kMaxTopK)
-        return fail(MOE_MX_ERR_INVALID_ARG, "max_top_k=%d must be in [1, min(E, %d)]", max_top_k, kMaxTopK);
+    if (max_top_k < 1 || max_top_k > kMaxTopK)
+        return fail(MOE_MX_ERR_INVALID_ARG, "max_top_k=%d must be in [1, %d]", max_top_k, kMaxTopK);
     int ndev = 0;
     cudaError_t ce = cudaGetDeviceCount(&ndev);
     if (ce != cudaSuccess)
@@ -321,24 +321,39 @@ int moe_mx_destroy(moe_mx_handle *h)
     return MOE_MX_OK;
 }
 
-int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, int num_tokens, const uint8_t *w1,
-                   const uint8_t *w1_scale, const uint8_t *w2, const uint8_t *w2_scale, int top_k, int act_dtype,
-                   void *out, void *stream)
+namespace {
+
+// The forward of both entry points: routing computed from router_logits, or (given_ids set)
+// the given global ids and weights restricted to the shard [id_offset, id_offset + E).
+int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, const int32_t *given_ids,
+                 const float *given_w, int id_offset, int num_tokens, const uint8_t *w1, const uint8_t *w1_scale,
+                 const uint8_t *w2, const uint8_t *w2_scale, int top_k, int act_dtype, void *out, int out_f32,
+                 void *stream)
 {
     g_last_error.clear();
     if (!h)
         return fail(MOE_MX_ERR_INVALID_ARG, "handle is NULL");
     if (num_tokens < 0 || num_tokens > h->maxT)
         return fail(MOE_MX_ERR_INVALID_ARG, "num_tokens=%d must be in [0, %d]", num_tokens, h->maxT);
-    if (top_k < 1 || top_k > h->maxK || top_k > h->E)
+    if (!given_ids && (top_k < 1 || top_k > h->maxK || top_k > h->E))
         return fail(MOE_MX_ERR_INVALID_ARG, "top_k=%d must be in [1, min(E=%d, max_top_k=%d)]", top_k, h->E,
                     h->maxK);
+    if (given_ids && (top_k < 1 || top_k > h->maxK))
+        return fail(MOE_MX_ERR_INVALID_ARG, "top_k=%d must be in [1, max_top_k=%d]", top_k, h->maxK);
+    if (given_ids && id_offset < 0)
+        return fail(MOE_MX_ERR_INVALID_ARG, "local_expert_offset=%d must be >= 0", id_offset);
     if (act_dtype != MOE_MX_ACT_BF16 && act_dtype != MOE_MX_ACT_MXFP8)
         return fail(MOE_MX_ERR_INVALID_ARG, "act_dtype=%d is not MOE_MX_ACT_BF16 or MOE_MX_ACT_MXFP8", act_dtype);
     if (num_tokens == 0)
         return MOE_MX_OK;
     int rc;
-    if ((rc = check_ptr(x, h->dev, "x")) || (rc = check_ptr(router_logits, h->dev, "router_logits")) ||
+    if (given_ids) {
+        if ((rc = check_ptr(given_ids, h->dev, "topk_ids")) || (rc = check_ptr(given_w, h->dev, "topk_w")))
+            return rc;
+    } else if ((rc = check_ptr(router_logits, h->dev, "router_logits"))) {
+        return rc;
+    }
+    if ((rc = check_ptr(x, h->dev, "x")) ||
         (rc = check_ptr(w1, h->dev, "w1")) || (rc = check_ptr(w1_scale, h->dev, "w1_scale")) ||
         (rc = check_ptr(w2, h->dev, "w2")) || (rc = check_ptr(w2_scale, h->dev, "w2_scale")) ||
         (rc = check_ptr(out, h->dev, "out")))
@@ -394,6 +409,9 @@ int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, 
         RouteGroupArgs ra{router_logits, T, E, k, h->topk_ids, h->topk_w, h->chunk_hist, h->counts,
                           h->pad_offsets, h->rowblocks, h->num_rowblocks, h->sorted_pair, h->pos_of_pair,
                           tile_rows, h->unit_counters};
+        ra.given_ids = given_ids;
+        ra.given_w = given_w;
+        ra.id_offset = id_offset;
         launch_route_and_group(ra, s);
         mark(1);
         const int mx8 = act_dtype == MOE_MX_ACT_MXFP8;
@@ -443,7 +461,7 @@ int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, 
         launch_fc_gemm(f2, h->map_H[f2.terms - 1], h->map_Hsw[f2.terms - 1][sw_idx], h->map_H16, h->map_w2,
                        h->num_sms, s);
         mark(4);
-        launch_combine(h->Y, T, H, k, h->pos_of_pair, h->topk_w, static_cast<__nv_bfloat16 *>(out), h->num_sms, s);
+        launch_combine(h->Y, T, H, k, h->pos_of_pair, h->topk_w, out, out_f32, h->num_sms, s);
         ce = cudaGetLastError();
         if (ce != cudaSuccess) {
             rc = cuda_fail(ce, "kernel launch");
@@ -459,6 +477,33 @@ done:
     if (prev != h->dev)
         cudaSetDevice(prev);
     return rc;
+}
+
+} // namespace
+
+int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, int num_tokens, const uint8_t *w1,
+                   const uint8_t *w1_scale, const uint8_t *w2, const uint8_t *w2_scale, int top_k, int act_dtype,
+                   void *out, void *stream)
+{
+    return forward_impl(h, x, router_logits, nullptr, nullptr, 0, num_tokens, w1, w1_scale, w2, w2_scale, top_k,
+                        act_dtype, out, 0, stream);
+}
+
+int moe_mx_forward_routed(moe_mx_handle *h, const void *x, const int32_t *topk_ids, const float *topk_w,
+                          int num_tokens, int top_k, int local_expert_offset, const uint8_t *w1,
+                          const uint8_t *w1_scale, const uint8_t *w2, const uint8_t *w2_scale, int act_dtype,
+                          void *out, int out_dtype, void *stream)
+{
+    if (out_dtype != MOE_MX_OUT_BF16 && out_dtype != MOE_MX_OUT_F32) {
+        g_last_error.clear();
+        return fail(MOE_MX_ERR_INVALID_ARG, "out_dtype=%d is not MOE_MX_OUT_BF16 or MOE_MX_OUT_F32", out_dtype);
+    }
+    if (!topk_ids || !topk_w) {
+        g_last_error.clear();
+        return fail(MOE_MX_ERR_INVALID_ARG, "topk_ids and topk_w must not be NULL");
+    }
+    return forward_impl(h, x, nullptr, topk_ids, topk_w, local_expert_offset, num_tokens, w1, w1_scale, w2, w2_scale,
+                        top_k, act_dtype, out, out_dtype == MOE_MX_OUT_F32, stream);
 }
 
 int moe_mx_sync_status(moe_mx_handle *h, void *stream)

@@ -32,13 +32,20 @@ struct RouteGroupArgs {
     int32_t *pos_of_pair;
     int split_rows; // rows per work block of the row-block list: 16, 32, 64 or kBlockRows
     int32_t *unit_counters; // optional: the GEMMs' 2 work-unit counters, zeroed here
+    // Routing given instead of computed (logits unused): global expert ids [T, k] and their
+    // weights; ids in [id_offset, id_offset + E) are this shard's local experts, any other id
+    // is left out of the grouping (local id -1, pos_of_pair -1).
+    const int32_t *given_ids = nullptr;
+    const float *given_w = nullptr;
+    int id_offset = 0;
 };
 
 void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s);
 void launch_gather(const __nv_bfloat16 *x, int P, int H, int k, const int32_t *pos_of_pair, uint8_t *aq,
                    uint8_t *asf, int act_rows, int act_mxfp8, int num_sms, cudaStream_t s);
-void launch_combine(const float *Y, int T, int H, int k, const int32_t *pos_of_pair, const float *topk_w,
-                    __nv_bfloat16 *out, int num_sms, cudaStream_t s);
+// out: bf16 [T, H], or (out_f32) float32 [T, H]; pairs with pos_of_pair -1 add nothing
+void launch_combine(const float *Y, int T, int H, int k, const int32_t *pos_of_pair, const float *topk_w, void *out,
+                    int out_f32, int num_sms, cudaStream_t s);
 void launch_mx_quantize(const float *src, int64_t rows, int64_t K, int fmt, uint8_t *codes, uint8_t *scales,
                         int num_sms, cudaStream_t s);
 

@@ -90,13 +90,33 @@ __device__ __forceinline__ void route_token(const float *__restrict__ row, int E
     }
 }
 
+// The given routing of one token (whole warp; lane j takes slot j, k <= 32): global ids mapped
+// to the local shard (-1 outside it), weights copied, local experts added to the histogram.
+__device__ __forceinline__ void take_given_token(const int32_t *__restrict__ gids, const float *__restrict__ gw,
+                                                 int E, int k, int off, int t, int lane,
+                                                 int32_t *__restrict__ topk_ids, float *__restrict__ topk_w,
+                                                 int32_t *hist)
+{
+    if (lane < k) {
+        const size_t p = (size_t)t * k + lane;
+        const int g = __ldg(gids + p);
+        const bool local = g >= off && g - off < E; // g >= off >= 0: no overflow in g - off
+        topk_ids[p] = local ? g - off : -1;
+        topk_w[p] = __ldg(gw + p);
+        if (local)
+            atomicAdd(&hist[g - off], 1);
+    }
+}
+
 // One warp per token; each CTA covers kRouteChunk tokens and also writes the
 // per-expert histogram of its chunk (the first level of the counting sort).
 template <int kPerLane>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float *__restrict__ logits, int T, int E,
                                                                int k, int32_t *__restrict__ topk_ids,
                                                                float *__restrict__ topk_w,
-                                                               int32_t *__restrict__ chunk_hist)
+                                                               int32_t *__restrict__ chunk_hist,
+                                                               const int32_t *__restrict__ gids,
+                                                               const float *__restrict__ gw, int off)
 {
     __shared__ int32_t hist[kMaxExperts];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -105,8 +125,12 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float *__res
     __syncthreads();
     const int t_begin = blockIdx.x * kRouteChunk;
     const int t_end = min(T, t_begin + kRouteChunk);
-    for (int t = t_begin + warp; t < t_end; t += kRouteThreads / 32)
-        route_token<kPerLane>(logits + (size_t)t * E, E, k, t, lane, topk_ids, topk_w, hist);
+    for (int t = t_begin + warp; t < t_end; t += kRouteThreads / 32) {
+        if (gids)
+            take_given_token(gids, gw, E, k, off, t, lane, topk_ids, topk_w, hist);
+        else
+            route_token<kPerLane>(logits + (size_t)t * E, E, k, t, lane, topk_ids, topk_w, hist);
+    }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x)
         chunk_hist[(size_t)blockIdx.x * E + e] = hist[e];
@@ -220,19 +244,23 @@ __device__ __forceinline__ void scatter_pairs(int p_begin, int p_end, const int3
     for (int base = p_begin; base < p_end; base += 32) {
         const int p = base + lane;
         const bool valid = p < p_end;
-        const int e = valid ? topk_ids[p] : -1 - lane; // invalid lanes never match each other
+        const int e_raw = valid ? topk_ids[p] : -1;
+        const bool placed = e_raw >= 0; // -1: a pair outside the local expert shard (given routing)
+        const int e = placed ? e_raw : -1 - lane; // lanes not placed never match each other
         const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
         const int rank = __popc(peers & lt_mask);
         int row = 0;
-        if (valid)
+        if (placed)
             row = cursor[e] + rank;
         __syncwarp();
-        if (valid && (32 - __clz(peers)) - 1 == lane) // highest lane of the group advances the cursor
+        if (placed && (32 - __clz(peers)) - 1 == lane) // highest lane of the group advances the cursor
             cursor[e] += __popc(peers);
         __syncwarp();
-        if (valid) {
+        if (placed) {
             sorted_pair[row] = p;
             pos_of_pair[p] = row;
+        } else if (valid) {
+            pos_of_pair[p] = -1;
         }
     }
 }
@@ -251,8 +279,12 @@ __global__ void __launch_bounds__(1024) route_group_small_kernel(const RouteGrou
     if (a.unit_counters && threadIdx.x < 2)
         a.unit_counters[threadIdx.x] = 0;
     __syncthreads();
-    for (int t = warp; t < a.T; t += 32)
-        route_token<kPerLane>(a.logits + (size_t)t * a.E, a.E, a.k, t, lane, a.topk_ids, a.topk_w, hist);
+    for (int t = warp; t < a.T; t += 32) {
+        if (a.given_ids)
+            take_given_token(a.given_ids, a.given_w, a.E, a.k, a.id_offset, t, lane, a.topk_ids, a.topk_w, hist);
+        else
+            route_token<kPerLane>(a.logits + (size_t)t * a.E, a.E, a.k, t, lane, a.topk_ids, a.topk_w, hist);
+    }
     __syncthreads(); // also makes lane 0's id writes visible to the whole CTA
     const int e = threadIdx.x;
     const int total = e < a.E ? hist[e] : 0;
@@ -323,6 +355,8 @@ __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16 *__rest
         mx_encode32(v, act_mxfp8, c0, c1, s0, s1); // the values are bf16 already: no rounding step
         for (int j = jg * group; j < (jg + 1) * group; ++j) {
             const int row = pos_of_pair[(size_t)t * k + j];
+            if (row < 0)
+                continue; // not in the local expert shard
             store_codes32(aq + (size_t)row * H + b * 32, c0);
             asf[sf_atom_byte(row, b * 32, H, 0)] = (uint8_t)s0;
             if (!act_mxfp8) {
@@ -337,10 +371,10 @@ __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16 *__rest
 // out[t, n] = bf16( sum_{j<k} w[t,j] * Y[pos(t,j), n] ), j ascending, f32.
 // Y is kept in f32 so the only rounding of the result is the final one.
 // One thread per 8 consecutive outputs (2 x 16-byte loads per slot, one 16-byte store).
+template <bool kOutF32>
 __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ Y, int T, int H, int k,
                                                       const int32_t *__restrict__ pos_of_pair,
-                                                      const float *__restrict__ topk_w,
-                                                      __nv_bfloat16 *__restrict__ out)
+                                                      const float *__restrict__ topk_w, void *__restrict__ out)
 {
     const int vec_per_row = H / 8;
     const long long total = (long long)T * vec_per_row;
@@ -355,6 +389,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
         for (int j = 0; j < k; ++j) {
             const float w = __ldg(topk_w + (size_t)t * k + j);
             const int row = __ldg(pos_of_pair + (size_t)t * k + j);
+            if (row < 0)
+                continue; // a pair outside the local expert shard: no contribution
             const float4 *src = reinterpret_cast<const float4 *>(Y + (size_t)row * H) + 2 * c;
             const float4 a0 = __ldg(src), a1 = __ldg(src + 1);
             acc[0] = fmaf(w, a0.x, acc[0]);
@@ -366,12 +402,19 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
             acc[6] = fmaf(w, a1.z, acc[6]);
             acc[7] = fmaf(w, a1.w, acc[7]);
         }
-        uint4 o;
-        __nv_bfloat162 *o2 = reinterpret_cast<__nv_bfloat162 *>(&o);
+        if (kOutF32) {
+            // a shard's partial output, kept in float32 for the sum over shards
+            float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(out) + (size_t)t * H) + 2 * c;
+            dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        } else {
+            uint4 o;
+            __nv_bfloat162 *o2 = reinterpret_cast<__nv_bfloat162 *>(&o);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            o2[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-        reinterpret_cast<uint4 *>(out + (size_t)t * H)[c] = o;
+            for (int i = 0; i < 4; ++i)
+                o2[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+            reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + (size_t)t * H)[c] = o;
+        }
     }
 }
 
@@ -379,8 +422,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
 void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s)
 {
     // the top-k scan visits 32 * kPerLane candidates per token: size it to the expert count
+    // (the given routing visits no candidates: the smallest instance serves it)
+    const bool narrow = a.given_ids != nullptr || a.E <= 256;
     if (a.T <= kSmallRouteTokens) {
-        if (a.E <= 256)
+        if (narrow)
             route_group_small_kernel<8><<<1, 1024, 0, s>>>(a);
         else if (a.E <= 512)
             route_group_small_kernel<16><<<1, 1024, 0, s>>>(a);
@@ -389,12 +434,15 @@ void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s)
         return;
     }
     const int nchunks = (a.T + kRouteChunk - 1) / kRouteChunk;
-    if (a.E <= 256)
-        route_kernel<8><<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist);
+    if (narrow)
+        route_kernel<8><<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist,
+                                                          a.given_ids, a.given_w, a.id_offset);
     else if (a.E <= 512)
-        route_kernel<16><<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist);
+        route_kernel<16><<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist,
+                                                          a.given_ids, a.given_w, a.id_offset);
     else
-        route_kernel<32><<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist);
+        route_kernel<32><<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist,
+                                                          a.given_ids, a.given_w, a.id_offset);
     scan_kernel<<<1, 1024, 0, s>>>(a.E, nchunks, a.split_rows, a.chunk_hist, a.counts, a.pad_offsets, a.rowblocks,
                                    a.num_rowblocks, a.sorted_pair, a.unit_counters);
     scatter_kernel<<<nchunks, 32, 0, s>>>(a.T, a.E, a.k, a.topk_ids, a.chunk_hist, a.sorted_pair, a.pos_of_pair);
@@ -413,13 +461,16 @@ void launch_gather(const __nv_bfloat16 *x, int P, int H, int k, const int32_t *p
                                                       act_mxfp8);
 }
 
-void launch_combine(const float *Y, int T, int H, int k, const int32_t *pos_of_pair, const float *topk_w,
-                    __nv_bfloat16 *out, int num_sms, cudaStream_t s)
+void launch_combine(const float *Y, int T, int H, int k, const int32_t *pos_of_pair, const float *topk_w, void *out,
+                    int out_f32, int num_sms, cudaStream_t s)
 {
     const long long work = (long long)T * (H / 8);
     const long long want = (work + 255) / 256;
     const int grid = (int)(want < (long long)num_sms * 8 ? want : (long long)num_sms * 8);
-    combine_kernel<<<grid > 0 ? grid : 1, 256, 0, s>>>(Y, T, H, k, pos_of_pair, topk_w, out);
+    if (out_f32)
+        combine_kernel<true><<<grid > 0 ? grid : 1, 256, 0, s>>>(Y, T, H, k, pos_of_pair, topk_w, out);
+    else
+        combine_kernel<false><<<grid > 0 ? grid : 1, 256, 0, s>>>(Y, T, H, k, pos_of_pair, topk_w, out);
 }
 
 } // namespace moe_mx

@@ -27,6 +27,8 @@ MOE_MX_ERR_TIMEOUT = -4
 MOE_MX_ERR_NO_MEMORY = -5
 MOE_MX_ACT_BF16 = 0
 MOE_MX_ACT_MXFP8 = 1
+MOE_MX_OUT_BF16 = 0
+MOE_MX_OUT_F32 = 1
 MOE_MX_FMT_MXFP4 = 0
 MOE_MX_FMT_MXFP8 = 1
 MOE_MX_SCALES_ROW_MAJOR = 0
@@ -39,6 +41,7 @@ _P, _I, _I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
 SIGNATURES = {
     "moe_mx_create": (_I, [ctypes.POINTER(_P), _I, _I, _I, _I, _I, _I]),
     "moe_mx_forward": (_I, [_P, _P, _P, _I, _P, _P, _P, _P, _I, _I, _P, _P]),
+    "moe_mx_forward_routed": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _I, _P, _I, _P]),
     "moe_mx_destroy": (_I, [_P]),
     "moe_mx_last_error": (ctypes.c_char_p, []),
     "moe_mx_sync_status": (_I, [_P, _P]),
@@ -131,6 +134,14 @@ def moe_mx_forward(handle: int, x, router_logits, num_tokens: int, w1, w1_scale,
                                          _stream(stream)))
 
 
+def moe_mx_forward_routed(handle: int, x, topk_ids, topk_w, num_tokens: int, top_k: int, local_expert_offset: int,
+                          w1, w1_scale, w2, w2_scale, act_dtype: int, out, out_dtype: int = MOE_MX_OUT_BF16,
+                          stream=None) -> None:
+    _check(load_library().moe_mx_forward_routed(handle, _ptr(x), _ptr(topk_ids), _ptr(topk_w), num_tokens, top_k,
+                                                local_expert_offset, _ptr(w1), _ptr(w1_scale), _ptr(w2),
+                                                _ptr(w2_scale), act_dtype, _ptr(out), out_dtype, _stream(stream)))
+
+
 def moe_mx_sync_status(handle: int, stream=None) -> int:
     """Returns the status code (does not raise on MOE_MX_ERR_TIMEOUT)."""
     return load_library().moe_mx_sync_status(handle, _stream(stream))
@@ -197,6 +208,21 @@ class MoeMxLayer:
         if out is None:
             out = torch.empty(T, self.H, dtype=torch.bfloat16, device=x.device)
         moe_mx_forward(self.handle, x, router_logits, T, w1, w1_scale, w2, w2_scale, top_k, act_dtype, out, stream)
+        return out
+
+    def forward_routed(self, x: torch.Tensor, topk_ids: torch.Tensor, topk_w: torch.Tensor, w1, w1_scale, w2,
+                       w2_scale, local_expert_offset: int = 0, act_dtype: int = MOE_MX_ACT_BF16,
+                       out_dtype: int = MOE_MX_OUT_BF16, out: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+        """The layer with the routing given (global ids, weights) for the local shard of E experts
+        starting at global id local_expert_offset; MOE_MX_OUT_F32 returns the shard's float32
+        partial output."""
+        T, k = topk_ids.shape
+        if out is None:
+            dt = torch.float32 if out_dtype == MOE_MX_OUT_F32 else torch.bfloat16
+            out = torch.empty(T, self.H, dtype=dt, device=x.device)
+        moe_mx_forward_routed(self.handle, x, topk_ids, topk_w, T, k, local_expert_offset, w1, w1_scale, w2,
+                              w2_scale, act_dtype, out, out_dtype, stream)
         return out
 
     def prepare_scales(self, w1_scale: torch.Tensor, w2_scale: torch.Tensor, stream=None):

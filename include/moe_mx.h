@@ -76,6 +76,10 @@ extern "C" {
 #define MOE_MX_ACT_BF16 0  /* w4a16: bf16 activations x MXFP4 weights */
 #define MOE_MX_ACT_MXFP8 1 /* w4a8: activations quantised to MXFP8 E4M3 before FC1 */
 
+/* Output element type of moe_mx_forward_routed (out_dtype). */
+#define MOE_MX_OUT_BF16 0 /* bf16 [T, H] */
+#define MOE_MX_OUT_F32 1  /* float32 [T, H]: a shard's partial output, for a sum over shards */
+
 /* Element formats for moe_mx_quantize. */
 #define MOE_MX_FMT_MXFP4 0 /* E2M1 codes, two per byte */
 #define MOE_MX_FMT_MXFP8 1 /* E4M3 codes, one per byte */
@@ -94,12 +98,13 @@ typedef struct moe_mx_handle moe_mx_handle;
  * Create a layer handle for fixed dimensions and allocate its workspace on
  * `device` (the workspace is sized once, for max_tokens tokens and
  * max_top_k slots; moe_mx_forward never allocates).
- *   hidden      H, the model dimension: a multiple of 256, 256..16384.
+ *   hidden      H, the model dimension: a multiple of 128, 128..16384.
  *   inter       I, the expert intermediate dimension: a multiple of 128,
  *               128..8192.
  *   num_experts E: 1..1024.
  *   max_tokens  largest num_tokens a forward will be given: 1..65536.
- *   max_top_k   largest top_k a forward will be given: 1..min(E, 32).
+ *   max_top_k   largest top_k a forward will be given: 1..32 (moe_mx_forward
+ *               also needs top_k <= E; moe_mx_forward_routed does not).
  *   device      CUDA device ordinal; must be compute capability 10.0.
  * On success *out receives the handle (caller owns it; free it with
  * moe_mx_destroy).  Errors: INVALID_ARG, UNSUPPORTED, NO_MEMORY, CUDA.
@@ -133,6 +138,44 @@ MOE_MX_API int moe_mx_create(moe_mx_handle **out, int hidden, int inter, int num
 MOE_MX_API int moe_mx_forward(moe_mx_handle *h, const void *x, const float *router_logits, int num_tokens,
                    const uint8_t *w1, const uint8_t *w1_scale, const uint8_t *w2,
                    const uint8_t *w2_scale, int top_k, int act_dtype, void *out, void *stream);
+
+/*
+ * Run the layer with the routing given instead of computed, for one contiguous
+ * shard of the experts: precomputed, unpacked top-k (global expert ids and
+ * their weights), experts outside the shard filtered out, and the shard's
+ * partial output written (tokenspeed-situ package description, "Supported
+ * contract": precomputed top-k routing, global expert ids, contiguous local
+ * expert shards with a local expert offset, the native routing filtering out
+ * other shards' experts into a partial output the caller all-reduces).  The
+ * handle's E is the number of local experts; the weights hold those E experts.
+ *   x                    bf16 [T, H] activations.
+ *   topk_ids             int32 [T, k] global expert ids; an id in
+ *                        [local_expert_offset, local_expert_offset + E) selects
+ *                        local expert id - local_expert_offset, any other value
+ *                        (another shard's expert, or no expert) adds nothing.
+ *                        Ids of one token need not be distinct or ordered.
+ *   topk_w               float32 [T, k] the routing weights, used as given (no
+ *                        renormalisation).
+ *   num_tokens           T: 0..max_tokens (0: MOE_MX_OK, nothing enqueued).
+ *   top_k                k: 1..max_top_k (may exceed E).
+ *   local_expert_offset  >= 0: global id of local expert 0.
+ *   w1, w1_scale, w2, w2_scale, act_dtype: as for moe_mx_forward, [E, ...].
+ *   out                  [T, H], written (not accumulated), must not alias x:
+ *                        bf16 (out_dtype MOE_MX_OUT_BF16) or float32
+ *                        (MOE_MX_OUT_F32, the partial sum before rounding, so
+ *                        that the partial outputs of all shards add up to the
+ *                        layer's output with one rounding at the end).
+ *                        out[t] = sum over slots j of token t whose expert is
+ *                        local, j ascending, of topk_w[t,j] * FC2(SwiGLU(FC1(x[t]))).
+ * moe_mx_get_routing afterwards reports the local ids (-1 for slots outside
+ * the shard) and the given weights; counts and the grouping cover the local
+ * pairs only.  Allocation, synchronisation, graph capture and errors as for
+ * moe_mx_forward (INVALID_ARG also for a bad out_dtype or a negative offset).
+ */
+MOE_MX_API int moe_mx_forward_routed(moe_mx_handle *h, const void *x, const int32_t *topk_ids, const float *topk_w,
+                                     int num_tokens, int top_k, int local_expert_offset, const uint8_t *w1,
+                                     const uint8_t *w1_scale, const uint8_t *w2, const uint8_t *w2_scale,
+                                     int act_dtype, void *out, int out_dtype, void *stream);
 
 /* Free the handle and its workspace (waits for the device).  NULL is a no-op. */
 MOE_MX_API int moe_mx_destroy(moe_mx_handle *h);

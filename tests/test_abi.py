@@ -57,9 +57,13 @@ def test_host_validation_without_gpu(lib):
     h = ctypes.c_void_p()
     assert lib.moe_mx_create(ctypes.byref(h), 200, 128, 8, 16, 2, 0) == moe_mx.MOE_MX_ERR_UNSUPPORTED
     assert lib.moe_mx_create(ctypes.byref(h), 256, 100, 8, 16, 2, 0) == moe_mx.MOE_MX_ERR_UNSUPPORTED
-    assert lib.moe_mx_create(ctypes.byref(h), 256, 128, 8, 16, 9, 0) == moe_mx.MOE_MX_ERR_INVALID_ARG
+    assert lib.moe_mx_create(ctypes.byref(h), 256, 128, 8, 16, 33, 0) == moe_mx.MOE_MX_ERR_INVALID_ARG
     assert lib.moe_mx_create(ctypes.byref(h), 256, 128, 2000, 16, 2, 0) == moe_mx.MOE_MX_ERR_UNSUPPORTED
     assert lib.moe_mx_create(None, 256, 128, 8, 16, 2, 0) == moe_mx.MOE_MX_ERR_INVALID_ARG
+    fr = lib.moe_mx_forward_routed
+    assert fr(None, None, None, None, 1, 1, 0, None, None, None, None, 0, None, 0, None) == moe_mx.MOE_MX_ERR_INVALID_ARG
+    assert fr(None, None, None, None, 1, 1, 0, None, None, None, None, 0, None, 5, None) == moe_mx.MOE_MX_ERR_INVALID_ARG
+    assert b"out_dtype" in lib.moe_mx_last_error()
     assert lib.moe_mx_block_rows() == 128
     assert lib.moe_mx_destroy(None) == moe_mx.MOE_MX_OK
     assert lib.moe_mx_debug_watchdog(None, 10, None) == moe_mx.MOE_MX_ERR_INVALID_ARG
