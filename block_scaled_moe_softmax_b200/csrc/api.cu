@@ -137,6 +137,7 @@ struct moe_mx_handle {
     int64_t max_rows;
     int swap_rows;
     int tile_rows; // 0: by token count; else 16, 32, 64 or 128 (MOE_MX_TILE_ROWS)
+    int pdl;       // launch the kernels after the router as programmatic dependents (MOE_MX_PDL, default 1)
     int scale_layout; // MOE_MX_SCALES_ROW_MAJOR or MOE_MX_SCALES_TILED
     unsigned long long timeout_ns;
     void *ws;
@@ -225,6 +226,7 @@ int moe_mx_create(moe_mx_handle **out, int hidden, int inter, int num_experts, i
     h->tile_rows = env_int("MOE_MX_TILE_ROWS", 0);
     if (h->tile_rows != 16 && h->tile_rows != 32 && h->tile_rows != 64 && h->tile_rows != kBlockRows)
         h->tile_rows = 0;
+    h->pdl = env_int("MOE_MX_PDL", 1) != 0;
     h->swap_rows = env_int("MOE_MX_SWAP_ROWS", 64);
     if (h->swap_rows < 0)
         h->swap_rows = 0;
@@ -412,11 +414,15 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
         ra.given_ids = given_ids;
         ra.given_w = given_w;
         ra.id_offset = id_offset;
-        launch_route_and_group(ra, s);
+        // Each kernel after the router may launch while its predecessor still runs (programmatic
+        // dependent launch): the FC GEMMs start streaming their weights early.  Stage timing
+        // records events between the kernels, so timed forwards launch them one after another.
+        const bool pdl = h->pdl && !evset;
+        launch_route_and_group(ra, s, pdl);
         mark(1);
         const int mx8 = act_dtype == MOE_MX_ACT_MXFP8;
         launch_gather(static_cast<const __nv_bfloat16 *>(x), (int)pairs, H, k, h->pos_of_pair, h->Aq, h->Asf,
-                      (int)h->max_rows, mx8, h->num_sms, s);
+                      (int)h->max_rows, mx8, h->num_sms, s, pdl);
 
         FcGemmArgs f1{};
         f1.rowblocks = h->rowblocks;
@@ -444,7 +450,7 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
         mark(2);
         const int sw_idx = tile_rows <= 16 ? 0 : tile_rows <= 32 ? 1 : 2; // box rows min(tile rows, 64)
         launch_fc_gemm(f1, h->map_A[f1.terms - 1], h->map_Asw[f1.terms - 1][sw_idx], h->map_A16, h->map_w1, h->num_sms,
-                       s);
+                       s, pdl);
         mark(3);
 
         FcGemmArgs f2 = f1;
@@ -459,9 +465,9 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
         f2.act_mxfp8 = 0;
         // the maps' plane count must equal the copy's terms: the stage barrier expects exactly those bytes
         launch_fc_gemm(f2, h->map_H[f2.terms - 1], h->map_Hsw[f2.terms - 1][sw_idx], h->map_H16, h->map_w2,
-                       h->num_sms, s);
+                       h->num_sms, s, pdl);
         mark(4);
-        launch_combine(h->Y, T, H, k, h->pos_of_pair, h->topk_w, out, out_f32, h->num_sms, s);
+        launch_combine(h->Y, T, H, k, h->pos_of_pair, h->topk_w, out, out_f32, h->num_sms, s, pdl);
         ce = cudaGetLastError();
         if (ce != cudaSuccess) {
             rc = cuda_fail(ce, "kernel launch");

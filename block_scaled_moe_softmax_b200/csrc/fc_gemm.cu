@@ -267,6 +267,11 @@ struct Ctx {
 // compile-time role index so that every operand of the TMA issue stays warp-uniform).
 // Consecutive stages come from different warps at nearly the same time, so the two 64-byte
 // halves of a weight row's 128-byte line are requested close together.
+// Launched as a programmatic dependent, the kernel may start while the kernel ahead of it (which
+// writes this GEMM's activations) still runs; the producers wait for it (grid_dep_wait) before
+// their first copy.  (Issuing the first pass's weight copies before that wait and deferring only
+// the activation copies measured slower: the extra paths cost the steady-state loop more than
+// the early weights gained.)
 template <int kActRows, int kMmaW, int kWTiles, int kTm, int PI>
 __device__ __forceinline__ void producer_role(const FcGemmArgs &a, const Ctx &c, const CUtensorMap *act_map,
                                               const CUtensorMap *act_map_sw, const CUtensorMap *act_map16,
@@ -284,6 +289,7 @@ __device__ __forceinline__ void producer_role(const FcGemmArgs &a, const Ctx &c,
     bool ok = true;
     const int scl_ld = a.K / 32;
     const UnitRing<kStages> ring{bars, c.units};
+    grid_dep_wait();
     for (uint32_t i = 0; ok; ++i) {
         const int4 blk = ring.take(i, a.err, tmo, lane);
         if (blk.w < 0)
@@ -570,6 +576,11 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(gsm + kOffTmemSlot);
+    // The next kernel may launch now: what it reads of this kernel's output it reads after its
+    // own grid_dep_wait; what it reads before (the row-block list, the work-unit counters) was
+    // written two kernels back, which had completed before this kernel could launch.
+    if (threadIdx.x == 0)
+        grid_dep_launch();
 
     const int nrb = *a.num_rowblocks;
     const int n_groups = a.n_tiles / P::kWT; // the launch guarantees n_tiles % kWT == 0
@@ -720,6 +731,10 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads,
     }
 
     tc_fence_before();
+    // every CTA waits for the kernel before it at least once, also a CTA that got no work (only
+    // the producers wait otherwise), so that this grid completes only after its predecessor has
+    if (threadIdx.x == 0)
+        grid_dep_wait();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
@@ -746,14 +761,15 @@ cudaError_t fc_gemm_prepare()
 
 template <int kActRows, int kMmaW, int kWTiles, int kTm>
 static void launch_one(const FcGemmArgs &a, const CUtensorMap &act_map, const CUtensorMap &act_map_sw,
-                       const CUtensorMap &act_map16, const CUtensorMap &w_map, int grid, cudaStream_t s)
+                       const CUtensorMap &act_map16, const CUtensorMap &w_map, int grid, cudaStream_t s, bool pdl)
 {
-    fc_gemm_kernel<kActRows, kMmaW, kWTiles, kTm><<<grid, Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads, Plan<kActRows, kMmaW, kWTiles, kTm>::kSmemBytes, s>>>(
-        a, act_map, act_map_sw, act_map16, w_map);
+    using P = Plan<kActRows, kMmaW, kWTiles, kTm>;
+    launch_kernel(fc_gemm_kernel<kActRows, kMmaW, kWTiles, kTm>, dim3(grid), dim3(P::kThreads), (size_t)P::kSmemBytes,
+                  s, pdl, a, act_map, act_map_sw, act_map16, w_map);
 }
 
 void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUtensorMap &act_map_sw,
-                    const CUtensorMap &act_map16, const CUtensorMap &w_map, int grid, cudaStream_t s)
+                    const CUtensorMap &act_map16, const CUtensorMap &w_map, int grid, cudaStream_t s, bool pdl)
 {
     // Row blocks of at most 16 / 32 / 64 rows run with their tokens on N; smaller activation
     // tiles leave room for more pipeline stages (bytes in flight) in the weight-streaming shapes.
@@ -763,26 +779,26 @@ void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUten
     const bool wt2 = !a.fc1 && a.n_tiles % 2 == 0;
     if (a.max_block_rows <= 16) {
         if (a.fc1)
-            launch_one<16, 2, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+            launch_one<16, 2, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
         else if (wt2)
-            launch_one<16, 1, 2, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+            launch_one<16, 1, 2, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
         else
-            launch_one<16, 1, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+            launch_one<16, 1, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
     } else if (a.max_block_rows <= 32) {
         if (a.fc1)
-            launch_one<32, 2, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+            launch_one<32, 2, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
         else if (wt2)
-            launch_one<32, 1, 2, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+            launch_one<32, 1, 2, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
         else
-            launch_one<32, 1, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+            launch_one<32, 1, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
     } else if (a.max_block_rows <= 64) {
-        launch_one<64, 1, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+        launch_one<64, 1, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
     } else if (a.terms == 1) {
         // single-term activations (w4a8 FC1): the smaller stages leave room for 6 of them
         // instead of 4, i.e. more bytes in flight per SM
-        launch_one<128, 1, 1, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+        launch_one<128, 1, 1, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
     } else {
-        launch_one<128, 1, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s);
+        launch_one<128, 1, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
     }
 }
 

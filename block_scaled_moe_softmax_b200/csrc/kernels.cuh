@@ -7,9 +7,30 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "ptx.cuh"
 
 namespace moe_mx {
+
+// Launch `kernel` on `s`; with pdl, as a programmatic dependent of the kernel before it in the
+// stream (it may start early: everything it reads from that kernel comes after grid_dep_wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                 bool pdl, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 32;
@@ -40,12 +61,16 @@ struct RouteGroupArgs {
     int id_offset = 0;
 };
 
-void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s);
+// Launchers of the forward's kernels.  pdl: launch as programmatic dependents of the kernel
+// before them in the stream (each waits for its predecessor before reading its output and lets
+// its own successor launch right after that wait); the first kernel of a forward, the router,
+// is always an ordinary launch.
+void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s, bool pdl = false);
 void launch_gather(const __nv_bfloat16 *x, int P, int H, int k, const int32_t *pos_of_pair, uint8_t *aq,
-                   uint8_t *asf, int act_rows, int act_mxfp8, int num_sms, cudaStream_t s);
+                   uint8_t *asf, int act_rows, int act_mxfp8, int num_sms, cudaStream_t s, bool pdl = false);
 // out: bf16 [T, H], or (out_f32) float32 [T, H]; pairs with pos_of_pair -1 add nothing
 void launch_combine(const float *Y, int T, int H, int k, const int32_t *pos_of_pair, const float *topk_w, void *out,
-                    int out_f32, int num_sms, cudaStream_t s);
+                    int out_f32, int num_sms, cudaStream_t s, bool pdl = false);
 void launch_mx_quantize(const float *src, int64_t rows, int64_t K, int fmt, uint8_t *codes, uint8_t *scales,
                         int num_sms, cudaStream_t s);
 
@@ -84,7 +109,7 @@ struct FcGemmArgs {
 // act_map16 = 16-row boxes of one plane (tokens on N, blocks beyond that); w_map = FC1: the
 // gate and up halves of a 64-row weight slice in one box, FC2: 128-row boxes.
 void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUtensorMap &act_map_sw,
-                    const CUtensorMap &act_map16, const CUtensorMap &w_map, int grid, cudaStream_t s);
+                    const CUtensorMap &act_map16, const CUtensorMap &w_map, int grid, cudaStream_t s, bool pdl = false);
 cudaError_t fc_gemm_prepare();
 
 // Rearrange row-major E8M0 weight scales [E][R][K/32] into the tiled atom layout the GEMM reads:

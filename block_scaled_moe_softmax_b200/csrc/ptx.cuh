@@ -93,6 +93,22 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
+// ----------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start before the kernel ahead
+// of it in the stream has finished.  griddepcontrol.wait blocks the executing thread until
+// every prerequisite grid has completed and its memory operations are visible (it returns at
+// once when there is none); griddepcontrol.launch_dependents lets the next such kernel launch
+// once every CTA of this grid has issued it or exited.
+__device__ __forceinline__ void grid_dep_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void grid_dep_launch()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ----------------------------------------------------------------- TMA / cp.async
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int32_t x, int32_t y,
                                             uint32_t bar)

@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float *__res
                                                                const int32_t *__restrict__ gids,
                                                                const float *__restrict__ gw, int off)
 {
+    grid_dep_launch(); // the next kernel (the scan) waits for this grid before reading its output
     __shared__ int32_t hist[kMaxExperts];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int e = threadIdx.x; e < E; e += blockDim.x)
@@ -206,6 +207,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(int E, int nchunks, int spli
                                                     int4 *__restrict__ rowblocks, int32_t *__restrict__ num_rowblocks,
                                                     int32_t *__restrict__ sorted_pair, int32_t *__restrict__ unit_counters)
 {
+    grid_dep_wait(); // the chunk histograms of the router
+    grid_dep_launch();
     __shared__ unsigned long long s_warp[32];
     const int e = threadIdx.x;
     if (unit_counters && e < 2) // the GEMMs' work-unit counters start at zero
@@ -271,6 +274,7 @@ __device__ __forceinline__ void scatter_pairs(int p_begin, int p_end, const int3
 template <int kPerLane>
 __global__ void __launch_bounds__(1024) route_group_small_kernel(const RouteGroupArgs a)
 {
+    grid_dep_launch(); // the next kernel (the gather) waits for this grid before reading its output
     __shared__ int32_t hist[kMaxExperts]; // counts, then cursors
     __shared__ unsigned long long s_warp[32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -305,6 +309,8 @@ __global__ void __launch_bounds__(32) scatter_kernel(int T, int E, int k, const 
                                                      int32_t *__restrict__ sorted_pair,
                                                      int32_t *__restrict__ pos_of_pair)
 {
+    grid_dep_wait(); // the scan's per-chunk bases (and, through it, the router's ids)
+    grid_dep_launch();
     __shared__ int32_t cursor[kMaxExperts];
     const int lane = threadIdx.x;
     for (int e = lane; e < E; e += 32)
@@ -327,6 +333,8 @@ __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16 *__rest
                                                      uint8_t *__restrict__ aq, uint8_t *__restrict__ asf, int act_rows,
                                                      int act_mxfp8)
 {
+    grid_dep_wait(); // pos_of_pair from the grouping
+    grid_dep_launch();
     const int blocks_per_row = H / 32, groups = k / group;
     const long long total = (long long)T * blocks_per_row * groups;
     for (long long g = blockIdx.x * (long long)blockDim.x + threadIdx.x; g < total;
@@ -376,6 +384,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
                                                       const int32_t *__restrict__ pos_of_pair,
                                                       const float *__restrict__ topk_w, void *__restrict__ out)
 {
+    grid_dep_wait(); // Y from FC2
     const int vec_per_row = H / 8;
     const long long total = (long long)T * vec_per_row;
     for (long long g = blockIdx.x * (long long)blockDim.x + threadIdx.x; g < total;
@@ -419,10 +428,11 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
 }
 
 // ---------------------------------------------------------------- launchers
-void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s)
+void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s, bool pdl)
 {
     // the top-k scan visits 32 * kPerLane candidates per token: size it to the expert count
-    // (the given routing visits no candidates: the smallest instance serves it)
+    // (the given routing visits no candidates: the smallest instance serves it).  The first
+    // kernel is an ordinary launch; those after it are programmatic dependents (pdl).
     const bool narrow = a.given_ids != nullptr || a.E <= 256;
     if (a.T <= kSmallRouteTokens) {
         if (narrow)
@@ -443,13 +453,14 @@ void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s)
     else
         route_kernel<32><<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist,
                                                           a.given_ids, a.given_w, a.id_offset);
-    scan_kernel<<<1, 1024, 0, s>>>(a.E, nchunks, a.split_rows, a.chunk_hist, a.counts, a.pad_offsets, a.rowblocks,
-                                   a.num_rowblocks, a.sorted_pair, a.unit_counters);
-    scatter_kernel<<<nchunks, 32, 0, s>>>(a.T, a.E, a.k, a.topk_ids, a.chunk_hist, a.sorted_pair, a.pos_of_pair);
+    launch_kernel(scan_kernel, dim3(1), dim3(1024), 0, s, pdl, a.E, nchunks, a.split_rows, a.chunk_hist, a.counts,
+                  a.pad_offsets, a.rowblocks, a.num_rowblocks, a.sorted_pair, a.unit_counters);
+    launch_kernel(scatter_kernel, dim3(nchunks), dim3(32), 0, s, pdl, a.T, a.E, a.k, (const int32_t *)a.topk_ids,
+                  (const int32_t *)a.chunk_hist, a.sorted_pair, a.pos_of_pair);
 }
 
 void launch_gather(const __nv_bfloat16 *x, int P, int H, int k, const int32_t *pos_of_pair, uint8_t *aq,
-                   uint8_t *asf, int act_rows, int act_mxfp8, int num_sms, cudaStream_t s)
+                   uint8_t *asf, int act_rows, int act_mxfp8, int num_sms, cudaStream_t s, bool pdl)
 {
     // encode each block once per token when that still fills the GPU, else once per pair
     const long long token_blocks = (long long)(P / k) * (H / 32);
@@ -457,20 +468,18 @@ void launch_gather(const __nv_bfloat16 *x, int P, int H, int k, const int32_t *p
     const long long work = token_blocks * (k / group);
     const long long want = (work + 255) / 256;
     const int grid = (int)(want < (long long)num_sms * 8 ? want : (long long)num_sms * 8);
-    gather_kernel<<<grid > 0 ? grid : 1, 256, 0, s>>>(x, P / k, H, k, group, pos_of_pair, aq, asf, act_rows,
-                                                      act_mxfp8);
+    launch_kernel(gather_kernel, dim3(grid > 0 ? grid : 1), dim3(256), 0, s, pdl, x, P / k, H, k, group, pos_of_pair,
+                  aq, asf, act_rows, act_mxfp8);
 }
 
 void launch_combine(const float *Y, int T, int H, int k, const int32_t *pos_of_pair, const float *topk_w, void *out,
-                    int out_f32, int num_sms, cudaStream_t s)
+                    int out_f32, int num_sms, cudaStream_t s, bool pdl)
 {
     const long long work = (long long)T * (H / 8);
     const long long want = (work + 255) / 256;
     const int grid = (int)(want < (long long)num_sms * 8 ? want : (long long)num_sms * 8);
-    if (out_f32)
-        combine_kernel<true><<<grid > 0 ? grid : 1, 256, 0, s>>>(Y, T, H, k, pos_of_pair, topk_w, out);
-    else
-        combine_kernel<false><<<grid > 0 ? grid : 1, 256, 0, s>>>(Y, T, H, k, pos_of_pair, topk_w, out);
+    launch_kernel(out_f32 ? combine_kernel<true> : combine_kernel<false>, dim3(grid > 0 ? grid : 1), dim3(256), 0, s,
+                  pdl, Y, T, H, k, pos_of_pair, topk_w, out);
 }
 
 } // namespace moe_mx

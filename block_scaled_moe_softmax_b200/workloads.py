@@ -76,6 +76,9 @@ WORKLOADS = {
                             "prefill-shaped, w4a16, 64 experts, 2048 tokens (profiling case)"),
     "prefill_w4a8": Workload("prefill_w4a8", 16384, 4096, 1536, 128, 8, "mxfp8", "none", 0,
                              "prefill, w4a8: T=16384 H=4096 I=1536 E=128 top-8"),
+    # the w4a8 prefill shape with 4096 tokens: a capture-sized case (about 2.5 GB on the device)
+    "prefill_w4a8_t4k": Workload("prefill_w4a8_t4k", 4096, 4096, 1536, 128, 8, "mxfp8", "none", 0,
+                                 "prefill-shaped, w4a8, 4096 tokens (profiling case)"),
     # the hidden size, expert count and top-k of the TokenSpeed SiTU bundle's supported contract, with the
     # routing given as precomputed top-k: TP8 (all 896 experts, intermediate shard 384) and the
     # first EP8 shard (112 local experts of 896, intermediate 3072); 128 tokens

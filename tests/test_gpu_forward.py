@@ -185,3 +185,22 @@ def test_watchdog_reports_timeout_and_context_survives(monkeypatch):
     ref, _, _ = helpers.oracle_forward(inp, wl.top_k, 0)
     helpers.check_output(out, ref, "after watchdog")
     layer2.close()
+
+
+@pytest.mark.parametrize("name", ["tiny", "multi"])
+@pytest.mark.parametrize("act_mode", [0, 1], ids=["w4a16", "w4a8"])
+def test_dependent_launch_gives_same_bits(name, act_mode, monkeypatch):
+    """Kernels launched as programmatic dependents (the default) and one after another
+    (MOE_MX_PDL=0) give bit-identical routing and outputs."""
+    wl = SHAPES[name]
+    inp = helpers.host_inputs(wl)
+    outs = []
+    for pdl in ("1", "0"):
+        monkeypatch.setenv("MOE_MX_PDL", pdl)
+        layer, _, out = _run(wl, act_mode, monkeypatch, inp=inp)
+        outs.append((out.clone(), [a.clone() for a in layer.routing(wl.T, wl.top_k)]))
+        layer.close()
+    assert torch.equal(outs[0][0].view(torch.int16), outs[1][0].view(torch.int16))
+    for a, b in zip(outs[0][1], outs[1][1]):
+        assert torch.equal(a, b)
+
