@@ -16,6 +16,8 @@ function states the passage of the pages it follows in the C source:
 * FC1 -> SwiGLU -> FC2 -> weighted combine with MXFP4 weights
   (tokenspeed-situ description, intro, "Supported contract", "Activation
   precision (w4a16 vs w4a8)"; mxfp6-sm120 description, "Execution model");
+* a shared expert added to every token with weight 1, held as extra expert slots
+  (mxfp6-sm120 description, path table: routed/shared reduction);
 * the same layer with the routing given (precomputed top-k, global expert ids)
   for one contiguous local expert shard, whose partial outputs add up to the
   layer (tokenspeed-situ description, "Supported contract");
@@ -84,6 +86,8 @@ def _load():
         lib.oracle_group.restype = None
         lib.oracle_moe_forward.argtypes = [i32] * 6 + [P] * 6 + [P, i32, P, P, P, P, i32]
         lib.oracle_moe_forward.restype = i32
+        lib.oracle_moe_forward_shared.argtypes = [i32] * 7 + [P] * 6 + [P, i32, P, P, P, P, i32]
+        lib.oracle_moe_forward_shared.restype = i32
         lib.oracle_moe_forward_routed.argtypes = [i32] * 6 + [P, P, P, i32] + [P] * 4 + [P, i32, P, P, P, P, i32]
         lib.oracle_moe_forward_routed.restype = i32
         _lib = lib
@@ -179,24 +183,26 @@ def group(ids: np.ndarray, E: int):
 # ---------------------------------------------------------------- the layer
 def moe_forward(x_bf16_bits: np.ndarray, logits: np.ndarray, w1: np.ndarray, w1s: np.ndarray,
                 w2: np.ndarray, w2s: np.ndarray, top_k: int, act_mode: int = ACT_BF16,
-                tokens=None, nthreads: int | None = None, exact: bool = False):
+                tokens=None, nthreads: int | None = None, exact: bool = False, num_shared: int = 0):
     """Evaluate the layer per token.
 
     x_bf16_bits: uint16 [T, H] (bf16 bit patterns); logits f32 [T, E];
-    w1 u8 [E, 2I, H/2], w1s u8 [E, 2I, H/32]; w2 u8 [E, H, I/2], w2s u8 [E, H, I/32].
+    w1 u8 [E + S, 2I, H/2], w1s u8 [E + S, 2I, H/32]; w2 u8 [E + S, H, I/2], w2s u8 [E + S, H, I/32],
+    S = num_shared: the shared expert's chunks in slots E.. (added to every token with weight 1).
     tokens: optional list of token indices to evaluate (default: all).
-    Returns (out bf16 bits uint16 [n, H], ids i32 [n, k], w f32 [n, k]), plus, with
+    Returns (out bf16 bits uint16 [n, H], ids i32 [n, k + S], w f32 [n, k + S]), plus, with
     exact=True, the float64 output before its final bf16 rounding as a fourth item.
     """
     x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
     logits = np.ascontiguousarray(logits, dtype=np.float32)
     T, H = x.shape
     E = logits.shape[1]
+    S = int(num_shared)
     I = w2.shape[2] * 2
     for a in (w1, w1s, w2, w2s):
         assert a.dtype == np.uint8 and a.flags["C_CONTIGUOUS"]
-    assert w1.shape == (E, 2 * I, H // 2) and w1s.shape == (E, 2 * I, H // 32)
-    assert w2.shape == (E, H, I // 2) and w2s.shape == (E, H, I // 32)
+    assert w1.shape == (E + S, 2 * I, H // 2) and w1s.shape == (E + S, 2 * I, H // 32)
+    assert w2.shape == (E + S, H, I // 2) and w2s.shape == (E + S, H, I // 32)
     if tokens is None:
         tok_arr = None
         n = T
@@ -204,13 +210,17 @@ def moe_forward(x_bf16_bits: np.ndarray, logits: np.ndarray, w1: np.ndarray, w1s
         tok_arr = np.ascontiguousarray(tokens, dtype=np.int32)
         n = int(tok_arr.shape[0])
     out = np.empty((n, H), dtype=np.uint16)
-    ids = np.empty((n, top_k), dtype=np.int32)
-    w = np.empty((n, top_k), dtype=np.float32)
+    ids = np.empty((n, top_k + S), dtype=np.int32)
+    w = np.empty((n, top_k + S), dtype=np.float32)
     out_exact = np.empty((n, H), dtype=np.float64) if exact else None
-    rc = _load().oracle_moe_forward(
-        T, H, I, E, top_k, act_mode, _ptr(x), _ptr(logits), _ptr(w1), _ptr(w1s), _ptr(w2), _ptr(w2s),
-        _ptr(tok_arr) if tok_arr is not None else None, n, _ptr(out), _ptr(ids), _ptr(w),
-        _ptr(out_exact) if exact else None, nthreads or default_threads())
+    tail = (_ptr(tok_arr) if tok_arr is not None else None, n, _ptr(out), _ptr(ids), _ptr(w),
+            _ptr(out_exact) if exact else None, nthreads or default_threads())
+    if S:
+        rc = _load().oracle_moe_forward_shared(T, H, I, E, S, top_k, act_mode, _ptr(x), _ptr(logits), _ptr(w1),
+                                               _ptr(w1s), _ptr(w2), _ptr(w2s), *tail)
+    else:
+        rc = _load().oracle_moe_forward(T, H, I, E, top_k, act_mode, _ptr(x), _ptr(logits), _ptr(w1), _ptr(w1s),
+                                        _ptr(w2), _ptr(w2s), *tail)
     if rc != 0:
         raise ValueError("oracle_moe_forward rejected its arguments")
     if exact:

@@ -368,6 +368,7 @@ void oracle_group(int T, int k, int E, const int32_t *ids, int32_t *counts, int3
 
 typedef struct {
     int T, H, I, E, k, act_mode;
+    int n_shared;               /* shared-expert slots E..E+n_shared-1, weight 1 for every token */
     const uint16_t *x;
     const float *logits;        /* router logits [T,E], or NULL when the routing is given: */
     const int32_t *given_ids;   /* [T,k] global expert ids (routed form), */
@@ -422,10 +423,6 @@ static void forward_token(const fwd_job *jb, int64_t slot)
             w[j] = jb->given_w[(int64_t)t * k + j];
         }
     }
-    if (jb->ids_out)
-        memcpy(jb->ids_out + slot * k, ids, sizeof(int32_t) * (size_t)k);
-    if (jb->w_out)
-        memcpy(jb->w_out + slot * k, w, sizeof(float) * (size_t)k);
 
     double *a = (double *)malloc(sizeof(double) * (size_t)H);
     double *h = (double *)malloc(sizeof(double) * (size_t)I);
@@ -435,7 +432,19 @@ static void forward_token(const fwd_job *jb, int64_t slot)
     if (jb->act_mode == 1)
         mxfp8_roundtrip(a, H);
 
-    for (int j = 0; j < k - (ORACLE_PLANT_MISTAKE == 7); ++j) { /* plant: last slot dropped */
+    /* the shared expert: slots k..k+n_shared-1 hold its n_shared chunks (experts E..), weight 1
+     * [mxfp6-sm120 package description, path table: "shared-expert combine and routed/shared
+     * reduction"] */
+    const int S = jb->n_shared;
+    for (int c = 0; c < S; ++c) {
+        ids[k + c] = E + c;
+        w[k + c] = ORACLE_PLANT_MISTAKE == 11 ? 0.5f : 1.0f; /* plant: shared expert half-weighted */
+    }
+    if (jb->ids_out)
+        memcpy(jb->ids_out + slot * (k + S), ids, sizeof(int32_t) * (size_t)(k + S));
+    if (jb->w_out)
+        memcpy(jb->w_out + slot * (k + S), w, sizeof(float) * (size_t)(k + S));
+    for (int j = 0; j < k + S - (ORACLE_PLANT_MISTAKE == 7); ++j) { /* plant: last slot dropped */
         const int64_t e = ids[j];
         if (e < 0)
             continue; /* routed form: an expert outside the local shard */
@@ -498,13 +507,13 @@ static void *forward_worker(void *arg)
  * [0,I), up rows [I,2I)), w1s [E,2I,H/32]; w2 codes [E,H,I/2], w2s [E,H,I/32].
  * Returns 0, or -1 on bad arguments.
  */
-static int run_forward(int T, int H, int I, int E, int k, int act_mode, const uint16_t *x, const float *logits,
+static int run_forward(int T, int H, int I, int E, int S, int k, int act_mode, const uint16_t *x, const float *logits,
                        const int32_t *given_ids, const float *given_w, int local_offset, const uint8_t *w1,
                        const uint8_t *w1s, const uint8_t *w2, const uint8_t *w2s, const int32_t *tokens, int n_eval,
                        uint16_t *out, int32_t *ids_out, float *w_out, double *out_exact, int nthreads)
 {
-    if (T < 0 || H <= 0 || I <= 0 || H % 32 || I % 32 || E < 1 || E > 1024 || k < 1 || k > 1024 || (logits && k > E) ||
-        (act_mode != 0 && act_mode != 1) || n_eval < 0 || !out)
+    if (T < 0 || H <= 0 || I <= 0 || H % 32 || I % 32 || E < 1 || S < 0 || E + S > 1024 || k < 1 ||
+        k + S > 1024 || (logits && k > E) || (act_mode != 0 && act_mode != 1) || n_eval < 0 || !out)
         return -1;
     if (n_eval == 0)
         return 0;
@@ -520,7 +529,7 @@ static int run_forward(int T, int H, int I, int E, int k, int act_mode, const ui
     pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
     fwd_job *jobs = (fwd_job *)malloc(sizeof(fwd_job) * (size_t)nthreads);
     for (int i = 0; i < nthreads; ++i) {
-        jobs[i] = (fwd_job){T, H, I, E, k, act_mode, x, logits, given_ids, given_w, local_offset, w1, w1s, w2, w2s,
+        jobs[i] = (fwd_job){T, H, I, E, k, act_mode, S, x, logits, given_ids, given_w, local_offset, w1, w1s, w2, w2s,
                             tokens, out, out_exact, ids_out, w_out, (int64_t)n_eval * i / nthreads,
                             (int64_t)n_eval * (i + 1) / nthreads};
         pthread_create(&th[i], NULL, forward_worker, &jobs[i]);
@@ -539,8 +548,32 @@ int oracle_moe_forward(int T, int H, int I, int E, int k, int act_mode, const ui
 {
     if (!logits)
         return -1;
-    return run_forward(T, H, I, E, k, act_mode, x, logits, NULL, NULL, 0, w1, w1s, w2, w2s, tokens, n_eval, out,
+    return run_forward(T, H, I, E, 0, k, act_mode, x, logits, NULL, NULL, 0, w1, w1s, w2, w2s, tokens, n_eval, out,
                        ids_out, w_out, out_exact, nthreads);
+}
+
+/*
+ * The layer with a shared expert: every token also passes through the shared
+ * expert, a SwiGLU MLP of intermediate size n_shared * I, and its output is added
+ * to the routed sum with weight 1 (the routed/shared reduction of the mxfp6-sm120
+ * package description's routed-MoE path).  The shared expert is held as n_shared
+ * chunks of I in expert slots E..E+n_shared-1 of w1..w2s ([E + n_shared, ...]):
+ * chunk c holds gate rows c*I..(c+1)*I-1 of the shared W1 followed by the matching
+ * up rows, and columns c*I..(c+1)*I-1 of the shared W2.  (SwiGLU is elementwise
+ * over the intermediate index, so the chunks' outputs add up to the shared MLP.)
+ * The router sees the E routed experts only (logits [T, E]).  ids_out / w_out
+ * ([n, k + n_shared]) list the routed slots, then the shared slots (ids E..,
+ * weight 1).  Returns 0, or -1 on bad arguments.
+ */
+int oracle_moe_forward_shared(int T, int H, int I, int E, int n_shared, int k, int act_mode, const uint16_t *x,
+                              const float *logits, const uint8_t *w1, const uint8_t *w1s, const uint8_t *w2,
+                              const uint8_t *w2s, const int32_t *tokens, int n_eval, uint16_t *out, int32_t *ids_out,
+                              float *w_out, double *out_exact, int nthreads)
+{
+    if (!logits)
+        return -1;
+    return run_forward(T, H, I, E, n_shared, k, act_mode, x, logits, NULL, NULL, 0, w1, w1s, w2, w2s, tokens, n_eval,
+                       out, ids_out, w_out, out_exact, nthreads);
 }
 
 /*
@@ -563,6 +596,6 @@ int oracle_moe_forward_routed(int T, int H, int I, int E, int k, int act_mode, c
 {
     if (!topk_ids || !topk_w || k > 1024)
         return -1;
-    return run_forward(T, H, I, E, k, act_mode, x, NULL, topk_ids, topk_w, local_offset, w1, w1s, w2, w2s, tokens,
+    return run_forward(T, H, I, E, 0, k, act_mode, x, NULL, topk_ids, topk_w, local_offset, w1, w1s, w2, w2s, tokens,
                        n_eval, out, ids_out, w_out, out_exact, nthreads);
 }

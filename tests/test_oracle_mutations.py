@@ -25,6 +25,7 @@ PLANTS = [
     (8, "weights not renormalised", "tests/test_oracle_routing.py"),
     (9, "grouping not stable", "tests/test_oracle_routing.py"),
     (10, "given routing: local expert offset ignored", "tests/test_oracle_routed.py"),
+    (11, "shared expert added with weight 1/2", "tests/test_oracle_shared.py"),
 ]
 
 
