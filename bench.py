@@ -86,14 +86,17 @@ def workload_desc(wl):
                  f"[{wl.local_offset}, {wl.local_offset + wl.E})")
     else:
         route = f"logit bias {wl.bias}"
+    if wl.shared:
+        route += f", plus a shared expert of intermediate {wl.shared * wl.I}"
     return (f"{wl.name}: T={wl.T} H={wl.H} I={wl.I} E={wl.E} top-{wl.top_k} "
             f"{'w4a8' if wl.act == 'mxfp8' else 'w4a16'}, {route}")
 
 
 # ------------------------------------------------------------------ inputs
 def make_gpu_weights(wl, dev):
-    """Draw float32 weights per expert on the GPU and quantise them with the library's MX quantiser."""
-    E, H, I = wl.E, wl.H, wl.I
+    """Draw float32 weights per expert (and shared-expert chunk) on the GPU and quantise them with
+    the library's MX quantiser."""
+    E, H, I = wl.slots, wl.H, wl.I
     w1 = torch.empty(E, 2 * I, H // 2, dtype=torch.uint8, device=dev)
     w1s = torch.empty(E, 2 * I, H // 32, dtype=torch.uint8, device=dev)
     w2 = torch.empty(E, H, I // 2, dtype=torch.uint8, device=dev)
@@ -110,7 +113,7 @@ def make_gpu_weights(wl, dev):
 def oracle_weights_for(wl, experts, dev):
     """Oracle-quantised weights (host, numpy) for the given experts; other experts stay zero."""
     import oracle
-    E, H, I = wl.E, wl.H, wl.I
+    E, H, I = wl.slots, wl.H, wl.I
     w1 = np.zeros((E, 2 * I, H // 2), np.uint8)
     w1s = np.zeros((E, 2 * I, H // 32), np.uint8)
     w2 = np.zeros((E, H, I // 2), np.uint8)
@@ -212,7 +215,8 @@ def oracle_time_tokens(wl, xb, route_np, wq, tokens, nthreads):
         ids, w = route_np
         oracle.moe_forward_routed(xb, ids, w, wl.local_offset, *wq, act, tokens=tokens, nthreads=nthreads)
     else:
-        oracle.moe_forward(xb, route_np, *wq, wl.top_k, act, tokens=tokens, nthreads=nthreads)
+        oracle.moe_forward(xb, route_np, *wq, wl.top_k, act, tokens=tokens, nthreads=nthreads,
+                           num_shared=wl.shared)
     return time.perf_counter() - t0
 
 
@@ -228,7 +232,7 @@ def cpu_sample_setup(wl, sample_tokens):
     else:
         logits = workloads.draw_logits(wl)
         ids, _ = oracle.route(logits.numpy()[sample_tokens], wl.top_k)
-        experts = sorted(set(int(e) for e in ids.reshape(-1)))
+        experts = sorted(set(int(e) for e in ids.reshape(-1))) + list(range(wl.E, wl.slots))
         route_np = logits.numpy()
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     wq = oracle_weights_for(wl, experts, dev)
@@ -343,7 +347,7 @@ def run_ours(args, wl):
     route_host = workloads.draw_topk(wl) if given else (workloads.draw_logits(wl),)
     route_in = tuple(a.to(dev) for a in route_host)
     out = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=dev)
-    layer = moe_mx.MoeMxLayer(wl.H, wl.I, wl.E, wl.T, wl.top_k, device=dev.index)
+    layer = moe_mx.MoeMxLayer(wl.H, wl.I, wl.E, wl.T, wl.top_k, device=dev.index, num_shared=wl.shared)
     # weight preparation, once, like the quantisation: the E8M0 scales in the tiled layout
     w1s, w2s = layer.prepare_scales(w1s, w2s)
     torch.cuda.synchronize()

@@ -133,7 +133,9 @@ int env_int(const char *name, int dflt)
 } // namespace
 
 struct moe_mx_handle {
-    int H, I, E, maxT, maxK, dev, num_sms;
+    // E: expert slots of the weights (routed experts, then the shared expert's S chunks);
+    // maxK: the largest routed top-k; a token has top_k + S slots
+    int H, I, E, S, maxT, maxK, dev, num_sms;
     int64_t max_rows;
     int swap_rows;
     int tile_rows; // 0: by token count; else 16, 32, 64 or 128 (MOE_MX_TILE_ROWS)
@@ -175,11 +177,17 @@ int64_t moe_mx_max_grouped_rows(const moe_mx_handle *h, int num_tokens, int top_
 {
     if (!h || num_tokens < 0 || top_k < 1)
         return 0;
-    return grouped_rows_bound(h->E, (int64_t)num_tokens * top_k);
+    return grouped_rows_bound(h->E, (int64_t)num_tokens * (top_k + h->S));
 }
 
 int moe_mx_create(moe_mx_handle **out, int hidden, int inter, int num_experts, int max_tokens, int max_top_k,
                   int device)
+{
+    return moe_mx_create_ex(out, hidden, inter, num_experts, 0, max_tokens, max_top_k, device);
+}
+
+int moe_mx_create_ex(moe_mx_handle **out, int hidden, int inter, int num_experts, int num_shared, int max_tokens,
+                     int max_top_k, int device)
 {
     g_last_error.clear();
     if (!out)
@@ -195,6 +203,10 @@ int moe_mx_create(moe_mx_handle **out, int hidden, int inter, int num_experts, i
         return fail(MOE_MX_ERR_INVALID_ARG, "max_tokens=%d must be in [1, 65536]", max_tokens);
     if (max_top_k < 1 || max_top_k > kMaxTopK)
         return fail(MOE_MX_ERR_INVALID_ARG, "max_top_k=%d must be in [1, %d]", max_top_k, kMaxTopK);
+    if (num_shared < 0 || num_experts + num_shared > kMaxExperts || max_top_k + num_shared > kMaxTopK)
+        return fail(MOE_MX_ERR_UNSUPPORTED,
+                    "num_shared=%d: need num_experts + num_shared <= %d and max_top_k + num_shared <= %d",
+                    num_shared, kMaxExperts, kMaxTopK);
     int ndev = 0;
     cudaError_t ce = cudaGetDeviceCount(&ndev);
     if (ce != cudaSuccess)
@@ -215,13 +227,14 @@ int moe_mx_create(moe_mx_handle **out, int hidden, int inter, int num_experts, i
     moe_mx_handle *h = new moe_mx_handle();
     h->H = hidden;
     h->I = inter;
-    h->E = num_experts;
+    h->E = num_experts + num_shared;
+    h->S = num_shared;
     h->maxT = max_tokens;
     h->maxK = max_top_k;
     h->dev = device;
     h->num_sms = prop.multiProcessorCount;
-    const int64_t pairs = (int64_t)max_tokens * max_top_k;
-    h->max_rows = grouped_rows_bound(num_experts, pairs);
+    const int64_t pairs = (int64_t)max_tokens * (max_top_k + num_shared);
+    h->max_rows = grouped_rows_bound(h->E, pairs);
     h->scale_layout = MOE_MX_SCALES_ROW_MAJOR;
     h->tile_rows = env_int("MOE_MX_TILE_ROWS", 0);
     if (h->tile_rows != 16 && h->tile_rows != 32 && h->tile_rows != 64 && h->tile_rows != kBlockRows)
@@ -241,9 +254,9 @@ int moe_mx_create(moe_mx_handle **out, int hidden, int inter, int num_experts, i
     } parts[] = {
         {(void **)&h->topk_ids, sizeof(int32_t) * pairs},
         {(void **)&h->topk_w, sizeof(float) * pairs},
-        {(void **)&h->chunk_hist, sizeof(int32_t) * nchunks * num_experts},
-        {(void **)&h->counts, sizeof(int32_t) * num_experts},
-        {(void **)&h->pad_offsets, sizeof(int32_t) * (num_experts + 1)},
+        {(void **)&h->chunk_hist, sizeof(int32_t) * nchunks * h->E},
+        {(void **)&h->counts, sizeof(int32_t) * h->E},
+        {(void **)&h->pad_offsets, sizeof(int32_t) * (h->E + 1)},
         {(void **)&h->rowblocks, sizeof(int4) * (h->max_rows / 16)}, // work blocks: >= 16 padded rows each
         {(void **)&h->num_rowblocks, sizeof(int32_t)},
         {(void **)&h->unit_counters, 2 * sizeof(int32_t)}, // FC1, FC2 work-unit counters
@@ -337,9 +350,12 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
         return fail(MOE_MX_ERR_INVALID_ARG, "handle is NULL");
     if (num_tokens < 0 || num_tokens > h->maxT)
         return fail(MOE_MX_ERR_INVALID_ARG, "num_tokens=%d must be in [0, %d]", num_tokens, h->maxT);
-    if (!given_ids && (top_k < 1 || top_k > h->maxK || top_k > h->E))
-        return fail(MOE_MX_ERR_INVALID_ARG, "top_k=%d must be in [1, min(E=%d, max_top_k=%d)]", top_k, h->E,
-                    h->maxK);
+    if (!given_ids && (top_k < 1 || top_k > h->maxK || top_k > h->E - h->S))
+        return fail(MOE_MX_ERR_INVALID_ARG, "top_k=%d must be in [1, min(E=%d, max_top_k=%d)]", top_k,
+                    h->E - h->S, h->maxK);
+    if (given_ids && h->S > 0)
+        return fail(MOE_MX_ERR_UNSUPPORTED, "the routed form takes no shared expert (handle has %d shared chunks)",
+                    h->S);
     if (given_ids && (top_k < 1 || top_k > h->maxK))
         return fail(MOE_MX_ERR_INVALID_ARG, "top_k=%d must be in [1, max_top_k=%d]", top_k, h->maxK);
     if (given_ids && id_offset < 0)
@@ -365,7 +381,8 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
     if (reinterpret_cast<uintptr_t>(w1) % 32 != 0 || reinterpret_cast<uintptr_t>(w2) % 32 != 0)
         return fail(MOE_MX_ERR_INVALID_ARG, "w1 and w2 must be 32-byte aligned");
 
-    const int H = h->H, I = h->I, E = h->E, T = num_tokens, k = top_k;
+    // E: expert slots; k: slots per token (the routed top_k, then the shared expert's chunks)
+    const int H = h->H, I = h->I, E = h->E, T = num_tokens, k = top_k + h->S;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int prev = 0;
     cudaGetDevice(&prev);
@@ -414,6 +431,7 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
         ra.given_ids = given_ids;
         ra.given_w = given_w;
         ra.id_offset = id_offset;
+        ra.n_shared = h->S;
         // Each kernel after the router may launch while its predecessor still runs (programmatic
         // dependent launch): the FC GEMMs start streaming their weights early.  Stage timing
         // records events between the kernels, so timed forwards launch them one after another.

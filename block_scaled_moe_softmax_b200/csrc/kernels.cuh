@@ -40,8 +40,8 @@ constexpr int kRouteThreads = 1024; // 32 warps: two tokens of a 64-token chunk 
 constexpr int kSmallRouteTokens = 64; // at most this many tokens: routing and grouping in one CTA
 
 struct RouteGroupArgs {
-    const float *logits;
-    int T, E, k;
+    const float *logits;   // [T, E - n_shared]: the routed experts' logits
+    int T, E, k;           // E, k: expert slots and slots per token, shared ones included
     int32_t *topk_ids;
     float *topk_w;
     int32_t *chunk_hist;
@@ -59,6 +59,10 @@ struct RouteGroupArgs {
     const int32_t *given_ids = nullptr;
     const float *given_w = nullptr;
     int id_offset = 0;
+    // Shared expert: its n_shared chunks are expert slots E - n_shared.., and every token's
+    // last n_shared slots route to them with weight 1 (the router picks k - n_shared routed
+    // experts among the first E - n_shared).  Logits form only.
+    int n_shared = 0;
 };
 
 // Launchers of the forward's kernels.  pdl: launch as programmatic dependents of the kernel

@@ -25,9 +25,11 @@ namespace moe_mx {
 // Route one token (whole warp): the k experts in descending logit order, the lowest index
 // first among equal logits, and their weights = the softmax over the selected logits.  Lane j
 // (j < k) writes the j-th id and weight and adds it to the block's expert histogram.
+// With n_shared > 0 the token has k + n_shared slots: after the k routed ones, the shared
+// expert's chunks (expert slots E.., weight 1).
 template <int kPerLane> // experts per lane: E <= 32 * kPerLane
-__device__ __forceinline__ void route_token(const float *__restrict__ row, int E, int k, int t, int lane,
-                                            int32_t *__restrict__ topk_ids, float *__restrict__ topk_w,
+__device__ __forceinline__ void route_token(const float *__restrict__ row, int E, int k, int n_shared, int t,
+                                            int lane, int32_t *__restrict__ topk_ids, float *__restrict__ topk_w,
                                             int32_t *hist)
 {
     float v[kPerLane];
@@ -83,10 +85,15 @@ __device__ __forceinline__ void route_token(const float *__restrict__ row, int E
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1)
         z += __shfl_xor_sync(0xFFFFFFFFu, z, off);
+    const int slots = k + n_shared;
     if (lane < k) {
-        topk_ids[(size_t)t * k + lane] = my_id;
-        topk_w[(size_t)t * k + lane] = u / z;
+        topk_ids[(size_t)t * slots + lane] = my_id;
+        topk_w[(size_t)t * slots + lane] = u / z;
         atomicAdd(&hist[my_id], 1);
+    } else if (lane < slots) {
+        topk_ids[(size_t)t * slots + lane] = E + (lane - k);
+        topk_w[(size_t)t * slots + lane] = 1.0f;
+        atomicAdd(&hist[E + (lane - k)], 1);
     }
 }
 
@@ -116,7 +123,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float *__res
                                                                float *__restrict__ topk_w,
                                                                int32_t *__restrict__ chunk_hist,
                                                                const int32_t *__restrict__ gids,
-                                                               const float *__restrict__ gw, int off)
+                                                               const float *__restrict__ gw, int off, int n_shared)
 {
     grid_dep_launch(); // the next kernel (the scan) waits for this grid before reading its output
     __shared__ int32_t hist[kMaxExperts];
@@ -130,7 +137,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float *__res
         if (gids)
             take_given_token(gids, gw, E, k, off, t, lane, topk_ids, topk_w, hist);
         else
-            route_token<kPerLane>(logits + (size_t)t * E, E, k, t, lane, topk_ids, topk_w, hist);
+            route_token<kPerLane>(logits + (size_t)t * (E - n_shared), E - n_shared, k - n_shared, n_shared, t, lane,
+                                  topk_ids, topk_w, hist);
     }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x)
@@ -287,7 +295,8 @@ __global__ void __launch_bounds__(1024) route_group_small_kernel(const RouteGrou
         if (a.given_ids)
             take_given_token(a.given_ids, a.given_w, a.E, a.k, a.id_offset, t, lane, a.topk_ids, a.topk_w, hist);
         else
-            route_token<kPerLane>(a.logits + (size_t)t * a.E, a.E, a.k, t, lane, a.topk_ids, a.topk_w, hist);
+            route_token<kPerLane>(a.logits + (size_t)t * (a.E - a.n_shared), a.E - a.n_shared, a.k - a.n_shared,
+                                  a.n_shared, t, lane, a.topk_ids, a.topk_w, hist);
     }
     __syncthreads(); // also makes lane 0's id writes visible to the whole CTA
     const int e = threadIdx.x;
@@ -446,13 +455,13 @@ void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s, bool pdl)
     const int nchunks = (a.T + kRouteChunk - 1) / kRouteChunk;
     if (narrow)
         route_kernel<8><<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist,
-                                                          a.given_ids, a.given_w, a.id_offset);
+                                                          a.given_ids, a.given_w, a.id_offset, a.n_shared);
     else if (a.E <= 512)
         route_kernel<16><<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist,
-                                                          a.given_ids, a.given_w, a.id_offset);
+                                                          a.given_ids, a.given_w, a.id_offset, a.n_shared);
     else
         route_kernel<32><<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist,
-                                                          a.given_ids, a.given_w, a.id_offset);
+                                                          a.given_ids, a.given_w, a.id_offset, a.n_shared);
     launch_kernel(scan_kernel, dim3(1), dim3(1024), 0, s, pdl, a.E, nchunks, a.split_rows, a.chunk_hist, a.counts,
                   a.pad_offsets, a.rowblocks, a.num_rowblocks, a.sorted_pair, a.unit_counters);
     launch_kernel(scatter_kernel, dim3(nchunks), dim3(32), 0, s, pdl, a.T, a.E, a.k, (const int32_t *)a.topk_ids,

@@ -40,6 +40,7 @@ MOE_MX_W2 = 1
 _P, _I, _I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
 SIGNATURES = {
     "moe_mx_create": (_I, [ctypes.POINTER(_P), _I, _I, _I, _I, _I, _I]),
+    "moe_mx_create_ex": (_I, [ctypes.POINTER(_P), _I, _I, _I, _I, _I, _I, _I]),
     "moe_mx_forward": (_I, [_P, _P, _P, _I, _P, _P, _P, _P, _I, _I, _P, _P]),
     "moe_mx_forward_routed": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _I, _P, _I, _P]),
     "moe_mx_destroy": (_I, [_P]),
@@ -123,6 +124,14 @@ def moe_mx_create(hidden: int, inter: int, num_experts: int, max_tokens: int, ma
     return h.value
 
 
+def moe_mx_create_ex(hidden: int, inter: int, num_experts: int, num_shared: int, max_tokens: int, max_top_k: int,
+                     device: int = 0) -> int:
+    h = ctypes.c_void_p()
+    _check(load_library().moe_mx_create_ex(ctypes.byref(h), hidden, inter, num_experts, num_shared, max_tokens,
+                                           max_top_k, device))
+    return h.value
+
+
 def moe_mx_destroy(handle: int) -> None:
     _check(load_library().moe_mx_destroy(handle))
 
@@ -197,10 +206,12 @@ class MoeMxLayer:
     """Owns a moe_mx handle for fixed (H, I, E) and runs forwards on torch tensors."""
 
     def __init__(self, hidden: int, inter: int, num_experts: int, max_tokens: int, max_top_k: int,
-                 device: int | None = None):
-        self.H, self.I, self.E = hidden, inter, num_experts
+                 device: int | None = None, num_shared: int = 0):
+        """num_experts routed experts; num_shared > 0 adds a shared expert held as that many
+        extra expert slots of the weights (see moe_mx_create_ex)."""
+        self.H, self.I, self.E, self.S = hidden, inter, num_experts, num_shared
         self.device = torch.cuda.current_device() if device is None else device
-        self.handle = moe_mx_create(hidden, inter, num_experts, max_tokens, max_top_k, self.device)
+        self.handle = moe_mx_create_ex(hidden, inter, num_experts, num_shared, max_tokens, max_top_k, self.device)
 
     def forward(self, x: torch.Tensor, router_logits: torch.Tensor, w1, w1_scale, w2, w2_scale, top_k: int,
                 act_dtype: int = MOE_MX_ACT_BF16, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
@@ -237,10 +248,11 @@ class MoeMxLayer:
         """The routing/grouping state of the most recent forward (device tensors)."""
         dev = torch.device("cuda", self.device)
         rows = moe_mx_max_grouped_rows(self.handle, T, top_k)
-        ids = torch.empty(T, top_k, dtype=torch.int32, device=dev)
-        w = torch.empty(T, top_k, dtype=torch.float32, device=dev)
-        counts = torch.empty(self.E, dtype=torch.int32, device=dev)
-        pad = torch.empty(self.E + 1, dtype=torch.int32, device=dev)
+        slots = top_k + self.S  # the routed slots, then the shared expert's chunks
+        ids = torch.empty(T, slots, dtype=torch.int32, device=dev)
+        w = torch.empty(T, slots, dtype=torch.float32, device=dev)
+        counts = torch.empty(self.E + self.S, dtype=torch.int32, device=dev)
+        pad = torch.empty(self.E + self.S + 1, dtype=torch.int32, device=dev)
         sp = torch.empty(rows, dtype=torch.int32, device=dev)
         moe_mx_get_routing(self.handle, ids, w, counts, pad, sp, stream)
         return ids, w, counts, pad, sp

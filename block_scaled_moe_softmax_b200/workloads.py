@@ -20,6 +20,8 @@ Workloads with the routing given (precomputed top-k) draw it instead of logits:
          (the weights a router would hand over: positive, summing to 1)
 Such a workload runs one contiguous shard of E local experts, global ids
 [local_offset, local_offset + E); its weights are drawn per local expert.
+A workload with a shared expert draws its `shared` chunks like experts
+E..E+shared-1 (the same per-expert N(0, 0.02) generators).
 The float32 weights are then quantised to MXFP4 along the reduction dim by the
 caller (the oracle's quantiser in tests, the library's quantiser in the bench;
 the two are checked bit-exact against each other).
@@ -50,6 +52,12 @@ class Workload:
     routing: str = "logits"    # "logits" (router) or "given" (precomputed top-k, global ids)
     experts_global: int = 0    # given routing: experts of the whole layer (0: E)
     local_offset: int = 0      # given routing: global id of local expert 0
+    shared: int = 0            # shared-expert chunks of I, held as weight slots E..E+shared-1
+
+    @property
+    def slots(self) -> int:
+        """Expert weight slots: the routed experts, then the shared expert's chunks."""
+        return self.E + self.shared
 
     @property
     def pairs(self) -> int:
@@ -79,6 +87,9 @@ WORKLOADS = {
     # the w4a8 prefill shape with 4096 tokens: a capture-sized case (about 2.5 GB on the device)
     "prefill_w4a8_t4k": Workload("prefill_w4a8_t4k", 4096, 4096, 1536, 128, 8, "mxfp8", "none", 0,
                                  "prefill-shaped, w4a8, 4096 tokens (profiling case)"),
+    # the decode shape with a shared expert of intermediate size I added to every token
+    "decode_shared": Workload("decode_shared", 16, 7168, 2048, 384, 8, "bf16", "none", 0,
+                              "decode-shaped, w4a16, plus one shared expert (I = 2048)", shared=1),
     # the hidden size, expert count and top-k of the TokenSpeed SiTU bundle's supported contract, with the
     # routing given as precomputed top-k: TP8 (all 896 experts, intermediate shard 384) and the
     # first EP8 shard (112 local experts of 896, intermediate 3072); 128 tokens

@@ -113,6 +113,29 @@ MOE_MX_API int moe_mx_create(moe_mx_handle **out, int hidden, int inter, int num
                   int max_top_k, int device);
 
 /*
+ * moe_mx_create with a shared expert (mxfp6-sm120 package description, routed-MoE
+ * path: "shared-expert combine and routed/shared reduction"): every token also
+ * passes through a shared SwiGLU expert of intermediate size num_shared * inter,
+ * whose output is added to the routed sum with weight 1 in the same combine.
+ *   num_shared  S >= 0: the shared expert is held as S chunks of `inter` in
+ *               expert slots num_experts .. num_experts + S - 1 of the weight
+ *               tensors, which then hold num_experts + S slots ([E + S, ...]).
+ *               Chunk c holds gate rows c*I .. c*I + I - 1 of the shared W1
+ *               followed by the matching up rows, and columns c*I .. c*I + I - 1
+ *               of the shared W2 (SwiGLU acts element by element along the
+ *               intermediate dimension, so the chunks' outputs add up to the
+ *               shared expert's output).  S = 0 is moe_mx_create.
+ * The router sees the routed experts only: router_logits stay [T, num_experts].
+ * A token has top_k + S slots; moe_mx_get_routing reports them in that order
+ * (the shared slots: ids num_experts.., weight 1) and counts / pad_offsets over
+ * all E + S slots.  num_experts + S <= 1024 and max_top_k + S <= 32, else
+ * MOE_MX_ERR_UNSUPPORTED.  moe_mx_forward_routed takes no shared expert
+ * (a handle with S > 0 rejects it with MOE_MX_ERR_UNSUPPORTED).
+ */
+MOE_MX_API int moe_mx_create_ex(moe_mx_handle **out, int hidden, int inter, int num_experts, int num_shared,
+                                int max_tokens, int max_top_k, int device);
+
+/*
  * Run the layer: out = MoE(x) for num_tokens tokens, enqueued on `stream`.
  *   x              bf16 [T, H] activations.
  *   router_logits  float32 [T, E] router logits (any per-expert bias already
@@ -217,9 +240,10 @@ MOE_MX_API int moe_mx_quantize(const float *src, int64_t rows, int64_t K, int fm
 MOE_MX_API int moe_mx_block_rows(void);
 
 /*
- * Number of rows of the padded grouped layout the most recent forward of T
- * tokens and top_k slots may occupy at most: T*k + E*(block_rows-1), rounded
- * up to block_rows.  Host-only arithmetic.
+ * Number of rows of the padded grouped layout a forward of T tokens and top_k
+ * routed slots may occupy at most: P + min(P, E)*(block_rows-1) with P = T*(top_k
+ * + S) pairs (S shared chunks, E expert slots), rounded up to block_rows.
+ * Host-only arithmetic.
  */
 MOE_MX_API int64_t moe_mx_max_grouped_rows(const moe_mx_handle *h, int num_tokens, int top_k);
 

@@ -17,7 +17,7 @@ def quantize_weights_cpu(wl, experts=None, fp32_override=None):
     Returns dict with w1, w1s, w2, w2s (numpy uint8, the C-ABI layouts).
     fp32_override: optional (w1_f32 [E,2I,H], w2_f32 [E,H,I]) numpy arrays to quantise instead.
     """
-    E, H, I = wl.E, wl.H, wl.I
+    E, H, I = wl.slots, wl.H, wl.I  # routed experts, then the shared expert's chunks
     w1 = np.zeros((E, 2 * I, H // 2), np.uint8)
     w1s = np.zeros((E, 2 * I, H // 32), np.uint8)
     w2 = np.zeros((E, H, I // 2), np.uint8)
@@ -88,7 +88,8 @@ def oracle_forward(inp, top_k, act_mode, tokens=None):
     the final bf16 rounding -- a bf16 result is measured against the value it rounds, not
     against a second, independent rounding of it -- plus the ids and weights."""
     _, ids, w, exact = oracle.moe_forward(inp["xb"], inp["logits"].numpy(), inp["w1"], inp["w1s"], inp["w2"],
-                                          inp["w2s"], top_k, act_mode, tokens=tokens, exact=True)
+                                          inp["w2s"], top_k, act_mode, tokens=tokens, exact=True,
+                                          num_shared=inp["w1"].shape[0] - inp["logits"].shape[1])
     return exact, ids, w
 
 
