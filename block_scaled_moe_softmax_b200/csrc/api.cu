@@ -140,6 +140,7 @@ struct moe_mx_handle {
     int swap_rows;
     int tile_rows; // 0: by token count; else 16, 32, 64 or 128 (MOE_MX_TILE_ROWS)
     int pdl;       // launch the kernels after the router as programmatic dependents (MOE_MX_PDL, default 1)
+    int wide;      // 128-row GEMM blocks: the two-tile (N = 256) variant (MOE_MX_WIDE, default 1)
     int scale_layout; // MOE_MX_SCALES_ROW_MAJOR or MOE_MX_SCALES_TILED
     unsigned long long timeout_ns;
     void *ws;
@@ -240,6 +241,7 @@ int moe_mx_create_ex(moe_mx_handle **out, int hidden, int inter, int num_experts
     if (h->tile_rows != 16 && h->tile_rows != 32 && h->tile_rows != 64 && h->tile_rows != kBlockRows)
         h->tile_rows = 0;
     h->pdl = env_int("MOE_MX_PDL", 1) != 0;
+    h->wide = env_int("MOE_MX_WIDE", 1) != 0;
     h->swap_rows = env_int("MOE_MX_SWAP_ROWS", 64);
     if (h->swap_rows < 0)
         h->swap_rows = 0;
@@ -465,6 +467,7 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
         f1.act_mxfp8 = mx8;
         f1.swap_rows = h->swap_rows;
         f1.max_block_rows = tile_rows;
+        f1.wide = h->wide;
         mark(2);
         const int sw_idx = tile_rows <= 16 ? 0 : tile_rows <= 32 ? 1 : 2; // box rows min(tile rows, 64)
         launch_fc_gemm(f1, h->map_A[f1.terms - 1], h->map_Asw[f1.terms - 1][sw_idx], h->map_A16, h->map_w1, h->num_sms,

@@ -105,9 +105,19 @@ template <int kActRows, int kMmaW, int kWTiles, int kTm> struct Plan {
     static constexpr int kMma = kMmaW;
     static_assert(kMma == 1 || kStages % 2 == 0, "alternating MMA warps need an even stage count");
     static_assert(kMma == 1 || kActRows <= 32, "two accumulators per buffer need N <= 64");
-    static_assert(kWT == 1 || (kWT == 2 && kMma == 1 && kActRows <= 32), "two weight tiles: one MMA warp, N <= 64");
-    // warps: producer 0, MMA 0, 4 epilogue, producers 1.., MMA 1 (if any), the scheduler
-    static constexpr int kThreads = 32 * (2 + 4 + (kProd - 1) + (kMma - 1) + 1);
+    static_assert(kWT == 1 || (kWT == 2 && kMma == 1 && (kActRows <= 32 || kActRows == 128)),
+                  "two weight tiles: one MMA warp, N <= 64 or the wide 128-row variant");
+    // The wide variant (128 token rows against two weight tiles, tokens on M): one M = 128,
+    // N = 256 MMA per K block covers both tiles, so each activation byte brought into shared
+    // memory feeds twice the MMA work.  Its 256-column accumulator leaves no room in TMEM for a
+    // second one beside the scale factors, so it is single-buffered; 8 epilogue warps (two per
+    // TMEM lane quarter, one per tile) copy it to registers and release it at once.
+    static constexpr bool kWide = kActRows == 128 && kWT == 2;
+    static constexpr int kEpiWarps = kWide ? 8 : 4;
+    // warps: producer 0, MMA 0, 4 epilogue, producers 1.., MMA 1 (if any), 4 more epilogue
+    // (wide), the scheduler
+    static constexpr int kEpi2 = 5 + kProd + (kMma - 1); // first warp of the second epilogue group
+    static constexpr int kThreads = 32 * (2 + kEpiWarps + (kProd - 1) + (kMma - 1) + 1);
     static constexpr int kOffAct = 0;
     static constexpr int kOffW = kOffAct + kStages * kActBytes;
     static constexpr int kOffAsf = kOffW + kStages * kWStage;
@@ -295,7 +305,7 @@ __device__ __forceinline__ void producer_role(const FcGemmArgs &a, const Ctx &c,
         if (blk.w < 0)
             break;
         const int nt0 = (blk.w % c.n_groups) * kWT; // the unit's first weight tile
-        const bool swap = kActRows < 128 || blk.z <= a.swap_rows;
+        const bool swap = !P::kWide && (kActRows < 128 || blk.z <= a.swap_rows); // wide: tokens on M always
         const int npad = (blk.z + 15) & ~15;
         const bool comb = swap && terms > 1 && npad <= P::kT2; // both terms on N of one MMA
         const int rb = blk.y / 128, o = blk.y & 127;
@@ -529,6 +539,146 @@ __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
     mbar_wait_bounded(bars.mma_done(), 0, nullptr, kDrainTimeoutNs);
 }
 
+// MMA role of the wide variant (warp 1): per K block one M = 128 (token rows) x N = 256 (both
+// weight tiles, contiguous in shared memory) block-scaled MMA per activation term, into the
+// single accumulator at TMEM columns 0..255.  Scale factors: the two weight atoms at kSfCol and
+// kSfCol + 4 (rows 0..127 and 128..255 of N), the activation atoms after them.
+template <int kActRows, int kMmaW, int kWTiles, int kTm>
+__device__ __forceinline__ void mma_role_wide(const FcGemmArgs &a, const Ctx &c)
+{
+    using P = Plan<kActRows, kMmaW, kWTiles, kTm>;
+    constexpr int kStages = P::kStages, kTermBytes = P::kTermBytes, kActBytes = P::kActBytes;
+    const Bars<kStages> bars{c.base + P::kOffBar};
+    const uint32_t base = c.base, tmem_base = c.tmem_base;
+    const int kst = c.kst, terms = c.terms;
+    const unsigned long long tmo = c.tmo;
+    uint32_t g = 0, cnt = 0;
+    bool ok = true;
+    const uint32_t sf_w = tmem_base + kSfCol, sf_act = sf_w + 8;
+    const uint64_t dact0 = smem_desc_sw128(base + P::kOffAct), dw0 = smem_desc_sw128(base + P::kOffW);
+    static_assert(P::kSmemBytes + 1024 < (1 << 18), "descriptor start field arithmetic needs addresses < 2^18");
+    const uint32_t idesc0 = idesc_mx(kFmtE4M3, kFmtE2M1, 128, 256, 0);
+    const UnitRing<kStages> ring{bars, c.units};
+    const int lane = threadIdx.x & 31;
+    for (; ok; ++cnt) {
+        const int4 blk = ring.take(cnt, a.err, tmo, lane);
+        if (blk.w < 0)
+            break;
+        // the accumulator is free once the epilogue has copied the previous unit's out of TMEM
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.acc_empty(0), (cnt & 1) ^ 1, a.err, tmo))) {
+            ok = false;
+            break;
+        }
+        tc_fence_after();
+        for (int kk = 0; kk < kst; ++kk, ++g) {
+            const int s = g % kStages;
+            const uint32_t ph = (g / kStages) & 1;
+            const uint32_t wsf_s = base + P::kOffWsf + s * P::kWsfStage;
+            const uint32_t asf_s = base + P::kOffAsf + s * kAsfBytes;
+            const uint64_t ds_act = dact0 + (uint64_t)((s * kActBytes) >> 4);
+            const uint64_t ds_w = dw0 + (uint64_t)((s * P::kWStage) >> 4);
+            uint64_t opa[4][2], opb[4];
+            uint32_t idesc[4], accf[4];
+#pragma unroll
+            for (int k32 = 0; k32 < 4; ++k32) {
+                idesc[k32] = idesc0 | ((uint32_t)k32 << 4) | ((uint32_t)k32 << 29);
+                accf[k32] = (kk == 0 && k32 == 0) ? 0u : 1u;
+                opb[k32] = ds_w + 2u * k32; // +32 bytes per K block
+#pragma unroll
+                for (int t = 0; t < 2; ++t)
+                    opa[k32][t] = ds_act + (uint64_t)((t * kTermBytes) >> 4) + 2u * k32;
+            }
+            const uint32_t empty_s = bars.empty(s);
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.full(s), ph, a.err, tmo))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            if (elect_one()) {
+                tmem_cp_sf_atom(sf_w, wsf_s);
+                tmem_cp_sf_atom(sf_w + 4, wsf_s + kWsfBytes);
+                tmem_cp_sf_atom(sf_act, asf_s);
+                if (terms > 1)
+                    tmem_cp_sf_atom(sf_act + 4, asf_s + 512);
+#pragma unroll
+                for (int k32 = 0; k32 < 4; ++k32) {
+                    umma_mx(tmem_base, opa[k32][0], opb[k32], idesc[k32], sf_act, sf_w, accf[k32]);
+                    if (terms > 1)
+                        umma_mx(tmem_base, opa[k32][1], opb[k32], idesc[k32], sf_act + 4, sf_w, 1u);
+                }
+                umma_commit(empty_s);
+            }
+            __syncwarp();
+        }
+        if (ok && elect_one())
+            umma_commit(bars.acc_full(0));
+        __syncwarp();
+    }
+    // all MMAs must have completed before TMEM is released
+    if (elect_one())
+        umma_commit(bars.mma_done());
+    __syncwarp();
+    mbar_wait_bounded(bars.mma_done(), 0, nullptr, kDrainTimeoutNs);
+}
+
+// Epilogue of the wide variant: 8 warps, two per TMEM lane quarter; the warps of the first
+// group (2..5) take weight tile 0 of the unit (accumulator columns 0..127), those of the second
+// (kEpi2..kEpi2+3) tile 1 (columns 128..255).  A thread owns one token row: it copies its 128
+// columns to registers, releases the accumulator, then forms its output (FC1: h = silu(gate) *
+// up for the tile's 64 gate / 64 up rows, written as FC2's operand; FC2: f32 rows of Y).
+template <int kActRows, int kMmaW, int kWTiles, int kTm>
+__device__ __forceinline__ void epilogue_wide(const FcGemmArgs &a, const Ctx &c, int warp, int lane)
+{
+    using P = Plan<kActRows, kMmaW, kWTiles, kTm>;
+    const Bars<P::kStages> bars{c.base + P::kOffBar};
+    const UnitRing<P::kStages> ring{bars, c.units};
+    const int q = warp & 3;                     // TMEM lane quarter this warp may access
+    const int half = warp >= P::kEpi2 ? 1 : 0;  // the unit's weight tile this warp writes
+    for (uint32_t cnt = 0;; ++cnt) {
+        const int4 blk = ring.take(cnt, a.err, c.tmo, lane);
+        // the eight epilogue warps leave together (they share named barrier 2)
+        if (!named_bar_all(2, 256, blk.w >= 0))
+            break;
+        const int nt = (blk.w % c.n_groups) * 2 + half;
+        const bool got = mbar_wait_bounded(bars.acc_full(0), cnt & 1, a.err, c.tmo);
+        if (!named_bar_all(2, 256, got))
+            break;
+        tc_fence_after();
+        const uint32_t tb = c.tmem_base + ((uint32_t)(32 * q) << 16) + 128u * half;
+        uint32_t v[8][16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            tmem_ld16(tb + 16 * j, v[j]);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bars.acc_empty(0)); // the MMA warp may overwrite the accumulator now
+        const int rl = 32 * q + lane;
+        const bool valid = rl < blk.z;
+        const int row = blk.y + rl;
+        if (a.fc1) {
+            // columns 0..63: gate rows nt*64 + i, columns 64..127: the matching up rows
+#pragma unroll
+            for (int c32 = 0; c32 < 2; ++c32) {
+                float h[32];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    h[i] = silu_mul(__uint_as_float(v[2 * c32][i]), __uint_as_float(v[4 + 2 * c32][i]));
+                    h[16 + i] = silu_mul(__uint_as_float(v[2 * c32 + 1][i]), __uint_as_float(v[5 + 2 * c32][i]));
+                }
+                if (valid)
+                    store_act_block32(a.hq, a.hsf, a.hq_rows, a.out_ld, row, nt * 64 + 32 * c32, h, a.act_mxfp8);
+            }
+        } else if (valid) {
+            uint4 *dst = reinterpret_cast<uint4 *>(a.y + (size_t)row * a.out_ld + nt * 128);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[4 * j + i] = make_uint4(v[j][4 * i], v[j][4 * i + 1], v[j][4 * i + 2], v[j][4 * i + 3]);
+        }
+    }
+}
+
 template <int kActRows, int kMmaW, int kWTiles, int kTm>
 __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads, 1)
     fc_gemm_kernel(const FcGemmArgs a, const __grid_constant__ CUtensorMap act_map,
@@ -555,11 +705,11 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads,
         mbar_init(bars.mma_done(), kMma);
         for (int b = 0; b < 2; ++b) {
             mbar_init(bars.acc_full(b), kMma); // every MMA warp commits every unit
-            mbar_init(bars.acc_empty(b), 128);
+            mbar_init(bars.acc_empty(b), 32 * P::kEpiWarps);
         }
         for (int r = 0; r < kRing; ++r) {
-            mbar_init(bars.ring_full(r), 1);                  // the scheduler's publish
-            mbar_init(bars.ring_empty(r), kProd + kMma + 4);  // one release per reading warp
+            mbar_init(bars.ring_full(r), 1);                             // the scheduler's publish
+            mbar_init(bars.ring_empty(r), kProd + kMma + P::kEpiWarps);  // one release per reading warp
         }
         fence_mbar_init();
         fence_proxy_async_smem();
@@ -602,7 +752,12 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads,
         else if (warp == 8)
             producer_role<kActRows, kMmaW, kWTiles, kTm, 3 % kProd>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
     } else if (warp == 1) {
-        mma_role<kActRows, kMmaW, kWTiles, kTm, 0>(a, ctx);
+        if constexpr (P::kWide)
+            mma_role_wide<kActRows, kMmaW, kWTiles, kTm>(a, ctx);
+        else
+            mma_role<kActRows, kMmaW, kWTiles, kTm, 0>(a, ctx);
+    } else if (P::kWide && ((warp >= 2 && warp < 6) || (warp >= P::kEpi2 && warp < P::kEpi2 + 4))) {
+        epilogue_wide<kActRows, kMmaW, kWTiles, kTm>(a, ctx, warp, lane);
     } else if (kMma > 1 && warp == 5 + kProd) {
         mma_role<kActRows, kMmaW, kWTiles, kTm, (kMma > 1 ? 1 : 0)>(a, ctx);
     } else if (warp == P::kThreads / 32 - 1) {
@@ -754,9 +909,10 @@ cudaError_t fc_gemm_prepare()
     if ((e = prepare_one<16, 1, 1, 2>()) != cudaSuccess || (e = prepare_one<16, 2, 1, 2>()) != cudaSuccess ||
         (e = prepare_one<16, 1, 2, 2>()) != cudaSuccess || (e = prepare_one<32, 1, 1, 2>()) != cudaSuccess ||
         (e = prepare_one<32, 2, 1, 2>()) != cudaSuccess || (e = prepare_one<32, 1, 2, 2>()) != cudaSuccess ||
-        (e = prepare_one<64, 1, 1, 2>()) != cudaSuccess || (e = prepare_one<128, 1, 1, 2>()) != cudaSuccess)
+        (e = prepare_one<64, 1, 1, 2>()) != cudaSuccess || (e = prepare_one<128, 1, 1, 2>()) != cudaSuccess ||
+        (e = prepare_one<128, 1, 1, 1>()) != cudaSuccess || (e = prepare_one<128, 1, 2, 2>()) != cudaSuccess)
         return e;
-    return prepare_one<128, 1, 1, 1>();
+    return prepare_one<128, 1, 2, 1>();
 }
 
 template <int kActRows, int kMmaW, int kWTiles, int kTm>
@@ -793,6 +949,14 @@ void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUten
             launch_one<32, 1, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
     } else if (a.max_block_rows <= 64) {
         launch_one<64, 1, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
+    } else if (a.wide && a.n_tiles % 2 == 0) {
+        // the wide variant (two weight tiles per unit, N = 256 MMAs): half the activation bytes
+        // per MMA of the one-tile variant (the 128-row GEMMs were bound by the shared-memory fill
+        // from L2, not by the tensor pipe)
+        if (a.terms == 1)
+            launch_one<128, 1, 2, 1>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
+        else
+            launch_one<128, 1, 2, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
     } else if (a.terms == 1) {
         // single-term activations (w4a8 FC1): the smaller stages leave room for 6 of them
         // instead of 4, i.e. more bytes in flight per SM

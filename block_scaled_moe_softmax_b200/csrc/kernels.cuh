@@ -106,6 +106,8 @@ struct FcGemmArgs {
     int wsf_tiled;               // 1: wscale is in the tiled atom layout (one bulk copy per stage)
     int max_block_rows;          // upper bound on any row block's rows: 16, 32, 64 or 128; selects
                                  // the kernel variant (activation tile rows per term)
+    int wide;                    // 128-row blocks: two weight tiles per work unit (tokens on M) when
+                                 // n_tiles is even
 };
 
 // Tensor maps: act_map = both term planes, 128-row boxes ([terms][128][128] codes, tokens

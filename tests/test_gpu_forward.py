@@ -36,11 +36,13 @@ SHAPES = {
 }
 
 
-def _run(wl, act_mode, monkeypatch, swap_rows=None, inp=None, tile_rows=None):
+def _run(wl, act_mode, monkeypatch, swap_rows=None, inp=None, tile_rows=None, wide=None):
     if swap_rows is not None:
         monkeypatch.setenv("MOE_MX_SWAP_ROWS", str(swap_rows))
     if tile_rows is not None:
         monkeypatch.setenv("MOE_MX_TILE_ROWS", str(tile_rows))
+    if wide is not None:
+        monkeypatch.setenv("MOE_MX_WIDE", str(wide))
     inp = inp or helpers.host_inputs(wl)
     d = helpers.to_device(inp)
     layer = moe_mx.MoeMxLayer(wl.H, wl.I, wl.E, max(wl.T, 1), wl.top_k)
@@ -49,11 +51,13 @@ def _run(wl, act_mode, monkeypatch, swap_rows=None, inp=None, tile_rows=None):
     return layer, inp, out
 
 
-# (tile rows, swap rows): the 128-row variant in both orientations and mixed, each smaller
-# variant (always tokens on N), and the automatic choice by token count
+# (tile rows, swap rows, wide): the 128-row blocks on the wide two-tile variant (tokens always on
+# M, whatever the swap setting) and on the one-tile variant in both orientations and mixed, each
+# smaller variant (always tokens on N), and the automatic choice by token count
 VARIANTS = {
-    "t128_tokens_on_M": (128, 0), "t128_weights_on_M": (128, 128), "t128_mixed": (128, 64),
-    "t64": (64, None), "t32": (32, None), "t16": (16, None), "auto": (None, None),
+    "t128_wide": (128, 0, None), "t128_wide_swaprows": (128, 128, None),
+    "t128_tokens_on_M": (128, 0, 0), "t128_weights_on_M": (128, 128, 0), "t128_mixed": (128, 64, 0),
+    "t64": (64, None, None), "t32": (32, None, None), "t16": (16, None, None), "auto": (None, None, None),
 }
 
 
@@ -62,8 +66,8 @@ VARIANTS = {
 @pytest.mark.parametrize("variant", list(VARIANTS))
 def test_forward_matches_oracle(name, act_mode, variant, monkeypatch):
     wl = SHAPES[name]
-    tile_rows, swap_rows = VARIANTS[variant]
-    layer, inp, out = _run(wl, act_mode, monkeypatch, swap_rows, tile_rows=tile_rows)
+    tile_rows, swap_rows, wide = VARIANTS[variant]
+    layer, inp, out = _run(wl, act_mode, monkeypatch, swap_rows, tile_rows=tile_rows, wide=wide)
     helpers.check_routing(layer, wl.T, wl.top_k, wl.E, inp["logits"].numpy())
     ref, _, _ = helpers.oracle_forward(inp, wl.top_k, act_mode)
     helpers.check_output(out, ref, f"{name}/{act_mode}/{variant}")
@@ -76,8 +80,8 @@ def test_forward_matches_oracle(name, act_mode, variant, monkeypatch):
 def test_tiled_scales_match_row_major(name, act_mode, variant, monkeypatch):
     """The tiled weight-scale layout (moe_mx_prepare_scales) gives bit-identical outputs."""
     wl = SHAPES[name]
-    tile_rows, swap_rows = VARIANTS[variant]
-    layer, inp, out_rm = _run(wl, act_mode, monkeypatch, swap_rows, tile_rows=tile_rows)
+    tile_rows, swap_rows, wide = VARIANTS[variant]
+    layer, inp, out_rm = _run(wl, act_mode, monkeypatch, swap_rows, tile_rows=tile_rows, wide=wide)
     d = helpers.to_device(inp)
     t1, t2 = layer.prepare_scales(d["w1s"], d["w2s"])
     out_t = layer.forward(d["x"], d["logits"], d["w1"], t1, d["w2"], t2, wl.top_k, act_mode)
