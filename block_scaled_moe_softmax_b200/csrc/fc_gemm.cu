@@ -86,7 +86,9 @@ template <int kActRows, int kMmaW, int kWTiles, int kTm> struct Plan {
     static constexpr int kWT = kWTiles;
     static constexpr int kWStage = kWT * kWBytes, kWsfStage = kWT * kWsfBytes;
     static constexpr int kStageBytes = kActBytes + kWStage + kAsfBytes + kWsfStage;
-    static constexpr int kStages = (kSmemLimit - 1024 - kXBytes - 256) / kStageBytes;
+    // wide variant: a 2 KB staging buffer per epilogue warp for FC2's f32 output rows
+    static constexpr int kYBytes = (kActRows == 128 && kWTiles == 2) ? 8 * 2048 : 0;
+    static constexpr int kStages = (kSmemLimit - 1024 - kXBytes - kYBytes - 256) / kStageBytes;
     // The per-stage copy issue is split over several producer warps (groups of two stages
     // round robin): each TMA instruction and each warp-wide 4-byte scale copy occupies its
     // issuing warp for about a hundred cycles (measured: the cost is per warp, not per SM).
@@ -123,7 +125,8 @@ template <int kActRows, int kMmaW, int kWTiles, int kTm> struct Plan {
     static constexpr int kOffAsf = kOffW + kStages * kWStage;
     static constexpr int kOffWsf = kOffAsf + kStages * kAsfBytes;
     static constexpr int kOffX = kOffWsf + kStages * kWsfStage;
-    static constexpr int kOffBar = kOffX + kXBytes;
+    static constexpr int kOffY = kOffX + kXBytes;
+    static constexpr int kOffBar = kOffY + kYBytes;
     static constexpr int kNumBars = 2 * kStages + 1 + 4 + 2 * kRing;
     static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
     static constexpr int kOffUnits = kOffTmemSlot + 16;                 // the work-unit ring
@@ -268,6 +271,7 @@ __device__ __forceinline__ float silu_mul(float g, float u)
 struct Ctx {
     uint32_t base;        // shared-memory base (1024-byte aligned, shared window)
     volatile int *units;  // the work-unit ring (generic pointer to shared memory)
+    uint8_t *ystage;      // wide variant: the epilogue warps' FC2 staging buffers (shared memory)
     uint32_t tmem_base;
     int total_units, n_groups, kst, terms; // n_groups: work units per row block (tile groups)
     unsigned long long tmo;
@@ -652,10 +656,10 @@ __device__ __forceinline__ void epilogue_wide(const FcGemmArgs &a, const Ctx &c,
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(bars.acc_empty(0)); // the MMA warp may overwrite the accumulator now
-        const int rl = 32 * q + lane;
-        const bool valid = rl < blk.z;
-        const int row = blk.y + rl;
         if (a.fc1) {
+            const int rl = 32 * q + lane;
+            const bool valid = rl < blk.z;
+            const int row = blk.y + rl;
             // columns 0..63: gate rows nt*64 + i, columns 64..127: the matching up rows
 #pragma unroll
             for (int c32 = 0; c32 < 2; ++c32) {
@@ -668,13 +672,31 @@ __device__ __forceinline__ void epilogue_wide(const FcGemmArgs &a, const Ctx &c,
                 if (valid)
                     store_act_block32(a.hq, a.hsf, a.hq_rows, a.out_ld, row, nt * 64 + 32 * c32, h, a.act_mxfp8);
             }
-        } else if (valid) {
-            uint4 *dst = reinterpret_cast<uint4 *>(a.y + (size_t)row * a.out_ld + nt * 128);
+        } else {
+            // FC2: f32 rows of Y.  Stored straight from registers, each store instruction of the
+            // warp would write 32 rows' 16-byte pieces (half sectors, 32 segments).  Instead each
+            // 16-column chunk goes through this warp's 2 KB buffer ([32 rows][4 x 16 bytes], the
+            // 16-byte column index xor-ed with row % 4: conflict-free both ways) and comes back
+            // out as 8 rows x 64 contiguous bytes per instruction: whole sectors.
+            uint4 *stg = reinterpret_cast<uint4 *>(c.ystage + 2048 * (half * 4 + (warp & 3)));
+            const int r0 = lane >> 2, ch = lane & 3;
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
+            for (int j = 0; j < 8; ++j) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
-                    dst[4 * j + i] = make_uint4(v[j][4 * i], v[j][4 * i + 1], v[j][4 * i + 2], v[j][4 * i + 3]);
+                    stg[lane * 4 + (i ^ (lane & 3))] =
+                        make_uint4(v[j][4 * i], v[j][4 * i + 1], v[j][4 * i + 2], v[j][4 * i + 3]);
+                __syncwarp();
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const int r = 8 * p + r0; // row of this warp's 32
+                    const uint4 val = stg[r * 4 + (ch ^ (r & 3))];
+                    if (32 * q + r < blk.z)
+                        *reinterpret_cast<uint4 *>(a.y + (size_t)(blk.y + 32 * q + r) * a.out_ld + nt * 128 + 16 * j +
+                                                   4 * ch) = val;
+                }
+                __syncwarp();
+            }
         }
     }
 }
@@ -739,8 +761,8 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads,
     const int terms = kTm == 1 ? 1 : a.terms; // activation terms per row: 1 (w4a8) or 2 (w4a16)
     const unsigned long long tmo = a.timeout_ns;
 
-    const Ctx ctx{base, reinterpret_cast<volatile int *>(gsm + P::kOffUnits), tmem_base, total_units, n_groups, kst, terms,
-                  tmo};
+    const Ctx ctx{base, reinterpret_cast<volatile int *>(gsm + P::kOffUnits), gsm + P::kOffY, tmem_base, total_units,
+                  n_groups, kst, terms, tmo};
     if (warp == 0) {
         producer_role<kActRows, kMmaW, kWTiles, kTm, 0>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
     } else if (warp >= 6 && warp < 5 + kProd) {
