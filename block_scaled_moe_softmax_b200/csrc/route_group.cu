@@ -337,6 +337,34 @@ __global__ void __launch_bounds__(32) scatter_kernel(int T, int E, int k, const 
 // and encoded once; group = 1 for small batches, which need the parallelism more).  One thread
 // per (token, 32-element block, pair group): 64 bytes in, group x (32 or 2 x 32) code bytes and
 // group x (1 or 2) scale bytes out.
+// Codes of one 32-element block, packed four to a word.
+__device__ __forceinline__ void pack_codes32(const uint8_t (&c)[32], uint4 &lo, uint4 &hi)
+{
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        w[i] = (uint32_t)c[4 * i] | ((uint32_t)c[4 * i + 1] << 8) | ((uint32_t)c[4 * i + 2] << 16) |
+               ((uint32_t)c[4 * i + 3] << 24);
+    lo = make_uint4(w[0], w[1], w[2], w[3]);
+    hi = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
+// Warp-wide rearrangement of 32 consecutive blocks' codes (lane l holds block l's 32 bytes,
+// i.e. 16-byte chunks 2l and 2l + 1 of the warp's 1 KB) so that lane l then holds chunks l and
+// l + 32: each 16-byte store instruction of the warp writes 512 contiguous bytes.  Chunk c sits
+// at position c ^ ((c >> 3) & 1) of the buffer: no bank conflicts on either side.
+__device__ __forceinline__ void transpose_codes(uint4 *stg, int lane, uint4 &lo, uint4 &hi)
+{
+    const int c0 = 2 * lane, c1 = 2 * lane + 1;
+    stg[c0 ^ ((c0 >> 3) & 1)] = lo;
+    stg[c1 ^ ((c1 >> 3) & 1)] = hi;
+    __syncwarp();
+    const int d0 = lane, d1 = lane + 32;
+    lo = stg[d0 ^ ((d0 >> 3) & 1)];
+    hi = stg[d1 ^ ((d1 >> 3) & 1)];
+    __syncwarp();
+}
+
 __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H, int k,
                                                      int group, const int32_t *__restrict__ pos_of_pair,
                                                      uint8_t *__restrict__ aq, uint8_t *__restrict__ asf, int act_rows,
@@ -344,12 +372,77 @@ __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16 *__rest
 {
     grid_dep_wait(); // pos_of_pair from the grouping
     grid_dep_launch();
+    __shared__ __align__(16) uint4 stage[8][2][64]; // per warp and term: 32 blocks' codes
     const int blocks_per_row = H / 32, groups = k / group;
     const long long total = (long long)T * blocks_per_row * groups;
-    for (long long g = blockIdx.x * (long long)blockDim.x + threadIdx.x; g < total;
-         g += (long long)gridDim.x * blockDim.x) {
+    const long long per_group = (long long)T * blocks_per_row;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (blocks_per_row % 32 == 0) {
+        // A warp takes 32 consecutive blocks of one token row (rows are whole multiples of 32
+        // blocks, and total a multiple of 32, so every lane has work): the codes of each term go
+        // through the warp's buffer once and leave as 512-byte rows per store instruction, to
+        // each of the group's grouped rows; the four scale bytes of a 128-element chunk leave as
+        // one word from the chunk's first lane.
+        for (long long wb = (long long)blockIdx.x * blockDim.x + 32 * warp; wb < total; wb += stride) {
+            const long long g = wb + lane;
+            const int jg = (int)(g / per_group);
+            const long long tb = g % per_group;
+            const int t = (int)(tb / blocks_per_row);
+            const int b = (int)(tb % blocks_per_row);
+            const int b0 = b - lane; // the warp's first block
+            const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H + (size_t)b * 32);
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint4 raw = __ldg(src + i);
+                const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 f = __bfloat1622float2(h2[j]);
+                    v[8 * i + 2 * j] = f.x;
+                    v[8 * i + 2 * j + 1] = f.y;
+                }
+            }
+            uint8_t c0[32], c1[32];
+            uint32_t s0, s1;
+            mx_encode32(v, act_mxfp8, c0, c1, s0, s1); // the values are bf16 already: no rounding step
+            uint4 a_lo, a_hi, b_lo = make_uint4(0, 0, 0, 0), b_hi = b_lo;
+            pack_codes32(c0, a_lo, a_hi);
+            transpose_codes(stage[warp][0], lane, a_lo, a_hi);
+            if (!act_mxfp8) {
+                pack_codes32(c1, b_lo, b_hi);
+                transpose_codes(stage[warp][1], lane, b_lo, b_hi);
+            }
+            // the scale bytes of blocks 4m .. 4m + 3 (one 128-element chunk) as one word
+            uint32_t w0 = s0, w1 = s1;
+#pragma unroll
+            for (int i = 1; i < 4; ++i) {
+                w0 |= __shfl_down_sync(0xFFFFFFFFu, s0, i) << (8 * i);
+                w1 |= __shfl_down_sync(0xFFFFFFFFu, s1, i) << (8 * i);
+            }
+            for (int j = jg * group; j < (jg + 1) * group; ++j) {
+                const int row = pos_of_pair[(size_t)t * k + j]; // the same for the whole warp
+                if (row < 0)
+                    continue; // not in the local expert shard
+                uint4 *dst = reinterpret_cast<uint4 *>(aq + (size_t)row * H + (size_t)b0 * 32);
+                dst[lane] = a_lo;
+                dst[lane + 32] = a_hi;
+                if ((lane & 3) == 0)
+                    *reinterpret_cast<uint32_t *>(asf + sf_atom_byte(row, b * 32, H, 0)) = w0;
+                if (!act_mxfp8) {
+                    uint4 *dst1 = reinterpret_cast<uint4 *>(aq + ((size_t)act_rows + row) * H + (size_t)b0 * 32);
+                    dst1[lane] = b_lo;
+                    dst1[lane + 32] = b_hi;
+                    if ((lane & 3) == 0)
+                        *reinterpret_cast<uint32_t *>(asf + sf_atom_byte(row, b * 32, H, 1)) = w1;
+                }
+            }
+        }
+        return;
+    }
+    for (long long g = blockIdx.x * (long long)blockDim.x + threadIdx.x; g < total; g += stride) {
         // consecutive threads take consecutive blocks of one row: coalesced loads and stores
-        const long long per_group = (long long)T * blocks_per_row;
         const int jg = (int)(g / per_group);
         const long long tb = g % per_group;
         const int t = (int)(tb / blocks_per_row);
