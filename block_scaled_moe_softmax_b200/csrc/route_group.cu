@@ -209,7 +209,10 @@ __device__ __forceinline__ int scan_experts(int E, int split, int total, int32_t
 }
 
 // One CTA: per-expert totals over the chunk histograms, the scan, and per-chunk base rows
-// for the scatter; also zeroes the GEMMs' work-unit counters (optional).
+// for the scatter; also zeroes the GEMMs' work-unit counters (optional).  Each expert's chunks
+// are split into contiguous ranges over a group of tpe threads (a power of two up to 32, as
+// many as 1024 threads allow), so the chunk loop runs tpe-way parallel: the ranges' sums, a
+// scan within the group, then (after the expert scan) each range writes its chunks' base rows.
 __global__ void __launch_bounds__(1024) scan_kernel(int E, int nchunks, int split, int32_t *__restrict__ chunk_hist,
                                                     int32_t *__restrict__ counts, int32_t *__restrict__ pad_offsets,
                                                     int4 *__restrict__ rowblocks, int32_t *__restrict__ num_rowblocks,
@@ -218,31 +221,61 @@ __global__ void __launch_bounds__(1024) scan_kernel(int E, int nchunks, int spli
     grid_dep_wait(); // the chunk histograms of the router
     grid_dep_launch();
     __shared__ unsigned long long s_warp[32];
-    const int e = threadIdx.x;
-    if (unit_counters && e < 2) // the GEMMs' work-unit counters start at zero
-        unit_counters[e] = 0;
-    int total = 0;
-    if (e < E) {
-        // exclusive prefix within the expert over the chunks; the loads go out in groups of
-        // kBatch so that their latencies overlap
-        constexpr int kBatch = 16;
-        for (int c0 = 0; c0 < nchunks; c0 += kBatch) {
+    __shared__ int32_t s_tot[kMaxExperts];
+    const int tid = threadIdx.x;
+    if (unit_counters && tid < 2) // the GEMMs' work-unit counters start at zero
+        unit_counters[tid] = 0;
+    int tpe = 1;
+    while (tpe < 32 && 2 * tpe * E <= (int)blockDim.x)
+        tpe *= 2;
+    const int ex = tid / tpe, sub = tid % tpe;
+    const bool mine = ex < E;
+    const int len = (nchunks + tpe - 1) / tpe;
+    const int c_lo = min(nchunks, sub * len), c_hi = min(nchunks, c_lo + len);
+    constexpr int kBatch = 16; // loads in flight together
+    int part = 0;
+    if (mine)
+        for (int c0 = c_lo; c0 < c_hi; c0 += kBatch) {
             int h[kBatch];
 #pragma unroll
             for (int i = 0; i < kBatch; ++i)
-                h[i] = c0 + i < nchunks ? chunk_hist[(size_t)(c0 + i) * E + e] : 0;
+                h[i] = c0 + i < c_hi ? chunk_hist[(size_t)(c0 + i) * E + ex] : 0;
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i)
+                part += h[i];
+        }
+    // inclusive scan of the ranges within the expert's group of tpe lanes (groups never straddle
+    // a warp: tpe divides 32)
+    int incl = part;
+    for (int off = 1; off < tpe; off <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if (sub >= off)
+            incl += y;
+    }
+    if (mine && sub == tpe - 1)
+        s_tot[ex] = incl;
+    __syncthreads();
+    const int base = scan_experts(E, split, tid < E ? s_tot[tid] : 0, counts, pad_offsets, rowblocks, num_rowblocks,
+                                  sorted_pair, s_warp);
+    __syncthreads();
+    if (tid < E)
+        s_tot[tid] = base; // now: each expert's first grouped row
+    __syncthreads();
+    if (mine) {
+        int run = s_tot[ex] + incl - part; // exclusive prefix within the expert, plus its base row
+        for (int c0 = c_lo; c0 < c_hi; c0 += kBatch) {
+            int h[kBatch];
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i)
+                h[i] = c0 + i < c_hi ? chunk_hist[(size_t)(c0 + i) * E + ex] : 0;
 #pragma unroll
             for (int i = 0; i < kBatch; ++i) {
-                if (c0 + i < nchunks)
-                    chunk_hist[(size_t)(c0 + i) * E + e] = total;
-                total += h[i];
+                if (c0 + i < c_hi)
+                    chunk_hist[(size_t)(c0 + i) * E + ex] = run;
+                run += h[i];
             }
         }
     }
-    const int base = scan_experts(E, split, total, counts, pad_offsets, rowblocks, num_rowblocks, sorted_pair, s_warp);
-    if (e < E)
-        for (int c = 0; c < nchunks; ++c)
-            chunk_hist[(size_t)c * E + e] += base;
 }
 
 // Stable placement of pairs [p_begin, p_end) by one warp: each pair goes to its expert's
@@ -252,26 +285,35 @@ __device__ __forceinline__ void scatter_pairs(int p_begin, int p_end, const int3
                                               int32_t *__restrict__ pos_of_pair, int lane)
 {
     const unsigned lt_mask = (1u << lane) - 1u;
-    for (int base = p_begin; base < p_end; base += 32) {
-        const int p = base + lane;
-        const bool valid = p < p_end;
-        const int e_raw = valid ? topk_ids[p] : -1;
-        const bool placed = e_raw >= 0; // -1: a pair outside the local expert shard (given routing)
-        const int e = placed ? e_raw : -1 - lane; // lanes not placed never match each other
-        const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
-        const int rank = __popc(peers & lt_mask);
-        int row = 0;
-        if (placed)
-            row = cursor[e] + rank;
-        __syncwarp();
-        if (placed && (32 - __clz(peers)) - 1 == lane) // highest lane of the group advances the cursor
-            cursor[e] += __popc(peers);
-        __syncwarp();
-        if (placed) {
-            sorted_pair[row] = p;
-            pos_of_pair[p] = row;
-        } else if (valid) {
-            pos_of_pair[p] = -1;
+    constexpr int kB = 8; // rounds of 32 pairs whose ids are loaded together
+    for (int base = p_begin; base < p_end; base += 32 * kB) {
+        int ev[kB];
+#pragma unroll
+        for (int i = 0; i < kB; ++i) {
+            const int p = base + 32 * i + lane;
+            ev[i] = p < p_end ? topk_ids[p] : -1;
+        }
+#pragma unroll
+        for (int i = 0; i < kB; ++i) {
+            const int p = base + 32 * i + lane;
+            const bool valid = p < p_end;
+            const bool placed = ev[i] >= 0; // -1: a pair outside the local expert shard (given routing)
+            const int e = placed ? ev[i] : -1 - lane; // lanes not placed never match each other
+            const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+            const int rank = __popc(peers & lt_mask);
+            int row = 0;
+            if (placed)
+                row = cursor[e] + rank;
+            __syncwarp();
+            if (placed && (32 - __clz(peers)) - 1 == lane) // highest lane of the group advances the cursor
+                cursor[e] += __popc(peers);
+            __syncwarp();
+            if (placed) {
+                sorted_pair[row] = p;
+                pos_of_pair[p] = row;
+            } else if (valid) {
+                pos_of_pair[p] = -1;
+            }
         }
     }
 }
