@@ -153,3 +153,23 @@ def test_page_contract_shapes(name):
     assert helpers.rel_frobenius(got, ref) <= helpers.TOL_REL_FRO, name
     assert helpers.max_abs_over_rms(got, ref) <= helpers.TOL_MAX_OVER_RMS, name
     layer.close()
+
+
+def test_expert_parallel_forward_two_shards_on_one_gpu():
+    """ep.ep_forward per rank of a 2-way expert split (run one after another on one GPU, with no
+    process group, so each returns its own partial output): their sum is the whole layer."""
+    from block_scaled_moe_softmax_b200 import ep
+    wl, x, ids, w, wq = _setup(40, 8, 4)
+    total = torch.zeros(40, wl.H, dtype=torch.float64)
+    for rank in range(2):
+        off, n = ep.shard_range(wl.E, 2, rank)
+        layer = moe_mx.MoeMxLayer(wl.H, wl.I, n, wl.T, 4)
+        d = _dev({k: np.ascontiguousarray(v[off:off + n]) for k, v in wq.items()})
+        part = ep.ep_forward(layer, x.cuda(), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(), d["w1"],
+                             d["w1s"], d["w2"], d["w2s"], wl.E, rank, 2)
+        assert layer.sync_status() == moe_mx.MOE_MX_OK, moe_mx.moe_mx_last_error()
+        total += part.double().cpu()
+        layer.close()
+    _, ref, _ = oracle.moe_forward_routed(workloads.bf16_bits(x), ids, w, 0, wq["w1"], wq["w1s"], wq["w2"], wq["w2s"])
+    assert helpers.rel_frobenius(total.numpy(), ref) <= helpers.TOL_REL_FRO
+    assert helpers.max_abs_over_rms(total.numpy(), ref) <= helpers.TOL_MAX_OVER_RMS

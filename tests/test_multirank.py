@@ -1,9 +1,14 @@
-"""Host logic of the multi-process bench path on CPU: two gloo ranks.
+"""Host logic of the multi-process paths on CPU: gloo ranks.
 
 bench.py runs one independent replica of the layer per GPU; its only
 cross-rank steps are a barrier around the timed region and a max over ranks of
 the measured time.  These run here with the gloo backend (world size 2), and the
 reference arm's non-zero ranks must exit without work.
+
+Expert parallelism (block_scaled_moe_softmax_b200.ep): each rank's partial output
+over its contiguous expert shard, summed over the ranks, must equal the whole
+layer.  Here the partial outputs come from the oracle (no GPU), the sum from
+ep.reduce_partials over gloo ranks (world sizes 2 and 4).
 """
 import os
 import subprocess
@@ -64,3 +69,59 @@ def test_max_over_ranks_single_rank_is_identity(world):
     sys.path.insert(0, ROOT)
     import bench
     assert bench.max_over_ranks(3.25, world) == 3.25
+
+
+def _ep_rank_main(rank, world, port, results):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import oracle
+    from block_scaled_moe_softmax_b200 import ep, workloads
+    from tests import helpers
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        wl = workloads.Workload("ep", 12, 64, 32, 8, 4, seed=5, routing="given", experts_global=8)
+        x = workloads.draw_x(wl)
+        ids, w = (a.numpy() for a in workloads.draw_topk(wl))
+        wq = helpers.quantize_weights_cpu(wl)
+        off, n = ep.shard_range(wl.E, world, rank)
+        shard = {k: np.ascontiguousarray(v[off:off + n]) for k, v in wq.items()}
+        _, part, _ = oracle.moe_forward_routed(workloads.bf16_bits(x), ids, w, off, shard["w1"], shard["w1s"],
+                                               shard["w2"], shard["w2s"])
+        total = ep.reduce_partials(torch.from_numpy(part).to(torch.float32))
+        _, full, _ = oracle.moe_forward_routed(workloads.bf16_bits(x), ids, w, 0, wq["w1"], wq["w1s"], wq["w2"],
+                                               wq["w2s"])
+        results[rank] = (float(np.abs(total.double().numpy() - full).max()), float(np.abs(full).max()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_expert_parallel_partials_sum_to_the_layer(world):
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    results = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_ep_rank_main, args=(r, world, port, results)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=300)
+        assert p.exitcode == 0
+    for r in range(world):
+        err, scale = results[r]
+        assert err <= 1e-6 * scale  # float32 rounding of the shards' sums only
+
+
+def test_shard_range():
+    sys.path.insert(0, ROOT)
+    from block_scaled_moe_softmax_b200 import ep
+    assert ep.shard_range(896, 8, 3) == (336, 112)
+    assert ep.shard_range(8, 1, 0) == (0, 8)
+    with pytest.raises(ValueError):
+        ep.shard_range(10, 4, 0)
+    with pytest.raises(ValueError):
+        ep.shard_range(8, 2, 2)
+
