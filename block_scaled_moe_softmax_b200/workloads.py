@@ -76,6 +76,11 @@ WORKLOADS = {
                                "batched decode, w4a16: T=256, logits + N(0,0.5) expert bias"),
     "prefill": Workload("prefill", 8192, 7168, 2048, 384, 8, "bf16", "zipf", 0,
                         "prefill, w4a16: T=8192, Zipf-like expert bias"),
+    # the decode shape at 1 and 4 tokens (the small-batch end of decode)
+    "decode_t1": Workload("decode_t1", 1, 7168, 2048, 384, 8, "bf16", "none", 0,
+                          "decode-shaped, w4a16, a single token"),
+    "decode_t4": Workload("decode_t4", 4, 7168, 2048, 384, 8, "bf16", "none", 0,
+                          "decode-shaped, w4a16, 4 tokens"),
     # the decode shape with 64 experts: a capture-sized case (about 1.5 GB of weights) for profiling
     "decode_e64": Workload("decode_e64", 16, 7168, 2048, 64, 8, "bf16", "none", 0,
                            "decode-shaped, w4a16, 64 experts (profiling case)"),
