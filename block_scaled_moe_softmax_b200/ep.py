@@ -1,5 +1,6 @@
-"""Expert parallelism over ranks: the layer's experts split into contiguous shards, one per
-rank, and the shards' partial outputs summed.
+"""Expert and tensor parallelism over ranks: the layer's experts split into contiguous shards
+(or every expert's intermediate dimension split into slices), one per rank, and the ranks'
+partial outputs summed.
 
 TokenSpeed SiTU package description, "Supported contract": every rank routes with the
 global expert ids, the layer filters them to its contiguous shard of local experts (local
@@ -8,6 +9,14 @@ all-reduces the partial outputs over the expert-parallel group.  On one rank the
 and the float32 partial output are moe_mx_forward_routed (CUDA); this module adds the
 shard bookkeeping and the sum over ranks (torch.distributed; NCCL on GPUs).  The result
 is the float32 sum; rounding it to bf16, if wanted, is the caller's.
+
+Tensor parallelism (the same page's TP8 configuration: all experts on every rank, each with
+a slice of the intermediate dimension) needs no kernel of its own: SwiGLU acts element by
+element along the intermediate index, so a rank holding gate/up rows and W2 columns of one
+slice computes that slice's share of every expert's output, and the shares add up.
+tp_shard_weights cuts a rank's slice out of the full weights; the rank then runs
+moe_mx_forward_routed on all experts (offset 0) with inter = I / world and a float32 output,
+and reduce_partials sums the ranks' outputs.
 """
 from __future__ import annotations
 
@@ -47,3 +56,31 @@ def ep_forward(layer: moe_mx.MoeMxLayer, x, topk_ids, topk_w, w1, w1_scale, w2, 
     partial = layer.forward_routed(x, topk_ids, topk_w, w1, w1_scale, w2, w2_scale, offset, act_dtype,
                                    moe_mx.MOE_MX_OUT_F32)
     return reduce_partials(partial, group)
+
+
+def tp_shard_weights(w1, w1_scale, w2, w2_scale, rank: int, world: int):
+    """Rank `rank`'s slice of the intermediate dimension of every expert: w1 [E, 2I, H/2] and its
+    scales keep gate rows and up rows [rank * I/world, (rank + 1) * I/world) (gate rows first,
+    as the layer expects); w2 [E, H, I/2] and its scales keep the matching columns.  I / world
+    must be a multiple of 128 (the layer's smallest intermediate tile).  Works on numpy arrays and
+    torch tensors alike; returns contiguous copies."""
+    E, two_i = w1.shape[0], w1.shape[1]
+    I = two_i // 2
+    if I % world or (I // world) % 128:
+        raise ValueError(f"intermediate size {I} does not split into {world} slices of a multiple of 128")
+    n = I // world
+    lo = rank * n
+
+    def rows(a):  # gate rows then up rows of the slice
+        g, u = a[:, lo:lo + n], a[:, I + lo:I + lo + n]
+        if isinstance(a, torch.Tensor):
+            return torch.cat([g, u], dim=1).contiguous()
+        import numpy as np
+        return np.ascontiguousarray(np.concatenate([g, u], axis=1))
+
+    def cols(a, per):  # columns of the slice along the last dim, `per` elements per stored unit
+        c = a[:, :, lo // per:(lo + n) // per]
+        return c.contiguous() if isinstance(c, torch.Tensor) else __import__("numpy").ascontiguousarray(c)
+
+    return rows(w1), rows(w1_scale), cols(w2, 2), cols(w2_scale, 32)
+

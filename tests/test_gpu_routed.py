@@ -173,3 +173,24 @@ def test_expert_parallel_forward_two_shards_on_one_gpu():
     _, ref, _ = oracle.moe_forward_routed(workloads.bf16_bits(x), ids, w, 0, wq["w1"], wq["w1s"], wq["w2"], wq["w2s"])
     assert helpers.rel_frobenius(total.numpy(), ref) <= helpers.TOL_REL_FRO
     assert helpers.max_abs_over_rms(total.numpy(), ref) <= helpers.TOL_MAX_OVER_RMS
+
+
+def test_tensor_parallel_slices_on_one_gpu():
+    """ep.tp_shard_weights: two ranks' slices of every expert's intermediate dimension, each run
+    through moe_mx_forward_routed with a float32 output (one after another on one GPU); their sum
+    is the whole layer."""
+    from block_scaled_moe_softmax_b200 import ep
+    wl, x, ids, w, wq = _setup(24, 4, 2, H=256, I=256)
+    total = torch.zeros(24, wl.H, dtype=torch.float64)
+    for rank in range(2):
+        s1, s1s, s2, s2s = ep.tp_shard_weights(*(torch.from_numpy(wq[n]).cuda() for n in ("w1", "w1s", "w2", "w2s")),
+                                               rank, 2)
+        layer = moe_mx.MoeMxLayer(wl.H, wl.I // 2, wl.E, wl.T, 2)
+        part = layer.forward_routed(x.cuda(), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(), s1, s1s, s2,
+                                    s2s, 0, 0, moe_mx.MOE_MX_OUT_F32)
+        assert layer.sync_status() == moe_mx.MOE_MX_OK, moe_mx.moe_mx_last_error()
+        total += part.double().cpu()
+        layer.close()
+    _, ref, _ = oracle.moe_forward_routed(workloads.bf16_bits(x), ids, w, 0, wq["w1"], wq["w1s"], wq["w2"], wq["w2s"])
+    assert helpers.rel_frobenius(total.numpy(), ref) <= helpers.TOL_REL_FRO
+    assert helpers.max_abs_over_rms(total.numpy(), ref) <= helpers.TOL_MAX_OVER_RMS

@@ -125,3 +125,57 @@ def test_shard_range():
     with pytest.raises(ValueError):
         ep.shard_range(8, 2, 2)
 
+
+def _tp_rank_main(rank, world, port, results):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import oracle
+    from block_scaled_moe_softmax_b200 import ep, workloads
+    from tests import helpers
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        wl = workloads.Workload("tp", 10, 64, 256, 4, 2, seed=6, routing="given", experts_global=4)
+        x = workloads.draw_x(wl)
+        ids, w = (a.numpy() for a in workloads.draw_topk(wl))
+        wq = helpers.quantize_weights_cpu(wl)
+        s1, s1s, s2, s2s = ep.tp_shard_weights(wq["w1"], wq["w1s"], wq["w2"], wq["w2s"], rank, world)
+        _, part, _ = oracle.moe_forward_routed(workloads.bf16_bits(x), ids, w, 0, s1, s1s, s2, s2s)
+        total = ep.reduce_partials(torch.from_numpy(part).to(torch.float32))
+        _, full, _ = oracle.moe_forward_routed(workloads.bf16_bits(x), ids, w, 0, wq["w1"], wq["w1s"], wq["w2"],
+                                               wq["w2s"])
+        results[rank] = (float(np.abs(total.double().numpy() - full).max()), float(np.abs(full).max()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_tensor_parallel_slices_sum_to_the_layer():
+    """Two ranks, each with half of every expert's intermediate dimension (gate/up rows and W2
+    columns of one slice): their partial outputs (oracle) summed over gloo equal the layer, as
+    SwiGLU acts element by element along the intermediate index."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    results = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_tp_rank_main, args=(r, world, port, results)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=300)
+        assert p.exitcode == 0
+    for r in range(world):
+        err, scale = results[r]
+        assert err <= 1e-6 * scale
+
+
+def test_tp_shard_weights_rejects_uneven_slices():
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    from block_scaled_moe_softmax_b200 import ep
+    w1 = np.zeros((2, 2 * 256, 32), np.uint8)
+    with pytest.raises(ValueError):
+        ep.tp_shard_weights(w1, w1, np.zeros((2, 64, 128), np.uint8), np.zeros((2, 64, 8), np.uint8), 0, 4)
+
