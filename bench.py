@@ -251,33 +251,73 @@ def cpu_baseline(wl, cores):
                       f"one oracle call, {n_tok} threads, {dt:.1f} s wall"}
 
 
+def reference_pairs(wl, sample_tokens):
+    """The (token, slot) pairs of the sampled tokens that the layer evaluates -- the routed slots
+    (the oracle's router, or the given routing restricted to the local shard) and the shared
+    expert's slots -- as (token, local expert, weight); and the pairs per token of the whole
+    workload, to convert pairs/s to tokens/s."""
+    import oracle
+    if wl.routing == "given":
+        ids, w = (a.numpy() for a in workloads.draw_topk(wl))
+        loc = ids - wl.local_offset
+        inside = (loc >= 0) & (loc < wl.E)
+        per_token = float(inside.sum()) / wl.T
+    else:
+        ids, w = oracle.route(workloads.draw_logits(wl).numpy()[sample_tokens], wl.top_k)
+        loc, inside = ids, np.ones(ids.shape, bool)
+        per_token = float(wl.top_k)
+    pairs = []
+    for i, t in enumerate(sample_tokens):
+        row = t if wl.routing == "given" else i
+        pairs += [(t, int(loc[row, j]), float(w[row, j])) for j in range(wl.top_k) if inside[row, j]]
+        pairs += [(t, wl.E + c, 1.0) for c in range(wl.shared)]
+    return pairs, per_token + wl.shared
+
+
 def run_reference(args, wl):
-    """The oracle as the reference arm: one token of the workload per step; steps run in batches of
-    up to `cores` concurrent steps (one thread each), so K steps take about K/cores token-times."""
+    """The oracle as the reference arm.  One step = one (token, slot) pair of the workload: the
+    FC1, SwiGLU and FC2 of one token through one expert, weighted -- the unit of the layer's work
+    (a token of the decode shapes is k of them), small enough that K steps take a few minutes.
+    The pairs come from the first `cores` tokens (their routing taken once, outside the timed
+    steps) and run in batches of up to `cores` concurrent steps, one thread each, through the
+    oracle's routed form with one slot per evaluated row.  tokens/s = pairs/s / pairs per token."""
+    import oracle
     cores = len(os.sched_getaffinity(0))
     sample = list(range(min(wl.T, cores)))
-    xb, route_np, wq, experts = cpu_sample_setup(wl, sample)
+    pairs, per_token = reference_pairs(wl, sample)
+    experts = sorted({e for _, e, _ in pairs})
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    wq = oracle_weights_for(wl, [e for e in experts if e < wl.E] + list(range(wl.E, wl.slots)), dev)
+    xb = workloads.bf16_bits(workloads.draw_x(wl))
+    act = 1 if wl.act == "mxfp8" else 0
 
     def run_steps(n):
         done, wall = 0, 0.0
         while done < n:
             batch = min(cores, n - done)
-            toks = [sample[(done + i) % len(sample)] for i in range(batch)]
-            wall += oracle_time_tokens(wl, xb, route_np, wq, toks, batch)
+            sel = [pairs[(done + i) % len(pairs)] for i in range(batch)]
+            xs = np.ascontiguousarray(xb[[t for t, _, _ in sel]])
+            ids = np.array([[e] for _, e, _ in sel], np.int32)
+            ws = np.array([[w] for _, _, w in sel], np.float32)
+            t0 = time.perf_counter()
+            oracle.moe_forward_routed(xs, ids, ws, 0, *wq, act, nthreads=batch)
+            wall += time.perf_counter() - t0
             done += batch
         return wall
 
     run_steps(args.warmup)
     total = run_steps(args.steps)
-    value = args.steps / total
+    value = args.steps / total / per_token
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 0,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": workload_desc(wl), "tokens_per_step": 1},
+        "data": "synthetic",
+        "config": {"workload": workload_desc(wl), "pairs_per_step": 1, "pairs_per_token": per_token},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": min(cores, args.steps), "kind": "oracle",
-                         "sample": f"one token of {wl.name} per step (tokens 0..{len(sample) - 1} cycled, "
-                                   f"{len(experts)} experts hit), up to {cores} steps concurrently"},
+                         "sample": f"one (token, slot) pair of {wl.name} per step: the {len(pairs)} pairs of tokens "
+                                   f"0..{len(sample) - 1} cycled ({len(experts)} experts), up to {cores} steps "
+                                   f"concurrently; {per_token:g} pairs per token"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
