@@ -340,14 +340,17 @@ def layer_weight_bytes(wl, hit):
     return hit * (3 * wl.I * wl.H // 2 + 3 * wl.I * wl.H // 32)
 
 
+# the sources the FC GEMM kernel is built from (the kernel the traffic record describes)
+FC_GEMM_SOURCES = ("fc_gemm.cu", "kernels.cuh", "ptx.cuh")
+
+
 def kernel_source_sha():
-    """sha256 (first 16 hex digits) over every CUDA source of the library, in name order."""
+    """sha256 (first 16 hex digits) over the FC GEMM kernel's CUDA sources, in name order."""
     csrc = os.path.join(ROOT, "block_scaled_moe_softmax_b200", "csrc")
     h = hashlib.sha256()
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in sorted(FC_GEMM_SOURCES):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 

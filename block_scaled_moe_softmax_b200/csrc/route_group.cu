@@ -22,6 +22,21 @@
 namespace moe_mx {
 
 // ---------------------------------------------------------------- router
+// Order-preserving map of a float onto uint32 (a < b <=> key(a) < key(b); -0 and +0, which
+// compare equal, share a key), and its inverse.
+__device__ __forceinline__ uint32_t order_key(float x)
+{
+    if (x == 0.f)
+        x = 0.f;
+    const uint32_t u = __float_as_uint(x);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float order_value(uint32_t k)
+{
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 // Route one token (whole warp): the k experts in descending logit order, the lowest index
 // first among equal logits, and their weights = the softmax over the selected logits.  Lane j
 // (j < k) writes the j-th id and weight and adds it to the block's expert histogram.
@@ -60,16 +75,13 @@ __device__ __forceinline__ void route_token(const float *__restrict__ row, int E
                 bi = e;
             }
         }
-        // warp arg-max with the lowest index winning ties
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
-            const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, off);
-            if (ov > bv || (ov == bv && oi < bi)) {
-                bv = ov;
-                bi = oi;
-            }
-        }
+        // warp arg-max with the lowest index winning ties: the largest value through an
+        // order-preserving integer key (one warp reduction), then the lowest index among the
+        // lanes holding it (another)
+        const uint32_t key = order_key(bv);
+        const uint32_t kmax = __reduce_max_sync(0xFFFFFFFFu, key);
+        bi = (int)__reduce_min_sync(0xFFFFFFFFu, key == kmax ? (uint32_t)bi : 0xFFFFFFFFu);
+        bv = order_value(kmax);
         if ((bi & 31) == lane)
             taken |= 1u << (bi >> 5);
         if (lane == j) {
@@ -295,6 +307,8 @@ __device__ __forceinline__ void scatter_pairs(int p_begin, int p_end, const int3
         }
 #pragma unroll
         for (int i = 0; i < kB; ++i) {
+            if (base + 32 * i >= p_end)
+                break; // no pair left in this round (warp-uniform)
             const int p = base + 32 * i + lane;
             const bool valid = p < p_end;
             const bool placed = ev[i] >= 0; // -1: a pair outside the local expert shard (given routing)

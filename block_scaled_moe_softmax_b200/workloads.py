@@ -81,6 +81,10 @@ WORKLOADS = {
                           "decode-shaped, w4a16, a single token"),
     "decode_t4": Workload("decode_t4", 4, 7168, 2048, 384, 8, "bf16", "none", 0,
                           "decode-shaped, w4a16, 4 tokens"),
+    # the decode routing (16 tokens, 384 experts, top-8) with small expert matrices: a profiling case
+    # for the routing and grouping kernel
+    "route_e384": Workload("route_e384", 16, 256, 128, 384, 8, "bf16", "none", 0,
+                           "decode routing shape with small experts (profiling case)"),
     # the decode shape with 64 experts: a capture-sized case (about 1.5 GB of weights) for profiling
     "decode_e64": Workload("decode_e64", 16, 7168, 2048, 64, 8, "bf16", "none", 0,
                            "decode-shaped, w4a16, 64 experts (profiling case)"),
