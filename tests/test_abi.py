@@ -60,6 +60,10 @@ def test_host_validation_without_gpu(lib):
     assert lib.moe_mx_create(ctypes.byref(h), 256, 128, 8, 16, 33, 0) == moe_mx.MOE_MX_ERR_INVALID_ARG
     assert lib.moe_mx_create(ctypes.byref(h), 256, 128, 2000, 16, 2, 0) == moe_mx.MOE_MX_ERR_UNSUPPORTED
     assert lib.moe_mx_create(None, 256, 128, 8, 16, 2, 0) == moe_mx.MOE_MX_ERR_INVALID_ARG
+    ce = lib.moe_mx_create_ex
+    assert ce(ctypes.byref(h), 256, 128, 1000, 30, 16, 2, 0) == moe_mx.MOE_MX_ERR_UNSUPPORTED  # E + S > 1024
+    assert ce(ctypes.byref(h), 256, 128, 8, 4, 16, 30, 0) == moe_mx.MOE_MX_ERR_UNSUPPORTED     # top_k + S > 32
+    assert ce(ctypes.byref(h), 256, 128, 8, -1, 16, 2, 0) == moe_mx.MOE_MX_ERR_UNSUPPORTED
     fr = lib.moe_mx_forward_routed
     assert fr(None, None, None, None, 1, 1, 0, None, None, None, None, 0, None, 0, None) == moe_mx.MOE_MX_ERR_INVALID_ARG
     assert fr(None, None, None, None, 1, 1, 0, None, None, None, None, 0, None, 5, None) == moe_mx.MOE_MX_ERR_INVALID_ARG
