@@ -1,0 +1,64 @@
+"""Host-side logic of bench.py (CPU only): the algorithmic work it divides by, the reference
+arm's sampling, and the JSON line of the reference arm."""
+import json
+import os
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from block_scaled_moe_softmax_b200 import workloads  # noqa: E402
+
+
+def test_algorithmic_work_closed_forms():
+    wl = workloads.WORKLOADS["decode"]
+    counts = np.zeros(wl.E, np.int64)
+    counts[[3, 7, 11]] = [5, 1, 10]            # 3 experts hit, 16 pairs
+    b, hit = bench.fc1_algorithmic_bytes(wl, counts)
+    assert hit == 3
+    # MXFP4 gate+up rows (half a byte per element) and their E8M0 scales, plus bf16 rows in and out
+    per_expert = 2 * wl.I * wl.H // 2 + 2 * wl.I * wl.H // 32
+    assert b == 3 * per_expert + 16 * (wl.H + wl.I) * 2
+    assert bench.fc1_algorithmic_flops(wl, counts) == 2.0 * 16 * 2 * wl.I * wl.H
+    assert bench.layer_weight_bytes(wl, 3) == 3 * (3 * wl.I * wl.H // 2 + 3 * wl.I * wl.H // 32)
+    assert per_expert == 15_597_568  # 15.60 MB per hit expert at H = 7168, I = 2048
+
+
+def test_kernels_per_forward():
+    assert bench.kernels_per_forward(16) == 5 and bench.kernels_per_forward(64) == 5
+    assert bench.kernels_per_forward(65) == 7
+
+
+def test_reference_pairs():
+    wl = workloads.WORKLOADS["tiny"]
+    pairs, per_token = bench.reference_pairs(wl, [0, 1, 2])
+    assert per_token == wl.top_k and len(pairs) == 3 * wl.top_k
+    assert all(0 <= e < wl.E for _, e, _ in pairs)
+    for t in range(3):  # a token's routed weights sum to 1
+        assert abs(sum(w for tt, _, w in pairs if tt == t) - 1.0) < 1e-6
+    sh = workloads.Workload("sh", 16, 256, 128, 8, 2, shared=2)
+    pairs, per_token = bench.reference_pairs(sh, [0])
+    assert per_token == 4 and [(e, w) for _, e, w in pairs[2:]] == [(8, 1.0), (9, 1.0)]
+    ep = workloads.WORKLOADS["situ_ep8"]
+    pairs, per_token = bench.reference_pairs(ep, list(range(8)))
+    ids, _ = workloads.draw_topk(ep)
+    ids = ids.numpy()
+    assert per_token == pytest.approx(((ids >= 0) & (ids < ep.E)).sum() / ep.T)
+    assert len(pairs) == int(((ids[:8] >= 0) & (ids[:8] < ep.E)).sum())
+
+
+def test_reference_arm_json_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                        "--steps", "6", "--warmup", "3"], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr
+    d = json.loads(r.stdout.strip().splitlines()[-1])
+    assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["steps"] == 6 and d["warmup"] == 3
+    assert d["value"] > 0 and d["higher_is_better"] is True and d["vs_baseline"] is None
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["config"]["pairs_per_token"] == 2.0
