@@ -297,14 +297,20 @@ uint16_t oracle_bf16_bits(double v) { return double_to_bf16_bits(v); }
  */
 void oracle_route(const float *logits, int E, int k, int32_t *ids, float *w)
 {
+    /* A NaN logit ranks below every number and gets probability 0: it is read as -inf (the
+     * pages do not say; this keeps the selection a total order).  A row with no finite logit
+     * has no defined softmax; its weights come out NaN. */
+    double *l = (double *)malloc(sizeof(double) * (size_t)E);
+    for (int e = 0; e < E; ++e)
+        l[e] = isnan(logits[e]) ? -INFINITY : (double)logits[e];
     unsigned char *taken = (unsigned char *)calloc((size_t)E, 1);
     for (int j = 0; j < k; ++j) {
         int best = -1;
         for (int e = 0; e < E; ++e) {
             if (taken[e])
                 continue;
-            if (best < 0 || logits[e] > logits[best] ||
-                (ORACLE_PLANT_MISTAKE == 3 && logits[e] == logits[best])) /* plant: highest index wins */
+            if (best < 0 || l[e] > l[best] ||
+                (ORACLE_PLANT_MISTAKE == 3 && l[e] == l[best])) /* plant: highest index wins */
                 best = e;
         }
         taken[best] = 1;
@@ -313,17 +319,18 @@ void oracle_route(const float *logits, int E, int k, int32_t *ids, float *w)
     free(taken);
     double mx = -INFINITY;
     for (int e = 0; e < E; ++e)
-        if ((double)logits[e] > mx)
-            mx = (double)logits[e];
+        if (l[e] > mx)
+            mx = l[e];
     double z = 0.0;
     for (int e = 0; e < E; ++e)
-        z += exp((double)logits[e] - mx);
+        z += exp(l[e] - mx);
     double p[1024];
     double psum = 0.0;
     for (int j = 0; j < k; ++j) {
-        p[j] = exp((double)logits[ids[j]] - mx) / z;
+        p[j] = exp(l[ids[j]] - mx) / z;
         psum += p[j];
     }
+    free(l);
     for (int j = 0; j < k; ++j)
         w[j] = (float)(ORACLE_PLANT_MISTAKE == 8 ? p[j] : p[j] / psum); /* plant: no renormalisation */
 }

@@ -208,3 +208,31 @@ def test_dependent_launch_gives_same_bits(name, act_mode, monkeypatch):
     for a, b in zip(outs[0][1], outs[1][1]):
         assert torch.equal(a, b)
 
+
+
+def test_router_matches_hand_derived_cases():
+    """The router on the hand-derived cases of tests/golden/routing_cases.txt (ties, -0 / +0, NaN
+    and -inf logits, k = E), each padded to 8 experts with -inf logits and run as one token of a
+    batch: ids as written, weights within 2e-6."""
+    from tests.test_oracle_routing import _golden_routing_cases
+    cases = _golden_routing_cases()
+    E, T = 8, len(cases)
+    k = max(c[0] for c in cases)
+    layer = moe_mx.MoeMxLayer(256, 128, E, T, k)
+    x = torch.zeros(T, 256, dtype=torch.bfloat16, device="cuda")
+    w1 = torch.zeros(E, 256, 128, dtype=torch.uint8, device="cuda")
+    w1s = torch.full((E, 256, 8), 127, dtype=torch.uint8, device="cuda")
+    w2 = torch.zeros(E, 256, 64, dtype=torch.uint8, device="cuda")
+    w2s = torch.full((E, 256, 4), 127, dtype=torch.uint8, device="cuda")
+    for kk in sorted({c[0] for c in cases}):
+        rows = [i for i, c in enumerate(cases) if c[0] == kk]
+        lg = torch.full((len(rows), E), float("-inf"), dtype=torch.float32)
+        for r, i in enumerate(rows):
+            lg[r, :len(cases[i][1])] = torch.tensor(cases[i][1], dtype=torch.float32)
+        layer.forward(x[:len(rows)], lg.cuda(), w1, w1s, w2, w2s, kk)
+        assert layer.sync_status() == moe_mx.MOE_MX_OK, moe_mx.moe_mx_last_error()
+        ids, w = [a.cpu().numpy() for a in layer.routing(len(rows), kk)[:2]]
+        for r, i in enumerate(rows):
+            assert ids[r].tolist() == cases[i][2], (cases[i], ids[r])
+            np.testing.assert_allclose(w[r], cases[i][3], rtol=2e-6, atol=1e-7)
+    layer.close()

@@ -7,6 +7,8 @@ stability").  The pins: library routines (torch.topk / torch.softmax on
 tie-free rows, numpy's stable argsort), invariants, brute force on ties and
 the k = E special case.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -105,3 +107,23 @@ def test_group_degenerate():
     ids = np.zeros((0, 2), np.int32)
     counts, offsets, sp = oracle.group(ids, 4)
     assert counts.tolist() == [0, 0, 0, 0] and offsets.tolist() == [0] * 5 and sp.size == 0
+
+
+def _golden_routing_cases():
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "routing_cases.txt")
+    cases = []
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        k, lg, ids, w = (f.strip() for f in line.split("|"))
+        cases.append((int(k), [float(v) for v in lg.split(",")], [int(v) for v in ids.split(",")],
+                      [float(v) for v in w.split(",")]))
+    return cases
+
+
+@pytest.mark.parametrize("k,logits,ids,w", _golden_routing_cases())
+def test_route_hand_derived_cases(k, logits, ids, w):
+    got_ids, got_w = oracle.route(np.array([logits], np.float32), k)
+    assert got_ids[0].tolist() == ids
+    np.testing.assert_allclose(got_w[0], w, rtol=2e-7, atol=1e-9)
