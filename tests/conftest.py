@@ -13,6 +13,14 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "slow: full-size workloads (minutes)")
 
 
+@pytest.fixture(scope="session", autouse=True)
+def _library_built():
+    """Build libmoe_mx.so (and nothing else) if it is missing or older than its sources, so
+    that the tests always load the library built from the sources they test."""
+    from block_scaled_moe_softmax_b200 import build as lib_build
+    lib_build.build()
+
+
 @pytest.fixture(scope="session")
 def cuda_available():
     import torch
