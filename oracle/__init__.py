@@ -24,8 +24,10 @@ function states the passage of the pages it follows in the C source:
 * MX codecs per the OCP Microscaling Formats v1.0 specification.
 
 Parity pins (what ties this oracle to something other than itself) are in
-``tests/test_oracle_mx.py``, ``tests/test_oracle_routing.py`` and
-``tests/test_oracle_layer.py``.
+``tests/test_oracle_mx.py``, ``tests/test_oracle_routing.py``,
+``tests/test_oracle_layer.py``, ``tests/test_oracle_routed.py`` and
+``tests/test_oracle_shared.py``; ``tests/test_oracle_mutations.py`` shows that
+they catch planted mistakes.
 """
 from __future__ import annotations
 

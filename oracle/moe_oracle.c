@@ -33,7 +33,9 @@
  * specification (E2M1, E4M3, E8M0 definitions and the shared-scale rule
  * floor(log2(amax)) - emax_elem).
  *
- * Parity pins for every function live in tests/test_oracle_*.py.
+ * Parity pins for every function live in tests/test_oracle_*.py (MX codecs, routing and
+ * grouping, the layer, the routed form, the shared expert), with hand-derived fixtures in
+ * tests/golden/.
  */
 #include <math.h>
 #include <pthread.h>
