@@ -20,6 +20,7 @@ and reduce_partials sums the ranks' outputs.
 """
 from __future__ import annotations
 
+import numpy as np
 import torch
 
 from . import moe_mx
@@ -75,12 +76,11 @@ def tp_shard_weights(w1, w1_scale, w2, w2_scale, rank: int, world: int):
         g, u = a[:, lo:lo + n], a[:, I + lo:I + lo + n]
         if isinstance(a, torch.Tensor):
             return torch.cat([g, u], dim=1).contiguous()
-        import numpy as np
         return np.ascontiguousarray(np.concatenate([g, u], axis=1))
 
-    def cols(a, per):  # columns of the slice along the last dim, `per` elements per stored unit
+    def cols(a, per):  # columns of the slice along the last dim, `per` elements per stored byte
         c = a[:, :, lo // per:(lo + n) // per]
-        return c.contiguous() if isinstance(c, torch.Tensor) else __import__("numpy").ascontiguousarray(c)
+        return c.contiguous() if isinstance(c, torch.Tensor) else np.ascontiguousarray(c)
 
     return rows(w1), rows(w1_scale), cols(w2, 2), cols(w2_scale, 32)
 
