@@ -2,6 +2,7 @@
 """Benchmark of the fused MXFP4 routed-MoE layer on B200; prints ONE JSON line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    (K defaults to 1000, or 200 for the reference arm)
                     [--workload decode|tiny|batched_decode|prefill|prefill_w4a8]
 
 Other workloads: the batched-decode and prefill configurations, and shards of the
@@ -541,7 +542,8 @@ def run_ours(args, wl):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 1000; 200 for --impl reference, whose step is a CPU pair-evaluation)")
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(workloads.WORKLOADS), default="decode")
@@ -550,6 +552,8 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     wl = workloads.WORKLOADS[args.workload]
+    if args.steps is None:
+        args.steps = 200 if args.impl == "reference" else 1000
     if args.impl == "reference":
         if int(os.environ.get("RANK", "0")) != 0:
             return
