@@ -61,12 +61,6 @@ from block_scaled_moe_softmax_b200 import moe_mx, workloads  # noqa: E402
 
 METRIC = "MoE layer tokens/s; % of HBM roofline (decode) / MMA peak (prefill)"
 FLUSH_BYTES = 512 << 20
-def kernels_per_forward(T):
-    """Kernel launches of one forward: routing+grouping (one kernel up to 64 tokens, else route,
-    scan and scatter), gather, FC1, FC2, combine."""
-    return (1 if T <= 64 else 3) + 4
-
-
 def log(*a):
     print(*a, file=sys.stderr, flush=True)
 
@@ -208,50 +202,6 @@ def max_over_ranks(v, world):
 
 
 # ------------------------------------------------------------------ CPU oracle timing
-def oracle_time_tokens(wl, xb, route_np, wq, tokens, nthreads):
-    import oracle
-    act = 1 if wl.act == "mxfp8" else 0
-    t0 = time.perf_counter()
-    if wl.routing == "given":
-        ids, w = route_np
-        oracle.moe_forward_routed(xb, ids, w, wl.local_offset, *wq, act, tokens=tokens, nthreads=nthreads)
-    else:
-        oracle.moe_forward(xb, route_np, *wq, wl.top_k, act, tokens=tokens, nthreads=nthreads,
-                           num_shared=wl.shared)
-    return time.perf_counter() - t0
-
-
-def cpu_sample_setup(wl, sample_tokens):
-    """Host inputs for the oracle on a token sample: x, the routing input (logits, or given ids
-    and weights), oracle-quantised weights of the experts the sample reaches, those experts."""
-    import oracle
-    if wl.routing == "given":
-        ids, w = (a.numpy() for a in workloads.draw_topk(wl))
-        loc = ids[sample_tokens] - wl.local_offset
-        experts = sorted(set(int(e) for e in loc.reshape(-1) if 0 <= e < wl.E))
-        route_np = (ids, w)
-    else:
-        logits = workloads.draw_logits(wl)
-        ids, _ = oracle.route(logits.numpy()[sample_tokens], wl.top_k)
-        experts = sorted(set(int(e) for e in ids.reshape(-1))) + list(range(wl.E, wl.slots))
-        route_np = logits.numpy()
-    dev = "cuda" if torch.cuda.is_available() else "cpu"
-    wq = oracle_weights_for(wl, experts, dev)
-    xb = workloads.bf16_bits(workloads.draw_x(wl))
-    return xb, route_np, wq, experts
-
-
-def cpu_baseline(wl, cores):
-    """The oracle on a bounded sample (about 10-30 s of CPU work): a few tokens, one thread each."""
-    n_tok = max(1, min(4, cores, wl.T))
-    tokens = list(range(n_tok))
-    xb, route_np, wq, experts = cpu_sample_setup(wl, tokens)
-    dt = oracle_time_tokens(wl, xb, route_np, wq, tokens, n_tok)
-    return {"value": n_tok / dt, "unit": "tokens/s", "cores": n_tok, "kind": "oracle",
-            "sample": f"tokens 0..{n_tok - 1} of the {wl.name} workload ({len(experts)} experts hit), "
-                      f"one oracle call, {n_tok} threads, {dt:.1f} s wall"}
-
-
 def reference_pairs(wl, sample_tokens):
     """The (token, slot) pairs of the sampled tokens that the layer evaluates -- the routed slots
     (the oracle's router, or the given routing restricted to the local shard) and the shared
@@ -275,50 +225,80 @@ def reference_pairs(wl, sample_tokens):
     return pairs, per_token + wl.shared
 
 
-def run_reference(args, wl):
-    """The oracle as the reference arm.  One step = one (token, slot) pair of the workload: the
-    FC1, SwiGLU and FC2 of one token through one expert, weighted -- the unit of the layer's work
-    (a token of the decode shapes is k of them), small enough that K steps take a few minutes.
-    The pairs come from the first `cores` tokens (their routing taken once, outside the timed
-    steps) and run in batches of up to `cores` concurrent steps, one thread each, through the
-    oracle's routed form with one slot per evaluated row.  tokens/s = pairs/s / pairs per token."""
-    import oracle
-    cores = len(os.sched_getaffinity(0))
-    sample = list(range(min(wl.T, cores)))
-    pairs, per_token = reference_pairs(wl, sample)
-    experts = sorted({e for _, e, _ in pairs})
-    dev = "cuda" if torch.cuda.is_available() else "cpu"
-    wq = oracle_weights_for(wl, [e for e in experts if e < wl.E] + list(range(wl.E, wl.slots)), dev)
-    xb = workloads.bf16_bits(workloads.draw_x(wl))
-    act = 1 if wl.act == "mxfp8" else 0
+class PairSampler:
+    """The oracle on (token, slot) pairs of a workload: one pair = one token's FC1, SwiGLU and FC2
+    through one expert, weighted -- the unit of the layer's work (a decode token is k of them).
+    The pairs are those of the given sample tokens (their routing taken once, here, outside any
+    timed region); batches of up to `threads` pairs run concurrently, one thread each, through the
+    oracle's routed form with one slot per evaluated row."""
 
-    def run_steps(n):
-        done, wall = 0, 0.0
-        while done < n:
-            batch = min(cores, n - done)
-            sel = [pairs[(done + i) % len(pairs)] for i in range(batch)]
-            xs = np.ascontiguousarray(xb[[t for t, _, _ in sel]])
+    def __init__(self, wl, sample_tokens, threads):
+        self.wl, self.threads = wl, threads
+        self.pairs, self.per_token = reference_pairs(wl, sample_tokens)
+        self.experts = sorted({e for _, e, _ in self.pairs})
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        self.wq = oracle_weights_for(wl, [e for e in self.experts if e < wl.E] + list(range(wl.E, wl.slots)), dev)
+        self.xb = workloads.bf16_bits(workloads.draw_x(wl))
+        self.act = 1 if wl.act == "mxfp8" else 0
+        self.done = 0
+
+    def run(self, n):
+        """Evaluate the next n pairs (cycling); returns the wall seconds of the oracle calls."""
+        import oracle
+        wall = 0.0
+        end = self.done + n
+        while self.done < end:
+            batch = min(self.threads, end - self.done)
+            sel = [self.pairs[(self.done + i) % len(self.pairs)] for i in range(batch)]
+            xs = np.ascontiguousarray(self.xb[[t for t, _, _ in sel]])
             ids = np.array([[e] for _, e, _ in sel], np.int32)
             ws = np.array([[w] for _, _, w in sel], np.float32)
             t0 = time.perf_counter()
-            oracle.moe_forward_routed(xs, ids, ws, 0, *wq, act, nthreads=batch)
+            oracle.moe_forward_routed(xs, ids, ws, 0, *self.wq, self.act, nthreads=batch)
             wall += time.perf_counter() - t0
-            done += batch
+            self.done += batch
         return wall
 
-    run_steps(args.warmup)
-    total = run_steps(args.steps)
-    value = args.steps / total / per_token
+
+def cpu_baseline(wl, cores, min_wall=3.0):
+    """The oracle on a bounded sample of the workload, on all the host's cores: batches of one
+    (token, slot) pair per core, one thread each, until at least min_wall seconds of oracle time;
+    tokens/s = pairs/s / pairs per token."""
+    n_tok = min(wl.T, max(1, -(-cores // max(1, wl.top_k))))
+    ps = PairSampler(wl, list(range(n_tok)), cores)
+    wall, pairs = 0.0, 0
+    while wall < min_wall:
+        wall += ps.run(cores)
+        pairs += cores
+    return {"value": pairs / wall / ps.per_token, "unit": "tokens/s", "cores": cores, "threads": cores,
+            "kind": "oracle",
+            "sample": f"{pairs} (token, slot) pairs of the {wl.name} workload (the {len(ps.pairs)} pairs of tokens "
+                      f"0..{n_tok - 1} cycled, {len(ps.experts)} experts), {cores} at a time, one thread per core "
+                      f"on {cores} cores, {wall:.1f} s of oracle wall time; {ps.per_token:g} pairs per token"}
+
+
+def run_reference(args, wl):
+    """The oracle as the reference arm.  One step = one (token, slot) pair of the workload (see
+    PairSampler), small enough that K steps take a few minutes.  The pairs come from the first
+    `cores` tokens and run up to `cores` at a time, one thread each.
+    tokens/s = pairs/s / pairs per token."""
+    cores = len(os.sched_getaffinity(0))
+    sample = list(range(min(wl.T, cores)))
+    ps = PairSampler(wl, sample, cores)
+    ps.run(args.warmup)
+    total = ps.run(args.steps)
+    value = args.steps / total / ps.per_token
+    used = min(cores, args.steps)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 0,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": workload_desc(wl), "pairs_per_step": 1, "pairs_per_token": per_token},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": min(cores, args.steps), "kind": "oracle",
-                         "sample": f"one (token, slot) pair of {wl.name} per step: the {len(pairs)} pairs of tokens "
-                                   f"0..{len(sample) - 1} cycled ({len(experts)} experts), up to {cores} steps "
-                                   f"concurrently; {per_token:g} pairs per token"},
+        "config": {"workload": workload_desc(wl), "pairs_per_step": 1, "pairs_per_token": ps.per_token},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used, "threads": used, "kind": "oracle",
+                         "sample": f"one (token, slot) pair of {wl.name} per step: the {len(ps.pairs)} pairs of "
+                                   f"tokens 0..{len(sample) - 1} cycled ({len(ps.experts)} experts), up to {cores} "
+                                   f"steps concurrently on {cores} cores; {ps.per_token:g} pairs per token"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -377,14 +357,32 @@ def traffic_record(wl, fc1_bytes):
     return None
 
 
-def run_ours(args, wl):
-    world, rank, local = dist_setup(args.gpus)
+class WeightCache:
+    """One resident weight set at a time: the decode, batched-decode and prefill workloads share
+    theirs (same H, I, E, seed), so the default run draws and quantises it once."""
+
+    def __init__(self, dev):
+        self.dev, self.key, self.w = dev, None, None
+
+    def get(self, wl):
+        key = (wl.H, wl.I, wl.E, wl.shared, wl.seed)
+        if key != self.key:
+            self.w = None
+            torch.cuda.empty_cache()
+            log(f"generating weights for {workload_desc(wl)}")
+            self.w = make_gpu_weights(wl, self.dev)
+            self.key = key
+        return self.w
+
+
+def measure(args, wl, weights, world, rank, with_e2e=True):
+    """Time one workload: K steps device-resident (the value), then the same steps with events
+    between the kernels (each kernel's own duration), then K steps end to end from pinned host
+    buffers.  Returns the workload's record (rank 0's view of the max-over-ranks times)."""
     dev = torch.device("cuda", torch.cuda.current_device())
     hbm_peak, bf16_peak, bf16_sustained, peak_src = measured_peaks()
     act = moe_mx.MOE_MX_ACT_MXFP8 if wl.act == "mxfp8" else moe_mx.MOE_MX_ACT_BF16
-
-    log(f"[rank {rank}] generating weights for {workload_desc(wl)}")
-    w1, w1s, w2, w2s = make_gpu_weights(wl, dev)
+    w1, w1s_rm, w2, w2s_rm = weights
     x = workloads.draw_x(wl).to(dev)
     given = wl.routing == "given"
     # the routing input: router logits, or the given top-k (global ids and weights)
@@ -393,7 +391,7 @@ def run_ours(args, wl):
     out = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=dev)
     layer = moe_mx.MoeMxLayer(wl.H, wl.I, wl.E, wl.T, wl.top_k, device=dev.index, num_shared=wl.shared)
     # weight preparation, once, like the quantisation: the E8M0 scales in the tiled layout
-    w1s, w2s = layer.prepare_scales(w1s, w2s)
+    w1s, w2s = layer.prepare_scales(w1s_rm, w2s_rm)
     torch.cuda.synchronize()
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
@@ -405,12 +403,9 @@ def run_ours(args, wl):
         else:
             moe_mx.moe_mx_forward(layer.handle, xin, rin[0], wl.T, w1, w1s, w2, w2s, wl.top_k, act, out, stream)
 
-    def fwd():
-        forward(x, route_in)
-
     for _ in range(args.warmup):
         flush.zero_()
-        fwd()
+        forward(x, route_in)
     torch.cuda.synchronize()
     status = layer.sync_status()
     assert status == moe_mx.MOE_MX_OK, moe_mx.moe_mx_last_error()
@@ -426,17 +421,20 @@ def run_ours(args, wl):
     torch.cuda.synchronize()
     if sampler:
         sampler.start()
+    launches0 = moe_mx.moe_mx_launch_count(layer.handle)
     for i in range(args.steps):
         flush.zero_()
         evs[i][0].record(stream)
-        fwd()
+        forward(x, route_in)
         evs[i][1].record(stream)
+    launches = moe_mx.moe_mx_launch_count(layer.handle) - launches0
     torch.cuda.synchronize()
     barrier(world)
     clocks = sampler.stop() if sampler else None
     step_ms = [a.elapsed_time(b) for a, b in evs]
     assert layer.sync_status() == moe_mx.MOE_MX_OK, moe_mx.moe_mx_last_error()
-    ms = statistics.mean(step_ms)
+    ms_all = max_over_ranks(statistics.mean(step_ms), world)
+    value = world * wl.T / (ms_all / 1000.0)
 
     # ---------------- per-kernel times: the same steps with CUDA events between the kernels.
     # (In the timed steps above each kernel may launch while the one before it still runs, and
@@ -446,36 +444,40 @@ def run_ours(args, wl):
     moe_mx.moe_mx_set_stage_timing(layer.handle, True)
     for i in range(stage_steps):
         flush.zero_()
-        fwd()
+        forward(x, route_in)
     stage = moe_mx.moe_mx_get_stage_times(layer.handle)
     moe_mx.moe_mx_set_stage_timing(layer.handle, False)
     assert layer.sync_status() == moe_mx.MOE_MX_OK, moe_mx.moe_mx_last_error()
-    ms_all = max_over_ranks(ms, world)
-    value = world * wl.T / (ms_all / 1000.0)
 
     # ---------------- end to end through the public API with host buffers
-    x_h = workloads.draw_x(wl).pin_memory()
-    r_h = tuple(a.pin_memory() for a in route_host)
-    o_h = torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory()
-    x_d = torch.empty_like(x)
-    r_d = tuple(torch.empty_like(a) for a in route_in)
-    e2e_steps = max(3, min(args.steps, 200))
-    e2e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    for i in range(e2e_steps):
-        flush.zero_()
-        e2e_evs[i][0].record(stream)
-        x_d.copy_(x_h, non_blocking=True)
-        for dst, src in zip(r_d, r_h):
-            dst.copy_(src, non_blocking=True)
-        forward(x_d, r_d)
-        o_h.copy_(out, non_blocking=True)
-        e2e_evs[i][1].record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in e2e_evs), world)
-    assert torch.equal(o_h.view(torch.int16), out.cpu().view(torch.int16))
+    e2e = None
+    if with_e2e:
+        x_h = workloads.draw_x(wl).pin_memory()
+        r_h = tuple(a.pin_memory() for a in route_host)
+        o_h = torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory()
+        x_d = torch.empty_like(x)
+        r_d = tuple(torch.empty_like(a) for a in route_in)
+        e2e_steps = max(3, min(args.steps, 200))
+        e2e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(e2e_steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        for i in range(e2e_steps):
+            flush.zero_()
+            e2e_evs[i][0].record(stream)
+            x_d.copy_(x_h, non_blocking=True)
+            for dst, src in zip(r_d, r_h):
+                dst.copy_(src, non_blocking=True)
+            forward(x_d, r_d)
+            o_h.copy_(out, non_blocking=True)
+            e2e_evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in e2e_evs), world)
+        assert torch.equal(o_h.view(torch.int16), out.cpu().view(torch.int16))
+        e2e = {"value": world * wl.T / (e2e_ms / 1000.0), "unit": "tokens/s",
+               "h2d_bytes_per_step": wl.T * wl.H * 2 + sum(a.numel() * a.element_size() for a in route_host),
+               "d2h_bytes_per_step": wl.T * wl.H * 2}
 
     fc1_ms = stage["fc1"]
     layer_bytes = layer_weight_bytes(wl, hit)
@@ -509,31 +511,56 @@ def run_ours(args, wl):
         layer_roofline = {"bound": "hbm", "weight_bytes": layer_bytes,
                           "achieved_gbs": layer_bytes / (ms_all / 1000.0) / 1e9,
                           "frac": layer_bytes / (ms_all / 1000.0) / 1e9 / hbm_peak}
+    rec = {"workload": workload_desc(wl), "ms_per_step": ms_all, "tokens_per_s": value, "hit_experts": hit,
+           "gpu_launches": launches, "roofline": roofline, "layer_roofline": layer_roofline, "stage_ms": stage,
+           "stage_ms_steps": stage_steps, "clocks": clocks, "e2e": e2e,
+           "weight_bytes_resident": (w1.numel() + w1s.numel() + w2.numel() + w2s.numel())}
+    layer.close()
+    return rec
+
+
+# the five configurations of the layer, measured by the default run (the first is the headline)
+DEFAULT_SET = ("decode", "tiny", "batched_decode", "prefill", "prefill_w4a8")
+
+
+def run_ours(args):
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    names = [args.workload] if args.workload else list(DEFAULT_SET)
+    cache = WeightCache(dev)
+    recs = {}
+    for name in names:
+        wl = workloads.WORKLOADS[name]
+        recs[name] = measure(args, wl, cache.get(wl), world, rank)
+    head_name = names[0]
+    wl = workloads.WORKLOADS[head_name]
+    head = recs[head_name]
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_all, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": workload_desc(wl), "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "top_k": wl.top_k,
-                   "act": wl.act, "hit_experts": hit, "global_batch": wl.T * world, "parallelism": f"replicas{world}",
-                   "l2": f"weights {(w1.numel() + w1s.numel() + w2.numel() + w2s.numel()) / 1e9:.2f} GB, "
-                         "a 512 MiB L2 flush before every timed step",
+        "metric": METRIC, "value": head["tokens_per_s"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": head["workload"], "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "top_k": wl.top_k,
+                   "act": wl.act, "hit_experts": head["hit_experts"], "global_batch": wl.T * world,
+                   "parallelism": f"replicas{world}",
+                   "l2": f"weights {head['weight_bytes_resident'] / 1e9:.2f} GB, a 512 MiB L2 flush before every "
+                         "timed step",
                    "weight_scales": "tiled layout (moe_mx_prepare_scales, once before timing)"},
-        "e2e": {"value": world * wl.T / (e2e_ms / 1000.0), "unit": "tokens/s",
-                "h2d_bytes_per_step": wl.T * wl.H * 2 + sum(a.numel() * a.element_size() for a in route_host),
-                "d2h_bytes_per_step": wl.T * wl.H * 2},
-        "gpu_launches": kernels_per_forward(wl.T) * args.steps,
-        "roofline": roofline,
-        "layer_roofline": layer_roofline,
-        "stage_ms": stage,
-        "stage_ms_steps": stage_steps,
-        "clocks": clocks,
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
+        "roofline": head["roofline"],
+        "layer_roofline": head["layer_roofline"],
+        "stage_ms": head["stage_ms"],
+        "stage_ms_steps": head["stage_ms_steps"],
+        "clocks": head["clocks"],
     }
+    if len(recs) > 1:
+        line["per_config"] = {n: {k: v for k, v in r.items() if k != "weight_bytes_resident"}
+                              for n, r in recs.items()}
     if rank == 0 and not args.no_cpu_baseline:
         cores = len(os.sched_getaffinity(0))
         line["cpu_baseline"] = cpu_baseline(wl, cores)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    layer.close()
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -546,12 +573,14 @@ def main():
                     help="timed steps (default 1000; 200 for --impl reference, whose step is a CPU pair-evaluation)")
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(workloads.WORKLOADS), default="decode")
+    ap.add_argument("--workload", choices=sorted(workloads.WORKLOADS), default=None,
+                    help="one workload only (default: decode as the headline, plus the other four "
+                         "configurations in per_config)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    wl = workloads.WORKLOADS[args.workload]
+    wl = workloads.WORKLOADS[args.workload or DEFAULT_SET[0]]
     if args.steps is None:
         args.steps = 200 if args.impl == "reference" else 1000
     if args.impl == "reference":
@@ -561,7 +590,7 @@ def main():
         return
     from block_scaled_moe_softmax_b200 import build as lib_build
     lib_build.build()
-    run_ours(args, wl)
+    run_ours(args)
 
 
 if __name__ == "__main__":

@@ -157,6 +157,7 @@ struct moe_mx_handle {
     const void *w1_key, *w2_key;
     CUtensorMap map_w1, map_w2;
     int last_T, last_k;
+    long long launches; // kernels launched by this handle's forwards since create
     // stage timing: a ring of kTimingRing event sets, one set per timed forward
     cudaEvent_t *ev;
     bool timing;
@@ -438,7 +439,7 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
         // dependent launch): the FC GEMMs start streaming their weights early.  Stage timing
         // records events between the kernels, so timed forwards launch them one after another.
         const bool pdl = h->pdl && !evset;
-        launch_route_and_group(ra, s, pdl);
+        h->launches += launch_route_and_group(ra, s, pdl);
         mark(1);
         const int mx8 = act_dtype == MOE_MX_ACT_MXFP8;
         launch_gather(static_cast<const __nv_bfloat16 *>(x), (int)pairs, H, k, h->pos_of_pair, h->Aq, h->Asf,
@@ -489,6 +490,7 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
                        h->num_sms, s, pdl);
         mark(4);
         launch_combine(h->Y, T, H, k, h->pos_of_pair, h->topk_w, out, out_f32, h->num_sms, s, pdl);
+        h->launches += 4; // gather, FC1, FC2, combine
         ce = cudaGetLastError();
         if (ce != cudaSuccess) {
             rc = cuda_fail(ce, "kernel launch");
@@ -620,6 +622,70 @@ int moe_mx_get_routing(const moe_mx_handle *h, int32_t *topk_ids, float *topk_w,
     }
     return MOE_MX_OK;
 }
+
+int moe_mx_get_intermediate(const moe_mx_handle *h, int which, void *dst, void *stream)
+{
+    g_last_error.clear();
+    if (!h)
+        return fail(MOE_MX_ERR_INVALID_ARG, "handle is NULL");
+    if (which < MOE_MX_INTER_AQ || which > MOE_MX_INTER_Y)
+        return fail(MOE_MX_ERR_INVALID_ARG, "which=%d is not one of MOE_MX_INTER_*", which);
+    const int64_t rows = grouped_rows_bound(h->E, (int64_t)h->last_T * h->last_k);
+    if (rows == 0)
+        return MOE_MX_OK;
+    if (!is_device_ptr(dst, h->dev))
+        return fail(MOE_MX_ERR_INVALID_ARG, "dst must be a device pointer on device %d", h->dev);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t K = (which == MOE_MX_INTER_AQ || which == MOE_MX_INTER_ASF) ? h->H : h->I;
+    cudaError_t ce = cudaSuccess;
+    uint8_t *d = static_cast<uint8_t *>(dst);
+    if (which == MOE_MX_INTER_AQ || which == MOE_MX_INTER_HQ) {
+        // two term planes of `rows` rows each, packed; in the workspace they sit max_rows apart
+        const uint8_t *src = which == MOE_MX_INTER_AQ ? h->Aq : h->Hq;
+        for (int t = 0; t < 2 && ce == cudaSuccess; ++t)
+            ce = cudaMemcpyAsync(d + t * rows * K, src + t * h->max_rows * K, (size_t)(rows * K),
+                                 cudaMemcpyDeviceToDevice, s);
+    } else if (which == MOE_MX_INTER_ASF || which == MOE_MX_INTER_HSF) {
+        const uint8_t *src = which == MOE_MX_INTER_ASF ? h->Asf : h->Hsf;
+        ce = cudaMemcpyAsync(d, src, (size_t)((rows / 128) * (K / 128) * 1024), cudaMemcpyDeviceToDevice, s);
+    } else {
+        ce = cudaMemcpyAsync(d, h->Y, (size_t)(rows * h->H) * sizeof(float), cudaMemcpyDeviceToDevice, s);
+    }
+    if (ce != cudaSuccess)
+        return cuda_fail(ce, "cudaMemcpyAsync(intermediate)");
+    return MOE_MX_OK;
+}
+
+int moe_mx_debug_encode_act(const float *src, int rows, int K, int act_dtype, int method, uint8_t *codes,
+                            uint8_t *scale_atoms, void *stream)
+{
+    g_last_error.clear();
+    if (rows < 0 || K < 128 || K % 128 != 0)
+        return fail(MOE_MX_ERR_INVALID_ARG, "rows=%d K=%d: need rows >= 0 and K a positive multiple of 128", rows, K);
+    if (act_dtype != MOE_MX_ACT_BF16 && act_dtype != MOE_MX_ACT_MXFP8)
+        return fail(MOE_MX_ERR_INVALID_ARG, "act_dtype=%d is not MOE_MX_ACT_BF16 or MOE_MX_ACT_MXFP8", act_dtype);
+    if (method != 0 && method != 1)
+        return fail(MOE_MX_ERR_INVALID_ARG, "method=%d is not 0 or 1", method);
+    if (rows == 0)
+        return MOE_MX_OK;
+    int dev = 0;
+    cudaError_t ce = cudaGetDevice(&dev);
+    if (ce != cudaSuccess)
+        return cuda_fail(ce, "cudaGetDevice");
+    int rc;
+    if ((rc = check_ptr(src, dev, "src")) || (rc = check_ptr(codes, dev, "codes")) ||
+        (rc = check_ptr(scale_atoms, dev, "scale_atoms")))
+        return rc;
+    int nsm = 148;
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    launch_encode_act(src, rows, K, act_dtype == MOE_MX_ACT_MXFP8, method, codes, scale_atoms, nsm,
+                      static_cast<cudaStream_t>(stream));
+    if ((ce = cudaGetLastError()) != cudaSuccess)
+        return cuda_fail(ce, "encoder launch");
+    return MOE_MX_OK;
+}
+
+long long moe_mx_launch_count(const moe_mx_handle *h) { return h ? h->launches : -1; }
 
 int moe_mx_set_scale_layout(moe_mx_handle *h, int layout)
 {

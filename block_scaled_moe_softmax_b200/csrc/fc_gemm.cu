@@ -660,17 +660,20 @@ __device__ __forceinline__ void epilogue_wide(const FcGemmArgs &a, const Ctx &c,
             const int rl = 32 * q + lane;
             const bool valid = rl < blk.z;
             const int row = blk.y + rl;
-            // columns 0..63: gate rows nt*64 + i, columns 64..127: the matching up rows
+            // columns 0..63: gate rows nt*64 + i, columns 64..127: the matching up rows.  Both halves'
+            // h first, so that the accumulator registers are dead before the encoder runs.
+            float h[2][32];
 #pragma unroll
-            for (int c32 = 0; c32 < 2; ++c32) {
-                float h[32];
+            for (int c32 = 0; c32 < 2; ++c32)
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    h[i] = silu_mul(__uint_as_float(v[2 * c32][i]), __uint_as_float(v[4 + 2 * c32][i]));
-                    h[16 + i] = silu_mul(__uint_as_float(v[2 * c32 + 1][i]), __uint_as_float(v[5 + 2 * c32][i]));
+                    h[c32][i] = silu_mul(__uint_as_float(v[2 * c32][i]), __uint_as_float(v[4 + 2 * c32][i]));
+                    h[c32][16 + i] = silu_mul(__uint_as_float(v[2 * c32 + 1][i]), __uint_as_float(v[5 + 2 * c32][i]));
                 }
-                if (valid)
-                    store_act_block32(a.hq, a.hsf, a.hq_rows, a.out_ld, row, nt * 64 + 32 * c32, h, a.act_mxfp8);
+            if (valid) {
+#pragma unroll
+                for (int c32 = 0; c32 < 2; ++c32)
+                    store_act_block32(a.hq, a.hsf, a.hq_rows, a.out_ld, row, nt * 64 + 32 * c32, h[c32], a.act_mxfp8);
             }
         } else {
             // FC2: f32 rows of Y.  Stored straight from registers, each store instruction of the

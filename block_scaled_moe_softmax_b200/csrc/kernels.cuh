@@ -69,7 +69,8 @@ struct RouteGroupArgs {
 // before them in the stream (each waits for its predecessor before reading its output and lets
 // its own successor launch right after that wait); the first kernel of a forward, the router,
 // is always an ordinary launch.
-void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s, bool pdl = false);
+// Returns the number of kernels launched (1 for small batches, else 3).
+int launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s, bool pdl = false);
 void launch_gather(const __nv_bfloat16 *x, int P, int H, int k, const int32_t *pos_of_pair, uint8_t *aq,
                    uint8_t *asf, int act_rows, int act_mxfp8, int num_sms, cudaStream_t s, bool pdl = false);
 // out: bf16 [T, H], or (out_f32) float32 [T, H]; pairs with pos_of_pair -1 add nothing
@@ -127,34 +128,11 @@ void launch_tile_scales(const uint8_t *src, uint8_t *dst, int E, int R, int K, i
 
 void launch_watchdog(uint32_t *err, unsigned long long timeout_ns, cudaStream_t s);
 
-// ---------------------------------------------------------------- MX device helpers
-// Quantise 32 values to MXFP8 E4M3 with the shared-scale rule of the OCP MX
-// specification (s = floor(log2 amax) - 8, clamped to [-127, 127]); returns the
-// scale byte and writes the 32 codes.
-__device__ __forceinline__ uint32_t mx_quantize32_e4m3(const float (&v)[32], uint8_t (&codes)[32])
-{
-    float amax = 0.f;
-    bool finite = true;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const float a = fabsf(v[i]);
-        finite = finite && (a <= 3.402823466e38f);
-        amax = fmaxf(amax, a);
-    }
-    if (!finite) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-            codes[i] = 0;
-        return 0xFF;
-    }
-    int s = (amax == 0.f) ? -127 : floor_log2_pos(amax) - 8;
-    s = max(-127, min(127, s));
-    const float inv = exp2_int(-s);
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-        codes[i] = (uint8_t)f32_to_e4m3(__fmul_rn(v[i], inv));
-    return (uint32_t)(s + 127);
-}
+// Encode float32 rows [rows, K] (K a multiple of 128) into codes [2][rows][K] and scale atoms
+// [ceil(rows/128)][K/128][2][512] with the forward's activation encoders: method 0 =
+// store_act_block32, 1 = store_act_warp32 (test entry moe_mx_debug_encode_act).
+void launch_encode_act(const float *src, int rows, int K, int act_mxfp8, int method, uint8_t *q, uint8_t *sf,
+                       int num_sms, cudaStream_t s);
 
 // ---------------------------------------------------------------- activation operand format
 // Activations reach the tensor core as MXFP8 E4M3 codes in [term][row][K]
@@ -181,22 +159,38 @@ __device__ __forceinline__ int mx_block_exp(float amax, int emax_shift)
     return max(-127, min(127, s));
 }
 
+// Largest finite float: a value compares <= to it only if it is neither infinite nor NaN.
+constexpr float kMaxFinite = 3.402823466e38f;
+
 // Encode 32 values as MXFP8 terms.  act_mxfp8 = 1: the OCP rule (shared
 // exponent floor(log2 amax) - 8, round-to-nearest-even, saturating) -- one term,
-// the w4a8 activation.  act_mxfp8 = 0: an exact two-term expansion of bf16
-// values, v = x1 + x2: x1 takes exponent floor(log2 amax) - 7 (the block max
-// lands in [128, 256), below the E4M3 maximum, so nothing saturates) and keeps
-// the top 4 significant bits of every element; x2 encodes the remainder v - x1,
-// which has at most 4 significant bits, with its own block exponent.  Elements
-// within 2^-13 of the block maximum are represented exactly; smaller ones keep
-// an absolute error below 2^-20 of the block maximum.
+// the w4a8 activation, and the MXFP8 path of moe_mx_quantize.  act_mxfp8 = 0: an
+// exact two-term expansion of bf16 values, v = x1 + x2: x1 takes exponent
+// floor(log2 amax) - 7 (the block max lands in [128, 256), below the E4M3
+// maximum, so nothing saturates) and keeps the top 4 significant bits of every
+// element; x2 encodes the remainder v - x1, which has at most 4 significant
+// bits, with its own block exponent.  Elements within 2^-13 of the block maximum
+// are represented exactly; smaller ones keep an absolute error below 2^-20 of
+// the block maximum.  A block that holds a NaN or an infinity has no finite
+// scale: every term gets the E8M0 NaN byte 0xFF and zero codes (the OCP
+// quantiser's rule for such a block).
 __device__ __forceinline__ void mx_encode32(const float (&v)[32], int act_mxfp8, uint8_t (&c0)[32], uint8_t (&c1)[32],
                                             uint32_t &s0, uint32_t &s1)
 {
+    // amax with NaN propagated: the block is finite exactly when amax <= the largest float
     float amax = 0.f;
 #pragma unroll
     for (int i = 0; i < 32; ++i)
-        amax = fmaxf(amax, fabsf(v[i]));
+        amax = fmax_nan(amax, fabsf(v[i]));
+    if (!(amax <= kMaxFinite)) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            c0[i] = 0;
+            c1[i] = 0;
+        }
+        s0 = s1 = 0xFFu;
+        return;
+    }
     const int e0 = mx_block_exp(amax, act_mxfp8 ? 8 : 7);
     const float inv0 = exp2_int(-e0), sc0 = exp2_int(e0);
     float r[32];
@@ -253,31 +247,33 @@ __device__ __forceinline__ void store_act_block32(uint8_t *q, uint8_t *sf, int p
 }
 
 // The 32 lanes of a warp write one 32-element block of `row`, lane l holding
-// element col0 + l (col0 = col rounded down to 32).
+// element col0 + l (col0 = col rounded down to 32): the encoding of
+// store_act_block32 computed with warp reductions (same rule, same results).
 __device__ __forceinline__ void store_act_warp32(uint8_t *q, uint8_t *sf, int plane_rows, int K, int row, int col,
                                                  float v, int act_mxfp8, int lane)
 {
     if (!act_mxfp8)
         v = __bfloat162float(__float2bfloat16_rn(v));
+    const bool finite = __all_sync(0xFFFFFFFFu, fabsf(v) <= kMaxFinite);
     float amax = fabsf(v);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1)
         amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-    const int e0 = mx_block_exp(amax, act_mxfp8 ? 8 : 7);
-    const uint32_t c0 = f32_to_e4m3(__fmul_rn(v, exp2_int(-e0)));
+    const int e0 = finite ? mx_block_exp(amax, act_mxfp8 ? 8 : 7) : 0;
+    const uint32_t c0 = finite ? f32_to_e4m3(__fmul_rn(v, exp2_int(-e0))) : 0u;
     q[(size_t)row * K + col] = (uint8_t)c0;
     if (lane == 0)
-        sf[sf_atom_byte(row, col, K, 0)] = (uint8_t)(e0 + 127);
+        sf[sf_atom_byte(row, col, K, 0)] = finite ? (uint8_t)(e0 + 127) : (uint8_t)0xFF;
     if (!act_mxfp8) {
-        const float r = __fsub_rn(v, __fmul_rn(e4m3_to_f32(c0), exp2_int(e0)));
+        const float r = finite ? __fsub_rn(v, __fmul_rn(e4m3_to_f32(c0), exp2_int(e0))) : 0.f;
         float amax1 = fabsf(r);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1)
             amax1 = fmaxf(amax1, __shfl_xor_sync(0xFFFFFFFFu, amax1, off));
         const int e1 = mx_block_exp(amax1, 7);
-        q[((size_t)plane_rows + row) * K + col] = (uint8_t)f32_to_e4m3(__fmul_rn(r, exp2_int(-e1)));
+        q[((size_t)plane_rows + row) * K + col] = finite ? (uint8_t)f32_to_e4m3(__fmul_rn(r, exp2_int(-e1))) : 0u;
         if (lane == 0)
-            sf[sf_atom_byte(row, col, K, 1)] = (uint8_t)(e1 + 127);
+            sf[sf_atom_byte(row, col, K, 1)] = finite ? (uint8_t)(e1 + 127) : (uint8_t)0xFF;
     }
 }
 

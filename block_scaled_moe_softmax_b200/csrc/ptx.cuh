@@ -175,18 +175,6 @@ __device__ __forceinline__ void tc_fence_after()
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, both operands K-major, kind::f16.
-__device__ __forceinline__ void umma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                            uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 // Arrive once on an mbarrier when all previously issued tcgen05 async ops of
 // this thread have completed.
 __device__ __forceinline__ void umma_commit(uint32_t bar)
@@ -227,16 +215,6 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr)
     return d;
 }
 
-// Instruction descriptor, kind::f16: bf16 A and B (K-major), f32 accumulator.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N)
-{
-    return (1u << 4)            // D format f32
-           | (1u << 7)          // A format bf16
-           | (1u << 10)         // B format bf16
-           | ((N >> 3) << 17)   // N / 8
-           | ((M >> 4) << 24);  // M / 16
-}
-
 // ----------------------------------------------------------------- MX helpers
 // floor(log2(a)) for a finite a > 0, read from the float's bits (handles subnormals).
 __device__ __forceinline__ int floor_log2_pos(float a)
@@ -255,6 +233,14 @@ __device__ __forceinline__ float exp2_int(int n)
     if (n >= -126)
         return __uint_as_float((uint32_t)(n + 127) << 23);
     return __uint_as_float(1u << (n + 149));
+}
+
+// max(a, b) that propagates NaN (a NaN operand gives NaN; fmaxf would drop it).
+__device__ __forceinline__ float fmax_nan(float a, float b)
+{
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
 }
 
 // Round to the nearest E4M3 code (ties to even), saturating to +-448.
@@ -284,18 +270,6 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code)
     uint16_t in = (uint16_t)((code & 0xFF) * 0x0101u); // same code in both bytes
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
     return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFF)));
-}
-
-// bf16 bit pattern of an E2M1 code scaled by 2^(sb-127), for scale bytes
-// sb in [2, 252] (the result is then a normal bf16 number, exactly).
-__device__ __forceinline__ uint32_t e2m1_bf16_bits(uint32_t nib, uint32_t sb)
-{
-    const uint32_t c = nib & 7;
-    // magnitude codes: 1 -> 0.5, 2/3 -> 1/1.5, 4/5 -> 2/3, 6/7 -> 4/6
-    const uint32_t expo = sb + (c >> 1) - 1;         // biased bf16 exponent
-    const uint32_t mant = (c > 1) ? ((c & 1) << 6) : 0u;
-    const uint32_t mag = (c == 0) ? 0u : ((expo << 7) | mant);
-    return mag | ((nib & 8) << 12);
 }
 
 } // namespace moe_mx

@@ -2,8 +2,9 @@
 // Formats v1.0: per 32-element block, shared scale exponent
 // s = floor(log2(amax)) - emax_elem clamped to [-127, 127], stored as the E8M0
 // byte s + 127; elements rounded to nearest-even onto the element grid,
-// saturating).  Used to prepare MXFP4 weights; the forward's activation
-// quantisation shares mx_quantize32_e4m3.
+// saturating; a block holding a NaN or an infinity gets scale byte 0xFF and zero
+// codes).  Used to prepare MXFP4 weights.  The MXFP8 path runs mx_encode32, the
+// encoder the forward's gather and FC1 epilogue run on activations.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -18,7 +19,7 @@ __device__ __forceinline__ uint32_t mx_quantize32_e2m1(const float (&v)[32], uin
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
         const float a = fabsf(v[i]);
-        finite = finite && (a <= 3.402823466e38f);
+        finite = finite && (a <= kMaxFinite);
         amax = fmaxf(amax, a);
     }
     if (!finite) {
@@ -64,8 +65,10 @@ __global__ void __launch_bounds__(256) mx_quantize_kernel(const float *__restric
                 ob[i] = p[i];
             reinterpret_cast<uint4 *>(codes)[b] = o;
         } else {
-            uint8_t c[32];
-            scales[b] = (uint8_t)mx_quantize32_e4m3(v, c);
+            uint8_t c[32], unused[32];
+            uint32_t s0, s1;
+            mx_encode32(v, 1, c, unused, s0, s1);
+            scales[b] = (uint8_t)s0;
             uint4 o[2];
             uint8_t *ob = reinterpret_cast<uint8_t *>(o);
 #pragma unroll
@@ -87,6 +90,50 @@ void launch_mx_quantize(const float *src, int64_t rows, int64_t K, int fmt, uint
     const long long cap = (long long)num_sms * 16;
     const int grid = (int)(want < cap ? want : cap);
     mx_quantize_kernel<<<grid > 0 ? grid : 1, 256, 0, s>>>(src, nblocks, fmt, codes, scales);
+}
+
+// ---------------------------------------------------------------- activation encoders (test entry)
+// Encode float32 rows [rows, K] into the activation operand format with the encoders the
+// forward runs: method 0 = store_act_block32 (one thread per 32-element block: the gather, which
+// encodes bf16 values, and the FC1 epilogue of units with the tokens on M), method 1 =
+// store_act_warp32 (one warp per block: the FC1 epilogue of units with the tokens on N).
+__global__ void __launch_bounds__(256) encode_act_kernel(const float *__restrict__ src, int rows, int K, int act_mxfp8,
+                                                         int method, uint8_t *__restrict__ q, uint8_t *__restrict__ sf)
+{
+    const long long nblocks = (long long)rows * (K / 32);
+    const long long gid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    if (method == 0) {
+        for (long long b = gid; b < nblocks; b += stride) {
+            const int row = (int)(b / (K / 32)), col = (int)(b % (K / 32)) * 32;
+            float v[32];
+            const float4 *s4 = reinterpret_cast<const float4 *>(src + (size_t)row * K + col);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 f = __ldg(s4 + i);
+                v[4 * i] = f.x;
+                v[4 * i + 1] = f.y;
+                v[4 * i + 2] = f.z;
+                v[4 * i + 3] = f.w;
+            }
+            store_act_block32(q, sf, rows, K, row, col, v, act_mxfp8);
+        }
+    } else {
+        const int lane = threadIdx.x & 31;
+        for (long long wb = gid >> 5; wb < nblocks; wb += stride >> 5) { // warp-uniform
+            const int row = (int)(wb / (K / 32)), col = (int)(wb % (K / 32)) * 32 + lane;
+            store_act_warp32(q, sf, rows, K, row, col, __ldg(src + (size_t)row * K + col), act_mxfp8, lane);
+        }
+    }
+}
+
+void launch_encode_act(const float *src, int rows, int K, int act_mxfp8, int method, uint8_t *q, uint8_t *sf,
+                       int num_sms, cudaStream_t s)
+{
+    const long long threads = (long long)rows * (K / 32) * (method == 0 ? 1 : 32);
+    const long long want = (threads + 255) / 256;
+    const int grid = (int)(want < (long long)num_sms * 16 ? want : (long long)num_sms * 16);
+    encode_act_kernel<<<grid > 0 ? grid : 1, 256, 0, s>>>(src, rows, K, act_mxfp8, method, q, sf);
 }
 
 // ---------------------------------------------------------------- scale tiling

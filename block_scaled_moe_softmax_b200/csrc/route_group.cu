@@ -586,7 +586,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
 }
 
 // ---------------------------------------------------------------- launchers
-void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s, bool pdl)
+int launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s, bool pdl)
 {
     // the top-k scan visits 32 * kPerLane candidates per token: size it to the expert count
     // (the given routing visits no candidates: the smallest instance serves it).  The first
@@ -599,7 +599,7 @@ void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s, bool pdl)
             route_group_small_kernel<16><<<1, 1024, 0, s>>>(a);
         else
             route_group_small_kernel<32><<<1, 1024, 0, s>>>(a);
-        return;
+        return 1;
     }
     const int nchunks = (a.T + kRouteChunk - 1) / kRouteChunk;
     if (narrow)
@@ -615,6 +615,7 @@ void launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s, bool pdl)
                   a.pad_offsets, a.rowblocks, a.num_rowblocks, a.sorted_pair, a.unit_counters);
     launch_kernel(scatter_kernel, dim3(nchunks), dim3(32), 0, s, pdl, a.T, a.E, a.k, (const int32_t *)a.topk_ids,
                   (const int32_t *)a.chunk_hist, a.sorted_pair, a.pos_of_pair);
+    return 3;
 }
 
 void launch_gather(const __nv_bfloat16 *x, int P, int H, int k, const int32_t *pos_of_pair, uint8_t *aq,

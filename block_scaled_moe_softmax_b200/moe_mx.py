@@ -35,6 +35,11 @@ MOE_MX_SCALES_ROW_MAJOR = 0
 MOE_MX_SCALES_TILED = 1
 MOE_MX_W1 = 0
 MOE_MX_W2 = 1
+MOE_MX_INTER_AQ = 0
+MOE_MX_INTER_ASF = 1
+MOE_MX_INTER_HQ = 2
+MOE_MX_INTER_HSF = 3
+MOE_MX_INTER_Y = 4
 
 # Every symbol include/moe_mx.h declares: name -> (restype, argtypes)
 _P, _I, _I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
@@ -56,6 +61,9 @@ SIGNATURES = {
     "moe_mx_route_group_noalloc": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
     "moe_mx_prepare_scales": (_I, [_P, _I, _P, _P, _P]),
     "moe_mx_set_scale_layout": (_I, [_P, _I]),
+    "moe_mx_get_intermediate": (_I, [_P, _I, _P, _P]),
+    "moe_mx_launch_count": (ctypes.c_longlong, [_P]),
+    "moe_mx_debug_encode_act": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
 }
 STAGES = ("route", "gather", "fc1", "fc2", "combine")
 
@@ -178,6 +186,23 @@ def moe_mx_route_group_noalloc(router_logits, num_tokens: int, num_experts: int,
         _ptr(pad_offsets), _ptr(sorted_pair), _ptr(pos_of_pair), _stream(stream)))
 
 
+def moe_mx_launch_count(handle: int) -> int:
+    """Kernels launched by the handle's forwards since it was created (host-side count)."""
+    return load_library().moe_mx_launch_count(handle)
+
+
+def moe_mx_get_intermediate(handle: int, which: int, dst, stream=None) -> None:
+    """Copy one intermediate buffer of the last forward (MOE_MX_INTER_*) into dst (see the header)."""
+    _check(load_library().moe_mx_get_intermediate(handle, which, _ptr(dst), _stream(stream)))
+
+
+def moe_mx_debug_encode_act(src, rows: int, K: int, act_dtype: int, method: int, codes, scale_atoms,
+                            stream=None) -> None:
+    """The forward's activation encoders on float32 rows (see the header)."""
+    _check(load_library().moe_mx_debug_encode_act(_ptr(src), rows, K, act_dtype, method, _ptr(codes),
+                                                  _ptr(scale_atoms), _stream(stream)))
+
+
 def moe_mx_prepare_scales(handle: int, which: int, src, dst, stream=None) -> None:
     """Rearrange one row-major E8M0 weight-scale tensor into the tiled layout (see the header)."""
     _check(load_library().moe_mx_prepare_scales(handle, which, _ptr(src), _ptr(dst), _stream(stream)))
@@ -256,6 +281,25 @@ class MoeMxLayer:
         sp = torch.empty(rows, dtype=torch.int32, device=dev)
         moe_mx_get_routing(self.handle, ids, w, counts, pad, sp, stream)
         return ids, w, counts, pad, sp
+
+    def intermediates(self, T: int, top_k: int, stream=None) -> dict:
+        """The intermediate buffers of the most recent forward of T tokens (device tensors):
+        aq [2, rows, H] / hq [2, rows, I] uint8 E4M3 codes, asf / hsf uint8 scale atoms,
+        y float32 [rows, H]; rows = moe_mx_max_grouped_rows(T, top_k)."""
+        dev = torch.device("cuda", self.device)
+        rows = moe_mx_max_grouped_rows(self.handle, T, top_k)
+        bufs = {
+            "aq": torch.empty(2, rows, self.H, dtype=torch.uint8, device=dev),
+            "asf": torch.empty(rows // 128 * (self.H // 128) * 1024, dtype=torch.uint8, device=dev),
+            "hq": torch.empty(2, rows, self.I, dtype=torch.uint8, device=dev),
+            "hsf": torch.empty(rows // 128 * (self.I // 128) * 1024, dtype=torch.uint8, device=dev),
+            "y": torch.empty(rows, self.H, dtype=torch.float32, device=dev),
+        }
+        which = {"aq": MOE_MX_INTER_AQ, "asf": MOE_MX_INTER_ASF, "hq": MOE_MX_INTER_HQ, "hsf": MOE_MX_INTER_HSF,
+                 "y": MOE_MX_INTER_Y}
+        for name, t in bufs.items():
+            moe_mx_get_intermediate(self.handle, which[name], t, stream)
+        return bufs
 
     def sync_status(self, stream=None) -> int:
         return moe_mx_sync_status(self.handle, stream)

@@ -150,9 +150,13 @@ MOE_MX_API int moe_mx_create_ex(moe_mx_handle **out, int hidden, int inter, int 
  *   act_dtype      MOE_MX_ACT_BF16 or MOE_MX_ACT_MXFP8.
  *   out            bf16 [T, H], written (not accumulated); must not alias x.
  * Only experts that receive at least one token have their weights read.
- * Dequantised weight values (code value * 2^(scale-127)) must be normal
- * bf16 numbers, i.e. weight scale bytes in [2, 252]; other scale bytes give
- * undefined (but finite-time, non-faulting) results.
+ * Weight scale bytes are E8M0 (2^(byte-127)); the tensor core applies them
+ * together with the activations' block scales and accumulates in float32.
+ * Every byte 0..254 is valid: products below float32's normal range may be
+ * flushed to zero and sums beyond its range become infinite; the NaN byte 0xFF
+ * makes every output it reaches NaN.  An activation block holding a NaN or an
+ * infinity is encoded with the NaN scale byte (see moe_mx_debug_encode_act),
+ * so the outputs of that token come out NaN.
  * The call does not synchronise the host, allocates nothing and may be
  * captured in a CUDA graph.  One forward may be in flight per handle.
  * Device-side failures (a bounded wait that gave up) surface through
@@ -224,8 +228,10 @@ MOE_MX_API int moe_mx_sync_status(moe_mx_handle *h, void *stream);
  * "Activation precision (w4a16 vs w4a8)".)
  *   fmt MOE_MX_FMT_MXFP4: codes [rows, K/2]; MOE_MX_FMT_MXFP8: codes [rows, K].
  *   scales [rows, K/32].
- * A utility for preparing weights; the forward quantises activations with
- * the same device code.  Errors: INVALID_ARG, CUDA.
+ * A block holding a NaN or an infinity gets scale byte 0xFF and zero codes.
+ * A utility for preparing weights; its MXFP8 path runs the same device encoder
+ * as the forward's w4a8 activation quantisation (moe_mx_debug_encode_act, method
+ * 0).  Errors: INVALID_ARG, CUDA.
  */
 MOE_MX_API int moe_mx_quantize(const float *src, int64_t rows, int64_t K, int fmt, uint8_t *codes,
                     uint8_t *scales, void *stream);
@@ -261,6 +267,68 @@ MOE_MX_API int64_t moe_mx_max_grouped_rows(const moe_mx_handle *h, int num_token
  */
 MOE_MX_API int moe_mx_get_routing(const moe_mx_handle *h, int32_t *topk_ids, float *topk_w, int32_t *counts,
                        int32_t *pad_offsets, int32_t *sorted_pair, void *stream);
+
+/* Intermediate buffers of a forward (moe_mx_get_intermediate). */
+#define MOE_MX_INTER_AQ 0  /* FC1's activation operand: E4M3 codes [2][rows][H] */
+#define MOE_MX_INTER_ASF 1 /* its E8M0 scale atoms [rows/128][H/128][2][512] */
+#define MOE_MX_INTER_HQ 2  /* FC2's activation operand (h): E4M3 codes [2][rows][I] */
+#define MOE_MX_INTER_HSF 3 /* its E8M0 scale atoms [rows/128][I/128][2][512] */
+#define MOE_MX_INTER_Y 4   /* FC2's output: float32 [rows][H] */
+
+/*
+ * Copy one intermediate buffer of the most recent forward into dst (a device
+ * buffer on the handle's device), for tests that check each stage on its own
+ * (test-only; the pages print no such interface, the hot-path scope of this
+ * library lists it beside moe_mx_get_routing).  rows =
+ * moe_mx_max_grouped_rows(h, T, top_k) of that forward; grouped row r holds
+ * the pair sorted_pair[r] (moe_mx_get_routing); rows past pad_offsets[E] and
+ * padding rows (sorted_pair -1) hold unspecified bytes.
+ *   MOE_MX_INTER_AQ / _HQ: the operand as E4M3 codes in two term planes of
+ *     rows x K bytes each (K = H for AQ, I for HQ), plane t at t * rows * K.
+ *     w4a16 (and h on every path but w4a8): value = term 0 + term 1, an exact
+ *     two-term expansion of the bf16 value (see moe_mx_debug_encode_act).
+ *     w4a8: term 0 alone is the OCP MXFP8 quantisation; plane 1 is unused.
+ *   MOE_MX_INTER_ASF / _HSF: the E8M0 scale bytes of those codes, (rows/128) x
+ *     (K/128) atoms of 1024 bytes: for grouped row r, 32-element block b of
+ *     the row and term t, the byte at ((r/128) * (K/128) + b/4) * 1024 + t * 512
+ *     + (r % 32) * 16 + ((r % 128) / 32) * 4 + b % 4.
+ *   MOE_MX_INTER_Y: FC2's float32 output rows before the weighted combine.
+ * Asynchronous on `stream`; call it after the forward on the same stream.
+ * Errors: INVALID_ARG (bad handle, `which` or dst), CUDA.
+ */
+MOE_MX_API int moe_mx_get_intermediate(const moe_mx_handle *h, int which, void *dst, void *stream);
+
+/*
+ * Run the forward's activation encoders on caller data (test-only; no
+ * counterpart on the pages): float32 rows src [rows, K] (K a multiple of 128)
+ * become E4M3 codes [2][rows][K] and E8M0 scale atoms [ceil(rows/128)][K/128][2][512]
+ * in the layout of MOE_MX_INTER_AQ / _ASF.  Per 32-element block of a row:
+ *   act_dtype MOE_MX_ACT_MXFP8: the OCP MXFP8 quantisation (scale exponent
+ *     floor(log2 amax) - 8, clamped to [-127, 127]; round-to-nearest-even,
+ *     saturating at 448), plane 0 only -- the w4a8 activations and h;
+ *   act_dtype MOE_MX_ACT_BF16: each value rounded to bf16, then split exactly
+ *     into two MXFP8 terms: term 0 with exponent floor(log2 amax) - 7 keeps the
+ *     top 4 significant bits of every element, term 1 the remainder with its own
+ *     block exponent (same rule); elements of at least 2^-13 of the block's
+ *     maximum are exact, smaller ones err by less than 2^-20 of it -- the w4a16
+ *     activations and h;
+ *   a block holding a NaN or an infinity: scale byte 0xFF and zero codes in
+ *     every term.
+ *   method 0: one thread per block, the encoder of the gather (on bf16 values)
+ *     and of FC1's epilogue for units with the tokens on the MMA's M side;
+ *   method 1: one warp per block, FC1's epilogue for units with the tokens on N.
+ * All pointers device memory of the current device, 16-byte aligned.
+ * Errors: INVALID_ARG, CUDA.
+ */
+MOE_MX_API int moe_mx_debug_encode_act(const float *src, int rows, int K, int act_dtype, int method, uint8_t *codes,
+                                       uint8_t *scale_atoms, void *stream);
+
+/*
+ * Number of kernels the handle's forwards have launched since moe_mx_create
+ * (host-side count; -1 for a NULL handle).  The difference across a region is
+ * that region's launch count.
+ */
+MOE_MX_API long long moe_mx_launch_count(const moe_mx_handle *h);
 
 /* Stages of one forward, in launch order (indices into moe_mx_get_stage_times). */
 #define MOE_MX_STAGE_ROUTE 0   /* routing, histogram, scan, stable scatter */
@@ -326,8 +394,7 @@ MOE_MX_API int moe_mx_debug_watchdog(moe_mx_handle *h, int timeout_us, void *str
  * Routing and grouping without a handle and without allocating: the router
  * (softmax, top-k with the lowest expert index winning ties, renormalised
  * weights) and the stable grouping by expert into 128-row padded segments --
- * the same kernels and results as the first stage of moe_mx_forward
- * (TokenSpeed-kernel README, "Public API": moe_route and moe_dispatch).  The
+ * the same kernels and results as the first stage of moe_mx_forward.  The
  * pages have no counterpart of this entry point; it exists for callers that
  * cannot allocate device memory at the point of the call and hold no handle
  * (for example an op whose device memory must all come from its framework's
@@ -344,7 +411,9 @@ MOE_MX_API int moe_mx_debug_watchdog(moe_mx_handle *h, int timeout_us, void *str
  *
  * The first call on a device looks up that device's scratch address
  * (cudaGetSymbolAddress), which may load the library's device code there: make
- * that first call outside any stream capture (e.g. at setup).  All calls on one
+ * that first call outside any stream capture (e.g. at setup).  The address is
+ * kept for the life of the process: after a cudaDeviceReset of that device it
+ * is stale, so do not call this entry point on a device that has been reset.  All calls on one
  * device share the scratch: calls whose executions overlap (unordered streams,
  * several host threads) race on it and corrupt each other's results; order
  * them (one stream, or events).

@@ -120,3 +120,44 @@ def check_routing(layer, T, k, E, logits_np):
         assert np.array_equal(seg[:counts_o[e]], sp_o[offs_o[e]:offs_o[e + 1]]), f"permutation differs at expert {e}"
         assert np.all(seg[counts_o[e]:] == -1), f"padding rows of expert {e} are not marked -1"
     return ids_o
+
+
+# ---------------------------------------------------------------- the activation operand format
+def atoms_to_rowmajor(atoms, rows, K):
+    """E8M0 scale bytes from the scale-atom layout the library documents (moe_mx.h,
+    MOE_MX_INTER_ASF): for row r, 32-element block b and term t, the byte at
+    ((r/128)*(K/128) + b/4)*1024 + t*512 + (r%32)*16 + ((r%128)/32)*4 + b%4.
+    Returns uint8 [2, rows, K/32]."""
+    atoms = np.asarray(atoms, np.uint8).reshape(-1)
+    r = np.arange(rows)[:, None]
+    b = np.arange(K // 32)[None, :]
+    out = np.empty((2, rows, K // 32), np.uint8)
+    for t in range(2):
+        idx = ((r // 128) * (K // 128) + b // 4) * 1024 + t * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + b % 4
+        out[t] = atoms[idx]
+    return out
+
+
+def check_two_term_split(codes2, scales2, ref, tag=""):
+    """The w4a16 operand: two E4M3 term planes (decoded with ml_dtypes) must add up to the bf16
+    values `ref` exactly wherever |ref| >= 2^-13 * the block's max |ref|, and within 2^-20 of the
+    block max elsewhere (the mathematics of the split: term 0 keeps each element's top 4
+    significant bits at block exponent floor(log2 amax) - 7, term 1 the remainder).
+    codes2 uint8 [2, n, K], scales2 uint8 [2, n, K/32], ref float64 [n, K] (finite)."""
+    ref = np.asarray(ref, np.float64)
+    got = dequant_mxfp8_lib(codes2[0], scales2[0]) + dequant_mxfp8_lib(codes2[1], scales2[1])
+    n, K = ref.shape
+    amax = np.repeat(np.abs(ref).reshape(n, K // 32, 32).max(axis=2), 32, axis=1)
+    big = np.abs(ref) >= amax * 2.0 ** -13
+    bad = big & (got != ref)
+    assert not bad.any(), f"{tag}: {int(bad.sum())} elements >= 2^-13 amax not exact, e.g. " \
+                          f"{ref[bad][:4]} -> {got[bad][:4]}"
+    err = np.abs(got - ref)
+    over = ~big & (err >= amax * 2.0 ** -20)
+    assert not over.any(), f"{tag}: {int(over.sum())} small elements err by >= 2^-20 amax"
+    return got
+
+
+def bf16_round(v):
+    """float32 -> nearest bf16 (ties to even) through ml_dtypes, as float64."""
+    return np.asarray(v, np.float32).astype(ml_dtypes.bfloat16).astype(np.float64)

@@ -43,9 +43,12 @@ def test_only_declared_symbols_are_exported(lib):
     assert exported == _declared_symbols()
 
 
-def test_library_is_built_for_sm100a(lib):
-    out = os.popen(f"/usr/local/cuda/bin/cuobjdump --list-elf {moe_mx.LIB_PATH} 2>&1").read()
-    assert "sm_100a" in out
+def test_library_is_built_for_sm100a_only(lib):
+    # every translation unit and the link are compiled for sm_100a alone (no PTX for other
+    # targets), so the GPU tests' launches only succeed on an sm_100 device
+    flags = build_mod.FLAGS
+    gencodes = [flags[i + 1] for i, f in enumerate(flags) if f == "-gencode"]
+    assert gencodes == ["arch=compute_100a,code=sm_100a"]
 
 
 def test_host_validation_without_gpu(lib):

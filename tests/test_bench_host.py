@@ -29,9 +29,11 @@ def test_algorithmic_work_closed_forms():
     assert per_expert == 15_597_568  # 15.60 MB per hit expert at H = 7168, I = 2048
 
 
-def test_kernels_per_forward():
-    assert bench.kernels_per_forward(16) == 5 and bench.kernels_per_forward(64) == 5
-    assert bench.kernels_per_forward(65) == 7
+def test_cpu_baseline_uses_every_core():
+    wl = workloads.WORKLOADS["tiny"]
+    cb = bench.cpu_baseline(wl, 4, min_wall=0.05)
+    assert cb["kind"] == "oracle" and cb["cores"] == 4 and cb["threads"] == 4 and cb["value"] > 0
+    assert "4 at a time" in cb["sample"]
 
 
 def test_reference_pairs():

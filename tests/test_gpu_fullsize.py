@@ -5,7 +5,8 @@ ids, per-expert counts, padded offsets and the permutation are compared with
 the oracle for EVERY token (bit-exact); the output is compared with the oracle's
 per-token evaluation on a sample of tokens (the oracle is too slow for all of
 them): the first and last tokens, tokens routed to the most- and least-loaded
-experts, and seeded random ones.  Tolerance as everywhere: relative Frobenius
+experts, seeded random ones, and tokens covering the last, partial work block
+of every expert segment whose rows are not a whole number of work blocks.  Tolerance as everywhere: relative Frobenius
 error <= 5e-3 and max |gpu - ref| <= 2e-2 * RMS(ref) over the sampled rows.
 
 Weights are drawn per expert on the GPU (float32, N(0, 0.02)), copied to the
@@ -59,7 +60,17 @@ def _weights(wl):
     return _WEIGHT_CACHE[key]
 
 
+def _work_block_rows(T):
+    """Rows per GEMM work block the library picks for T tokens (16 up to 16 tokens, 32 up to 512,
+    then whole 128-row segments)."""
+    return 16 if T <= 16 else 32 if T <= 512 else 128
+
+
 def _sample_tokens(ids, wl, n_random=8):
+    """First and last tokens, tokens of the most and least loaded experts, seeded random ones, and
+    a cover of every ragged segment tail: for each expert whose row count is not a multiple of the
+    work-block rows, at least one token whose row lies in that segment's last, partial work block
+    (chosen greedily, the token covering most uncovered tails first)."""
     T = wl.T
     counts = np.bincount(ids.reshape(-1), minlength=wl.E)
     hit = np.nonzero(counts)[0]
@@ -70,6 +81,22 @@ def _sample_tokens(ids, wl, n_random=8):
     toks.add(int(np.nonzero((ids == small).any(axis=1))[0][-1]))
     rng = np.random.default_rng(1234)
     toks.update(int(t) for t in rng.choice(T, size=min(n_random, T), replace=False))
+    split = _work_block_rows(T)
+    tails = {}  # ragged expert -> tokens whose rows sit in its last, partial work block
+    for e in hit:
+        if counts[e] % split == 0:
+            continue
+        members = np.nonzero((ids == e).any(axis=1))[0]   # ascending token = ascending grouped row
+        tails[int(e)] = set(int(t) for t in members[(counts[e] // split) * split:])
+    uncovered = {e for e, ts in tails.items() if not (ts & toks)}
+    while uncovered:
+        score = {}
+        for e in uncovered:
+            for t in tails[e]:
+                score[t] = score.get(t, 0) + 1
+        best = max(sorted(score), key=lambda t: score[t])
+        toks.add(best)
+        uncovered = {e for e in uncovered if best not in tails[e]}
     return sorted(toks)
 
 

@@ -1,8 +1,11 @@
 """GPU MX quantiser (moe_mx_quantize) against the oracle's quantiser: bit-exact.
 
-The same device code quantises the w4a8 activations inside the forward, so
-this also pins that step.  Inputs mix magnitudes over many binades, all-zero
-blocks, exact rounding ties, saturation, negative zeros and subnormals.
+Its MXFP8 path runs mx_encode32, the encoder of the forward's gather; the
+forward's own encoders (the gather and FC1's epilogue, on caller data and
+inside a forward) are pinned in tests/test_gpu_encoders.py and
+tests/test_gpu_intermediates.py.  Inputs mix magnitudes over many binades,
+all-zero blocks, exact rounding ties, saturation, negative zeros, subnormals
+and non-finite blocks (scale byte 0xFF, zero codes).
 """
 import numpy as np
 import pytest
@@ -34,6 +37,9 @@ def _inputs():
     v[5, :3] = [7.9, 7.0, 6.5]                       # saturation above 6
     v[6, :2] = [1e-40, -3e-39]                       # float32 subnormals
     v[7] = np.float32(1e-45)
+    v[8, 3] = np.nan                                 # non-finite blocks
+    v[9, 0] = np.inf
+    v[10, 31] = -np.inf
     return v.reshape(64, 2048)
 
 
