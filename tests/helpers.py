@@ -103,6 +103,27 @@ def check_output(got_bf16, ref_f64, tag=""):
     return rf, mx
 
 
+def check_output_rows(got_bf16, ref_f64, tag=""):
+    """The layer's tolerance applied to each token row against that row's own RMS.  For inputs
+    whose tokens differ in scale by orders of magnitude (outlier channels), the final bf16
+    rounding alone (2^-9 of each element) of the largest rows exceeds 2e-2 of the whole output's
+    RMS -- the oracle's own correctly rounded output does too -- so such cases are held to the
+    bound row by row, where the rounding is within it."""
+    got = got_bf16.float().cpu().double().numpy()
+    ref = np.asarray(ref_f64, np.float64)
+    assert np.all(np.isfinite(got)), f"{tag}: non-finite outputs"
+    worst_rf, worst_mx = 0.0, 0.0
+    for t in range(ref.shape[0]):
+        if not np.any(ref[t]):
+            assert not np.any(got[t]), f"{tag}: row {t} should be zero"
+            continue
+        rf, mx = rel_frobenius(got[t], ref[t]), max_abs_over_rms(got[t], ref[t])
+        assert rf <= TOL_REL_FRO, f"{tag}: row {t} relative Frobenius error {rf:.3e} > {TOL_REL_FRO}"
+        assert mx <= TOL_MAX_OVER_RMS, f"{tag}: row {t} max|gpu-ref|/RMS(row) {mx:.3e} > {TOL_MAX_OVER_RMS}"
+        worst_rf, worst_mx = max(worst_rf, rf), max(worst_mx, mx)
+    return worst_rf, worst_mx
+
+
 def check_routing(layer, T, k, E, logits_np):
     """Bit-exact ids/counts/offsets/permutation against the oracle; weights within 2e-6 relative."""
     ids_g, w_g, counts_g, pad_g, sp_g = [a.cpu().numpy() for a in layer.routing(T, k)]

@@ -51,7 +51,7 @@ def _inputs(seed=5):
     v[44, 0, 5] = np.nan                                                   # non-finite blocks
     v[44, 2, 0] = np.inf
     v[44, 3, 31] = -np.inf
-    v[45, :, :] = np.float32(3.0e38)                                      # rounds to bf16 infinity
+    v[45, :, :] = np.float32(3.4e38)                                      # rounds to bf16 infinity
     v[46, 0, :] = np.float32(2.0 ** 127) * np.linspace(-1, 1, 32, dtype=np.float32)
     return v.reshape(n, K)
 

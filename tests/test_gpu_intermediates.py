@@ -16,9 +16,13 @@
          bf16 rounding (w4a16) or the oracle's MXFP8 quantisation (w4a8) of the
          exact g * u, bit for bit -- the MMAs, the K order, the SwiGLU epilogue
          and its encoder, with the GPU's own float32 h known exactly;
-    (ii) x constant per token, every scale 2^0: h takes few significant bits, so
-         FC2's float32 rows Y must equal the decoded float64 matmul of W2 with
-         the GPU's own h operand exactly.
+    (ii) x constant per token, every scale 2^0: h takes few significant bits.
+    In both, FC2's float32 rows Y must equal the decoded float64 matmul of W2
+    with the GPU's own h operand exactly, and the output must meet the tolerance
+    against the exact weighted sum of those rows.  (The oracle's SwiGLU runs in
+    double, where 1 + exp(-g) is not 1: its h sits a hair below g * u and lands
+    on the other side of a rounding tie now and then, so the output is compared
+    with the oracle only where h needs no rounding: case (ii), w4a16.)
     Every kernel variant (activation tiles of 16, 32, 64 or 128 rows, the wide
     two-tile variant, both orientations) and both activation modes.
 """
@@ -49,14 +53,14 @@ def _set_variant(monkeypatch, variant):
 
 
 def _grouped_rows(layer, T, k, E):
-    """(grouped row, token, slot expert) of every real pair of the last forward."""
+    """(grouped row, token, expert, slot) of every real pair of the last forward."""
     ids, _, counts, pad, sp = [a.cpu().numpy() for a in layer.routing(T, k)]
     rows = []
     for e in range(E):
         for r in range(pad[e], pad[e] + counts[e]):
             p = int(sp[r])
-            rows.append((r, p // k, int(ids[p // k, p % k])))
-    return np.array(rows, dtype=np.int64).reshape(-1, 3)
+            rows.append((r, p // k, int(ids[p // k, p % k]), p % k))
+    return np.array(rows, dtype=np.int64).reshape(-1, 4)
 
 
 def _forward(wl, x_bf16, logits, w, act):
@@ -124,10 +128,11 @@ def test_w4a16_activation_operand_is_exact_split(name, variant, monkeypatch):
     codes, scales = _operand(inter, "aq", rows_total, wl.H)
     r, t = grows[:, 0], grows[:, 1]
     helpers.check_two_term_split(codes[:, r], scales[:, r], x.float().numpy().astype(np.float64)[t], name)
-    # and the layer's output still meets the tolerance against the oracle on this input
+    # and the layer's output still meets the tolerance against the oracle on this input (row by
+    # row: the outlier tokens' outputs are up to 10^6 times the others')
     inp2 = dict(inp, x=x, xb=workloads.bf16_bits(x))
     ref, _, _ = helpers.oracle_forward(inp2, wl.top_k, 0)
-    helpers.check_output(out, ref, f"{name} crafted x")
+    helpers.check_output_rows(out, ref, f"{name} crafted x")
     layer.close()
 
 
@@ -187,7 +192,7 @@ def test_exact_special_case(case, act, variant, monkeypatch):
     x = _exact_x(case, rng)
     logits = workloads.draw_logits(wl)
     layer, out, inter, grows = _forward(wl, x, logits, w, act)
-    r, t, e = grows[:, 0], grows[:, 1], grows[:, 2]
+    r, t, e, j = grows[:, 0], grows[:, 1], grows[:, 2], grows[:, 3]
     rows_total = inter["aq"].shape[1]
     xf = x.float().numpy().astype(np.float64)
     # FC1's operand: x is exactly representable (w4a16: term 0 alone; w4a8: one code per value)
@@ -213,15 +218,23 @@ def test_exact_special_case(case, act, variant, monkeypatch):
         assert np.array_equal(hscales[0][r], s_o), "h scale bytes != the oracle's MXFP8 quantisation of g * u"
         assert np.array_equal(hcodes[0][r], q_o), "h codes != the oracle's MXFP8 quantisation of g * u"
         h_dec = helpers.dequant_mxfp8_lib(q_o, s_o)
-    if case == "fc1_fc2":
-        w2d = helpers.dequant_mxfp4_lib(w["w2"], w["w2s"])             # [E, H, I]
-        y_ref = _per_expert_matmul(h_dec, w2d, e)
-        y = inter["y"][r].astype(np.float64)
-        assert np.array_equal(y, y_ref), f"FC2 rows differ from the exact matmul: max |d| = {np.abs(y - y_ref).max()}"
-    # the layer's output within the tolerance of the oracle, as always
-    inp = dict(xb=workloads.bf16_bits(x), logits=logits, **w)
-    ref, _, _ = helpers.oracle_forward(inp, wl.top_k, act)
-    helpers.check_output(out, ref, f"exact {case}")
+    # FC2's float32 rows equal the float64 matmul of W2 with the GPU's own h operand (the sums
+    # are exact in float32 by construction)
+    w2d = helpers.dequant_mxfp4_lib(w["w2"], w["w2s"])                 # [E, H, I]
+    y_ref = _per_expert_matmul(h_dec, w2d, e)
+    y = inter["y"][r].astype(np.float64)
+    assert np.array_equal(y, y_ref), f"FC2 rows differ from the exact matmul: max |d| = {np.abs(y - y_ref).max()}"
+    # the combine of those rows, within the tolerance of the exact weighted sum
+    w_g = layer.routing(wl.T, wl.top_k)[1].cpu().numpy().astype(np.float64)
+    exact_out = np.zeros((wl.T, wl.H))
+    np.add.at(exact_out, t, w_g[t, j][:, None] * y_ref)
+    helpers.check_output(out, exact_out, f"exact {case} combine")
+    if act == 0 and case == "fc1_fc2":
+        # here h needs no rounding, so the oracle (whose SwiGLU in double makes h = g * u * (1 - ~e^-g),
+        # on the other side of a rounding tie now and then) meets the same values: compare with it too
+        inp = dict(xb=workloads.bf16_bits(x), logits=logits, **w)
+        ref, _, _ = helpers.oracle_forward(inp, wl.top_k, act)
+        helpers.check_output(out, ref, f"exact {case}")
     layer.close()
 
 

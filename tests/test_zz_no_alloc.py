@@ -33,7 +33,8 @@ def _need_gpu():
 def _logits(T, E, seed):
     g = torch.Generator().manual_seed(seed)
     lg = torch.randn(T, E, generator=g, dtype=torch.float32)
-    lg[::7, 5] = lg[::7, 9]          # exact ties: the lower index must win
+    lo, hi = (5, 9) if E > 9 else (1, 6)
+    lg[::7, lo] = lg[::7, hi]        # exact ties: the lower index must win
     if T > 3:
         lg[3, :] = 0.0               # a row of all-equal logits
     return lg
