@@ -2,30 +2,35 @@
 """Benchmark of the fused MXFP4 routed-MoE layer on B200; prints ONE JSON line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--parallel replicas|ep] [--no-cpu-baseline]
                     (K defaults to 1000, or 200 for the reference arm)
-                    [--workload decode|tiny|batched_decode|prefill|prefill_w4a8]
 
-Other workloads: the batched-decode and prefill configurations, and shards of the
-896-expert, top-16 layer with the routing given as precomputed top-k (situ_tp8,
-situ_ep8; moe_mx_forward_routed).
+Default run: the decode-shaped layer is the headline (w4a16, T=16 tokens,
+H=7168, I=2048, E=384 experts, top-8), and all five configurations of the layer
+are measured in the same run under "per_config": tiny (T=16, H=256, I=128,
+E=8, top-2), decode, batched decode (T=256, logits + a N(0, 0.5) expert bias),
+prefill (T=8192, Zipf-like expert bias) and prefill w4a8 (T=16384, H=4096,
+I=1536, E=128).  --workload NAME measures one workload alone (also the
+small-batch decode shapes decode_t1 / decode_t4, the shared-expert decode, and
+shards of the 896-expert, top-16 layer with the routing given as precomputed
+top-k: situ_tp8, situ_ep8).  Inputs are synthetic and seeded (bf16 x ~ N(0,1),
+float32 logits ~ N(0,1) plus the workload's bias, weights N(0, 0.02) quantised
+to MXFP4 on the GPU by the library's quantiser).  One step = one whole forward
+(routing, grouping, FC1 + SwiGLU, FC2, combine) through the C ABI, inputs
+resident in HBM.  The decode weights (8.98 GB) are far larger than L2, and L2 is
+additionally flushed (512 MiB write) before every timed step; each step is
+timed with CUDA events on the launching stream.
 
-Workload (default): the decode-shaped layer, w4a16, T=16 tokens, H=7168,
-I=2048, E=384 experts, top-8; synthetic seeded inputs (bf16 x ~ N(0,1),
-float32 logits ~ N(0,1), weights N(0,0.02) quantised to MXFP4 on the GPU by the
-library's quantiser).  One step = one whole forward (routing, grouping, FC1 +
-SwiGLU, FC2, combine) through the C ABI, inputs resident in HBM.  The weights
-(8.98 GB) are far larger than L2 and L2 is additionally flushed (512 MiB write)
-before every timed step; each step is timed with CUDA events on the launching
-stream.
-
---impl ours (default): the CUDA path.  Reported: tokens/s (value), the same
-metric end to end with host buffers (e2e: pinned H2D of x and logits, forward,
-D2H of the output, all inside the timed step), the roofline of the dominant
-kernel (the FC1 grouped GEMM), and the CPU oracle timed on a bounded token
-sample on the host cores (cpu_baseline).  FC1's bound is whichever of its two
-costs is larger at the measured peaks: bytes (FP4 codes + E8M0 scales of the
-hit experts' W1 + activation rows read + h rows written) against the HBM copy
-bandwidth -- the decode shapes -- or FLOPs (2 * pairs * 2I * H) against the
+--impl ours (default): the CUDA path.  Reported per workload: tokens/s, the same
+metric end to end with host buffers (e2e: pinned H2D of x and the routing
+input, forward, D2H of the output, all inside the timed step), the roofline of
+the dominant kernel (the FC1 grouped GEMM) and of the whole step, the per-stage
+times, the clocks sampled during the timed region and the library's own count
+of kernel launches in it.  The headline also carries the CPU oracle timed on a
+bounded sample on all host cores (cpu_baseline).  FC1's bound is whichever of
+its two costs is larger at the measured peaks: bytes (FP4 codes + E8M0 scales of
+the hit experts' W1 + activation rows read + h rows written) against the HBM
+copy bandwidth -- the decode shapes -- or FLOPs (2 * pairs * 2I * H) against the
 sustained bf16 GEMM rate (x2 for w4a8's MXFP8 operands) -- the prefill shapes;
 achieved = that work / FC1's mean CUDA-event duration.  The timed steps carry no
 events between kernels (each kernel after the router may launch while the one
@@ -34,11 +39,16 @@ steps (at most 300) with events between the kernels, which the library then
 launches one after another.
 
 --impl reference: the CPU oracle (the only reference this path has), timed on
-the host cores on a bounded token sample of the same workload per step.
+the host cores on a bounded sample of the same workload per step.
 
-Multi-GPU (torchrun, one process per GPU): every rank runs an independent
-replica of the workload (the layer has no exchange step at this scope), timed
-between barriers; value = tokens of all ranks / max-over-ranks time.
+Multi-GPU (torchrun, one process per GPU).  --parallel replicas (default):
+every rank runs an independent replica of the workload, timed between
+barriers; value = tokens of all ranks / max-over-ranks time ("scaling": weak).
+--parallel ep: expert parallelism -- each rank holds a contiguous shard of the
+experts, routes all tokens of the one batch and runs the pairs of its shard
+(moe_mx_forward_shard, float32 partial output), and the partials are summed
+over the ranks by an NCCL all-reduce inside the step; value = the batch's
+tokens / max-over-ranks time ("scaling": strong).
 """
 from __future__ import annotations
 
@@ -88,19 +98,20 @@ def workload_desc(wl):
 
 
 # ------------------------------------------------------------------ inputs
-def make_gpu_weights(wl, dev):
+def make_gpu_weights(wl, dev, experts=None):
     """Draw float32 weights per expert (and shared-expert chunk) on the GPU and quantise them with
-    the library's MX quantiser."""
-    E, H, I = wl.slots, wl.H, wl.I
+    the library's MX quantiser; `experts` (a range of global ids) keeps only those slots."""
+    experts = range(wl.slots) if experts is None else experts
+    E, H, I = len(experts), wl.H, wl.I
     w1 = torch.empty(E, 2 * I, H // 2, dtype=torch.uint8, device=dev)
     w1s = torch.empty(E, 2 * I, H // 32, dtype=torch.uint8, device=dev)
     w2 = torch.empty(E, H, I // 2, dtype=torch.uint8, device=dev)
     w2s = torch.empty(E, H, I // 32, dtype=torch.uint8, device=dev)
-    for e in range(E):
+    for i, e in enumerate(experts):
         f1 = workloads.draw_w1_expert(wl, e, device=str(dev))
-        moe_mx.moe_mx_quantize(f1, 2 * I, H, moe_mx.MOE_MX_FMT_MXFP4, w1[e], w1s[e])
+        moe_mx.moe_mx_quantize(f1, 2 * I, H, moe_mx.MOE_MX_FMT_MXFP4, w1[i], w1s[i])
         f2 = workloads.draw_w2_expert(wl, e, device=str(dev))
-        moe_mx.moe_mx_quantize(f2, H, I, moe_mx.MOE_MX_FMT_MXFP4, w2[e], w2s[e])
+        moe_mx.moe_mx_quantize(f2, H, I, moe_mx.MOE_MX_FMT_MXFP4, w2[i], w2s[i])
     torch.cuda.synchronize(dev)
     return w1, w1s, w2, w2s
 
@@ -361,16 +372,18 @@ class WeightCache:
     """One resident weight set at a time: the decode, batched-decode and prefill workloads share
     theirs (same H, I, E, seed), so the default run draws and quantises it once."""
 
-    def __init__(self, dev):
+    def __init__(self, dev, experts_of=None):
         self.dev, self.key, self.w = dev, None, None
+        self.experts_of = experts_of  # workload -> the range of experts this rank holds (None: all)
 
     def get(self, wl):
-        key = (wl.H, wl.I, wl.E, wl.shared, wl.seed)
+        experts = self.experts_of(wl) if self.experts_of else None
+        key = (wl.H, wl.I, wl.E, wl.shared, wl.seed, None if experts is None else (experts.start, experts.stop))
         if key != self.key:
             self.w = None
             torch.cuda.empty_cache()
             log(f"generating weights for {workload_desc(wl)}")
-            self.w = make_gpu_weights(wl, self.dev)
+            self.w = make_gpu_weights(wl, self.dev, experts)
             self.key = key
         return self.w
 
@@ -378,18 +391,28 @@ class WeightCache:
 def measure(args, wl, weights, world, rank, with_e2e=True):
     """Time one workload: K steps device-resident (the value), then the same steps with events
     between the kernels (each kernel's own duration), then K steps end to end from pinned host
-    buffers.  Returns the workload's record (rank 0's view of the max-over-ranks times)."""
+    buffers.  Returns the workload's record (rank 0's view of the max-over-ranks times).
+    With --parallel ep each rank holds a contiguous shard of the experts; a step is every rank's
+    forward over its shard routed from all tokens' logits (moe_mx_forward_shard, float32 partial
+    output) and the sum of the partials over the ranks (NCCL all-reduce)."""
     dev = torch.device("cuda", torch.cuda.current_device())
     hbm_peak, bf16_peak, bf16_sustained, peak_src = measured_peaks()
     act = moe_mx.MOE_MX_ACT_MXFP8 if wl.act == "mxfp8" else moe_mx.MOE_MX_ACT_BF16
     w1, w1s_rm, w2, w2s_rm = weights
     x = workloads.draw_x(wl).to(dev)
     given = wl.routing == "given"
+    ep_mode = args.parallel == "ep"
+    if ep_mode and (given or wl.shared):
+        raise SystemExit(f"--parallel ep runs the logits form without a shared expert; {wl.name} is not one")
     # the routing input: router logits, or the given top-k (global ids and weights)
     route_host = workloads.draw_topk(wl) if given else (workloads.draw_logits(wl),)
     route_in = tuple(a.to(dev) for a in route_host)
-    out = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=dev)
-    layer = moe_mx.MoeMxLayer(wl.H, wl.I, wl.E, wl.T, wl.top_k, device=dev.index, num_shared=wl.shared)
+    E_local, offset = wl.E, 0
+    if ep_mode:
+        from block_scaled_moe_softmax_b200 import ep
+        offset, E_local = ep.shard_range(wl.E, world, rank)
+    out = torch.empty(wl.T, wl.H, dtype=torch.float32 if ep_mode else torch.bfloat16, device=dev)
+    layer = moe_mx.MoeMxLayer(wl.H, wl.I, E_local, wl.T, wl.top_k, device=dev.index, num_shared=wl.shared)
     # weight preparation, once, like the quantisation: the E8M0 scales in the tiled layout
     w1s, w2s = layer.prepare_scales(w1s_rm, w2s_rm)
     torch.cuda.synchronize()
@@ -397,7 +420,11 @@ def measure(args, wl, weights, world, rank, with_e2e=True):
     stream = torch.cuda.current_stream()
 
     def forward(xin, rin):
-        if given:
+        if ep_mode:
+            moe_mx.moe_mx_forward_shard(layer.handle, xin, rin[0], wl.T, wl.E, offset, w1, w1s, w2, w2s, wl.top_k,
+                                        act, out, moe_mx.MOE_MX_OUT_F32, stream)
+            ep.reduce_partials(out)
+        elif given:
             moe_mx.moe_mx_forward_routed(layer.handle, xin, rin[0], rin[1], wl.T, wl.top_k, wl.local_offset, w1, w1s,
                                          w2, w2s, act, out, moe_mx.MOE_MX_OUT_BF16, stream)
         else:
@@ -434,7 +461,9 @@ def measure(args, wl, weights, world, rank, with_e2e=True):
     step_ms = [a.elapsed_time(b) for a, b in evs]
     assert layer.sync_status() == moe_mx.MOE_MX_OK, moe_mx.moe_mx_last_error()
     ms_all = max_over_ranks(statistics.mean(step_ms), world)
-    value = world * wl.T / (ms_all / 1000.0)
+    # replicas: every rank its own batch; expert parallelism: one batch over all ranks
+    batch_tokens = wl.T if ep_mode else world * wl.T
+    value = batch_tokens / (ms_all / 1000.0)
 
     # ---------------- per-kernel times: the same steps with CUDA events between the kernels.
     # (In the timed steps above each kernel may launch while the one before it still runs, and
@@ -454,7 +483,7 @@ def measure(args, wl, weights, world, rank, with_e2e=True):
     if with_e2e:
         x_h = workloads.draw_x(wl).pin_memory()
         r_h = tuple(a.pin_memory() for a in route_host)
-        o_h = torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory()
+        o_h = torch.empty(wl.T, wl.H, dtype=out.dtype).pin_memory()
         x_d = torch.empty_like(x)
         r_d = tuple(torch.empty_like(a) for a in route_in)
         e2e_steps = max(3, min(args.steps, 200))
@@ -474,10 +503,11 @@ def measure(args, wl, weights, world, rank, with_e2e=True):
         torch.cuda.synchronize()
         barrier(world)
         e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in e2e_evs), world)
-        assert torch.equal(o_h.view(torch.int16), out.cpu().view(torch.int16))
-        e2e = {"value": world * wl.T / (e2e_ms / 1000.0), "unit": "tokens/s",
+        assert torch.equal(o_h, out.cpu()) if ep_mode else torch.equal(o_h.view(torch.int16),
+                                                                       out.cpu().view(torch.int16))
+        e2e = {"value": batch_tokens / (e2e_ms / 1000.0), "unit": "tokens/s",
                "h2d_bytes_per_step": wl.T * wl.H * 2 + sum(a.numel() * a.element_size() for a in route_host),
-               "d2h_bytes_per_step": wl.T * wl.H * 2}
+               "d2h_bytes_per_step": wl.T * wl.H * out.element_size()}
 
     fc1_ms = stage["fc1"]
     layer_bytes = layer_weight_bytes(wl, hit)
@@ -527,7 +557,14 @@ def run_ours(args):
     world, rank, local = dist_setup(args.gpus)
     dev = torch.device("cuda", torch.cuda.current_device())
     names = [args.workload] if args.workload else list(DEFAULT_SET)
-    cache = WeightCache(dev)
+    experts_of = None
+    if args.parallel == "ep":
+        from block_scaled_moe_softmax_b200 import ep
+
+        def experts_of(wl):
+            off, n = ep.shard_range(wl.E, world, rank)
+            return range(off, off + n)
+    cache = WeightCache(dev, experts_of)
     recs = {}
     for name in names:
         wl = workloads.WORKLOADS[name]
@@ -538,10 +575,12 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": head["tokens_per_s"], "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "strong" if args.parallel == "ep" else "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
         "config": {"workload": head["workload"], "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "top_k": wl.top_k,
-                   "act": wl.act, "hit_experts": head["hit_experts"], "global_batch": wl.T * world,
-                   "parallelism": f"replicas{world}",
+                   "act": wl.act, "hit_experts": head["hit_experts"],
+                   "global_batch": wl.T if args.parallel == "ep" else wl.T * world,
+                   "parallelism": f"ep{world}" if args.parallel == "ep" else f"replicas{world}",
                    "l2": f"weights {head['weight_bytes_resident'] / 1e9:.2f} GB, a 512 MiB L2 flush before every "
                          "timed step",
                    "weight_scales": "tiled layout (moe_mx_prepare_scales, once before timing)"},
@@ -577,6 +616,9 @@ def main():
                     help="one workload only (default: decode as the headline, plus the other four "
                          "configurations in per_config)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--parallel", choices=["replicas", "ep"], default="replicas",
+                    help="replicas: an independent batch per GPU (default); ep: one batch, the experts split "
+                         "into contiguous shards over the GPUs, partial outputs all-reduced (NCCL)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

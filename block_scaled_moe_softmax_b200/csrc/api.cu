@@ -141,11 +141,13 @@ struct moe_mx_handle {
     int tile_rows; // 0: by token count; else 16, 32, 64 or 128 (MOE_MX_TILE_ROWS)
     int pdl;       // launch the kernels after the router as programmatic dependents (MOE_MX_PDL, default 1)
     int wide;      // 128-row GEMM blocks: the two-tile (N = 256) variant (MOE_MX_WIDE, default 1)
+    int fuse_combine; // small batches: the combine runs in FC2's epilogue (MOE_MX_FUSE_COMBINE, default 1)
     int scale_layout; // MOE_MX_SCALES_ROW_MAJOR or MOE_MX_SCALES_TILED
     unsigned long long timeout_ns;
     void *ws;
     int32_t *topk_ids, *chunk_hist, *counts, *pad_offsets, *num_rowblocks, *sorted_pair, *pos_of_pair;
     int32_t *unit_counters;
+    int32_t *combine_cnt; // [max_tokens][H/128] pairs of each token and FC2 weight tile done (fused combine)
     float *topk_w;
     int4 *rowblocks;
     uint8_t *Aq, *Asf, *Hq, *Hsf; // MXFP8 operand planes [2][rows][K] and their scale atoms
@@ -243,6 +245,7 @@ int moe_mx_create_ex(moe_mx_handle **out, int hidden, int inter, int num_experts
         h->tile_rows = 0;
     h->pdl = env_int("MOE_MX_PDL", 1) != 0;
     h->wide = env_int("MOE_MX_WIDE", 1) != 0;
+    h->fuse_combine = env_int("MOE_MX_FUSE_COMBINE", 1) != 0;
     h->swap_rows = env_int("MOE_MX_SWAP_ROWS", 64);
     if (h->swap_rows < 0)
         h->swap_rows = 0;
@@ -263,6 +266,7 @@ int moe_mx_create_ex(moe_mx_handle **out, int hidden, int inter, int num_experts
         {(void **)&h->rowblocks, sizeof(int4) * (h->max_rows / 16)}, // work blocks: >= 16 padded rows each
         {(void **)&h->num_rowblocks, sizeof(int32_t)},
         {(void **)&h->unit_counters, 2 * sizeof(int32_t)}, // FC1, FC2 work-unit counters
+        {(void **)&h->combine_cnt, sizeof(int32_t) * max_tokens * (hidden / 128)},
         {(void **)&h->sorted_pair, sizeof(int32_t) * h->max_rows},
         {(void **)&h->pos_of_pair, sizeof(int32_t) * pairs},
         {(void **)&h->err, sizeof(uint32_t)},
@@ -341,21 +345,32 @@ int moe_mx_destroy(moe_mx_handle *h)
 
 namespace {
 
-// The forward of both entry points: routing computed from router_logits, or (given_ids set)
-// the given global ids and weights restricted to the shard [id_offset, id_offset + E).
+// The forward of every entry point: routing computed from router_logits, or (given_ids set)
+// the given global ids and weights restricted to the shard [id_offset, id_offset + E); with
+// route_E > 0 the logits cover route_E experts (the whole layer) and the routed pairs are
+// restricted to the shard [id_offset, id_offset + E) the handle holds.
 int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, const int32_t *given_ids,
                  const float *given_w, int id_offset, int num_tokens, const uint8_t *w1, const uint8_t *w1_scale,
                  const uint8_t *w2, const uint8_t *w2_scale, int top_k, int act_dtype, void *out, int out_f32,
-                 void *stream)
+                 void *stream, int route_E = 0)
 {
     g_last_error.clear();
     if (!h)
         return fail(MOE_MX_ERR_INVALID_ARG, "handle is NULL");
     if (num_tokens < 0 || num_tokens > h->maxT)
         return fail(MOE_MX_ERR_INVALID_ARG, "num_tokens=%d must be in [0, %d]", num_tokens, h->maxT);
-    if (!given_ids && (top_k < 1 || top_k > h->maxK || top_k > h->E - h->S))
-        return fail(MOE_MX_ERR_INVALID_ARG, "top_k=%d must be in [1, min(E=%d, max_top_k=%d)]", top_k,
-                    h->E - h->S, h->maxK);
+    if (route_E > 0 && h->S > 0)
+        return fail(MOE_MX_ERR_UNSUPPORTED, "the shard form takes no shared expert (handle has %d shared chunks)",
+                    h->S);
+    if (route_E > 0 && (route_E > kMaxExperts || id_offset < 0 || id_offset > route_E - h->E))
+        return fail(MOE_MX_ERR_INVALID_ARG,
+                    "num_experts_global=%d, local_expert_offset=%d: need the shard [offset, offset + %d) inside "
+                    "[0, num_experts_global) and num_experts_global <= %d",
+                    route_E, id_offset, h->E, kMaxExperts);
+    const int routed = route_E > 0 ? route_E : h->E - h->S; // experts the router chooses among
+    if (!given_ids && (top_k < 1 || top_k > h->maxK || top_k > routed))
+        return fail(MOE_MX_ERR_INVALID_ARG, "top_k=%d must be in [1, min(E=%d, max_top_k=%d)]", top_k, routed,
+                    h->maxK);
     if (given_ids && h->S > 0)
         return fail(MOE_MX_ERR_UNSUPPORTED, "the routed form takes no shared expert (handle has %d shared chunks)",
                     h->S);
@@ -435,6 +450,8 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
         ra.given_w = given_w;
         ra.id_offset = id_offset;
         ra.n_shared = h->S;
+        ra.shard = route_E > 0;
+        ra.route_E = route_E;
         // Each kernel after the router may launch while its predecessor still runs (programmatic
         // dependent launch): the FC GEMMs start streaming their weights early.  Stage timing
         // records events between the kernels, so timed forwards launch them one after another.
@@ -485,12 +502,23 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
         f2.out_ld = H;
         f2.fc1 = 0;
         f2.act_mxfp8 = 0;
+        // small batches of the logits form: every FC2 unit has its tokens on N, and its epilogue
+        // finishes the combine of the tokens whose k pairs it completes
+        const bool fuse = h->fuse_combine && !given_ids && route_E == 0 && tile_rows <= 64;
+        f2.fuse_combine = fuse;
+        f2.combine_cnt = h->combine_cnt;
+        f2.sorted_pair = h->sorted_pair;
+        f2.pos_of_pair = h->pos_of_pair;
+        f2.topk_w = h->topk_w;
+        f2.k = k;
+        f2.out = static_cast<__nv_bfloat16 *>(out);
         // the maps' plane count must equal the copy's terms: the stage barrier expects exactly those bytes
         launch_fc_gemm(f2, h->map_H[f2.terms - 1], h->map_Hsw[f2.terms - 1][sw_idx], h->map_H16, h->map_w2,
                        h->num_sms, s, pdl);
         mark(4);
-        launch_combine(h->Y, T, H, k, h->pos_of_pair, h->topk_w, out, out_f32, h->num_sms, s, pdl);
-        h->launches += 4; // gather, FC1, FC2, combine
+        if (!fuse)
+            launch_combine(h->Y, T, H, k, h->pos_of_pair, h->topk_w, out, out_f32, h->num_sms, s, pdl);
+        h->launches += fuse ? 3 : 4; // gather, FC1, FC2 (+ combine)
         ce = cudaGetLastError();
         if (ce != cudaSuccess) {
             rc = cuda_fail(ce, "kernel launch");
@@ -535,6 +563,23 @@ int moe_mx_forward_routed(moe_mx_handle *h, const void *x, const int32_t *topk_i
                         top_k, act_dtype, out, out_dtype == MOE_MX_OUT_F32, stream);
 }
 
+int moe_mx_forward_shard(moe_mx_handle *h, const void *x, const float *router_logits, int num_tokens,
+                         int num_experts_global, int local_expert_offset, const uint8_t *w1, const uint8_t *w1_scale,
+                         const uint8_t *w2, const uint8_t *w2_scale, int top_k, int act_dtype, void *out,
+                         int out_dtype, void *stream)
+{
+    if (out_dtype != MOE_MX_OUT_BF16 && out_dtype != MOE_MX_OUT_F32) {
+        g_last_error.clear();
+        return fail(MOE_MX_ERR_INVALID_ARG, "out_dtype=%d is not MOE_MX_OUT_BF16 or MOE_MX_OUT_F32", out_dtype);
+    }
+    if (num_experts_global < 1) {
+        g_last_error.clear();
+        return fail(MOE_MX_ERR_INVALID_ARG, "num_experts_global=%d must be >= 1", num_experts_global);
+    }
+    return forward_impl(h, x, router_logits, nullptr, nullptr, local_expert_offset, num_tokens, w1, w1_scale, w2,
+                        w2_scale, top_k, act_dtype, out, out_dtype == MOE_MX_OUT_F32, stream, num_experts_global);
+}
+
 int moe_mx_sync_status(moe_mx_handle *h, void *stream)
 {
     g_last_error.clear();
@@ -547,6 +592,8 @@ int moe_mx_sync_status(moe_mx_handle *h, void *stream)
     if ((ce = cudaMemcpy(&word, h->err, sizeof(word), cudaMemcpyDeviceToHost)) != cudaSuccess)
         return cuda_fail(ce, "cudaMemcpy(error word)");
     if (word != 0) {
+        // a forward cut short may leave the fused combine's counts behind: they start at zero again
+        cudaMemset(h->combine_cnt, 0, sizeof(int32_t) * h->maxT * (h->H / 128));
         cudaMemset(h->err, 0, sizeof(uint32_t));
         cudaDeviceSynchronize();
         return fail(MOE_MX_ERR_TIMEOUT, "a device-side wait gave up (error word 0x%x)", word);

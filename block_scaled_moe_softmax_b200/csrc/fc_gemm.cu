@@ -267,6 +267,44 @@ __device__ __forceinline__ float silu_mul(float g, float u)
 } // namespace
 
 
+// The combine fused into FC2's epilogue (small batches, every unit with its tokens on N), run by
+// the 128 epilogue threads (L = 0..127) after a unit's Y rows are stored.  Each (token, weight
+// tile) those rows belong to counts one more finished pair; the unit that completes a token's k
+// pairs of a tile sums the token's k rows of that tile in j order, out = bf16(sum_j w_j * Y_j)
+// with the combine kernel's arithmetic (same bits), and resets the count for the next forward.
+// Every Y store is fenced before its count, and the completing unit fences before it reads.
+__device__ __forceinline__ void fused_combine_unit(const FcGemmArgs &a, const int4 blk, int nt0, int kWT, int L,
+                                                   int *s_list)
+{
+    __threadfence();
+    if (L == 0)
+        s_list[128] = 0;
+    named_bar_sync(1, 128);
+    if (L < blk.z * kWT) { // one (row, weight tile) per thread: rows <= 64, kWT <= 2
+        const int n = L / kWT, tile = nt0 + L % kWT;
+        const int t = a.sorted_pair[blk.y + n] / a.k;
+        int *c = a.combine_cnt + (size_t)t * a.n_tiles + tile;
+        if (atomicAdd(c, 1) == a.k - 1) {
+            *c = 0; // the token's last pair of this tile: nothing else counts it in this forward
+            s_list[atomicAdd(&s_list[128], 1)] = t * a.n_tiles + tile;
+        }
+    }
+    named_bar_sync(1, 128);
+    __threadfence();
+    const int ne = s_list[128];
+    for (int i = 0; i < ne; ++i) {
+        const int t = s_list[i] / a.n_tiles, col = (s_list[i] % a.n_tiles) * 128 + L;
+        float acc = 0.f;
+        for (int j = 0; j < a.k; ++j) {
+            const float w = __ldg(a.topk_w + (size_t)t * a.k + j);
+            const int row = __ldg(a.pos_of_pair + (size_t)t * a.k + j);
+            acc = fmaf(w, __ldcg(a.y + (size_t)row * a.out_ld + col), acc);
+        }
+        a.out[(size_t)t * a.out_ld + col] = __float2bfloat16_rn(acc);
+    }
+    named_bar_sync(1, 128); // the list is rewritten by the next unit
+}
+
 // Per-CTA state the warp roles share (all values are CTA-uniform).
 struct Ctx {
     uint32_t base;        // shared-memory base (1024-byte aligned, shared window)
@@ -907,6 +945,8 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads,
             }
             tc_fence_before();
             mbar_arrive(bars.acc_empty(buf));
+            if (swap && !a.fc1 && a.fuse_combine)
+                fused_combine_unit(a, blk, nt0, P::kWT, 32 * q + lane, reinterpret_cast<int *>(xch));
         }
     }
 

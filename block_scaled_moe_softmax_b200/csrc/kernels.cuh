@@ -63,6 +63,11 @@ struct RouteGroupArgs {
     // last n_shared slots route to them with weight 1 (the router picks k - n_shared routed
     // experts among the first E - n_shared).  Logits form only.
     int n_shared = 0;
+    // Logits form over a shard: the router picks among route_E experts (the whole layer; the
+    // logits are [T, route_E]) and keeps the E of [id_offset, id_offset + E), the rest -1.
+    int shard = 0;
+    int route_E = 0;
+    __host__ __device__ int routeE() const { return shard ? route_E : E - n_shared; }
 };
 
 // Launchers of the forward's kernels.  pdl: launch as programmatic dependents of the kernel
@@ -109,6 +114,16 @@ struct FcGemmArgs {
                                  // the kernel variant (activation tile rows per term)
     int wide;                    // 128-row blocks: two weight tiles per work unit (tokens on M) when
                                  // n_tiles is even
+    // FC2 only, every unit with its tokens on N: the weighted combine fused into the epilogue
+    // (out = bf16(sum_j w[t,j] * Y[pos(t,j)]) written by the unit that completes a token's k pairs
+    // of a weight tile, counted in combine_cnt [T][n_tiles], zero before and after every forward)
+    int fuse_combine;
+    int *combine_cnt;
+    const int32_t *sorted_pair;  // grouped row -> pair t*k + j
+    const int32_t *pos_of_pair;  // pair -> grouped row
+    const float *topk_w;         // [T, k]
+    int k;                       // slots per token
+    __nv_bfloat16 *out;          // [T, H]
 };
 
 // Tensor maps: act_map = both term planes, 128-row boxes ([terms][128][128] codes, tokens

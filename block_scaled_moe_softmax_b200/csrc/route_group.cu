@@ -42,10 +42,14 @@ __device__ __forceinline__ float order_value(uint32_t k)
 // (j < k) writes the j-th id and weight and adds it to the block's expert histogram.
 // With n_shared > 0 the token has k + n_shared slots: after the k routed ones, the shared
 // expert's chunks (expert slots E.., weight 1).
+// With e_local >= 0 the E experts routed over are the whole layer's and this launch holds the
+// shard [off, off + e_local) of them: a selected expert inside it is written as its local id
+// (global - off) and counted, one outside as -1 (not grouped); the weights are the whole
+// layer's, as if unsharded.
 template <int kPerLane> // experts per lane: E <= 32 * kPerLane
 __device__ __forceinline__ void route_token(const float *__restrict__ row, int E, int k, int n_shared, int t,
                                             int lane, int32_t *__restrict__ topk_ids, float *__restrict__ topk_w,
-                                            int32_t *hist)
+                                            int32_t *hist, int off = 0, int e_local = -1)
 {
     float v[kPerLane];
     uint32_t taken = 0;
@@ -99,9 +103,12 @@ __device__ __forceinline__ void route_token(const float *__restrict__ row, int E
         z += __shfl_xor_sync(0xFFFFFFFFu, z, off);
     const int slots = k + n_shared;
     if (lane < k) {
-        topk_ids[(size_t)t * slots + lane] = my_id;
+        const int loc = my_id - off; // off = 0 unless sharded
+        const bool local = e_local < 0 || (loc >= 0 && loc < e_local);
+        topk_ids[(size_t)t * slots + lane] = local ? loc : -1;
         topk_w[(size_t)t * slots + lane] = u / z;
-        atomicAdd(&hist[my_id], 1);
+        if (local)
+            atomicAdd(&hist[loc], 1);
     } else if (lane < slots) {
         topk_ids[(size_t)t * slots + lane] = E + (lane - k);
         topk_w[(size_t)t * slots + lane] = 1.0f;
@@ -135,7 +142,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float *__res
                                                                float *__restrict__ topk_w,
                                                                int32_t *__restrict__ chunk_hist,
                                                                const int32_t *__restrict__ gids,
-                                                               const float *__restrict__ gw, int off, int n_shared)
+                                                               const float *__restrict__ gw, int off, int n_shared,
+                                                               int route_E, int shard)
 {
     grid_dep_launch(); // the next kernel (the scan) waits for this grid before reading its output
     __shared__ int32_t hist[kMaxExperts];
@@ -149,8 +157,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float *__res
         if (gids)
             take_given_token(gids, gw, E, k, off, t, lane, topk_ids, topk_w, hist);
         else
-            route_token<kPerLane>(logits + (size_t)t * (E - n_shared), E - n_shared, k - n_shared, n_shared, t, lane,
-                                  topk_ids, topk_w, hist);
+            route_token<kPerLane>(logits + (size_t)t * route_E, route_E, k - n_shared, n_shared, t, lane, topk_ids,
+                                  topk_w, hist, off, shard ? E : -1);
     }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x)
@@ -351,8 +359,8 @@ __global__ void __launch_bounds__(1024) route_group_small_kernel(const RouteGrou
         if (a.given_ids)
             take_given_token(a.given_ids, a.given_w, a.E, a.k, a.id_offset, t, lane, a.topk_ids, a.topk_w, hist);
         else
-            route_token<kPerLane>(a.logits + (size_t)t * (a.E - a.n_shared), a.E - a.n_shared, a.k - a.n_shared,
-                                  a.n_shared, t, lane, a.topk_ids, a.topk_w, hist);
+            route_token<kPerLane>(a.logits + (size_t)t * a.routeE(), a.routeE(), a.k - a.n_shared, a.n_shared, t, lane,
+                                  a.topk_ids, a.topk_w, hist, a.id_offset, a.shard ? a.E : -1);
     }
     __syncthreads(); // also makes lane 0's id writes visible to the whole CTA
     const int e = threadIdx.x;
@@ -591,11 +599,11 @@ int launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s, bool pdl)
     // the top-k scan visits 32 * kPerLane candidates per token: size it to the expert count
     // (the given routing visits no candidates: the smallest instance serves it).  The first
     // kernel is an ordinary launch; those after it are programmatic dependents (pdl).
-    const bool narrow = a.given_ids != nullptr || a.E <= 256;
+    const bool narrow = a.given_ids != nullptr || a.routeE() <= 256;
     if (a.T <= kSmallRouteTokens) {
         if (narrow)
             route_group_small_kernel<8><<<1, 1024, 0, s>>>(a);
-        else if (a.E <= 512)
+        else if (a.routeE() <= 512)
             route_group_small_kernel<16><<<1, 1024, 0, s>>>(a);
         else
             route_group_small_kernel<32><<<1, 1024, 0, s>>>(a);
@@ -604,13 +612,16 @@ int launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s, bool pdl)
     const int nchunks = (a.T + kRouteChunk - 1) / kRouteChunk;
     if (narrow)
         route_kernel<8><<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist,
-                                                          a.given_ids, a.given_w, a.id_offset, a.n_shared);
-    else if (a.E <= 512)
+                                                          a.given_ids, a.given_w, a.id_offset, a.n_shared, a.routeE(),
+                                                          a.shard);
+    else if (a.routeE() <= 512)
         route_kernel<16><<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist,
-                                                          a.given_ids, a.given_w, a.id_offset, a.n_shared);
+                                                          a.given_ids, a.given_w, a.id_offset, a.n_shared, a.routeE(),
+                                                          a.shard);
     else
         route_kernel<32><<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist,
-                                                          a.given_ids, a.given_w, a.id_offset, a.n_shared);
+                                                          a.given_ids, a.given_w, a.id_offset, a.n_shared, a.routeE(),
+                                                          a.shard);
     launch_kernel(scan_kernel, dim3(1), dim3(1024), 0, s, pdl, a.E, nchunks, a.split_rows, a.chunk_hist, a.counts,
                   a.pad_offsets, a.rowblocks, a.num_rowblocks, a.sorted_pair, a.unit_counters);
     launch_kernel(scatter_kernel, dim3(nchunks), dim3(32), 0, s, pdl, a.T, a.E, a.k, (const int32_t *)a.topk_ids,

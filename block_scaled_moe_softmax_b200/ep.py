@@ -5,10 +5,12 @@ partial outputs summed.
 TokenSpeed SiTU package description, "Supported contract": every rank routes with the
 global expert ids, the layer filters them to its contiguous shard of local experts (local
 expert offset = rank x experts per rank) and produces a partial output, and the caller
-all-reduces the partial outputs over the expert-parallel group.  On one rank the filtering
-and the float32 partial output are moe_mx_forward_routed (CUDA); this module adds the
-shard bookkeeping and the sum over ranks (torch.distributed; NCCL on GPUs).  The result
-is the float32 sum; rounding it to bf16, if wanted, is the caller's.
+all-reduces the partial outputs over the expert-parallel group.  On one rank the routing,
+the filtering and the float32 partial output are CUDA: moe_mx_forward_shard from the whole
+layer's router logits (every rank routes all tokens; ep_forward_logits), or
+moe_mx_forward_routed from precomputed global ids (ep_forward).  This module adds the shard
+bookkeeping and the sum over ranks (torch.distributed; NCCL on GPUs).  The result is the
+float32 sum; rounding it to bf16, if wanted, is the caller's.
 
 Tensor parallelism (the same page's TP8 configuration: all experts on every rank, each with
 a slice of the intermediate dimension) needs no kernel of its own: SwiGLU acts element by
@@ -56,6 +58,27 @@ def ep_forward(layer: moe_mx.MoeMxLayer, x, topk_ids, topk_w, w1, w1_scale, w2, 
         raise ValueError(f"layer holds {layer.E} experts, rank {rank}'s shard has {n}")
     partial = layer.forward_routed(x, topk_ids, topk_w, w1, w1_scale, w2, w2_scale, offset, act_dtype,
                                    moe_mx.MOE_MX_OUT_F32)
+    return reduce_partials(partial, group)
+
+
+def ep_forward_logits(layer, x, router_logits, w1, w1_scale, w2, w2_scale, top_k: int, num_experts: int,
+                      rank: int, world: int, group=None, act_dtype: int = moe_mx.MOE_MX_ACT_BF16,
+                      partial_fn=None) -> torch.Tensor:
+    """One expert-parallel forward routed from the whole layer's logits [T, num_experts]: this rank
+    routes every token over all experts, runs the pairs of its contiguous shard
+    (moe_mx_forward_shard: float32 partial output) and the partials are summed over the group.
+    `layer` holds this rank's shard (its E local experts' weights in w1..w2_scale).
+    partial_fn(offset, n) may replace the rank's partial computation (it must return the float32
+    partial [T, H] of the shard [offset, offset + n)); by default the layer computes it.
+    Returns the float32 sum of all ranks' partial outputs."""
+    offset, n = shard_range(num_experts, world, rank)
+    if partial_fn is None:
+        if layer.E != n:
+            raise ValueError(f"layer holds {layer.E} experts, rank {rank}'s shard has {n}")
+        partial = layer.forward_shard(x, router_logits, w1, w1_scale, w2, w2_scale, top_k, offset, act_dtype,
+                                      moe_mx.MOE_MX_OUT_F32)
+    else:
+        partial = partial_fn(offset, n)
     return reduce_partials(partial, group)
 
 

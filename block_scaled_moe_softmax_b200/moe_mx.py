@@ -48,6 +48,7 @@ SIGNATURES = {
     "moe_mx_create_ex": (_I, [ctypes.POINTER(_P), _I, _I, _I, _I, _I, _I, _I]),
     "moe_mx_forward": (_I, [_P, _P, _P, _I, _P, _P, _P, _P, _I, _I, _P, _P]),
     "moe_mx_forward_routed": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _I, _P, _I, _P]),
+    "moe_mx_forward_shard": (_I, [_P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _I, _I, _P, _I, _P]),
     "moe_mx_destroy": (_I, [_P]),
     "moe_mx_last_error": (ctypes.c_char_p, []),
     "moe_mx_sync_status": (_I, [_P, _P]),
@@ -159,6 +160,15 @@ def moe_mx_forward_routed(handle: int, x, topk_ids, topk_w, num_tokens: int, top
                                                 _ptr(w2_scale), act_dtype, _ptr(out), out_dtype, _stream(stream)))
 
 
+def moe_mx_forward_shard(handle: int, x, router_logits, num_tokens: int, num_experts_global: int,
+                         local_expert_offset: int, w1, w1_scale, w2, w2_scale, top_k: int, act_dtype: int, out,
+                         out_dtype: int = MOE_MX_OUT_F32, stream=None) -> None:
+    _check(load_library().moe_mx_forward_shard(handle, _ptr(x), _ptr(router_logits), num_tokens, num_experts_global,
+                                               local_expert_offset, _ptr(w1), _ptr(w1_scale), _ptr(w2),
+                                               _ptr(w2_scale), top_k, act_dtype, _ptr(out), out_dtype,
+                                               _stream(stream)))
+
+
 def moe_mx_sync_status(handle: int, stream=None) -> int:
     """Returns the status code (does not raise on MOE_MX_ERR_TIMEOUT)."""
     return load_library().moe_mx_sync_status(handle, _stream(stream))
@@ -259,6 +269,20 @@ class MoeMxLayer:
             out = torch.empty(T, self.H, dtype=dt, device=x.device)
         moe_mx_forward_routed(self.handle, x, topk_ids, topk_w, T, k, local_expert_offset, w1, w1_scale, w2,
                               w2_scale, act_dtype, out, out_dtype, stream)
+        return out
+
+    def forward_shard(self, x: torch.Tensor, router_logits: torch.Tensor, w1, w1_scale, w2, w2_scale, top_k: int,
+                      local_expert_offset: int, act_dtype: int = MOE_MX_ACT_BF16, out_dtype: int = MOE_MX_OUT_F32,
+                      out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """The layer routed from the whole layer's logits [T, E_global], over this handle's shard of
+        E experts starting at global id local_expert_offset: the shard's partial output (float32
+        by default, for a sum over the expert-parallel group)."""
+        T, E_global = router_logits.shape
+        if out is None:
+            dt = torch.float32 if out_dtype == MOE_MX_OUT_F32 else torch.bfloat16
+            out = torch.empty(T, self.H, dtype=dt, device=x.device)
+        moe_mx_forward_shard(self.handle, x, router_logits, T, E_global, local_expert_offset, w1, w1_scale, w2,
+                             w2_scale, top_k, act_dtype, out, out_dtype, stream)
         return out
 
     def prepare_scales(self, w1_scale: torch.Tensor, w2_scale: torch.Tensor, stream=None):

@@ -204,6 +204,38 @@ MOE_MX_API int moe_mx_forward_routed(moe_mx_handle *h, const void *x, const int3
                                      const uint8_t *w1_scale, const uint8_t *w2, const uint8_t *w2_scale,
                                      int act_dtype, void *out, int out_dtype, void *stream);
 
+/*
+ * Run the layer over one rank's contiguous shard of the experts, routed from the
+ * whole layer's router logits: expert parallelism as the tokenspeed-situ package
+ * description's "Supported contract" runs it (every rank sees global expert
+ * ids, keeps the pairs of its contiguous local shard, and writes a partial
+ * output that the caller all-reduces over the expert-parallel group), with the
+ * routing done here, on every rank, for all tokens.  The handle's E is the number
+ * of local experts; the weights hold those E experts.
+ *   router_logits       float32 [T, num_experts_global], the whole layer's logits.
+ *   num_experts_global  experts of the whole layer: 1..1024, >= local_expert_offset + E.
+ *   local_expert_offset global id of local expert 0 (>= 0).
+ *   top_k               1..min(num_experts_global, max_top_k): the whole layer's
+ *                       top-k (softmax, lowest index winning ties, weights
+ *                       renormalised over the k), as moe_mx_forward chooses it.
+ *   out                 [T, H], written: float32 (MOE_MX_OUT_F32: the shard's
+ *                       partial sum, sum over slots j whose expert is local of
+ *                       w[t,j] * FC2(SwiGLU(FC1(x[t]))), j ascending; the partial
+ *                       outputs of all shards add up to the layer's output before
+ *                       its rounding) or bf16 (MOE_MX_OUT_BF16).
+ *   x, w1, w1_scale, w2, w2_scale, act_dtype, num_tokens: as for moe_mx_forward.
+ * With the shard [0, E) of E experts this is moe_mx_forward (same routing, same
+ * output bits for bf16).  moe_mx_get_routing afterwards reports the local ids
+ * (-1 for a selected expert outside the shard) and the whole layer's weights.
+ * Allocation, synchronisation, graph capture and errors as for moe_mx_forward
+ * (INVALID_ARG also for a bad out_dtype or a shard outside the layer;
+ * UNSUPPORTED for a handle with a shared expert).
+ */
+MOE_MX_API int moe_mx_forward_shard(moe_mx_handle *h, const void *x, const float *router_logits, int num_tokens,
+                                    int num_experts_global, int local_expert_offset, const uint8_t *w1,
+                                    const uint8_t *w1_scale, const uint8_t *w2, const uint8_t *w2_scale, int top_k,
+                                    int act_dtype, void *out, int out_dtype, void *stream);
+
 /* Free the handle and its workspace (waits for the device).  NULL is a no-op. */
 MOE_MX_API int moe_mx_destroy(moe_mx_handle *h);
 

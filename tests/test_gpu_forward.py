@@ -236,3 +236,26 @@ def test_router_matches_hand_derived_cases():
             assert ids[r].tolist() == cases[i][2], (cases[i], ids[r])
             np.testing.assert_allclose(w[r], cases[i][3], rtol=2e-6, atol=1e-7)
     layer.close()
+
+
+@pytest.mark.parametrize("name", ["tiny", "multi"])
+@pytest.mark.parametrize("act_mode", [0, 1], ids=["w4a16", "w4a8"])
+@pytest.mark.parametrize("variant", ["auto", "t16", "t32", "t64"])
+def test_fused_combine_gives_same_bits(name, act_mode, variant, monkeypatch):
+    """Up to 512 tokens (every FC2 unit with its tokens on N) the combine runs in FC2's epilogue by
+    default; it must give exactly the bits of the separate combine kernel (MOE_MX_FUSE_COMBINE=0),
+    on two forwards in a row (its per-token counters must be back at zero after each)."""
+    wl = SHAPES[name]
+    tile_rows = VARIANTS[variant][0]
+    inp = helpers.host_inputs(wl)
+    outs = []
+    for fuse in ("1", "0"):
+        monkeypatch.setenv("MOE_MX_FUSE_COMBINE", fuse)
+        layer, _, out = _run(wl, act_mode, monkeypatch, inp=inp, tile_rows=tile_rows)
+        d = helpers.to_device(inp)
+        out2 = layer.forward(d["x"], d["logits"], d["w1"], d["w1s"], d["w2"], d["w2s"], wl.top_k, act_mode)
+        assert layer.sync_status() == moe_mx.MOE_MX_OK, moe_mx.moe_mx_last_error()
+        assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+        outs.append(out)
+        layer.close()
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))

@@ -121,6 +121,69 @@ def test_top_k_beyond_shard_and_foreign_routing():
     layer.close()
 
 
+@pytest.mark.parametrize("T", [12, 200])
+@pytest.mark.parametrize("act", [0, 1], ids=["w4a16", "w4a8"])
+def test_logits_shards_match_oracle_and_add_up(T, act):
+    """moe_mx_forward_shard: the whole layer's router on every token, the pairs of one contiguous
+    shard kept.  Local ids (-1 outside the shard) bit-exact and the whole layer's weights within
+    2e-6 of the oracle's router; counts and the grouping of the local pairs bit-exact; each shard's
+    float32 partial within the tolerance of the oracle's routed form at the shard's offset; the
+    partials of a partition adding up to the oracle's layer; and the shard [0, E) giving the bits
+    of moe_mx_forward."""
+    E, k = 8, 4
+    wl = workloads.Workload("shard", T, 256, 128, E, k, "bf16", "normal", 4)
+    x, logits = workloads.draw_x(wl), workloads.draw_logits(wl)
+    wq = helpers.quantize_weights_cpu(wl)
+    xb = workloads.bf16_bits(x)
+    ids_o, w_o = oracle.route(logits.numpy(), k)
+    total = torch.zeros(T, wl.H, dtype=torch.float64)
+    for lo, hi in ((0, 3), (3, 5), (5, 8)):
+        layer = moe_mx.MoeMxLayer(wl.H, wl.I, hi - lo, T, k)
+        d = _dev({n: np.ascontiguousarray(v[lo:hi]) for n, v in wq.items()})
+        part = layer.forward_shard(x.cuda(), logits.cuda(), d["w1"], d["w1s"], d["w2"], d["w2s"], k, lo, act)
+        assert layer.sync_status() == moe_mx.MOE_MX_OK, moe_mx.moe_mx_last_error()
+        ids_g, w_g = [a.cpu().numpy() for a in layer.routing(T, k)[:2]]
+        np.testing.assert_allclose(w_g, w_o, rtol=2e-6, atol=0)
+        _check_grouping(layer, T, k, hi - lo, ids_o, w_g, lo)
+        shard = {n: np.ascontiguousarray(v[lo:hi]) for n, v in wq.items()}
+        _, ref, _ = oracle.moe_forward_routed(xb, ids_o, w_o, lo, shard["w1"], shard["w1s"], shard["w2"],
+                                              shard["w2s"], act)
+        got = part.double().cpu()
+        assert helpers.rel_frobenius(got.numpy(), ref) <= helpers.TOL_REL_FRO
+        assert helpers.max_abs_over_rms(got.numpy(), ref) <= helpers.TOL_MAX_OVER_RMS
+        total += got
+        layer.close()
+    inp = dict(xb=xb, logits=logits, **wq)
+    ref_all, _, _ = helpers.oracle_forward(inp, k, act)
+    assert helpers.rel_frobenius(total.numpy(), ref_all) <= helpers.TOL_REL_FRO
+    assert helpers.max_abs_over_rms(total.numpy(), ref_all) <= helpers.TOL_MAX_OVER_RMS
+    # the shard of all experts, bf16 output: the bits of moe_mx_forward
+    layer = moe_mx.MoeMxLayer(wl.H, wl.I, E, T, k)
+    d = _dev(wq)
+    full = layer.forward(x.cuda(), logits.cuda(), d["w1"], d["w1s"], d["w2"], d["w2s"], k, act)
+    sh = layer.forward_shard(x.cuda(), logits.cuda(), d["w1"], d["w1s"], d["w2"], d["w2s"], k, 0, act,
+                             moe_mx.MOE_MX_OUT_BF16)
+    assert layer.sync_status() == moe_mx.MOE_MX_OK, moe_mx.moe_mx_last_error()
+    assert torch.equal(full.view(torch.int16), sh.view(torch.int16))
+    layer.close()
+
+
+def test_shard_form_rejects_bad_shards():
+    layer = moe_mx.MoeMxLayer(256, 128, 4, 8, 2)
+    x = torch.zeros(8, 256, dtype=torch.bfloat16, device="cuda")
+    lg = torch.zeros(8, 8, dtype=torch.float32, device="cuda")
+    w1 = torch.zeros(4, 256, 128, dtype=torch.uint8, device="cuda")
+    w1s = torch.full((4, 256, 8), 127, dtype=torch.uint8, device="cuda")
+    w2 = torch.zeros(4, 256, 64, dtype=torch.uint8, device="cuda")
+    w2s = torch.full((4, 256, 4), 127, dtype=torch.uint8, device="cuda")
+    out = torch.empty(8, 256, dtype=torch.float32, device="cuda")
+    for E_g, off in ((8, 5), (8, -1), (3, 0), (2000, 0)):   # shard beyond the layer, negative, too small, too many
+        with pytest.raises(moe_mx.MoeMxError) as ei:
+            moe_mx.moe_mx_forward_shard(layer.handle, x, lg, 8, E_g, off, w1, w1s, w2, w2s, 2, 0, out)
+        assert ei.value.code == moe_mx.MOE_MX_ERR_INVALID_ARG
+    layer.close()
+
+
 def _tokens(ids, E_local, offset, T, n_random=6):
     loc = (ids >= offset) & (ids < offset + E_local)
     n_local = loc.sum(axis=1)

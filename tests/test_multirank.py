@@ -115,6 +115,59 @@ def test_expert_parallel_partials_sum_to_the_layer(world):
         assert err <= 1e-6 * scale  # float32 rounding of the shards' sums only
 
 
+def _ep_logits_rank_main(rank, world, port, results):
+    """The logits-form chain (ep.ep_forward_logits) on one gloo rank, with the oracle standing in
+    for the rank's CUDA partial: every rank routes all tokens over all experts (the oracle's
+    router) and evaluates the pairs of its shard (the oracle's routed form at its offset)."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import oracle
+    from block_scaled_moe_softmax_b200 import ep, workloads
+    from tests import helpers
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        wl = workloads.Workload("ep_logits", 12, 64, 32, 8, 4, seed=9)
+        x = workloads.draw_x(wl)
+        logits = workloads.draw_logits(wl).numpy()
+        wq = helpers.quantize_weights_cpu(wl)
+        xb = workloads.bf16_bits(x)
+
+        def partial(offset, n):
+            ids, w = oracle.route(logits, wl.top_k)
+            shard = {k: np.ascontiguousarray(v[offset:offset + n]) for k, v in wq.items()}
+            _, part, _ = oracle.moe_forward_routed(xb, ids, w, offset, shard["w1"], shard["w1s"], shard["w2"],
+                                                   shard["w2s"])
+            return torch.from_numpy(part).to(torch.float32)
+
+        total = ep.ep_forward_logits(None, None, None, None, None, None, None, wl.top_k, wl.E, rank, world,
+                                     partial_fn=partial)
+        _, _, _, full = oracle.moe_forward(xb, logits, wq["w1"], wq["w1s"], wq["w2"], wq["w2s"], wl.top_k,
+                                           exact=True)
+        results[rank] = (float(np.abs(total.double().numpy() - full).max()), float(np.abs(full).max()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_expert_parallel_logits_chain_sums_to_the_layer(world):
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    results = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_ep_logits_rank_main, args=(r, world, port, results)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=300)
+        assert p.exitcode == 0
+    for r in range(world):
+        err, scale = results[r]
+        assert err <= 1e-6 * scale  # float32 rounding of the shards' sums only
+
+
 def test_shard_range():
     sys.path.insert(0, ROOT)
     from block_scaled_moe_softmax_b200 import ep
