@@ -328,6 +328,14 @@ def fc1_algorithmic_bytes(wl, counts):
     return w + P * wl.H * 2 + P * wl.I * 2, hit
 
 
+def fc2_algorithmic_bytes(wl, counts):
+    """FC2's bytes: the hit experts' W2 codes and scales, h rows read (bf16-equivalent) and the
+    float32 Y rows written."""
+    hit = int((counts > 0).sum())
+    P = int(counts.sum())
+    return hit * (wl.I * wl.H // 2 + wl.I * wl.H // 32) + P * wl.I * 2 + P * wl.H * 4
+
+
 def layer_weight_bytes(wl, hit):
     return hit * (3 * wl.I * wl.H // 2 + 3 * wl.I * wl.H // 32)
 
@@ -510,6 +518,13 @@ def measure(args, wl, weights, world, rank, with_e2e=True):
                "d2h_bytes_per_step": wl.T * wl.H * out.element_size()}
 
     fc1_ms = stage["fc1"]
+    kernel_name = "fc_gemm_kernel (FC1 + SwiGLU)"
+    if stage["fc2"] < 1e-3 <= fc1_ms:
+        # up to 16 tokens the library runs FC1 and FC2 as one launch (two phases): the roofline
+        # kernel is that launch, with both GEMMs' work
+        kernel_name = "fc_gemm_kernel (FC1 + SwiGLU, then FC2, one launch)"
+        fc1_bytes += fc2_algorithmic_bytes(wl, counts)
+        fc1_flops *= 1.5
     layer_bytes = layer_weight_bytes(wl, hit)
     # FC1 is bound by whichever of its weight stream and its MMA work takes longer at the
     # measured peaks.  The tensor peak is the bf16 one (the w4a16 path's two-term MXFP8
@@ -519,21 +534,21 @@ def measure(args, wl, weights, world, rank, with_e2e=True):
     traffic = traffic_record(wl, fc1_bytes)
     if fc1_flops / (mma_peak * 1e12) > fc1_bytes / (hbm_peak * 1e9):
         achieved = fc1_flops / (fc1_ms / 1000.0) / 1e12
-        roofline = {"bound": "tensor", "kernel": "fc_gemm_kernel (FC1 + SwiGLU)", "achieved": achieved,
+        roofline = {"bound": "tensor", "kernel": kernel_name, "achieved": achieved,
                     "peak": mma_peak, "unit": "TFLOP/s", "frac": achieved / mma_peak, "traffic": traffic,
                     "peak_source": f"{peak_src} sustained cuBLAS bf16 GEMM"
                                    + (" x 2 (MXFP8 / bf16 nominal ratio)" if wl.act == "mxfp8" else ""),
                     "algorithmic_flops_per_launch": fc1_flops, "algorithmic_bytes_per_launch": fc1_bytes}
     else:
         achieved = fc1_bytes / (fc1_ms / 1000.0) / 1e9
-        roofline = {"bound": "hbm", "kernel": "fc_gemm_kernel (FC1 + SwiGLU)", "achieved": achieved,
+        roofline = {"bound": "hbm", "kernel": kernel_name, "achieved": achieved,
                     "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": traffic,
                     "peak_source": f"{peak_src} HBM copy bandwidth",
                     "algorithmic_bytes_per_launch": fc1_bytes}
     # the whole step against the same bound: weight bytes of the hit experts (FC1 + FC2), or
     # the MMA work of both GEMMs (2 * pairs * 3I * H)
     if roofline["bound"] == "tensor":
-        layer_flops = 1.5 * fc1_flops
+        layer_flops = 6.0 * int(counts.sum()) * wl.I * wl.H
         layer_roofline = {"bound": "tensor", "flops": layer_flops,
                           "achieved_tflops": layer_flops / (ms_all / 1000.0) / 1e12,
                           "frac": layer_flops / (ms_all / 1000.0) / 1e12 / mma_peak}

@@ -142,12 +142,14 @@ struct moe_mx_handle {
     int pdl;       // launch the kernels after the router as programmatic dependents (MOE_MX_PDL, default 1)
     int wide;      // 128-row GEMM blocks: the two-tile (N = 256) variant (MOE_MX_WIDE, default 1)
     int fuse_combine; // small batches: the combine runs in FC2's epilogue (MOE_MX_FUSE_COMBINE, default 1)
+    int two_phase;    // up to 16 tokens: FC1 and FC2 in one launch (MOE_MX_TWO_PHASE, default 1)
     int scale_layout; // MOE_MX_SCALES_ROW_MAJOR or MOE_MX_SCALES_TILED
     unsigned long long timeout_ns;
     void *ws;
     int32_t *topk_ids, *chunk_hist, *counts, *pad_offsets, *num_rowblocks, *sorted_pair, *pos_of_pair;
     int32_t *unit_counters;
     int32_t *combine_cnt; // [max_tokens][H/128] pairs of each token and FC2 weight tile done (fused combine)
+    int32_t *rb_done;     // [max_rows/16] FC1 units done per row block (two-phase launch)
     float *topk_w;
     int4 *rowblocks;
     uint8_t *Aq, *Asf, *Hq, *Hsf; // MXFP8 operand planes [2][rows][K] and their scale atoms
@@ -246,6 +248,7 @@ int moe_mx_create_ex(moe_mx_handle **out, int hidden, int inter, int num_experts
     h->pdl = env_int("MOE_MX_PDL", 1) != 0;
     h->wide = env_int("MOE_MX_WIDE", 1) != 0;
     h->fuse_combine = env_int("MOE_MX_FUSE_COMBINE", 1) != 0;
+    h->two_phase = env_int("MOE_MX_TWO_PHASE", 1) != 0;
     h->swap_rows = env_int("MOE_MX_SWAP_ROWS", 64);
     if (h->swap_rows < 0)
         h->swap_rows = 0;
@@ -267,6 +270,7 @@ int moe_mx_create_ex(moe_mx_handle **out, int hidden, int inter, int num_experts
         {(void **)&h->num_rowblocks, sizeof(int32_t)},
         {(void **)&h->unit_counters, 2 * sizeof(int32_t)}, // FC1, FC2 work-unit counters
         {(void **)&h->combine_cnt, sizeof(int32_t) * max_tokens * (hidden / 128)},
+        {(void **)&h->rb_done, sizeof(int32_t) * (h->max_rows / 16)},
         {(void **)&h->sorted_pair, sizeof(int32_t) * h->max_rows},
         {(void **)&h->pos_of_pair, sizeof(int32_t) * pairs},
         {(void **)&h->err, sizeof(uint32_t)},
@@ -452,6 +456,15 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
         ra.n_shared = h->S;
         ra.shard = route_E > 0;
         ra.route_E = route_E;
+        // Up to 16 tokens routed from logits (the k experts of a token distinct), every expert's
+        // pairs fit one 16-row block: FC1 and FC2 then run as one launch (two phases), FC2's units
+        // waiting for their row block's FC1 units through rb_done, which the routing kernel (one
+        // CTA at this size) zeroes.  Row blocks: at most one per expert slot hit.
+        const bool two = h->two_phase && !given_ids && tile_rows == 16 && T <= 16 && T <= kSmallRouteTokens;
+        if (two) {
+            ra.zero_words = h->rb_done;
+            ra.zero_n = (int)((int64_t)T * k < E ? (int64_t)T * k : E);
+        }
         // Each kernel after the router may launch while its predecessor still runs (programmatic
         // dependent launch): the FC GEMMs start streaming their weights early.  Stage timing
         // records events between the kernels, so timed forwards launch them one after another.
@@ -488,8 +501,9 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
         f1.wide = h->wide;
         mark(2);
         const int sw_idx = tile_rows <= 16 ? 0 : tile_rows <= 32 ? 1 : 2; // box rows min(tile rows, 64)
-        launch_fc_gemm(f1, h->map_A[f1.terms - 1], h->map_Asw[f1.terms - 1][sw_idx], h->map_A16, h->map_w1, h->num_sms,
-                       s, pdl);
+        if (!two)
+            launch_fc_gemm(f1, h->map_A[f1.terms - 1], h->map_Asw[f1.terms - 1][sw_idx], h->map_A16, h->map_w1,
+                           h->num_sms, s, pdl);
         mark(3);
 
         FcGemmArgs f2 = f1;
@@ -513,12 +527,23 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
         f2.k = k;
         f2.out = static_cast<__nv_bfloat16 *>(out);
         // the maps' plane count must equal the copy's terms: the stage barrier expects exactly those bytes
-        launch_fc_gemm(f2, h->map_H[f2.terms - 1], h->map_Hsw[f2.terms - 1][sw_idx], h->map_H16, h->map_w2,
-                       h->num_sms, s, pdl);
+        if (two) {
+            // one launch, one work-unit counter: FC1's units first, then FC2's
+            f1.rb_done = f2.rb_done = h->rb_done;
+            f2.unit_counter = f1.unit_counter;
+            const CUtensorMap m1[4] = {h->map_A[f1.terms - 1], h->map_Asw[f1.terms - 1][sw_idx], h->map_A16,
+                                       h->map_w1};
+            const CUtensorMap m2[4] = {h->map_H[f2.terms - 1], h->map_Hsw[f2.terms - 1][sw_idx], h->map_H16,
+                                       h->map_w2};
+            launch_fc_gemm_two_phase(f1, m1, f2, m2, h->num_sms, s, pdl);
+        } else {
+            launch_fc_gemm(f2, h->map_H[f2.terms - 1], h->map_Hsw[f2.terms - 1][sw_idx], h->map_H16, h->map_w2,
+                           h->num_sms, s, pdl);
+        }
         mark(4);
         if (!fuse)
             launch_combine(h->Y, T, H, k, h->pos_of_pair, h->topk_w, out, out_f32, h->num_sms, s, pdl);
-        h->launches += fuse ? 3 : 4; // gather, FC1, FC2 (+ combine)
+        h->launches += 1 + (two ? 1 : 2) + (fuse ? 0 : 1); // gather, FC1 and FC2 (one launch or two), combine
         ce = cudaGetLastError();
         if (ce != cudaSuccess) {
             rc = cuda_fail(ce, "kernel launch");

@@ -167,8 +167,10 @@ template <int kStages> struct UnitRing {
             mbar_arrive(bars.ring_empty(r));
         return v;
     }
-    // Scheduler (one lane): publish the CTA's j-th unit; false once the work is exhausted.
-    __device__ bool fill(uint32_t j, const FcGemmArgs &a, int total_units, int n_groups, unsigned long long tmo) const
+    // Scheduler (one lane): publish the CTA's j-th unit; false once the work is exhausted.  Units
+    // [0, units0) belong to phase 0 (n_groups0 per row block), the rest to phase 1.
+    __device__ bool fill(uint32_t j, const FcGemmArgs &a, int total_units, int units0, int n_groups0,
+                         int n_groups1, unsigned long long tmo) const
     {
         const int r = (int)(j % kRing);
         const bool got = mbar_wait_bounded(bars.ring_empty(r), ((j / kRing) & 1) ^ 1, a.err, tmo);
@@ -177,7 +179,7 @@ template <int kStages> struct UnitRing {
         if (u >= total_units)
             u = -1;
         if (u >= 0)
-            blk = a.rowblocks[u / n_groups];
+            blk = a.rowblocks[u < units0 ? u / n_groups0 : (u - units0) / n_groups1];
         slots[4 * r] = blk.x;
         slots[4 * r + 1] = blk.y;
         slots[4 * r + 2] = blk.z;
@@ -305,15 +307,49 @@ __device__ __forceinline__ void fused_combine_unit(const FcGemmArgs &a, const in
     named_bar_sync(1, 128); // the list is rewritten by the next unit
 }
 
-// Per-CTA state the warp roles share (all values are CTA-uniform).
+// Per-CTA state the warp roles share (all values are CTA-uniform).  A launch runs one phase (one
+// GEMM) or two (FC1's units, then FC2's): per phase its arguments, tensor maps, work units per
+// row block (tile groups), K stages and activation terms; a unit's phase follows from its index.
 struct Ctx {
     uint32_t base;        // shared-memory base (1024-byte aligned, shared window)
     volatile int *units;  // the work-unit ring (generic pointer to shared memory)
     uint8_t *ystage;      // wide variant: the epilogue warps' FC2 staging buffers (shared memory)
     uint32_t tmem_base;
-    int total_units, n_groups, kst, terms; // n_groups: work units per row block (tile groups)
+    int total_units, units0; // all units; those of phase 0 (units0 == total_units: one phase)
+    const FcGemmArgs *args[2];
+    const CUtensorMap *maps[2][4]; // act_map, act_map_sw, act_map16, w_map
+    int n_groups[2], kst[2], terms[2];
     unsigned long long tmo;
+    uint32_t *err;
+    __device__ int phase(int u) const { return u >= units0 ? 1 : 0; }
+    __device__ int local(int u) const { return u >= units0 ? u - units0 : u; } // index within its phase
 };
+
+// Bounded wait (one thread) until *count >= target, read with acquire semantics at GPU scope, then
+// a proxy fence so that the caller's later TMA reads (async proxy) see what the counted writers
+// stored before counting.  False (and the error word set) if the limit ran out.
+__device__ __forceinline__ bool wait_count(const int32_t *count, int target, uint32_t *err,
+                                           unsigned long long timeout_ns)
+{
+    const long long t0 = clock64();
+    for (uint32_t it = 0;; ++it) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(count) : "memory");
+        if (v >= target)
+            break;
+        if ((it & 63) == 63) {
+            const unsigned long long dt = (unsigned long long)(clock64() - t0);
+            if (dt > 100000ull && *(volatile uint32_t *)err != 0)
+                return false;
+            if (dt > timeout_ns) {
+                atomicOr(err, kErrTimeout);
+                return false;
+            }
+        }
+    }
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    return true;
+}
 
 // Producer role, one of kProd warps taking stages g with g % kProd == PI (PI is a
 // compile-time role index so that every operand of the TMA issue stays warp-uniform).
@@ -325,9 +361,7 @@ struct Ctx {
 // the activation copies measured slower: the extra paths cost the steady-state loop more than
 // the early weights gained.)
 template <int kActRows, int kMmaW, int kWTiles, int kTm, int PI>
-__device__ __forceinline__ void producer_role(const FcGemmArgs &a, const Ctx &c, const CUtensorMap *act_map,
-                                              const CUtensorMap *act_map_sw, const CUtensorMap *act_map16,
-                                              const CUtensorMap *w_map, int lane)
+__device__ __forceinline__ void producer_role(const Ctx &c, int lane)
 {
     using P = Plan<kActRows, kMmaW, kWTiles, kTm>;
     constexpr int kStages = P::kStages, kProd = P::kProd, kWT = P::kWT;
@@ -335,18 +369,25 @@ __device__ __forceinline__ void producer_role(const FcGemmArgs &a, const Ctx &c,
     constexpr int kOffAct = P::kOffAct, kOffW = P::kOffW, kOffAsf = P::kOffAsf, kOffWsf = P::kOffWsf;
     const Bars<kStages> bars{c.base + P::kOffBar};
     const uint32_t base = c.base;
-    const int kst = c.kst, terms = c.terms;
     const unsigned long long tmo = c.tmo;
     uint32_t g = 0;
     bool ok = true;
-    const int scl_ld = a.K / 32;
     const UnitRing<kStages> ring{bars, c.units};
     grid_dep_wait();
     for (uint32_t i = 0; ok; ++i) {
-        const int4 blk = ring.take(i, a.err, tmo, lane);
+        const int4 blk = ring.take(i, c.err, tmo, lane);
         if (blk.w < 0)
             break;
-        const int nt0 = (blk.w % c.n_groups) * kWT; // the unit's first weight tile
+        const int ph = c.phase(blk.w), u = c.local(blk.w);
+        const FcGemmArgs &a = *c.args[ph];
+        const CUtensorMap *act_map = c.maps[ph][0], *act_map_sw = c.maps[ph][1], *act_map16 = c.maps[ph][2],
+                          *w_map = c.maps[ph][3];
+        const int kst = c.kst[ph], terms = c.terms[ph], scl_ld = a.K / 32;
+        // the unit's fields the stage loop reads, in registers
+        const bool fc1 = a.fc1 != 0, wsf_tiled = a.wsf_tiled != 0;
+        const int R = a.R, act_rows = a.act_rows;
+        const uint8_t *const wscale = a.wscale, *const act_sf = a.act_sf;
+        const int nt0 = (u % c.n_groups[ph]) * kWT; // the unit's first weight tile
         const bool swap = !P::kWide && (kActRows < 128 || blk.z <= a.swap_rows); // wide: tokens on M always
         const int npad = (blk.z + 15) & ~15;
         const bool comb = swap && terms > 1 && npad <= P::kT2; // both terms on N of one MMA
@@ -363,11 +404,22 @@ __device__ __forceinline__ void producer_role(const FcGemmArgs &a, const Ctx &c,
                             (a.wsf_tiled ? kWT * 512u : 0u);
         // tiled weight scales: the first tile's atoms, one per K stage, then the next tile's
         const uint8_t *wsf_tile = a.wscale + ((size_t)blk.x * a.n_tiles + nt0) * (size_t)kst * 512;
+        // the second phase of a two-phase launch (FC2) reads h, which the first phase (FC1) writes:
+        // it starts only once every FC1 unit of its row block has been counted
+        if (ph == 1 && a.rb_done) {
+            bool mine = true;
+            if (elect_one())
+                mine = wait_count(a.rb_done + u / c.n_groups[1], c.n_groups[0], c.err, tmo);
+            if (!__all_sync(0xFFFFFFFFu, mine)) {
+                ok = false;
+                break;
+            }
+        }
         for (int kk = 0; kk < kst; ++kk, ++g) {
             if ((int)(g % kProd) != PI)
                 continue; // another producer warp fills this stage
             const int s = g % kStages;
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.empty(s), ((g / kStages) & 1) ^ 1, a.err, tmo))) {
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.empty(s), ((g / kStages) & 1) ^ 1, c.err, tmo))) {
                 ok = false;
                 break;
             }
@@ -379,7 +431,7 @@ __device__ __forceinline__ void producer_role(const FcGemmArgs &a, const Ctx &c,
             const uint32_t wdst = base + kOffW + s * P::kWStage;
             const uint32_t wsf = base + kOffWsf + s * P::kWsfStage;
             const uint32_t asf_dst = base + kOffAsf + s * kAsfBytes;
-            const uint8_t *asf_src = a.act_sf + ((size_t)rb * kst + kk) * 1024;
+            const uint8_t *asf_src = act_sf + ((size_t)rb * kst + kk) * 1024;
             const int kx = kk * 128;
             if (elect_one()) {
                 mbar_arrive_expect_tx(full_s, tx);
@@ -387,11 +439,11 @@ __device__ __forceinline__ void producer_role(const FcGemmArgs &a, const Ctx &c,
                 // 3-D box; FC2 = rows [128 nt, 128 nt + 128), one box
                 for (int wt = 0; wt < kWT; ++wt) {
                     const int nt = nt0 + wt;
-                    if (a.fc1)
+                    if (fc1)
                         tma_load_3d(wdst + wt * kWBytes, w_map, kx, nt * 64, 2 * blk.x, full_s);
                     else
-                        tma_load_2d(wdst + wt * kWBytes, w_map, kx, blk.x * a.R + nt * 128, full_s);
-                    if (a.wsf_tiled)
+                        tma_load_2d(wdst + wt * kWBytes, w_map, kx, blk.x * R + nt * 128, full_s);
+                    if (wsf_tiled)
                         bulk_copy_g2s(wsf + wt * kWsfBytes, wsf_tile + ((size_t)wt * kst + kk) * 512, 512u, full_s);
                 }
                 if (!swap) {
@@ -403,20 +455,20 @@ __device__ __forceinline__ void producer_role(const FcGemmArgs &a, const Ctx &c,
                     for (int r16 = 0; r16 < npad; r16 += 16) {
                         tma_load_2d(act + r16 * 128, act_map16, kx, blk.y + r16, full_s);
                         if (terms > 1)
-                            tma_load_2d(act + kTermBytes + r16 * 128, act_map16, kx, a.act_rows + blk.y + r16, full_s);
+                            tma_load_2d(act + kTermBytes + r16 * 128, act_map16, kx, act_rows + blk.y + r16, full_s);
                     }
                 }
             }
             __syncwarp();
-            if (!a.wsf_tiled) // weight scale bytes: 4 per row (the stage's 4 blocks) into the atom layout
+            if (!wsf_tiled) // weight scale bytes: 4 per row (the stage's 4 blocks) into the atom layout
                 for (int wt = 0; wt < kWT; ++wt) {
                     const int nt = nt0 + wt;
                     // tile rows as two 64-row halves: FC1 gate rows then the matching up rows
-                    const int wrow_a = blk.x * a.R + (a.fc1 ? nt * 64 : nt * 128);
-                    const int wrow_b = a.fc1 ? wrow_a + a.R / 2 : wrow_a + 64;
+                    const int wrow_a = blk.x * R + (fc1 ? nt * 64 : nt * 128);
+                    const int wrow_b = fc1 ? wrow_a + R / 2 : wrow_a + 64;
                     for (int r = lane; r < 128; r += 32) {
                         const int wr = r < 64 ? wrow_a + r : wrow_b + (r - 64);
-                        cp_async_4(wsf + wt * kWsfBytes + sf_atom_offset(r, 0), a.wscale + (size_t)wr * scl_ld + kk * 4);
+                        cp_async_4(wsf + wt * kWsfBytes + sf_atom_offset(r, 0), wscale + (size_t)wr * scl_ld + kk * 4);
                     }
                 }
             if (swap) {
@@ -443,12 +495,13 @@ __device__ __forceinline__ void producer_role(const FcGemmArgs &a, const Ctx &c,
 // counter and publishes them kLook units ahead of the first reader, off the producers' path
 // (the counter is a global atomic: a round trip of about a microsecond per unit).
 template <int kActRows, int kMmaW, int kWTiles, int kTm>
-__device__ __forceinline__ void scheduler_role(const FcGemmArgs &a, const Ctx &c, int lane)
+__device__ __forceinline__ void scheduler_role(const Ctx &c, int lane)
 {
     using P = Plan<kActRows, kMmaW, kWTiles, kTm>;
     const UnitRing<P::kStages> ring{Bars<P::kStages>{c.base + P::kOffBar}, c.units};
     if (lane == 0)
-        for (uint32_t j = 0; ring.fill(j, a, c.total_units, c.n_groups, c.tmo); ++j) {
+        for (uint32_t j = 0;
+             ring.fill(j, *c.args[0], c.total_units, c.units0, c.n_groups[0], c.n_groups[1], c.tmo); ++j) {
         }
     __syncwarp();
 }
@@ -456,7 +509,7 @@ __device__ __forceinline__ void scheduler_role(const FcGemmArgs &a, const Ctx &c
 // MMA role: warp 1 (MI = 0) and, with kMma = 2, warp 7 (MI = 1), taking stages g with
 // g % kMma == MI.  The whole warp runs the loop, one elected lane issues.
 template <int kActRows, int kMmaW, int kWTiles, int kTm, int MI>
-__device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
+__device__ __forceinline__ void mma_role(const Ctx &c)
 {
     using P = Plan<kActRows, kMmaW, kWTiles, kTm>;
     constexpr int kStages = P::kStages, kMma = P::kMma, kWT = P::kWT;
@@ -464,7 +517,6 @@ __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
     constexpr int kOffAct = P::kOffAct, kOffW = P::kOffW, kOffAsf = P::kOffAsf, kOffWsf = P::kOffWsf;
     const Bars<kStages> bars{c.base + P::kOffBar};
     const uint32_t base = c.base, tmem_base = c.tmem_base;
-    const int kst = c.kst, terms = c.terms;
     const unsigned long long tmo = c.tmo;
     uint32_t g = 0, cnt = 0;
     bool ok = true;
@@ -478,9 +530,12 @@ __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
     const UnitRing<kStages> ring{bars, c.units};
     const int lane = threadIdx.x & 31;
     for (; ok; ++cnt) {
-        const int4 blk = ring.take(cnt, a.err, tmo, lane);
+        const int4 blk = ring.take(cnt, c.err, tmo, lane);
         if (blk.w < 0)
             break;
+        const int phs = c.phase(blk.w); // the unit's phase (FC1 or FC2 in a two-phase launch)
+        const FcGemmArgs &a = *c.args[phs];
+        const int kst = c.kst[phs], terms = c.terms[phs];
         const bool swap = kActRows < 128 || blk.z <= a.swap_rows;
         const uint32_t npad = (uint32_t)((blk.z + 15) & ~15);
         const bool comb = swap && terms > 1 && npad <= (uint32_t)P::kT2;
@@ -500,7 +555,7 @@ __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
             }
         const int buf = cnt & 1;
         if (!__all_sync(0xFFFFFFFFu,
-                        mbar_wait_bounded(bars.acc_empty(buf), ((cnt >> 1) & 1) ^ 1, a.err, tmo))) {
+                        mbar_wait_bounded(bars.acc_empty(buf), ((cnt >> 1) & 1) ^ 1, c.err, tmo))) {
             ok = false;
             break;
         }
@@ -542,7 +597,7 @@ __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
                 }
             }
             const uint32_t empty_s = bars.empty(s);
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.full(s), ph, a.err, tmo))) {
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.full(s), ph, c.err, tmo))) {
                 ok = false;
                 break;
             }
@@ -586,13 +641,13 @@ __device__ __forceinline__ void mma_role(const FcGemmArgs &a, const Ctx &c)
 // single accumulator at TMEM columns 0..255.  Scale factors: the two weight atoms at kSfCol and
 // kSfCol + 4 (rows 0..127 and 128..255 of N), the activation atoms after them.
 template <int kActRows, int kMmaW, int kWTiles, int kTm>
-__device__ __forceinline__ void mma_role_wide(const FcGemmArgs &a, const Ctx &c)
+__device__ __forceinline__ void mma_role_wide(const Ctx &c)
 {
     using P = Plan<kActRows, kMmaW, kWTiles, kTm>;
     constexpr int kStages = P::kStages, kTermBytes = P::kTermBytes, kActBytes = P::kActBytes;
     const Bars<kStages> bars{c.base + P::kOffBar};
     const uint32_t base = c.base, tmem_base = c.tmem_base;
-    const int kst = c.kst, terms = c.terms;
+    const int kst = c.kst[0], terms = c.terms[0]; // one phase
     const unsigned long long tmo = c.tmo;
     uint32_t g = 0, cnt = 0;
     bool ok = true;
@@ -603,11 +658,11 @@ __device__ __forceinline__ void mma_role_wide(const FcGemmArgs &a, const Ctx &c)
     const UnitRing<kStages> ring{bars, c.units};
     const int lane = threadIdx.x & 31;
     for (; ok; ++cnt) {
-        const int4 blk = ring.take(cnt, a.err, tmo, lane);
+        const int4 blk = ring.take(cnt, c.err, tmo, lane);
         if (blk.w < 0)
             break;
         // the accumulator is free once the epilogue has copied the previous unit's out of TMEM
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.acc_empty(0), (cnt & 1) ^ 1, a.err, tmo))) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.acc_empty(0), (cnt & 1) ^ 1, c.err, tmo))) {
             ok = false;
             break;
         }
@@ -631,7 +686,7 @@ __device__ __forceinline__ void mma_role_wide(const FcGemmArgs &a, const Ctx &c)
                     opa[k32][t] = ds_act + (uint64_t)((t * kTermBytes) >> 4) + 2u * k32;
             }
             const uint32_t empty_s = bars.empty(s);
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.full(s), ph, a.err, tmo))) {
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.full(s), ph, c.err, tmo))) {
                 ok = false;
                 break;
             }
@@ -669,20 +724,21 @@ __device__ __forceinline__ void mma_role_wide(const FcGemmArgs &a, const Ctx &c)
 // columns to registers, releases the accumulator, then forms its output (FC1: h = silu(gate) *
 // up for the tile's 64 gate / 64 up rows, written as FC2's operand; FC2: f32 rows of Y).
 template <int kActRows, int kMmaW, int kWTiles, int kTm>
-__device__ __forceinline__ void epilogue_wide(const FcGemmArgs &a, const Ctx &c, int warp, int lane)
+__device__ __forceinline__ void epilogue_wide(const Ctx &c, int warp, int lane)
 {
+    const FcGemmArgs &a = *c.args[0]; // one phase
     using P = Plan<kActRows, kMmaW, kWTiles, kTm>;
     const Bars<P::kStages> bars{c.base + P::kOffBar};
     const UnitRing<P::kStages> ring{bars, c.units};
     const int q = warp & 3;                     // TMEM lane quarter this warp may access
     const int half = warp >= P::kEpi2 ? 1 : 0;  // the unit's weight tile this warp writes
     for (uint32_t cnt = 0;; ++cnt) {
-        const int4 blk = ring.take(cnt, a.err, c.tmo, lane);
+        const int4 blk = ring.take(cnt, c.err, c.tmo, lane);
         // the eight epilogue warps leave together (they share named barrier 2)
         if (!named_bar_all(2, 256, blk.w >= 0))
             break;
-        const int nt = (blk.w % c.n_groups) * 2 + half;
-        const bool got = mbar_wait_bounded(bars.acc_full(0), cnt & 1, a.err, c.tmo);
+        const int nt = (blk.w % c.n_groups[0]) * 2 + half;
+        const bool got = mbar_wait_bounded(bars.acc_full(0), cnt & 1, c.err, c.tmo);
         if (!named_bar_all(2, 256, got))
             break;
         tc_fence_after();
@@ -744,9 +800,11 @@ __device__ __forceinline__ void epilogue_wide(const FcGemmArgs &a, const Ctx &c,
 
 template <int kActRows, int kMmaW, int kWTiles, int kTm>
 __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads, 1)
-    fc_gemm_kernel(const FcGemmArgs a, const __grid_constant__ CUtensorMap act_map,
-                   const __grid_constant__ CUtensorMap act_map_sw, const __grid_constant__ CUtensorMap act_map16,
-                   const __grid_constant__ CUtensorMap w_map)
+    fc_gemm_kernel(const __grid_constant__ FcGemmArgs a0, const __grid_constant__ FcGemmArgs a1,
+                   const __grid_constant__ CUtensorMap act_map, const __grid_constant__ CUtensorMap act_map_sw,
+                   const __grid_constant__ CUtensorMap act_map16, const __grid_constant__ CUtensorMap w_map,
+                   const __grid_constant__ CUtensorMap act_map1, const __grid_constant__ CUtensorMap act_map_sw1,
+                   const __grid_constant__ CUtensorMap act_map16_1, const __grid_constant__ CUtensorMap w_map1)
 {
     using P = Plan<kActRows, kMmaW, kWTiles, kTm>;
     constexpr int kStages = P::kStages;
@@ -780,6 +838,12 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads,
         prefetch_tensormap(&act_map_sw);
         prefetch_tensormap(&act_map16);
         prefetch_tensormap(&w_map);
+        if (a0.rb_done) { // two phases: FC2's maps too
+            prefetch_tensormap(&act_map1);
+            prefetch_tensormap(&act_map_sw1);
+            prefetch_tensormap(&act_map16_1);
+            prefetch_tensormap(&w_map1);
+        }
     }
     if (warp == 1) {
         tmem_alloc(base + kOffTmemSlot, kTmemCols);
@@ -795,52 +859,78 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads,
     if (threadIdx.x == 0)
         grid_dep_launch();
 
-    const int nrb = *a.num_rowblocks;
-    const int n_groups = a.n_tiles / P::kWT; // the launch guarantees n_tiles % kWT == 0
-    const int total_units = nrb * n_groups;
-    const int kst = a.K / 128; // K stages of 128 elements (4 scale blocks)
-    const int terms = kTm == 1 ? 1 : a.terms; // activation terms per row: 1 (w4a8) or 2 (w4a16)
-    const unsigned long long tmo = a.timeout_ns;
-
-    const Ctx ctx{base, reinterpret_cast<volatile int *>(gsm + P::kOffUnits), gsm + P::kOffY, tmem_base, total_units,
-                  n_groups, kst, terms, tmo};
+    // one phase (a0 alone), or two (a0 = FC1, a1 = FC2; only such launches carry rb_done)
+    const bool two = a0.rb_done != nullptr;
+    const int nrb = *a0.num_rowblocks;
+    const unsigned long long tmo = a0.timeout_ns;
+    Ctx ctx;
+    ctx.base = base;
+    ctx.units = reinterpret_cast<volatile int *>(gsm + P::kOffUnits);
+    ctx.ystage = gsm + P::kOffY;
+    ctx.tmem_base = tmem_base;
+    ctx.args[0] = &a0;
+    ctx.args[1] = two ? &a1 : &a0;
+    ctx.maps[0][0] = &act_map;
+    ctx.maps[0][1] = &act_map_sw;
+    ctx.maps[0][2] = &act_map16;
+    ctx.maps[0][3] = &w_map;
+    ctx.maps[1][0] = two ? &act_map1 : &act_map;
+    ctx.maps[1][1] = two ? &act_map_sw1 : &act_map_sw;
+    ctx.maps[1][2] = two ? &act_map16_1 : &act_map16;
+    ctx.maps[1][3] = two ? &w_map1 : &w_map;
+    for (int ph = 0; ph < 2; ++ph) {
+        const FcGemmArgs &ap = *ctx.args[ph];
+        ctx.n_groups[ph] = ap.n_tiles / P::kWT;       // the launch guarantees n_tiles % kWT == 0
+        ctx.kst[ph] = ap.K / 128;                     // K stages of 128 elements (4 scale blocks)
+        ctx.terms[ph] = kTm == 1 ? 1 : ap.terms;      // activation terms per row: 1 (w4a8) or 2 (w4a16)
+    }
+    ctx.units0 = nrb * ctx.n_groups[0];
+    ctx.total_units = ctx.units0 + (two ? nrb * ctx.n_groups[1] : 0);
+    ctx.tmo = tmo;
+    ctx.err = a0.err;
     if (warp == 0) {
-        producer_role<kActRows, kMmaW, kWTiles, kTm, 0>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
+        producer_role<kActRows, kMmaW, kWTiles, kTm, 0>(ctx, lane);
     } else if (warp >= 6 && warp < 5 + kProd) {
         // further producer warps (compile-time role index: every TMA operand stays warp-uniform)
         if (warp == 6)
-            producer_role<kActRows, kMmaW, kWTiles, kTm, 1 % kProd>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
+            producer_role<kActRows, kMmaW, kWTiles, kTm, 1 % kProd>(ctx, lane);
         else if (warp == 7)
-            producer_role<kActRows, kMmaW, kWTiles, kTm, 2 % kProd>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
+            producer_role<kActRows, kMmaW, kWTiles, kTm, 2 % kProd>(ctx, lane);
         else if (warp == 8)
-            producer_role<kActRows, kMmaW, kWTiles, kTm, 3 % kProd>(a, ctx, &act_map, &act_map_sw, &act_map16, &w_map, lane);
+            producer_role<kActRows, kMmaW, kWTiles, kTm, 3 % kProd>(ctx, lane);
     } else if (warp == 1) {
         if constexpr (P::kWide)
-            mma_role_wide<kActRows, kMmaW, kWTiles, kTm>(a, ctx);
+            mma_role_wide<kActRows, kMmaW, kWTiles, kTm>(ctx);
         else
-            mma_role<kActRows, kMmaW, kWTiles, kTm, 0>(a, ctx);
+            mma_role<kActRows, kMmaW, kWTiles, kTm, 0>(ctx);
     } else if (P::kWide && ((warp >= 2 && warp < 6) || (warp >= P::kEpi2 && warp < P::kEpi2 + 4))) {
-        epilogue_wide<kActRows, kMmaW, kWTiles, kTm>(a, ctx, warp, lane);
+        epilogue_wide<kActRows, kMmaW, kWTiles, kTm>(ctx, warp, lane);
     } else if (kMma > 1 && warp == 5 + kProd) {
-        mma_role<kActRows, kMmaW, kWTiles, kTm, (kMma > 1 ? 1 : 0)>(a, ctx);
+        mma_role<kActRows, kMmaW, kWTiles, kTm, (kMma > 1 ? 1 : 0)>(ctx);
     } else if (warp == P::kThreads / 32 - 1) {
-        scheduler_role<kActRows, kMmaW, kWTiles, kTm>(a, ctx, lane);
+        scheduler_role<kActRows, kMmaW, kWTiles, kTm>(ctx, lane);
     } else if (warp >= 2 && warp < 6) {
         // ------------------------------------------------------------ epilogue (warps 2..5)
         const int q = warp & 3; // TMEM lane quarter this warp may access
         float *xch = reinterpret_cast<float *>(gsm + kOffX);
         const UnitRing<kStages> ring{bars, reinterpret_cast<volatile int *>(gsm + P::kOffUnits)};
+        uint32_t g_run = 0; // pipeline stages of the units before this one
         for (uint32_t cnt = 0;; ++cnt) {
-            const int4 blk = ring.take(cnt, a.err, tmo, lane);
+            const int4 blk = ring.take(cnt, ctx.err, tmo, lane);
             // the four epilogue warps leave together (they share named barriers below)
             if (!named_bar_all(2, 128, blk.w >= 0))
                 break;
-            const int nt0 = (blk.w % n_groups) * P::kWT; // the unit's first weight tile
+            const int phs = ctx.phase(blk.w), u = ctx.local(blk.w);
+            const FcGemmArgs &a = *ctx.args[phs];
+            const int kst = ctx.kst[phs], terms = ctx.terms[phs];
+            const uint32_t g0 = g_run; // the unit's first stage
+            g_run += (uint32_t)kst;
+            const int nt0 = (u % ctx.n_groups[phs]) * P::kWT; // the unit's first weight tile
             const int rows = blk.z;
             const bool swap = kActRows < 128 || rows <= a.swap_rows;
             const int buf = cnt & 1;
             // the four epilogue warps leave together or not at all (they share named barrier 1 below)
-            const bool got = mbar_wait_bounded(bars.acc_full(buf), (cnt >> 1) & 1, a.err, tmo);
+            const bool got = mbar_wait_bounded(bars.acc_full(buf), (cnt >> 1) & 1, ctx.err, tmo);
             if (!named_bar_all(2, 128, got))
                 break;
             tc_fence_after();
@@ -891,7 +981,6 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads,
                 const bool comb = terms > 1 && npad <= P::kT2;
                 // partial sums: per MMA warp with stages in this unit (with one K stage only the
                 // warp that took it), and per term when both terms sit side by side on N
-                const uint32_t g0 = cnt * (uint32_t)kst;
                 const bool acc0 = kMma == 1 || kst > 1 || (g0 & 1) == 0;
                 const bool acc1 = kMma > 1 && (kst > 1 || (g0 & 1) == 1);
                 for (int wt = 0; wt < P::kWT; ++wt) // each weight tile of the unit (64 columns apart)
@@ -945,6 +1034,16 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads,
             }
             tc_fence_before();
             mbar_arrive(bars.acc_empty(buf));
+            if (a.fc1 && a.rb_done) {
+                // two phases: count this FC1 unit done for its row block once every epilogue thread's h
+                // stores are visible device-wide (FC2's producers wait for the count, then copy h)
+                __threadfence();
+                named_bar_sync(1, 128);
+                if (q == 0 && lane == 0) {
+                    __threadfence();
+                    atomicAdd(a.rb_done + u / ctx.n_groups[0], 1);
+                }
+            }
             if (swap && !a.fc1 && a.fuse_combine)
                 fused_combine_unit(a, blk, nt0, P::kWT, 32 * q + lane, reinterpret_cast<int *>(xch));
         }
@@ -986,7 +1085,7 @@ static void launch_one(const FcGemmArgs &a, const CUtensorMap &act_map, const CU
 {
     using P = Plan<kActRows, kMmaW, kWTiles, kTm>;
     launch_kernel(fc_gemm_kernel<kActRows, kMmaW, kWTiles, kTm>, dim3(grid), dim3(P::kThreads), (size_t)P::kSmemBytes,
-                  s, pdl, a, act_map, act_map_sw, act_map16, w_map);
+                  s, pdl, a, a, act_map, act_map_sw, act_map16, w_map, act_map, act_map_sw, act_map16, w_map);
 }
 
 void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUtensorMap &act_map_sw,
@@ -1029,6 +1128,16 @@ void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUten
     } else {
         launch_one<128, 1, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
     }
+}
+
+void launch_fc_gemm_two_phase(const FcGemmArgs &a1, const CUtensorMap *maps1, const FcGemmArgs &a2,
+                              const CUtensorMap *maps2, int grid, cudaStream_t s, bool pdl)
+{
+    // tokens on N, 16-row blocks, two MMA warps: the small-batch FC1 variant serves both phases
+    // (FC2 units then take one weight tile each)
+    using P = Plan<16, 2, 1, 2>;
+    launch_kernel(fc_gemm_kernel<16, 2, 1, 2>, dim3(grid), dim3(P::kThreads), (size_t)P::kSmemBytes, s, pdl, a1, a2,
+                  maps1[0], maps1[1], maps1[2], maps1[3], maps2[0], maps2[1], maps2[2], maps2[3]);
 }
 
 // ---------------------------------------------------------------- watchdog self-test

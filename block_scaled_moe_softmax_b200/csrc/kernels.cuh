@@ -67,6 +67,9 @@ struct RouteGroupArgs {
     // logits are [T, route_E]) and keeps the E of [id_offset, id_offset + E), the rest -1.
     int shard = 0;
     int route_E = 0;
+    // optional: counts the one-CTA path zeroes (the FC GEMMs' per-row-block completion counts)
+    int32_t *zero_words = nullptr;
+    int zero_n = 0;
     __host__ __device__ int routeE() const { return shard ? route_E : E - n_shared; }
 };
 
@@ -124,6 +127,10 @@ struct FcGemmArgs {
     const float *topk_w;         // [T, k]
     int k;                       // slots per token
     __nv_bfloat16 *out;          // [T, H]
+    // One launch running FC1's units, then FC2's (launch_fc_gemm_two_phase): FC1's epilogue counts
+    // each row block's finished units in rb_done (zero before the forward), and an FC2 unit copies
+    // its row block's h only once all of them are counted.
+    int32_t *rb_done;
 };
 
 // Tensor maps: act_map = both term planes, 128-row boxes ([terms][128][128] codes, tokens
@@ -133,6 +140,12 @@ struct FcGemmArgs {
 void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUtensorMap &act_map_sw,
                     const CUtensorMap &act_map16, const CUtensorMap &w_map, int grid, cudaStream_t s, bool pdl = false);
 cudaError_t fc_gemm_prepare();
+// FC1 (a1, with its maps) and FC2 (a2) in one persistent launch, for row blocks of at most 16 rows:
+// the work units of FC1 come first, those of FC2 after them, and an FC2 unit waits (bounded) until
+// FC1 has finished every unit of its row block.  Both args carry the same rowblocks, rb_done,
+// unit counter (one) and error word.
+void launch_fc_gemm_two_phase(const FcGemmArgs &a1, const CUtensorMap *maps1, const FcGemmArgs &a2,
+                              const CUtensorMap *maps2, int grid, cudaStream_t s, bool pdl);
 
 // Rearrange row-major E8M0 weight scales [E][R][K/32] into the tiled atom layout the GEMM reads:
 // for expert e, 128-row weight tile nt and K stage kk (128 elements), one 512-byte atom at

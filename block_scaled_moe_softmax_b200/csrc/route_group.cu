@@ -354,6 +354,8 @@ __global__ void __launch_bounds__(1024) route_group_small_kernel(const RouteGrou
         hist[e] = 0;
     if (a.unit_counters && threadIdx.x < 2)
         a.unit_counters[threadIdx.x] = 0;
+    for (int i = threadIdx.x; i < a.zero_n; i += blockDim.x)
+        a.zero_words[i] = 0;
     __syncthreads();
     for (int t = warp; t < a.T; t += 32) {
         if (a.given_ids)

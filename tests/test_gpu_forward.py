@@ -259,3 +259,26 @@ def test_fused_combine_gives_same_bits(name, act_mode, variant, monkeypatch):
         outs.append(out)
         layer.close()
     assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 16, 4), (3, 384, 8), (16, 40, 8), (16, 8, 2)])
+@pytest.mark.parametrize("act_mode", [0, 1], ids=["w4a16", "w4a8"])
+def test_two_phase_launch_matches_oracle(T, E, k, act_mode, monkeypatch):
+    """Up to 16 tokens FC1 and FC2 run as one launch by default (FC2's units wait for their row
+    block's FC1 units); with MOE_MX_TWO_PHASE=0 as two.  Both meet the oracle's tolerance, the
+    routing is bit-exact, and two forwards in a row give the same bits (the per-row-block counts
+    start from zero every forward).  I = 128 makes FC2 a single K stage per unit."""
+    for I in (256, 128):
+        wl = workloads.Workload(f"two_phase{T}_{E}_{k}_{I}", T, 512, I, E, k, "bf16", "normal", 13)
+        inp = helpers.host_inputs(wl)
+        ref, _, _ = helpers.oracle_forward(inp, k, act_mode)
+        for two in ("1", "0"):
+            monkeypatch.setenv("MOE_MX_TWO_PHASE", two)
+            layer, _, out = _run(wl, act_mode, monkeypatch, inp=inp)
+            helpers.check_routing(layer, T, k, E, inp["logits"].numpy())
+            helpers.check_output(out, ref, f"{wl.name} two_phase={two}")
+            d = helpers.to_device(inp)
+            out2 = layer.forward(d["x"], d["logits"], d["w1"], d["w1s"], d["w2"], d["w2s"], k, act_mode)
+            assert layer.sync_status() == moe_mx.MOE_MX_OK, moe_mx.moe_mx_last_error()
+            assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+            layer.close()
