@@ -141,8 +141,9 @@ struct moe_mx_handle {
     int tile_rows; // 0: by token count; else 16, 32, 64 or 128 (MOE_MX_TILE_ROWS)
     int pdl;       // launch the kernels after the router as programmatic dependents (MOE_MX_PDL, default 1)
     int wide;      // 128-row GEMM blocks: the two-tile (N = 256) variant (MOE_MX_WIDE, default 1)
-    int fuse_combine; // small batches: the combine runs in FC2's epilogue (MOE_MX_FUSE_COMBINE, default 1)
-    int two_phase;    // up to 16 tokens: FC1 and FC2 in one launch (MOE_MX_TWO_PHASE, default 1)
+    int fuse_combine; // small batches: the combine in FC2's epilogue (MOE_MX_FUSE_COMBINE; off by default: slower)
+    int two_phase;    // small batches: FC1 and FC2 in one launch (MOE_MX_TWO_PHASE, default 1)
+    int two_phase_max_tokens; // ... up to this many tokens (at most 16)
     int scale_layout; // MOE_MX_SCALES_ROW_MAJOR or MOE_MX_SCALES_TILED
     unsigned long long timeout_ns;
     void *ws;
@@ -247,8 +248,14 @@ int moe_mx_create_ex(moe_mx_handle **out, int hidden, int inter, int num_experts
         h->tile_rows = 0;
     h->pdl = env_int("MOE_MX_PDL", 1) != 0;
     h->wide = env_int("MOE_MX_WIDE", 1) != 0;
-    h->fuse_combine = env_int("MOE_MX_FUSE_COMBINE", 1) != 0;
+    h->fuse_combine = env_int("MOE_MX_FUSE_COMBINE", 0) != 0;
     h->two_phase = env_int("MOE_MX_TWO_PHASE", 1) != 0;
+    // measured: one launch gains at a single token (0.090 -> 0.083 ms) and loses from 2 tokens on
+    // (its FC2 units are one weight tile each, and short); MOE_MX_TWO_PHASE_TOKENS (<= 16) moves
+    // the bound
+    h->two_phase_max_tokens = env_int("MOE_MX_TWO_PHASE_TOKENS", 1);
+    if (h->two_phase_max_tokens > 16)
+        h->two_phase_max_tokens = 16;
     h->swap_rows = env_int("MOE_MX_SWAP_ROWS", 64);
     if (h->swap_rows < 0)
         h->swap_rows = 0;
@@ -460,7 +467,7 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
         // pairs fit one 16-row block: FC1 and FC2 then run as one launch (two phases), FC2's units
         // waiting for their row block's FC1 units through rb_done, which the routing kernel (one
         // CTA at this size) zeroes.  Row blocks: at most one per expert slot hit.
-        const bool two = h->two_phase && !given_ids && tile_rows == 16 && T <= 16 && T <= kSmallRouteTokens;
+        const bool two = h->two_phase && !given_ids && tile_rows == 16 && T <= h->two_phase_max_tokens;
         if (two) {
             ra.zero_words = h->rb_done;
             ra.zero_n = (int)((int64_t)T * k < E ? (int64_t)T * k : E);
@@ -504,7 +511,8 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
         if (!two)
             launch_fc_gemm(f1, h->map_A[f1.terms - 1], h->map_Asw[f1.terms - 1][sw_idx], h->map_A16, h->map_w1,
                            h->num_sms, s, pdl);
-        mark(3);
+        if (!two)
+            mark(3);
 
         FcGemmArgs f2 = f1;
         f2.wscale = w2_scale;
@@ -536,6 +544,7 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
             const CUtensorMap m2[4] = {h->map_H[f2.terms - 1], h->map_Hsw[f2.terms - 1][sw_idx], h->map_H16,
                                        h->map_w2};
             launch_fc_gemm_two_phase(f1, m1, f2, m2, h->num_sms, s, pdl);
+            mark(3); // the FC1 stage's time covers both GEMMs; the FC2 stage is empty
         } else {
             launch_fc_gemm(f2, h->map_H[f2.terms - 1], h->map_Hsw[f2.terms - 1][sw_idx], h->map_H16, h->map_w2,
                            h->num_sms, s, pdl);

@@ -321,8 +321,9 @@ struct Ctx {
     int n_groups[2], kst[2], terms[2];
     unsigned long long tmo;
     uint32_t *err;
-    __device__ int phase(int u) const { return u >= units0 ? 1 : 0; }
-    __device__ int local(int u) const { return u >= units0 ? u - units0 : u; } // index within its phase
+    bool two; // a compile-time constant of the kernel (kTwo): one-phase kernels fold every phase to 0
+    __device__ int phase(int u) const { return two && u >= units0 ? 1 : 0; }
+    __device__ int local(int u) const { return two && u >= units0 ? u - units0 : u; } // index within its phase
 };
 
 // Bounded wait (one thread) until *count >= target, read with acquire semantics at GPU scope, then
@@ -363,6 +364,7 @@ __device__ __forceinline__ bool wait_count(const int32_t *count, int target, uin
 template <int kActRows, int kMmaW, int kWTiles, int kTm, int PI>
 __device__ __forceinline__ void producer_role(const Ctx &c, int lane)
 {
+    uint32_t *const err_w = c.err; // in a register: the stage loops wait with it
     using P = Plan<kActRows, kMmaW, kWTiles, kTm>;
     constexpr int kStages = P::kStages, kProd = P::kProd, kWT = P::kWT;
     constexpr int kTermBytes = P::kTermBytes, kActBytes = P::kActBytes;
@@ -375,7 +377,7 @@ __device__ __forceinline__ void producer_role(const Ctx &c, int lane)
     const UnitRing<kStages> ring{bars, c.units};
     grid_dep_wait();
     for (uint32_t i = 0; ok; ++i) {
-        const int4 blk = ring.take(i, c.err, tmo, lane);
+        const int4 blk = ring.take(i, err_w, tmo, lane);
         if (blk.w < 0)
             break;
         const int ph = c.phase(blk.w), u = c.local(blk.w);
@@ -409,7 +411,7 @@ __device__ __forceinline__ void producer_role(const Ctx &c, int lane)
         if (ph == 1 && a.rb_done) {
             bool mine = true;
             if (elect_one())
-                mine = wait_count(a.rb_done + u / c.n_groups[1], c.n_groups[0], c.err, tmo);
+                mine = wait_count(a.rb_done + u / c.n_groups[1], c.n_groups[0], err_w, tmo);
             if (!__all_sync(0xFFFFFFFFu, mine)) {
                 ok = false;
                 break;
@@ -419,7 +421,7 @@ __device__ __forceinline__ void producer_role(const Ctx &c, int lane)
             if ((int)(g % kProd) != PI)
                 continue; // another producer warp fills this stage
             const int s = g % kStages;
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.empty(s), ((g / kStages) & 1) ^ 1, c.err, tmo))) {
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.empty(s), ((g / kStages) & 1) ^ 1, err_w, tmo))) {
                 ok = false;
                 break;
             }
@@ -511,6 +513,7 @@ __device__ __forceinline__ void scheduler_role(const Ctx &c, int lane)
 template <int kActRows, int kMmaW, int kWTiles, int kTm, int MI>
 __device__ __forceinline__ void mma_role(const Ctx &c)
 {
+    uint32_t *const err_w = c.err; // in a register: the stage loops wait with it
     using P = Plan<kActRows, kMmaW, kWTiles, kTm>;
     constexpr int kStages = P::kStages, kMma = P::kMma, kWT = P::kWT;
     constexpr int kTermBytes = P::kTermBytes, kActBytes = P::kActBytes;
@@ -530,7 +533,7 @@ __device__ __forceinline__ void mma_role(const Ctx &c)
     const UnitRing<kStages> ring{bars, c.units};
     const int lane = threadIdx.x & 31;
     for (; ok; ++cnt) {
-        const int4 blk = ring.take(cnt, c.err, tmo, lane);
+        const int4 blk = ring.take(cnt, err_w, tmo, lane);
         if (blk.w < 0)
             break;
         const int phs = c.phase(blk.w); // the unit's phase (FC1 or FC2 in a two-phase launch)
@@ -555,7 +558,7 @@ __device__ __forceinline__ void mma_role(const Ctx &c)
             }
         const int buf = cnt & 1;
         if (!__all_sync(0xFFFFFFFFu,
-                        mbar_wait_bounded(bars.acc_empty(buf), ((cnt >> 1) & 1) ^ 1, c.err, tmo))) {
+                        mbar_wait_bounded(bars.acc_empty(buf), ((cnt >> 1) & 1) ^ 1, err_w, tmo))) {
             ok = false;
             break;
         }
@@ -597,7 +600,7 @@ __device__ __forceinline__ void mma_role(const Ctx &c)
                 }
             }
             const uint32_t empty_s = bars.empty(s);
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.full(s), ph, c.err, tmo))) {
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.full(s), ph, err_w, tmo))) {
                 ok = false;
                 break;
             }
@@ -643,6 +646,7 @@ __device__ __forceinline__ void mma_role(const Ctx &c)
 template <int kActRows, int kMmaW, int kWTiles, int kTm>
 __device__ __forceinline__ void mma_role_wide(const Ctx &c)
 {
+    uint32_t *const err_w = c.err; // in a register: the stage loops wait with it
     using P = Plan<kActRows, kMmaW, kWTiles, kTm>;
     constexpr int kStages = P::kStages, kTermBytes = P::kTermBytes, kActBytes = P::kActBytes;
     const Bars<kStages> bars{c.base + P::kOffBar};
@@ -658,11 +662,11 @@ __device__ __forceinline__ void mma_role_wide(const Ctx &c)
     const UnitRing<kStages> ring{bars, c.units};
     const int lane = threadIdx.x & 31;
     for (; ok; ++cnt) {
-        const int4 blk = ring.take(cnt, c.err, tmo, lane);
+        const int4 blk = ring.take(cnt, err_w, tmo, lane);
         if (blk.w < 0)
             break;
         // the accumulator is free once the epilogue has copied the previous unit's out of TMEM
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.acc_empty(0), (cnt & 1) ^ 1, c.err, tmo))) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.acc_empty(0), (cnt & 1) ^ 1, err_w, tmo))) {
             ok = false;
             break;
         }
@@ -686,7 +690,7 @@ __device__ __forceinline__ void mma_role_wide(const Ctx &c)
                     opa[k32][t] = ds_act + (uint64_t)((t * kTermBytes) >> 4) + 2u * k32;
             }
             const uint32_t empty_s = bars.empty(s);
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.full(s), ph, c.err, tmo))) {
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.full(s), ph, err_w, tmo))) {
                 ok = false;
                 break;
             }
@@ -726,6 +730,7 @@ __device__ __forceinline__ void mma_role_wide(const Ctx &c)
 template <int kActRows, int kMmaW, int kWTiles, int kTm>
 __device__ __forceinline__ void epilogue_wide(const Ctx &c, int warp, int lane)
 {
+    uint32_t *const err_w = c.err; // in a register: the stage loops wait with it
     const FcGemmArgs &a = *c.args[0]; // one phase
     using P = Plan<kActRows, kMmaW, kWTiles, kTm>;
     const Bars<P::kStages> bars{c.base + P::kOffBar};
@@ -733,12 +738,12 @@ __device__ __forceinline__ void epilogue_wide(const Ctx &c, int warp, int lane)
     const int q = warp & 3;                     // TMEM lane quarter this warp may access
     const int half = warp >= P::kEpi2 ? 1 : 0;  // the unit's weight tile this warp writes
     for (uint32_t cnt = 0;; ++cnt) {
-        const int4 blk = ring.take(cnt, c.err, c.tmo, lane);
+        const int4 blk = ring.take(cnt, err_w, c.tmo, lane);
         // the eight epilogue warps leave together (they share named barrier 2)
         if (!named_bar_all(2, 256, blk.w >= 0))
             break;
         const int nt = (blk.w % c.n_groups[0]) * 2 + half;
-        const bool got = mbar_wait_bounded(bars.acc_full(0), cnt & 1, c.err, c.tmo);
+        const bool got = mbar_wait_bounded(bars.acc_full(0), cnt & 1, err_w, c.tmo);
         if (!named_bar_all(2, 256, got))
             break;
         tc_fence_after();
@@ -798,7 +803,7 @@ __device__ __forceinline__ void epilogue_wide(const Ctx &c, int warp, int lane)
     }
 }
 
-template <int kActRows, int kMmaW, int kWTiles, int kTm>
+template <int kActRows, int kMmaW, int kWTiles, int kTm, bool kTwo>
 __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads, 1)
     fc_gemm_kernel(const __grid_constant__ FcGemmArgs a0, const __grid_constant__ FcGemmArgs a1,
                    const __grid_constant__ CUtensorMap act_map, const __grid_constant__ CUtensorMap act_map_sw,
@@ -838,7 +843,7 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads,
         prefetch_tensormap(&act_map_sw);
         prefetch_tensormap(&act_map16);
         prefetch_tensormap(&w_map);
-        if (a0.rb_done) { // two phases: FC2's maps too
+        if (kTwo) { // two phases: FC2's maps too
             prefetch_tensormap(&act_map1);
             prefetch_tensormap(&act_map_sw1);
             prefetch_tensormap(&act_map16_1);
@@ -859,8 +864,8 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads,
     if (threadIdx.x == 0)
         grid_dep_launch();
 
-    // one phase (a0 alone), or two (a0 = FC1, a1 = FC2; only such launches carry rb_done)
-    const bool two = a0.rb_done != nullptr;
+    // one phase (a0 alone), or two (kTwo: a0 = FC1, a1 = FC2)
+    constexpr bool two = kTwo;
     const int nrb = *a0.num_rowblocks;
     const unsigned long long tmo = a0.timeout_ns;
     Ctx ctx;
@@ -888,6 +893,7 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads,
     ctx.total_units = ctx.units0 + (two ? nrb * ctx.n_groups[1] : 0);
     ctx.tmo = tmo;
     ctx.err = a0.err;
+    ctx.two = kTwo;
     if (warp == 0) {
         producer_role<kActRows, kMmaW, kWTiles, kTm, 0>(ctx, lane);
     } else if (warp >= 6 && warp < 5 + kProd) {
@@ -912,11 +918,12 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads,
     } else if (warp >= 2 && warp < 6) {
         // ------------------------------------------------------------ epilogue (warps 2..5)
         const int q = warp & 3; // TMEM lane quarter this warp may access
+        uint32_t *const err_w = a0.err;
         float *xch = reinterpret_cast<float *>(gsm + kOffX);
         const UnitRing<kStages> ring{bars, reinterpret_cast<volatile int *>(gsm + P::kOffUnits)};
         uint32_t g_run = 0; // pipeline stages of the units before this one
         for (uint32_t cnt = 0;; ++cnt) {
-            const int4 blk = ring.take(cnt, ctx.err, tmo, lane);
+            const int4 blk = ring.take(cnt, err_w, tmo, lane);
             // the four epilogue warps leave together (they share named barriers below)
             if (!named_bar_all(2, 128, blk.w >= 0))
                 break;
@@ -930,7 +937,7 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads,
             const bool swap = kActRows < 128 || rows <= a.swap_rows;
             const int buf = cnt & 1;
             // the four epilogue warps leave together or not at all (they share named barrier 1 below)
-            const bool got = mbar_wait_bounded(bars.acc_full(buf), (cnt >> 1) & 1, ctx.err, tmo);
+            const bool got = mbar_wait_bounded(bars.acc_full(buf), (cnt >> 1) & 1, err_w, tmo);
             if (!named_bar_all(2, 128, got))
                 break;
             tc_fence_after();
@@ -1061,9 +1068,10 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads,
     }
 }
 
-template <int kActRows, int kMmaW, int kWTiles, int kTm> static cudaError_t prepare_one()
+template <int kActRows, int kMmaW, int kWTiles, int kTm, bool kTwo = false> static cudaError_t prepare_one()
 {
-    return cudaFuncSetAttribute(fc_gemm_kernel<kActRows, kMmaW, kWTiles, kTm>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(fc_gemm_kernel<kActRows, kMmaW, kWTiles, kTm, kTwo>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 Plan<kActRows, kMmaW, kWTiles, kTm>::kSmemBytes);
 }
 
@@ -1076,7 +1084,9 @@ cudaError_t fc_gemm_prepare()
         (e = prepare_one<64, 1, 1, 2>()) != cudaSuccess || (e = prepare_one<128, 1, 1, 2>()) != cudaSuccess ||
         (e = prepare_one<128, 1, 1, 1>()) != cudaSuccess || (e = prepare_one<128, 1, 2, 2>()) != cudaSuccess)
         return e;
-    return prepare_one<128, 1, 2, 1>();
+    if ((e = prepare_one<128, 1, 2, 1>()) != cudaSuccess)
+        return e;
+    return prepare_one<16, 2, 1, 2, true>();
 }
 
 template <int kActRows, int kMmaW, int kWTiles, int kTm>
@@ -1084,7 +1094,7 @@ static void launch_one(const FcGemmArgs &a, const CUtensorMap &act_map, const CU
                        const CUtensorMap &act_map16, const CUtensorMap &w_map, int grid, cudaStream_t s, bool pdl)
 {
     using P = Plan<kActRows, kMmaW, kWTiles, kTm>;
-    launch_kernel(fc_gemm_kernel<kActRows, kMmaW, kWTiles, kTm>, dim3(grid), dim3(P::kThreads), (size_t)P::kSmemBytes,
+    launch_kernel(fc_gemm_kernel<kActRows, kMmaW, kWTiles, kTm, false>, dim3(grid), dim3(P::kThreads), (size_t)P::kSmemBytes,
                   s, pdl, a, a, act_map, act_map_sw, act_map16, w_map, act_map, act_map_sw, act_map16, w_map);
 }
 
@@ -1136,7 +1146,7 @@ void launch_fc_gemm_two_phase(const FcGemmArgs &a1, const CUtensorMap *maps1, co
     // tokens on N, 16-row blocks, two MMA warps: the small-batch FC1 variant serves both phases
     // (FC2 units then take one weight tile each)
     using P = Plan<16, 2, 1, 2>;
-    launch_kernel(fc_gemm_kernel<16, 2, 1, 2>, dim3(grid), dim3(P::kThreads), (size_t)P::kSmemBytes, s, pdl, a1, a2,
+    launch_kernel(fc_gemm_kernel<16, 2, 1, 2, true>, dim3(grid), dim3(P::kThreads), (size_t)P::kSmemBytes, s, pdl, a1, a2,
                   maps1[0], maps1[1], maps1[2], maps1[3], maps2[0], maps2[1], maps2[2], maps2[3]);
 }
 

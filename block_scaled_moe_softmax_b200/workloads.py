@@ -85,6 +85,12 @@ WORKLOADS = {
     # for the routing and grouping kernel
     "route_e384": Workload("route_e384", 16, 256, 128, 384, 8, "bf16", "none", 0,
                            "decode routing shape with small experts (profiling case)"),
+    "decode_t2": Workload("decode_t2", 2, 7168, 2048, 384, 8, "bf16", "none", 0,
+                          "decode-shaped, w4a16, 2 tokens"),
+    # one decode token over 64 experts: a capture-sized case (about 1.5 GB of weights) with the GEMM
+    # work of the single-token decode (8 experts hit), for profiling
+    "decode_t1_e64": Workload("decode_t1_e64", 1, 7168, 2048, 64, 8, "bf16", "none", 0,
+                              "decode-shaped, w4a16, a single token, 64 experts (profiling case)"),
     # the decode shape with 64 experts: a capture-sized case (about 1.5 GB of weights) for profiling
     "decode_e64": Workload("decode_e64", 16, 7168, 2048, 64, 8, "bf16", "none", 0,
                            "decode-shaped, w4a16, 64 experts (profiling case)"),

@@ -365,8 +365,8 @@ MOE_MX_API long long moe_mx_launch_count(const moe_mx_handle *h);
 /* Stages of one forward, in launch order (indices into moe_mx_get_stage_times). */
 #define MOE_MX_STAGE_ROUTE 0   /* routing, histogram, scan, stable scatter */
 #define MOE_MX_STAGE_GATHER 1  /* gather of activation rows (+ MXFP8 quantisation) */
-#define MOE_MX_STAGE_FC1 2     /* FC1 grouped GEMM with the SwiGLU epilogue */
-#define MOE_MX_STAGE_FC2 3     /* FC2 grouped GEMM */
+#define MOE_MX_STAGE_FC1 2     /* FC1 grouped GEMM with the SwiGLU epilogue (up to 16 tokens: FC1 and FC2, one launch) */
+#define MOE_MX_STAGE_FC2 3     /* FC2 grouped GEMM (empty when it ran in FC1's launch) */
 #define MOE_MX_STAGE_COMBINE 4 /* weighted combine */
 #define MOE_MX_NUM_STAGES 5
 

@@ -242,9 +242,10 @@ def test_router_matches_hand_derived_cases():
 @pytest.mark.parametrize("act_mode", [0, 1], ids=["w4a16", "w4a8"])
 @pytest.mark.parametrize("variant", ["auto", "t16", "t32", "t64"])
 def test_fused_combine_gives_same_bits(name, act_mode, variant, monkeypatch):
-    """Up to 512 tokens (every FC2 unit with its tokens on N) the combine runs in FC2's epilogue by
-    default; it must give exactly the bits of the separate combine kernel (MOE_MX_FUSE_COMBINE=0),
-    on two forwards in a row (its per-token counters must be back at zero after each)."""
+    """Up to 512 tokens (every FC2 unit with its tokens on N) the combine may run in FC2's epilogue
+    (MOE_MX_FUSE_COMBINE=1; off by default, it measured slower); it must give exactly the bits of
+    the separate combine kernel, on two forwards in a row (its per-token counters must be back at
+    zero after each)."""
     wl = SHAPES[name]
     tile_rows = VARIANTS[variant][0]
     inp = helpers.host_inputs(wl)
@@ -264,14 +265,15 @@ def test_fused_combine_gives_same_bits(name, act_mode, variant, monkeypatch):
 @pytest.mark.parametrize("T,E,k", [(1, 16, 4), (3, 384, 8), (16, 40, 8), (16, 8, 2)])
 @pytest.mark.parametrize("act_mode", [0, 1], ids=["w4a16", "w4a8"])
 def test_two_phase_launch_matches_oracle(T, E, k, act_mode, monkeypatch):
-    """Up to 16 tokens FC1 and FC2 run as one launch by default (FC2's units wait for their row
-    block's FC1 units); with MOE_MX_TWO_PHASE=0 as two.  Both meet the oracle's tolerance, the
+    """FC1 and FC2 as one launch (FC2's units wait for their row block's FC1 units; by default up to
+    2 tokens, here forced up to 16) and as two launches (MOE_MX_TWO_PHASE=0).  Both meet the oracle's tolerance, the
     routing is bit-exact, and two forwards in a row give the same bits (the per-row-block counts
     start from zero every forward).  I = 128 makes FC2 a single K stage per unit."""
     for I in (256, 128):
         wl = workloads.Workload(f"two_phase{T}_{E}_{k}_{I}", T, 512, I, E, k, "bf16", "normal", 13)
         inp = helpers.host_inputs(wl)
         ref, _, _ = helpers.oracle_forward(inp, k, act_mode)
+        monkeypatch.setenv("MOE_MX_TWO_PHASE_TOKENS", "16")   # every T here through the one launch
         for two in ("1", "0"):
             monkeypatch.setenv("MOE_MX_TWO_PHASE", two)
             layer, _, out = _run(wl, act_mode, monkeypatch, inp=inp)
