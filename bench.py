@@ -10,7 +10,7 @@ H=7168, I=2048, E=384 experts, top-8), and all five configurations of the layer
 are measured in the same run under "per_config": tiny (T=16, H=256, I=128,
 E=8, top-2), decode, batched decode (T=256, logits + a N(0, 0.5) expert bias),
 prefill (T=8192, Zipf-like expert bias) and prefill w4a8 (T=16384, H=4096,
-I=1536, E=128).  --workload NAME measures one workload alone (also the
+I=1536, E=128), and the small-batch decode shapes (1 and 4 tokens).  --workload NAME measures one workload alone (also the
 small-batch decode shapes decode_t1 / decode_t4, the shared-expert decode, and
 shards of the 896-expert, top-16 layer with the routing given as precomputed
 top-k: situ_tp8, situ_ep8).  Inputs are synthetic and seeded (bf16 x ~ N(0,1),
@@ -565,7 +565,7 @@ def measure(args, wl, weights, world, rank, with_e2e=True):
 
 
 # the five configurations of the layer, measured by the default run (the first is the headline)
-DEFAULT_SET = ("decode", "tiny", "batched_decode", "prefill", "prefill_w4a8")
+DEFAULT_SET = ("decode", "tiny", "batched_decode", "prefill", "prefill_w4a8", "decode_t1", "decode_t4")
 
 
 def run_ours(args):

@@ -116,7 +116,7 @@ def test_forward_is_deterministic(monkeypatch):
 # ... including expert counts that take each top-k width (8, 16 and 32 candidates per lane) on
 # both routing paths (one CTA up to 256 tokens, three kernels beyond)
 @pytest.mark.parametrize("T,E,k", [(1, 8, 2), (3, 4, 4), (16, 8, 1), (130, 2, 2), (20, 1000, 4), (300, 600, 8),
-                                   (257, 300, 6), (40, 384, 8)])
+                                   (257, 300, 6), (40, 384, 8), (1, 384, 8), (2, 384, 8), (4, 384, 8), (8, 384, 8)])
 def test_edge_shapes(T, E, k, monkeypatch):
     wl = workloads.Workload(f"edge{T}_{E}_{k}", T, 256, 128, E, k, "bf16", "none", 7)
     layer, inp, out = _run(wl, 0, monkeypatch)

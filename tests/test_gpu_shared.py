@@ -44,7 +44,7 @@ def _check_routing(layer, T, k, wl, logits_np):
         assert np.all(seg[counts_o[e]:] == -1)
 
 
-@pytest.mark.parametrize("T", [12, 200])
+@pytest.mark.parametrize("T", [1, 12, 200])
 @pytest.mark.parametrize("S", [1, 2])
 @pytest.mark.parametrize("act", [0, 1], ids=["w4a16", "w4a8"])
 def test_shared_expert_matches_oracle(T, S, act):
