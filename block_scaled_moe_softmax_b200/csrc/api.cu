@@ -144,6 +144,8 @@ struct moe_mx_handle {
     int fuse_combine; // small batches: the combine in FC2's epilogue (MOE_MX_FUSE_COMBINE; off by default: slower)
     int two_phase;    // small batches: FC1 and FC2 in one launch (MOE_MX_TWO_PHASE, default 1)
     int two_phase_max_tokens; // ... up to this many tokens (at most 16)
+    int fc2_tiles;            // FC2 of blocks of <= 16 rows: weight tiles per unit (MOE_MX_FC2_TILES: 0 = by
+                              // token count, 2 or 4)
     int scale_layout; // MOE_MX_SCALES_ROW_MAJOR or MOE_MX_SCALES_TILED
     unsigned long long timeout_ns;
     void *ws;
@@ -254,6 +256,9 @@ int moe_mx_create_ex(moe_mx_handle **out, int hidden, int inter, int num_experts
     // (its FC2 units are one weight tile each, and short); MOE_MX_TWO_PHASE_TOKENS (<= 16) moves
     // the bound
     h->two_phase_max_tokens = env_int("MOE_MX_TWO_PHASE_TOKENS", 1);
+    h->fc2_tiles = env_int("MOE_MX_FC2_TILES", 0);
+    if (h->fc2_tiles != 2 && h->fc2_tiles != 4)
+        h->fc2_tiles = 0;
     if (h->two_phase_max_tokens > 16)
         h->two_phase_max_tokens = 16;
     h->swap_rows = env_int("MOE_MX_SWAP_ROWS", 64);
@@ -524,6 +529,10 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
         f2.out_ld = H;
         f2.fc1 = 0;
         f2.act_mxfp8 = 0;
+        // FC2 of 16-row blocks: four weight tiles per unit (3 stages of 4 tiles: 96 KB of weights in
+        // flight per SM, against 80 KB in 5 stages of 2) when there are many units to share out;
+        // measured at 16 tokens 164 -> 145 us, at 2 and 4 tokens no gain
+        f2.fc2_tiles = h->fc2_tiles ? h->fc2_tiles : (T > 4 ? 4 : 2);
         // small batches of the logits form: every FC2 unit has its tokens on N, and its epilogue
         // finishes the combine of the tokens whose k pairs it completes
         const bool fuse = h->fuse_combine && !given_ids && route_E == 0 && tile_rows <= 64;

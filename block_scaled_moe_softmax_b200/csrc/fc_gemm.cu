@@ -107,8 +107,12 @@ template <int kActRows, int kMmaW, int kWTiles, int kTm> struct Plan {
     static constexpr int kMma = kMmaW;
     static_assert(kMma == 1 || kStages % 2 == 0, "alternating MMA warps need an even stage count");
     static_assert(kMma == 1 || kActRows <= 32, "two accumulators per buffer need N <= 64");
-    static_assert(kWT == 1 || (kWT == 2 && kMma == 1 && (kActRows <= 32 || kActRows == 128)),
-                  "two weight tiles: one MMA warp, N <= 64 or the wide 128-row variant");
+    static_assert(kWT == 1 || (kWT == 2 && kMma == 1 && (kActRows <= 32 || kActRows == 128)) ||
+                      (kWT == 4 && kMma == 1 && kActRows <= 16),
+                  "two weight tiles: one MMA warp, N <= 64 or the wide 128-row variant; four: N <= 32");
+    // TMEM columns between the accumulators of a unit's weight tiles within one 128-column buffer:
+    // 64, or 32 for four tiles (N <= 32)
+    static constexpr int kAccW = kWT == 4 ? 32 : 64;
     // The wide variant (128 token rows against two weight tiles, tokens on M): one M = 128,
     // N = 256 MMA per K block covers both tiles, so each activation byte brought into shared
     // memory feeds twice the MMA work.  Its 256-column accumulator leaves no room in TMEM for a
@@ -617,10 +621,11 @@ __device__ __forceinline__ void mma_role(const Ctx &c)
                 for (int k32 = 0; k32 < 4; ++k32)
 #pragma unroll
                     for (int wt = 0; wt < kWT; ++wt) {
-                        umma_mx(d + 64u * wt, opa[k32][wt][0], opb[k32][wt][0], idesc[k32], sfa[wt][0], sfb[wt][0],
+                        umma_mx(d + (uint32_t)P::kAccW * wt, opa[k32][wt][0], opb[k32][wt][0], idesc[k32], sfa[wt][0],
+                                sfb[wt][0],
                                 accf[k32]);
                         if (t1)
-                            umma_mx(d + 64u * wt, opa[k32][wt][1], opb[k32][wt][1], idesc[k32], sfa[wt][1],
+                            umma_mx(d + (uint32_t)P::kAccW * wt, opa[k32][wt][1], opb[k32][wt][1], idesc[k32], sfa[wt][1],
                                     sfb[wt][1], 1u);
                     }
                 umma_commit(empty_s);
@@ -1002,7 +1007,7 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads,
                             continue;
                         for (int t = 0; t < (comb ? 2 : 1); ++t) {
                             uint32_t r[16];
-                            tmem_ld16(tb + 64 * (w + wt) + (t ? P::kT2 : 0) + n0, r);
+                            tmem_ld16(tb + 64 * w + P::kAccW * wt + (t ? P::kT2 : 0) + n0, r);
                             tmem_wait_ld();
 #pragma unroll
                             for (int j = 0; j < 16; ++j)
@@ -1079,7 +1084,8 @@ cudaError_t fc_gemm_prepare()
 {
     cudaError_t e;
     if ((e = prepare_one<16, 1, 1, 2>()) != cudaSuccess || (e = prepare_one<16, 2, 1, 2>()) != cudaSuccess ||
-        (e = prepare_one<16, 1, 2, 2>()) != cudaSuccess || (e = prepare_one<32, 1, 1, 2>()) != cudaSuccess ||
+        (e = prepare_one<16, 1, 2, 2>()) != cudaSuccess || (e = prepare_one<16, 1, 4, 2>()) != cudaSuccess ||
+        (e = prepare_one<32, 1, 1, 2>()) != cudaSuccess ||
         (e = prepare_one<32, 2, 1, 2>()) != cudaSuccess || (e = prepare_one<32, 1, 2, 2>()) != cudaSuccess ||
         (e = prepare_one<64, 1, 1, 2>()) != cudaSuccess || (e = prepare_one<128, 1, 1, 2>()) != cudaSuccess ||
         (e = prepare_one<128, 1, 1, 1>()) != cudaSuccess || (e = prepare_one<128, 1, 2, 2>()) != cudaSuccess)
@@ -1110,6 +1116,8 @@ void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUten
     if (a.max_block_rows <= 16) {
         if (a.fc1)
             launch_one<16, 2, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
+        else if (a.fc2_tiles == 4 && a.n_tiles % 4 == 0)
+            launch_one<16, 1, 4, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
         else if (wt2)
             launch_one<16, 1, 2, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
         else

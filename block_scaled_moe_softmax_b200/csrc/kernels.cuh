@@ -131,6 +131,7 @@ struct FcGemmArgs {
     // each row block's finished units in rb_done (zero before the forward), and an FC2 unit copies
     // its row block's h only once all of them are counted.
     int32_t *rb_done;
+    int fc2_tiles;               // FC2 with blocks of <= 16 rows: weight tiles per work unit (2 or 4)
 };
 
 // Tensor maps: act_map = both term planes, 128-row boxes ([terms][128][128] codes, tokens
