@@ -450,13 +450,14 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
         };
         mark(0);
         // activation tile rows per term of the GEMM variant; the segments are split into work
-        // blocks of at most that many rows (a segment holds one expert's tokens, so at 16 or 32
-        // tokens nothing is split).  Up to a few hundred tokens 32-row blocks, all with their
-        // tokens on N, are fastest (measured at 256 tokens: 1.61 ms against 1.90 ms with 64-row
-        // blocks): the variant has room for two MMA warps, and re-reading the weights of the
-        // few experts split into several blocks costs less than that gains.
+        // blocks of at most that many rows (a segment holds one expert's tokens, so at 16 tokens
+        // nothing is split).  Up to a few hundred tokens small blocks, all with their tokens on N,
+        // are fastest: re-reading the weights of the few experts split into several blocks costs
+        // less than the deeper pipelines gain.  Measured at 256 tokens: 32-row blocks 1.61 ms
+        // against 1.90 ms with 64-row ones, and 16-row blocks (FC2 then takes four weight tiles
+        // per unit) 1.48 ms against 1.56 ms with 32-row ones.
         const int tile_rows = h->tile_rows > 0 ? h->tile_rows
-                              : T <= 16        ? 16
+                              : T <= 256       ? 16
                               : T <= 512       ? 32
                                                : kBlockRows;
         RouteGroupArgs ra{router_logits, T, E, k, h->topk_ids, h->topk_w, h->chunk_hist, h->counts,
@@ -477,9 +478,11 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
             ra.zero_words = h->rb_done;
             ra.zero_n = (int)((int64_t)T * k < E ? (int64_t)T * k : E);
         }
-        // Each kernel after the router may launch while its predecessor still runs (programmatic
-        // dependent launch): the FC GEMMs start streaming their weights early.  Stage timing
-        // records events between the kernels, so timed forwards launch them one after another.
+        // Each kernel may launch while its predecessor still runs (programmatic dependent launch):
+        // the FC GEMMs start streaming their weights early, and the router's launch overlaps the
+        // tail of whatever precedes the forward in the stream (it waits for it before its work).
+        // Stage timing records events between the kernels, so timed forwards launch them one after
+        // another.
         const bool pdl = h->pdl && !evset;
         h->launches += launch_route_and_group(ra, s, pdl);
         mark(1);

@@ -146,6 +146,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float *__res
                                                                int route_E, int shard)
 {
     grid_dep_launch(); // the next kernel (the scan) waits for this grid before reading its output
+    grid_dep_wait();   // whatever precedes it (see route_group_small_kernel)
     __shared__ int32_t hist[kMaxExperts];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int e = threadIdx.x; e < E; e += blockDim.x)
@@ -347,6 +348,10 @@ template <int kPerLane>
 __global__ void __launch_bounds__(1024) route_group_small_kernel(const RouteGroupArgs a)
 {
     grid_dep_launch(); // the next kernel (the gather) waits for this grid before reading its output
+    // Launched as a programmatic dependent of whatever precedes it in the stream (the previous
+    // forward's combine, or the caller's kernel that writes the logits): wait for it before
+    // reading an input or writing the workspace that kernel may still read.
+    grid_dep_wait();
     __shared__ int32_t hist[kMaxExperts]; // counts, then cursors
     __shared__ unsigned long long s_warp[32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -599,31 +604,30 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
 int launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s, bool pdl)
 {
     // the top-k scan visits 32 * kPerLane candidates per token: size it to the expert count
-    // (the given routing visits no candidates: the smallest instance serves it).  The first
-    // kernel is an ordinary launch; those after it are programmatic dependents (pdl).
+    // (the given routing visits no candidates: the smallest instance serves it).  With pdl every
+    // kernel is a programmatic dependent of the one before it in the stream, the first one too
+    // (its launch overlaps the tail of whatever precedes it; it waits for that before its work).
     const bool narrow = a.given_ids != nullptr || a.routeE() <= 256;
     if (a.T <= kSmallRouteTokens) {
         if (narrow)
-            route_group_small_kernel<8><<<1, 1024, 0, s>>>(a);
+            launch_kernel(route_group_small_kernel<8>, dim3(1), dim3(1024), 0, s, pdl, a);
         else if (a.routeE() <= 512)
-            route_group_small_kernel<16><<<1, 1024, 0, s>>>(a);
+            launch_kernel(route_group_small_kernel<16>, dim3(1), dim3(1024), 0, s, pdl, a);
         else
-            route_group_small_kernel<32><<<1, 1024, 0, s>>>(a);
+            launch_kernel(route_group_small_kernel<32>, dim3(1), dim3(1024), 0, s, pdl, a);
         return 1;
     }
     const int nchunks = (a.T + kRouteChunk - 1) / kRouteChunk;
+    auto route = [&](auto kernel) {
+        launch_kernel(kernel, dim3(nchunks), dim3(kRouteThreads), 0, s, pdl, a.logits, a.T, a.E, a.k, a.topk_ids,
+                      a.topk_w, a.chunk_hist, a.given_ids, a.given_w, a.id_offset, a.n_shared, a.routeE(), a.shard);
+    };
     if (narrow)
-        route_kernel<8><<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist,
-                                                          a.given_ids, a.given_w, a.id_offset, a.n_shared, a.routeE(),
-                                                          a.shard);
+        route(route_kernel<8>);
     else if (a.routeE() <= 512)
-        route_kernel<16><<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist,
-                                                          a.given_ids, a.given_w, a.id_offset, a.n_shared, a.routeE(),
-                                                          a.shard);
+        route(route_kernel<16>);
     else
-        route_kernel<32><<<nchunks, kRouteThreads, 0, s>>>(a.logits, a.T, a.E, a.k, a.topk_ids, a.topk_w, a.chunk_hist,
-                                                          a.given_ids, a.given_w, a.id_offset, a.n_shared, a.routeE(),
-                                                          a.shard);
+        route(route_kernel<32>);
     launch_kernel(scan_kernel, dim3(1), dim3(1024), 0, s, pdl, a.E, nchunks, a.split_rows, a.chunk_hist, a.counts,
                   a.pad_offsets, a.rowblocks, a.num_rowblocks, a.sorted_pair, a.unit_counters);
     launch_kernel(scatter_kernel, dim3(nchunks), dim3(32), 0, s, pdl, a.T, a.E, a.k, (const int32_t *)a.topk_ids,
