@@ -492,8 +492,10 @@ __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16 *__rest
                 w0 |= __shfl_down_sync(0xFFFFFFFFu, s0, i) << (8 * i);
                 w1 |= __shfl_down_sync(0xFFFFFFFFu, s1, i) << (8 * i);
             }
-            for (int j = jg * group; j < (jg + 1) * group; ++j) {
-                const int row = pos_of_pair[(size_t)t * k + j]; // the same for the whole warp
+            // the group's grouped rows, one per lane, loaded together (not one round trip per row)
+            const int my_row = lane < group ? pos_of_pair[(size_t)t * k + jg * group + lane] : -1;
+            for (int j = 0; j < group; ++j) {
+                const int row = __shfl_sync(0xFFFFFFFFu, my_row, j); // the same for the whole warp
                 if (row < 0)
                     continue; // not in the local expert shard
                 uint4 *dst = reinterpret_cast<uint4 *>(aq + (size_t)row * H + (size_t)b0 * 32);
