@@ -344,13 +344,27 @@ def layer_weight_bytes(wl, hit):
 FC_GEMM_SOURCES = ("fc_gemm.cu", "kernels.cuh", "ptx.cuh")
 
 
-def kernel_source_sha():
-    """sha256 (first 16 hex digits) over the FC GEMM kernel's CUDA sources, in name order."""
+def _code_only(text: str) -> str:
+    """C/CUDA source with its comments removed and whitespace collapsed: what the compiler sees
+    of it, so that an edit of a comment does not count as a change of the kernel."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
+def kernel_source_sha(read=None):
+    """sha256 (first 16 hex digits) over the FC GEMM kernel's CUDA sources, in name order, code
+    only (comments and whitespace stripped).  read(name) returns a source's text (default: the
+    working tree)."""
     csrc = os.path.join(ROOT, "block_scaled_moe_softmax_b200", "csrc")
+    if read is None:
+        def read(name):
+            with open(os.path.join(csrc, name)) as f:
+                return f.read()
     h = hashlib.sha256()
     for name in sorted(FC_GEMM_SOURCES):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + b"\0" + f.read())
+        h.update(name.encode() + b"\0" + _code_only(read(name)).encode())
     return h.hexdigest()[:16]
 
 

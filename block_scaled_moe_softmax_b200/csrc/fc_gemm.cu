@@ -42,7 +42,13 @@
 // w4a16 terms sit side by side on N as well (term 2 from column kT2 on), so one
 // MMA per 32-element K block covers both: an M = 128 block-scaled MMA occupies
 // the tensor pipe about as long for N = 16 as for N = 128 (measured), so this
-// halves the pipe time of the weight-streaming shapes.  Every wait is bounded;
+// halves the pipe time of the weight-streaming shapes.  A work unit takes 1, 2 or 4
+// adjacent weight tiles (4 only with tokens on N at up to 16 rows, where four
+// 32-column accumulators share a 128-column TMEM buffer): fewer, larger stages
+// keep more weight bytes in flight per SM.
+// One launch may also run two phases (kTwo): FC1's units, then FC2's, claimed from
+// one counter; FC1's epilogue counts each row block's finished units and an FC2
+// unit's producers wait for that count before copying h.  Every wait is bounded;
 // a wait that gives up records an error word, and the CTA drains its own copies
 // and MMAs before freeing TMEM.
 #include "kernels.cuh"
