@@ -75,8 +75,8 @@ struct RouteGroupArgs {
 
 // Launchers of the forward's kernels.  pdl: launch as programmatic dependents of the kernel
 // before them in the stream (each waits for its predecessor before reading its output and lets
-// its own successor launch right after that wait); the first kernel of a forward, the router,
-// is always an ordinary launch.
+// its own successor launch right after that wait); the router, the first kernel of a forward,
+// waits for whatever precedes it before it reads the logits or writes the workspace.
 // Returns the number of kernels launched (1 for small batches, else 3).
 int launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s, bool pdl = false);
 void launch_gather(const __nv_bfloat16 *x, int P, int H, int k, const int32_t *pos_of_pair, uint8_t *aq,

@@ -61,9 +61,9 @@ def _weights(wl):
 
 
 def _work_block_rows(T):
-    """Rows per GEMM work block the library picks for T tokens (16 up to 16 tokens, 32 up to 512,
+    """Rows per GEMM work block the library picks for T tokens (16 up to 256 tokens, 32 up to 512,
     then whole 128-row segments)."""
-    return 16 if T <= 16 else 32 if T <= 512 else 128
+    return 16 if T <= 256 else 32 if T <= 512 else 128
 
 
 def _sample_tokens(ids, wl, n_random=8):
