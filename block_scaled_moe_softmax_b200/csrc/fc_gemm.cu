@@ -788,22 +788,24 @@ __device__ __forceinline__ void epilogue_wide(const Ctx &c, int warp, int lane)
         } else {
             // FC2: f32 rows of Y.  Stored straight from registers, each store instruction of the
             // warp would write 32 rows' 16-byte pieces (half sectors, 32 segments).  Instead each
-            // 16-column chunk goes through this warp's 2 KB buffer ([32 rows][4 x 16 bytes], the
-            // 16-byte column index xor-ed with row % 4: conflict-free both ways) and comes back
-            // out as 8 rows x 64 contiguous bytes per instruction: whole sectors.
+            // 16-column chunk goes through this warp's 2 KB buffer ([32 rows][4 x 16 bytes]) and
+            // comes back out as 8 rows x 64 contiguous bytes per instruction: whole sectors.  Row
+            // r's 16-byte piece i sits at position i ^ ((r >> 1) & 3): a 16-byte access serves 8
+            // lanes per shared-memory wavefront, and the 8 lanes of either side (rows l .. l + 7
+            // writing piece i; rows r, r + 1 reading pieces 0..3) then meet 8 distinct bank groups.
             uint4 *stg = reinterpret_cast<uint4 *>(c.ystage + 2048 * (half * 4 + (warp & 3)));
             const int r0 = lane >> 2, ch = lane & 3;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
-                    stg[lane * 4 + (i ^ (lane & 3))] =
+                    stg[lane * 4 + (i ^ ((lane >> 1) & 3))] =
                         make_uint4(v[j][4 * i], v[j][4 * i + 1], v[j][4 * i + 2], v[j][4 * i + 3]);
                 __syncwarp();
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
                     const int r = 8 * p + r0; // row of this warp's 32
-                    const uint4 val = stg[r * 4 + (ch ^ (r & 3))];
+                    const uint4 val = stg[r * 4 + (ch ^ ((r >> 1) & 3))];
                     if (32 * q + r < blk.z)
                         *reinterpret_cast<uint4 *>(a.y + (size_t)(blk.y + 32 * q + r) * a.out_ld + nt * 128 + 16 * j +
                                                    4 * ch) = val;

@@ -202,8 +202,9 @@ constexpr float kMaxFinite = 3.402823466e38f;
 // are represented exactly; smaller ones keep an absolute error below 2^-20 of
 // the block maximum.  A block that holds a NaN or an infinity has no finite
 // scale: every term gets the E8M0 NaN byte 0xFF and zero codes (the OCP
-// quantiser's rule for such a block).
-__device__ __forceinline__ void mx_encode32(const float (&v)[32], int act_mxfp8, uint8_t (&c0)[32], uint8_t (&c1)[32],
+// quantiser's rule for such a block).  The codes come out packed, four to a
+// word: element 4i + b in byte b of word i (w0: first term, w1: second).
+__device__ __forceinline__ void mx_encode32(const float (&v)[32], int act_mxfp8, uint32_t (&w0)[8], uint32_t (&w1)[8],
                                             uint32_t &s0, uint32_t &s1)
 {
     // amax with NaN propagated: the block is finite exactly when amax <= the largest float
@@ -213,10 +214,8 @@ __device__ __forceinline__ void mx_encode32(const float (&v)[32], int act_mxfp8,
         amax = fmax_nan(amax, fabsf(v[i]));
     if (!(amax <= kMaxFinite)) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            c0[i] = 0;
-            c1[i] = 0;
-        }
+        for (int i = 0; i < 8; ++i)
+            w0[i] = w1[i] = 0u;
         s0 = s1 = 0xFFu;
         return;
     }
@@ -225,33 +224,36 @@ __device__ __forceinline__ void mx_encode32(const float (&v)[32], int act_mxfp8,
     float r[32];
     float amax1 = 0.f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        c0[i] = (uint8_t)f32_to_e4m3(__fmul_rn(v[i], inv0));
-        r[i] = __fsub_rn(v[i], __fmul_rn(e4m3_to_f32(c0[i]), sc0));
-        amax1 = fmaxf(amax1, fabsf(r[i]));
+    for (int i = 0; i < 16; ++i) { // element pairs (2i, 2i + 1): one conversion each way
+        const uint32_t p = f32x2_to_e4m3x2(__fmul_rn(v[2 * i], inv0), __fmul_rn(v[2 * i + 1], inv0));
+        const float2 d = e4m3x2_to_f32x2(p);
+        r[2 * i] = __fsub_rn(v[2 * i], __fmul_rn(d.x, sc0));
+        r[2 * i + 1] = __fsub_rn(v[2 * i + 1], __fmul_rn(d.y, sc0));
+        amax1 = fmaxf(amax1, fmaxf(fabsf(r[2 * i]), fabsf(r[2 * i + 1])));
+        w0[i >> 1] = (i & 1) ? (w0[i >> 1] | (p << 16)) : p;
     }
     s0 = (uint32_t)(e0 + 127);
     if (act_mxfp8) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            w1[i] = 0u;
         s1 = 0;
         return;
     }
     const int e1 = mx_block_exp(amax1, 7);
     const float inv1 = exp2_int(-e1);
 #pragma unroll
-    for (int i = 0; i < 32; ++i)
-        c1[i] = (uint8_t)f32_to_e4m3(__fmul_rn(r[i], inv1));
+    for (int i = 0; i < 16; ++i) {
+        const uint32_t p = f32x2_to_e4m3x2(__fmul_rn(r[2 * i], inv1), __fmul_rn(r[2 * i + 1], inv1));
+        w1[i >> 1] = (i & 1) ? (w1[i >> 1] | (p << 16)) : p;
+    }
     s1 = (uint32_t)(e1 + 127);
 }
 
-__device__ __forceinline__ void store_codes32(uint8_t *dst, const uint8_t (&c)[32])
+__device__ __forceinline__ void store_codes32(uint8_t *dst, const uint32_t (&w)[8])
 {
-    uint4 w[2];
-    uint8_t *b = reinterpret_cast<uint8_t *>(w);
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-        b[i] = c[i];
-    reinterpret_cast<uint4 *>(dst)[0] = w[0];
-    reinterpret_cast<uint4 *>(dst)[1] = w[1];
+    reinterpret_cast<uint4 *>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    reinterpret_cast<uint4 *>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
 // One thread writes the 32-element block [col, col+32) of `row` (values v, f32):
@@ -264,7 +266,7 @@ __device__ __forceinline__ void store_act_block32(uint8_t *q, uint8_t *sf, int p
         for (int i = 0; i < 32; ++i)
             v[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
     }
-    uint8_t c0[32], c1[32];
+    uint32_t c0[8], c1[8];
     uint32_t s0, s1;
     mx_encode32(v, act_mxfp8, c0, c1, s0, s1);
     store_codes32(q + (size_t)row * K + col, c0);

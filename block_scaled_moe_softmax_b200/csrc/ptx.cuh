@@ -263,6 +263,26 @@ __device__ __forceinline__ uint32_t f32_to_e2m1(float t)
     return r & 0xF;
 }
 
+// Two values rounded to E4M3 codes (ties to even, saturating to +-448): a's code in
+// bits [0, 8), b's in bits [8, 16) (the conversion puts its first source operand in the
+// upper byte).
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float a, float b)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
+    return r;
+}
+
+// Values of the two E4M3 codes in bits [0, 8) (.x) and [8, 16) (.y) of p (exact), via
+// the hardware e4m3 -> f16 conversion, which keeps each byte's position.
+__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint32_t p)
+{
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)(p & 0xFFFF)));
+    return make_float2(__half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFF))),
+                       __half2float(__ushort_as_half((unsigned short)(h2 >> 16))));
+}
+
 // Value of an E4M3 code (exact), via the hardware e4m3 -> f16 conversion.
 __device__ __forceinline__ float e4m3_to_f32(uint32_t code)
 {

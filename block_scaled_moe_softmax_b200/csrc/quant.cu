@@ -65,17 +65,11 @@ __global__ void __launch_bounds__(256) mx_quantize_kernel(const float *__restric
                 ob[i] = p[i];
             reinterpret_cast<uint4 *>(codes)[b] = o;
         } else {
-            uint8_t c[32], unused[32];
+            uint32_t c[8], unused[8];
             uint32_t s0, s1;
             mx_encode32(v, 1, c, unused, s0, s1);
             scales[b] = (uint8_t)s0;
-            uint4 o[2];
-            uint8_t *ob = reinterpret_cast<uint8_t *>(o);
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-                ob[i] = c[i];
-            reinterpret_cast<uint4 *>(codes)[2 * b] = o[0];
-            reinterpret_cast<uint4 *>(codes)[2 * b + 1] = o[1];
+            store_codes32(codes + 32 * b, c);
         }
     }
 }

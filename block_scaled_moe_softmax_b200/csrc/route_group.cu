@@ -409,17 +409,6 @@ __global__ void __launch_bounds__(32) scatter_kernel(int T, int E, int k, const 
 // per (token, 32-element block, pair group): 64 bytes in, group x (32 or 2 x 32) code bytes and
 // group x (1 or 2) scale bytes out.
 // Codes of one 32-element block, packed four to a word.
-__device__ __forceinline__ void pack_codes32(const uint8_t (&c)[32], uint4 &lo, uint4 &hi)
-{
-    uint32_t w[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-        w[i] = (uint32_t)c[4 * i] | ((uint32_t)c[4 * i + 1] << 8) | ((uint32_t)c[4 * i + 2] << 16) |
-               ((uint32_t)c[4 * i + 3] << 24);
-    lo = make_uint4(w[0], w[1], w[2], w[3]);
-    hi = make_uint4(w[4], w[5], w[6], w[7]);
-}
-
 // Warp-wide rearrangement of 32 consecutive blocks' codes (lane l holds block l's 32 bytes,
 // i.e. 16-byte chunks 2l and 2l + 1 of the warp's 1 KB) so that lane l then holds chunks l and
 // l + 32: each 16-byte store instruction of the warp writes 512 contiguous bytes.  Chunk c sits
@@ -436,10 +425,27 @@ __device__ __forceinline__ void transpose_codes(uint4 *stg, int lane, uint4 &lo,
     __syncwarp();
 }
 
-__global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H, int k,
-                                                     int group, const int32_t *__restrict__ pos_of_pair,
-                                                     uint8_t *__restrict__ aq, uint8_t *__restrict__ asf, int act_rows,
-                                                     int act_mxfp8)
+// 32 bf16 values (four 16-byte pieces) as floats.
+__device__ __forceinline__ void bf16x32_to_f32(const uint4 (&raw)[4], float (&v)[32])
+{
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw[i]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(h2[j]);
+            v[8 * i + 2 * j] = f.x;
+            v[8 * i + 2 * j + 1] = f.y;
+        }
+    }
+}
+
+// At most 128 registers a thread, so that two CTAs (16 warps) share an SM: the kernel streams,
+// and its loads need warps in flight to cover their latency.
+__global__ void __launch_bounds__(256, 2) gather_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H, int k,
+                                                        int group, const int32_t *__restrict__ pos_of_pair,
+                                                        uint8_t *__restrict__ aq, uint8_t *__restrict__ asf,
+                                                        int act_rows, int act_mxfp8)
 {
     grid_dep_wait(); // pos_of_pair from the grouping
     grid_dep_launch();
@@ -454,37 +460,41 @@ __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16 *__rest
         // blocks, and total a multiple of 32, so every lane has work): the codes of each term go
         // through the warp's buffer once and leave as 512-byte rows per store instruction, to
         // each of the group's grouped rows; the four scale bytes of a 128-element chunk leave as
-        // one word from the chunk's first lane.
-        for (long long wb = (long long)blockIdx.x * blockDim.x + 32 * warp; wb < total; wb += stride) {
-            const long long g = wb + lane;
+        // one word from the chunk's first lane.  The x pieces and grouped rows of the warp's next
+        // 32 blocks are loaded while it encodes the current ones.
+        long long wb = (long long)blockIdx.x * blockDim.x + 32 * warp; // warp-uniform
+        uint4 raw[4];
+        int my_row = -1; // lane j < group: grouped row of the token's pair jg * group + j
+        auto load = [&](long long w) {
+            const long long g = w + lane;
             const int jg = (int)(g / per_group);
             const long long tb = g % per_group;
-            const int t = (int)(tb / blocks_per_row);
+            const int t = (int)(tb / blocks_per_row), b = (int)(tb % blocks_per_row);
+            const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H + (size_t)b * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                raw[i] = __ldg(src + i);
+            my_row = lane < group ? pos_of_pair[(size_t)t * k + jg * group + lane] : -1;
+        };
+        if (wb < total)
+            load(wb);
+        for (; wb < total; wb += stride) {
+            const long long tb = (wb + lane) % per_group;
             const int b = (int)(tb % blocks_per_row);
             const int b0 = b - lane; // the warp's first block
-            const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H + (size_t)b * 32);
             float v[32];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint4 raw = __ldg(src + i);
-                const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float2 f = __bfloat1622float2(h2[j]);
-                    v[8 * i + 2 * j] = f.x;
-                    v[8 * i + 2 * j + 1] = f.y;
-                }
-            }
-            uint8_t c0[32], c1[32];
+            bf16x32_to_f32(raw, v);
+            const int rows_now = my_row;
+            if (wb + stride < total)
+                load(wb + stride);
+            uint32_t c0[8], c1[8];
             uint32_t s0, s1;
             mx_encode32(v, act_mxfp8, c0, c1, s0, s1); // the values are bf16 already: no rounding step
-            uint4 a_lo, a_hi, b_lo = make_uint4(0, 0, 0, 0), b_hi = b_lo;
-            pack_codes32(c0, a_lo, a_hi);
+            uint4 a_lo = make_uint4(c0[0], c0[1], c0[2], c0[3]), a_hi = make_uint4(c0[4], c0[5], c0[6], c0[7]);
+            uint4 b_lo = make_uint4(c1[0], c1[1], c1[2], c1[3]), b_hi = make_uint4(c1[4], c1[5], c1[6], c1[7]);
             transpose_codes(stage[warp][0], lane, a_lo, a_hi);
-            if (!act_mxfp8) {
-                pack_codes32(c1, b_lo, b_hi);
+            if (!act_mxfp8)
                 transpose_codes(stage[warp][1], lane, b_lo, b_hi);
-            }
             // the scale bytes of blocks 4m .. 4m + 3 (one 128-element chunk) as one word
             uint32_t w0 = s0, w1 = s1;
 #pragma unroll
@@ -492,10 +502,8 @@ __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16 *__rest
                 w0 |= __shfl_down_sync(0xFFFFFFFFu, s0, i) << (8 * i);
                 w1 |= __shfl_down_sync(0xFFFFFFFFu, s1, i) << (8 * i);
             }
-            // the group's grouped rows, one per lane, loaded together (not one round trip per row)
-            const int my_row = lane < group ? pos_of_pair[(size_t)t * k + jg * group + lane] : -1;
             for (int j = 0; j < group; ++j) {
-                const int row = __shfl_sync(0xFFFFFFFFu, my_row, j); // the same for the whole warp
+                const int row = __shfl_sync(0xFFFFFFFFu, rows_now, j); // the same for the whole warp
                 if (row < 0)
                     continue; // not in the local expert shard
                 uint4 *dst = reinterpret_cast<uint4 *>(aq + (size_t)row * H + (size_t)b0 * 32);
@@ -521,19 +529,13 @@ __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16 *__rest
         const int t = (int)(tb / blocks_per_row);
         const int b = (int)(tb % blocks_per_row);
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H + (size_t)b * 32);
+        uint4 raw[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            raw[i] = __ldg(src + i);
         float v[32];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint4 raw = __ldg(src + i);
-            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float2 f = __bfloat1622float2(h2[j]);
-                v[8 * i + 2 * j] = f.x;
-                v[8 * i + 2 * j + 1] = f.y;
-            }
-        }
-        uint8_t c0[32], c1[32];
+        bf16x32_to_f32(raw, v);
+        uint32_t c0[8], c1[8];
         uint32_t s0, s1;
         mx_encode32(v, act_mxfp8, c0, c1, s0, s1); // the values are bf16 already: no rounding step
         for (int j = jg * group; j < (jg + 1) * group; ++j) {

@@ -94,6 +94,10 @@ WORKLOADS = {
     # the decode shape with 64 experts: a capture-sized case (about 1.5 GB of weights) for profiling
     "decode_e64": Workload("decode_e64", 16, 7168, 2048, 64, 8, "bf16", "none", 0,
                            "decode-shaped, w4a16, 64 experts (profiling case)"),
+    # the batched-decode routing mix (about 8 pairs per hit expert, some experts over 16 rows) with
+    # 64 experts and 64 tokens: a capture-sized case (about 1.5 GB of weights) for profiling
+    "batched_decode_e64": Workload("batched_decode_e64", 64, 7168, 2048, 64, 8, "bf16", "normal", 0,
+                                   "batched-decode-shaped, w4a16, 64 tokens, 64 experts (profiling case)"),
     # a prefill shape with 64 experts and 2048 tokens: a capture-sized case for profiling
     "prefill_e64": Workload("prefill_e64", 2048, 7168, 2048, 64, 8, "bf16", "none", 0,
                             "prefill-shaped, w4a16, 64 experts, 2048 tokens (profiling case)"),
