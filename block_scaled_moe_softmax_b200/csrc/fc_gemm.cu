@@ -95,15 +95,29 @@ template <int kActRows, int kMmaW, int kWTiles, int kTm> struct Plan {
     // wide variant: a 2 KB staging buffer per epilogue warp for FC2's f32 output rows
     static constexpr int kYBytes = (kActRows == 128 && kWTiles == 2) ? 8 * 2048 : 0;
     static constexpr int kStages = (kSmemLimit - 1024 - kXBytes - kYBytes - 256) / kStageBytes;
-    // The per-stage copy issue is split over several producer warps (groups of two stages
-    // round robin): each TMA instruction and each warp-wide 4-byte scale copy occupies its
-    // issuing warp for about a hundred cycles (measured: the cost is per warp, not per SM).
-    // A producer's consecutive stages are kProd apart; its parity waits on a slot's "empty"
-    // barrier are only sound while it cannot get two rounds ahead of that slot, which holds
-    // when kProd <= kStages.
+    // The per-stage copy issue is split over several producer warps: each TMA instruction and
+    // each warp-wide 4-byte scale copy occupies its issuing warp for about a hundred cycles
+    // (measured: the cost is per warp, not per SM).  Measured on the 16-row FC1 at decode: 2
+    // producer warps 25 % slower than 4, and 6 slower still (70 %), with producers then
+    // sharing the MMA warps' schedulers.  With single stages round robin a producer's
+    // consecutive stages are kProd apart; its parity waits on a slot's "empty" barrier are
+    // only sound while it cannot get two rounds ahead of that slot, which holds when
+    // kProd <= kStages.
     static constexpr int kProdWant = kActRows < 128 ? 4 : 2;
     static constexpr int kProd = kProdWant <= kStages ? kProdWant : kStages;
     static_assert(kProd >= 1 && kProd <= kStages, "producer warps vs pipeline stages");
+    // Weight-streaming variants hand out stages in pairs (2m, 2m + 1 to producer m % kProd): a
+    // K stage holds 64 bytes of each packed weight row, so one warp then requests both halves of
+    // a row's 128-byte line back to back (measured: batched decode FC1 0.971 -> 0.954 ms).  A
+    // producer's next stage after 2m + 1 is 2m + 2 kProd; its parity wait on that slot is sound
+    // while it cannot be two rounds ahead, i.e. while 2 kProd - 1 <= kStages (by induction over
+    // the stages it issued before, which were consumed in order).
+    static constexpr bool kPairStages = kActRows < 128 && 2 * kProd - 1 <= kStages;
+    // producer role index of stage g
+    static __device__ __forceinline__ int producer_of(uint32_t g)
+    {
+        return (int)((kPairStages ? (g >> 1) : g) % (uint32_t)kProd);
+    }
     // With at most 32 tokens per block (N <= 64) two MMA warps may take alternate stages,
     // each into its own accumulator (the epilogue adds them): one thread issues a block-scaled
     // MMA about every 64 cycles, and the second warp hides the per-stage wait and bookkeeping.
@@ -362,10 +376,10 @@ __device__ __forceinline__ bool wait_count(const int32_t *count, int target, uin
     return true;
 }
 
-// Producer role, one of kProd warps taking stages g with g % kProd == PI (PI is a
-// compile-time role index so that every operand of the TMA issue stays warp-uniform).
-// Consecutive stages come from different warps at nearly the same time, so the two 64-byte
-// halves of a weight row's 128-byte line are requested close together.
+// Producer role, one of kProd warps taking the stages g with Plan::producer_of(g) == PI (PI is
+// a compile-time role index so that every operand of the TMA issue stays warp-uniform): stage
+// pairs in the weight-streaming variants, so that the two 64-byte halves of a weight row's
+// 128-byte line are requested together, else single stages round robin.
 // Launched as a programmatic dependent, the kernel may start while the kernel ahead of it (which
 // writes this GEMM's activations) still runs; the producers wait for it (grid_dep_wait) before
 // their first copy.  (Issuing the first pass's weight copies before that wait and deferring only
@@ -428,7 +442,7 @@ __device__ __forceinline__ void producer_role(const Ctx &c, int lane)
             }
         }
         for (int kk = 0; kk < kst; ++kk, ++g) {
-            if ((int)(g % kProd) != PI)
+            if (P::producer_of(g) != PI)
                 continue; // another producer warp fills this stage
             const int s = g % kStages;
             if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars.empty(s), ((g / kStages) & 1) ^ 1, err_w, tmo))) {
@@ -499,7 +513,7 @@ __device__ __forceinline__ void producer_role(const Ctx &c, int lane)
     // drain: every stage this warp issued must have landed before the CTA may exit
     const uint32_t first = g > (uint32_t)kStages ? g - kStages : 0u;
     for (uint32_t q = first; q < g; ++q)
-        if ((int)(q % kProd) == PI)
+        if (P::producer_of(q) == PI)
             mbar_wait_bounded(bars.full(q % kStages), (q / kStages) & 1, nullptr, kDrainTimeoutNs);
 }
 
