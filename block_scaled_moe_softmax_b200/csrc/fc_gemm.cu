@@ -108,11 +108,20 @@ template <int kActRows, int kMmaW, int kWTiles, int kTm> struct Plan {
     static_assert(kProd >= 1 && kProd <= kStages, "producer warps vs pipeline stages");
     // Weight-streaming variants hand out stages in pairs (2m, 2m + 1 to producer m % kProd): a
     // K stage holds 64 bytes of each packed weight row, so one warp then requests both halves of
-    // a row's 128-byte line back to back (measured: batched decode FC1 0.971 -> 0.954 ms).  A
-    // producer's next stage after 2m + 1 is 2m + 2 kProd; its parity wait on that slot is sound
-    // while it cannot be two rounds ahead, i.e. while 2 kProd - 1 <= kStages (by induction over
-    // the stages it issued before, which were consumed in order).
-    static constexpr bool kPairStages = kActRows < 128 && 2 * kProd - 1 <= kStages;
+    // a row's 128-byte line back to back (measured: batched decode FC1 0.971 -> 0.954 ms).
+    // Soundness of a producer's parity wait for stage g (slot g % kStages): it passes early only
+    // if stage g - 2 kStages is still unconsumed.  By induction the producer's own earlier
+    // stages g' were issued after stage g' - kStages was consumed.  With one MMA warp stages are
+    // consumed in order, and its previous stage is at least g - (2 kProd - 1), which rules the
+    // early pass out when 2 kProd - 1 <= kStages.  With two MMA warps (one per stage parity,
+    // each in order, kStages even) the producer's previous pair holds a stage of g's parity at
+    // least g - 2 kProd: 2 kProd <= kStages.
+    static constexpr bool kPairStages =
+        kActRows < 128 && (kMmaW == 1 ? 2 * kProd - 1 <= kStages : 2 * kProd <= kStages);
+    // single stages round robin with two MMA warps: the producer's previous stage of g's parity
+    // is g - kProd (kProd even) or g - 2 kProd
+    static_assert(kMmaW == 1 || kPairStages || kProd % 2 == 0 || 2 * kProd <= kStages,
+                  "producer parity waits with two MMA warps");
     // producer role index of stage g
     static __device__ __forceinline__ int producer_of(uint32_t g)
     {
@@ -160,6 +169,8 @@ template <int kActRows, int kMmaW, int kWTiles, int kTm> struct Plan {
 };
 
 constexpr uint32_t kFmtE4M3 = 0, kFmtE2M1 = 5;
+
+
 
 template <int kStages> struct Bars {
     uint32_t base;
@@ -385,7 +396,7 @@ __device__ __forceinline__ bool wait_count(const int32_t *count, int target, uin
 // their first copy.  (Issuing the first pass's weight copies before that wait and deferring only
 // the activation copies measured slower: the extra paths cost the steady-state loop more than
 // the early weights gained.)
-template <int kActRows, int kMmaW, int kWTiles, int kTm, int PI>
+template <int kActRows, int kMmaW, int kWTiles, int kTm, int PI, bool kScalesN>
 __device__ __forceinline__ void producer_role(const Ctx &c, int lane)
 {
     uint32_t *const err_w = c.err; // in a register: the stage loops wait with it
@@ -423,10 +434,15 @@ __device__ __forceinline__ void producer_role(const Ctx &c, int lane)
         const bool sw3 = swap && npad <= P::kT2;
         const uint32_t act_bytes =
             (uint32_t)terms * (!swap ? (uint32_t)kTermBytes : sw3 ? (uint32_t)P::kT2 * 128u : (uint32_t)npad * 128u);
-        // activation scales: one bulk copy of the two 128-row atoms (tokens on M), or 4-byte copies
-        // of this block's rows into a stage atom laid out for N (tokens on N); weight scales: one
-        // bulk copy (tiled layout) or 4-byte copies (row-major)
-        const uint32_t tx = act_bytes + kWT * kWTxBytes + (swap ? 0u : (uint32_t)terms * 512u) +
+        // activation scales: one bulk copy of the two 128-row atoms (tokens on M); with the tokens
+        // on N one bulk copy of the block's atom in the N layout where the producer of the
+        // activations wrote one, else 4-byte copies of this block's rows into a stage atom laid
+        // out for N; weight scales: one bulk copy (tiled layout) or 4-byte copies (row-major)
+        const uint8_t *const act_sf_n =
+            kScalesN && swap && a.act_sf_n && a.n_rows == P::kT2 && npad <= P::kT2 && (comb || terms == 1)
+                ? a.act_sf_n + (size_t)(blk.y / P::kT2) * (size_t)kst * 512
+                : nullptr;
+        const uint32_t tx = act_bytes + kWT * kWTxBytes + (swap ? (act_sf_n ? 512u : 0u) : (uint32_t)terms * 512u) +
                             (a.wsf_tiled ? kWT * 512u : 0u);
         // tiled weight scales: the first tile's atoms, one per K stage, then the next tile's
         const uint8_t *wsf_tile = a.wscale + ((size_t)blk.x * a.n_tiles + nt0) * (size_t)kst * 512;
@@ -477,6 +493,9 @@ __device__ __forceinline__ void producer_role(const Ctx &c, int lane)
                     bulk_copy_g2s(asf_dst, asf_src, (uint32_t)terms * 512u, full_s);
                 } else if (sw3) {
                     tma_load_3d(act, act_map_sw, kx, blk.y, 0, full_s); // [terms][kT2 rows][128]
+                    if constexpr (kScalesN)
+                        if (act_sf_n)
+                            bulk_copy_g2s(asf_dst, act_sf_n + (size_t)kk * 512, 512u, full_s);
                 } else {
                     for (int r16 = 0; r16 < npad; r16 += 16) {
                         tma_load_2d(act + r16 * 128, act_map16, kx, blk.y + r16, full_s);
@@ -497,7 +516,7 @@ __device__ __forceinline__ void producer_role(const Ctx &c, int lane)
                         cp_async_4(wsf + wt * kWsfBytes + sf_atom_offset(r, 0), wscale + (size_t)wr * scl_ld + kk * 4);
                     }
                 }
-            if (swap) {
+            if (swap && !act_sf_n) {
                 // row j of term t: from row o + j of the term's 128-row atom to N row t * kT2 + j of
                 // one atom (both terms on N) or to row j of the term's own atom
                 for (int j = lane; j < npad; j += 32)
@@ -830,7 +849,11 @@ __device__ __forceinline__ void epilogue_wide(const Ctx &c, int warp, int lane)
     }
 }
 
-template <int kActRows, int kMmaW, int kWTiles, int kTm, bool kTwo>
+// kScalesN: the activation scales of units with their tokens on N may come in the N layout (one
+// bulk copy per stage), and FC1 writes h's scales in that layout too; a separate instantiation, so
+// that the kernels without it keep their code as it was (measured: carrying both forms in one
+// kernel slowed FC1 at 256 tokens by 2-8 %, and even a dead argument in its epilogue by 2 %).
+template <int kActRows, int kMmaW, int kWTiles, int kTm, bool kTwo, bool kScalesN>
 __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads, 1)
     fc_gemm_kernel(const __grid_constant__ FcGemmArgs a0, const __grid_constant__ FcGemmArgs a1,
                    const __grid_constant__ CUtensorMap act_map, const __grid_constant__ CUtensorMap act_map_sw,
@@ -922,15 +945,15 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads,
     ctx.err = a0.err;
     ctx.two = kTwo;
     if (warp == 0) {
-        producer_role<kActRows, kMmaW, kWTiles, kTm, 0>(ctx, lane);
+        producer_role<kActRows, kMmaW, kWTiles, kTm, 0, kScalesN>(ctx, lane);
     } else if (warp >= 6 && warp < 5 + kProd) {
         // further producer warps (compile-time role index: every TMA operand stays warp-uniform)
         if (warp == 6)
-            producer_role<kActRows, kMmaW, kWTiles, kTm, 1 % kProd>(ctx, lane);
+            producer_role<kActRows, kMmaW, kWTiles, kTm, 1 % kProd, kScalesN>(ctx, lane);
         else if (warp == 7)
-            producer_role<kActRows, kMmaW, kWTiles, kTm, 2 % kProd>(ctx, lane);
+            producer_role<kActRows, kMmaW, kWTiles, kTm, 2 % kProd, kScalesN>(ctx, lane);
         else if (warp == 8)
-            producer_role<kActRows, kMmaW, kWTiles, kTm, 3 % kProd>(ctx, lane);
+            producer_role<kActRows, kMmaW, kWTiles, kTm, 3 % kProd, kScalesN>(ctx, lane);
     } else if (warp == 1) {
         if constexpr (P::kWide)
             mma_role_wide<kActRows, kMmaW, kWTiles, kTm>(ctx);
@@ -1051,8 +1074,12 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads,
                                 if (n >= rows)
                                     break;
                                 const float hv = silu_mul(v[j], xch[L * 16 + j]);
-                                store_act_warp32(a.hq, a.hsf, a.hq_rows, a.out_ld, blk.y + n, i, hv, a.act_mxfp8,
-                                                 lane);
+                                if constexpr (kScalesN)
+                                    store_act_warp32(a.hq, a.hsf, a.hq_rows, a.out_ld, blk.y + n, i, hv,
+                                                     a.act_mxfp8, lane, a.hsf_n, a.n_rows);
+                                else
+                                    store_act_warp32(a.hq, a.hsf, a.hq_rows, a.out_ld, blk.y + n, i, hv,
+                                                     a.act_mxfp8, lane);
                             }
                         }
                         named_bar_sync(1, 128);
@@ -1095,9 +1122,10 @@ __global__ void __launch_bounds__(Plan<kActRows, kMmaW, kWTiles, kTm>::kThreads,
     }
 }
 
-template <int kActRows, int kMmaW, int kWTiles, int kTm, bool kTwo = false> static cudaError_t prepare_one()
+template <int kActRows, int kMmaW, int kWTiles, int kTm, bool kTwo = false, bool kScalesN = false>
+static cudaError_t prepare_one()
 {
-    return cudaFuncSetAttribute(fc_gemm_kernel<kActRows, kMmaW, kWTiles, kTm, kTwo>,
+    return cudaFuncSetAttribute(fc_gemm_kernel<kActRows, kMmaW, kWTiles, kTm, kTwo, kScalesN>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 Plan<kActRows, kMmaW, kWTiles, kTm>::kSmemBytes);
 }
@@ -1112,18 +1140,23 @@ cudaError_t fc_gemm_prepare()
         (e = prepare_one<64, 1, 1, 2>()) != cudaSuccess || (e = prepare_one<128, 1, 1, 2>()) != cudaSuccess ||
         (e = prepare_one<128, 1, 1, 1>()) != cudaSuccess || (e = prepare_one<128, 1, 2, 2>()) != cudaSuccess)
         return e;
-    if ((e = prepare_one<128, 1, 2, 1>()) != cudaSuccess)
+    if ((e = prepare_one<128, 1, 2, 1>()) != cudaSuccess || (e = prepare_one<16, 2, 1, 2, true>()) != cudaSuccess)
         return e;
-    return prepare_one<16, 2, 1, 2, true>();
+    if ((e = prepare_one<16, 2, 1, 2, false, true>()) != cudaSuccess ||
+        (e = prepare_one<16, 1, 2, 2, false, true>()) != cudaSuccess ||
+        (e = prepare_one<16, 1, 4, 2, false, true>()) != cudaSuccess)
+        return e;
+    return prepare_one<16, 2, 1, 2, true, true>();
 }
 
-template <int kActRows, int kMmaW, int kWTiles, int kTm>
+template <int kActRows, int kMmaW, int kWTiles, int kTm, bool kScalesN = false>
 static void launch_one(const FcGemmArgs &a, const CUtensorMap &act_map, const CUtensorMap &act_map_sw,
                        const CUtensorMap &act_map16, const CUtensorMap &w_map, int grid, cudaStream_t s, bool pdl)
 {
     using P = Plan<kActRows, kMmaW, kWTiles, kTm>;
-    launch_kernel(fc_gemm_kernel<kActRows, kMmaW, kWTiles, kTm, false>, dim3(grid), dim3(P::kThreads), (size_t)P::kSmemBytes,
-                  s, pdl, a, a, act_map, act_map_sw, act_map16, w_map, act_map, act_map_sw, act_map16, w_map);
+    launch_kernel(fc_gemm_kernel<kActRows, kMmaW, kWTiles, kTm, false, kScalesN>, dim3(grid), dim3(P::kThreads),
+                  (size_t)P::kSmemBytes, s, pdl, a, a, act_map, act_map_sw, act_map16, w_map, act_map, act_map_sw,
+                  act_map16, w_map);
 }
 
 void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUtensorMap &act_map_sw,
@@ -1135,11 +1168,20 @@ void launch_fc_gemm(const FcGemmArgs &a, const CUtensorMap &act_map, const CUten
     // units) with one MMA warp and two weight tiles per work unit when the tiles pair up.
     // Each choice measured fastest on the decode shapes.
     const bool wt2 = !a.fc1 && a.n_tiles % 2 == 0;
+    // the N-layout scales (a.act_sf_n, a.hsf_n) are read and written by the kScalesN
+    // instantiations only; the others ignore them
+    const bool sn = a.act_sf_n != nullptr || a.hsf_n != nullptr;
     if (a.max_block_rows <= 16) {
-        if (a.fc1)
+        if (a.fc1 && sn)
+            launch_one<16, 2, 1, 2, true>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
+        else if (a.fc1)
             launch_one<16, 2, 1, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
+        else if (a.fc2_tiles == 4 && a.n_tiles % 4 == 0 && sn)
+            launch_one<16, 1, 4, 2, true>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
         else if (a.fc2_tiles == 4 && a.n_tiles % 4 == 0)
             launch_one<16, 1, 4, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
+        else if (wt2 && sn)
+            launch_one<16, 1, 2, 2, true>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
         else if (wt2)
             launch_one<16, 1, 2, 2>(a, act_map, act_map_sw, act_map16, w_map, grid, s, pdl);
         else
@@ -1176,8 +1218,12 @@ void launch_fc_gemm_two_phase(const FcGemmArgs &a1, const CUtensorMap *maps1, co
     // tokens on N, 16-row blocks, two MMA warps: the small-batch FC1 variant serves both phases
     // (FC2 units then take one weight tile each)
     using P = Plan<16, 2, 1, 2>;
-    launch_kernel(fc_gemm_kernel<16, 2, 1, 2, true>, dim3(grid), dim3(P::kThreads), (size_t)P::kSmemBytes, s, pdl, a1, a2,
-                  maps1[0], maps1[1], maps1[2], maps1[3], maps2[0], maps2[1], maps2[2], maps2[3]);
+    if (a1.act_sf_n != nullptr || a1.hsf_n != nullptr)
+        launch_kernel(fc_gemm_kernel<16, 2, 1, 2, true, true>, dim3(grid), dim3(P::kThreads), (size_t)P::kSmemBytes, s,
+                      pdl, a1, a2, maps1[0], maps1[1], maps1[2], maps1[3], maps2[0], maps2[1], maps2[2], maps2[3]);
+    else
+        launch_kernel(fc_gemm_kernel<16, 2, 1, 2, true, false>, dim3(grid), dim3(P::kThreads), (size_t)P::kSmemBytes,
+                      s, pdl, a1, a2, maps1[0], maps1[1], maps1[2], maps1[3], maps2[0], maps2[1], maps2[2], maps2[3]);
 }
 
 // ---------------------------------------------------------------- watchdog self-test

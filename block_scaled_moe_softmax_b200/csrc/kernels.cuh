@@ -79,8 +79,10 @@ struct RouteGroupArgs {
 // waits for whatever precedes it before it reads the logits or writes the workspace.
 // Returns the number of kernels launched (1 for small batches, else 3).
 int launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s, bool pdl = false);
+// asf_n (optional): the scales again in the N layout of blocks of n_rows rows (sf_n_byte)
 void launch_gather(const __nv_bfloat16 *x, int P, int H, int k, const int32_t *pos_of_pair, uint8_t *aq,
-                   uint8_t *asf, int act_rows, int act_mxfp8, int num_sms, cudaStream_t s, bool pdl = false);
+                   uint8_t *asf, int act_rows, int act_mxfp8, uint8_t *asf_n, int n_rows, int num_sms,
+                   cudaStream_t s, bool pdl = false);
 // out: bf16 [T, H], or (out_f32) float32 [T, H]; pairs with pos_of_pair -1 add nothing
 void launch_combine(const float *Y, int T, int H, int k, const int32_t *pos_of_pair, const float *topk_w, void *out,
                     int out_f32, int num_sms, cudaStream_t s, bool pdl = false);
@@ -132,6 +134,12 @@ struct FcGemmArgs {
     // its row block's h only once all of them are counted.
     int32_t *rb_done;
     int fc2_tiles;               // FC2 with blocks of <= 16 rows: weight tiles per work unit (2 or 4)
+    // The activation scales also in the N layout (sf_n_byte) of blocks of n_rows rows, for units
+    // with their tokens on N: one 512-byte bulk copy per stage instead of 4-byte copies (nullptr:
+    // not written); FC1 writes h's scales in that layout too when hsf_n is set.
+    const uint8_t *act_sf_n;
+    uint8_t *hsf_n;
+    int n_rows;
 };
 
 // Tensor maps: act_map = both term planes, 128-row boxes ([terms][128][128] codes, tokens
@@ -178,6 +186,16 @@ __device__ __forceinline__ size_t sf_atom_byte(int row, int col, int K, int term
 {
     return ((size_t)(row >> 7) * (size_t)(K >> 7) + (size_t)(col >> 7)) * 1024 + (size_t)term * 512 +
            (size_t)sf_atom_offset(row & 127, (col >> 5) & 3);
+}
+
+// The N layout, for GEMM units that put a block of n_rows grouped rows (16 or 32, blocks starting
+// at multiples of n_rows) on the MMA's N side with both terms side by side: per block and
+// 128-element K stage one 512-byte atom, in which row j of term t is the atom's row
+// t * n_rows + j.  That is the stage's scale atom as the MMA reads it, so a unit copies it whole.
+__device__ __forceinline__ size_t sf_n_byte(int row, int col, int K, int term, int n_rows)
+{
+    return ((size_t)(row / n_rows) * (size_t)(K >> 7) + (size_t)(col >> 7)) * 512 +
+           (size_t)sf_atom_offset(term * n_rows + row % n_rows, (col >> 5) & 3);
 }
 
 // E8M0 exponent of a block: floor(log2(amax)) - emax_shift, clamped to [-127, 127]
@@ -280,8 +298,10 @@ __device__ __forceinline__ void store_act_block32(uint8_t *q, uint8_t *sf, int p
 // The 32 lanes of a warp write one 32-element block of `row`, lane l holding
 // element col0 + l (col0 = col rounded down to 32): the encoding of
 // store_act_block32 computed with warp reductions (same rule, same results).
+// sf_n (optional): the scale bytes again in the N layout of blocks of n_rows rows.
 __device__ __forceinline__ void store_act_warp32(uint8_t *q, uint8_t *sf, int plane_rows, int K, int row, int col,
-                                                 float v, int act_mxfp8, int lane)
+                                                 float v, int act_mxfp8, int lane, uint8_t *sf_n = nullptr,
+                                                 int n_rows = 0)
 {
     if (!act_mxfp8)
         v = __bfloat162float(__float2bfloat16_rn(v));
@@ -293,8 +313,11 @@ __device__ __forceinline__ void store_act_warp32(uint8_t *q, uint8_t *sf, int pl
     const int e0 = finite ? mx_block_exp(amax, act_mxfp8 ? 8 : 7) : 0;
     const uint32_t c0 = finite ? f32_to_e4m3(__fmul_rn(v, exp2_int(-e0))) : 0u;
     q[(size_t)row * K + col] = (uint8_t)c0;
-    if (lane == 0)
+    if (lane == 0) {
         sf[sf_atom_byte(row, col, K, 0)] = finite ? (uint8_t)(e0 + 127) : (uint8_t)0xFF;
+        if (sf_n)
+            sf_n[sf_n_byte(row, col, K, 0, n_rows)] = finite ? (uint8_t)(e0 + 127) : (uint8_t)0xFF;
+    }
     if (!act_mxfp8) {
         const float r = finite ? __fsub_rn(v, __fmul_rn(e4m3_to_f32(c0), exp2_int(e0))) : 0.f;
         float amax1 = fabsf(r);
@@ -303,8 +326,11 @@ __device__ __forceinline__ void store_act_warp32(uint8_t *q, uint8_t *sf, int pl
             amax1 = fmaxf(amax1, __shfl_xor_sync(0xFFFFFFFFu, amax1, off));
         const int e1 = mx_block_exp(amax1, 7);
         q[((size_t)plane_rows + row) * K + col] = finite ? (uint8_t)f32_to_e4m3(__fmul_rn(r, exp2_int(-e1))) : 0u;
-        if (lane == 0)
+        if (lane == 0) {
             sf[sf_atom_byte(row, col, K, 1)] = finite ? (uint8_t)(e1 + 127) : (uint8_t)0xFF;
+            if (sf_n)
+                sf_n[sf_n_byte(row, col, K, 1, n_rows)] = finite ? (uint8_t)(e1 + 127) : (uint8_t)0xFF;
+        }
     }
 }
 

@@ -445,7 +445,8 @@ __device__ __forceinline__ void bf16x32_to_f32(const uint4 (&raw)[4], float (&v)
 __global__ void __launch_bounds__(256, 2) gather_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H, int k,
                                                         int group, const int32_t *__restrict__ pos_of_pair,
                                                         uint8_t *__restrict__ aq, uint8_t *__restrict__ asf,
-                                                        int act_rows, int act_mxfp8)
+                                                        int act_rows, int act_mxfp8, uint8_t *__restrict__ asf_n,
+                                                        int n_rows)
 {
     grid_dep_wait(); // pos_of_pair from the grouping
     grid_dep_launch();
@@ -509,14 +510,20 @@ __global__ void __launch_bounds__(256, 2) gather_kernel(const __nv_bfloat16 *__r
                 uint4 *dst = reinterpret_cast<uint4 *>(aq + (size_t)row * H + (size_t)b0 * 32);
                 dst[lane] = a_lo;
                 dst[lane + 32] = a_hi;
-                if ((lane & 3) == 0)
+                if ((lane & 3) == 0) {
                     *reinterpret_cast<uint32_t *>(asf + sf_atom_byte(row, b * 32, H, 0)) = w0;
+                    if (asf_n)
+                        *reinterpret_cast<uint32_t *>(asf_n + sf_n_byte(row, b * 32, H, 0, n_rows)) = w0;
+                }
                 if (!act_mxfp8) {
                     uint4 *dst1 = reinterpret_cast<uint4 *>(aq + ((size_t)act_rows + row) * H + (size_t)b0 * 32);
                     dst1[lane] = b_lo;
                     dst1[lane + 32] = b_hi;
-                    if ((lane & 3) == 0)
+                    if ((lane & 3) == 0) {
                         *reinterpret_cast<uint32_t *>(asf + sf_atom_byte(row, b * 32, H, 1)) = w1;
+                        if (asf_n)
+                            *reinterpret_cast<uint32_t *>(asf_n + sf_n_byte(row, b * 32, H, 1, n_rows)) = w1;
+                    }
                 }
             }
         }
@@ -544,9 +551,13 @@ __global__ void __launch_bounds__(256, 2) gather_kernel(const __nv_bfloat16 *__r
                 continue; // not in the local expert shard
             store_codes32(aq + (size_t)row * H + b * 32, c0);
             asf[sf_atom_byte(row, b * 32, H, 0)] = (uint8_t)s0;
+            if (asf_n)
+                asf_n[sf_n_byte(row, b * 32, H, 0, n_rows)] = (uint8_t)s0;
             if (!act_mxfp8) {
                 store_codes32(aq + ((size_t)act_rows + row) * H + b * 32, c1);
                 asf[sf_atom_byte(row, b * 32, H, 1)] = (uint8_t)s1;
+                if (asf_n)
+                    asf_n[sf_n_byte(row, b * 32, H, 1, n_rows)] = (uint8_t)s1;
             }
         }
     }
@@ -640,7 +651,8 @@ int launch_route_and_group(const RouteGroupArgs &a, cudaStream_t s, bool pdl)
 }
 
 void launch_gather(const __nv_bfloat16 *x, int P, int H, int k, const int32_t *pos_of_pair, uint8_t *aq,
-                   uint8_t *asf, int act_rows, int act_mxfp8, int num_sms, cudaStream_t s, bool pdl)
+                   uint8_t *asf, int act_rows, int act_mxfp8, uint8_t *asf_n, int n_rows, int num_sms,
+                   cudaStream_t s, bool pdl)
 {
     // encode each block once per token when that still fills the GPU, else once per pair
     const long long token_blocks = (long long)(P / k) * (H / 32);
@@ -649,7 +661,7 @@ void launch_gather(const __nv_bfloat16 *x, int P, int H, int k, const int32_t *p
     const long long want = (work + 255) / 256;
     const int grid = (int)(want < (long long)num_sms * 8 ? want : (long long)num_sms * 8);
     launch_kernel(gather_kernel, dim3(grid > 0 ? grid : 1), dim3(256), 0, s, pdl, x, P / k, H, k, group, pos_of_pair,
-                  aq, asf, act_rows, act_mxfp8);
+                  aq, asf, act_rows, act_mxfp8, asf_n, n_rows);
 }
 
 void launch_combine(const float *Y, int T, int H, int k, const int32_t *pos_of_pair, const float *topk_w, void *out,
