@@ -22,13 +22,15 @@
 //
 // Per CTA (one per SM, persistent; work units u = (row block, weight tile) handed
 // out at run time through a global counter):
-//   producers   2 to 4 warps, taking pipeline stages round robin: TMA of the
-//               weight tile (E2M1 codes unpacked to 8-bit containers; for FC1
-//               the gate and up halves in one 3-D box), TMA of both activation
-//               term planes in one 3-D box, the stage's weight scale atom (one
-//               bulk copy in the tiled layout, else 4-byte copies) and the
-//               activation scale atom (bulk copy, or 4-byte copies laid out for
-//               N when the tokens sit on N);
+//   producers   2 to 4 warps, taking pipeline stages round robin (in pairs in
+//               the weight-streaming variants): TMA of the weight tile (E2M1
+//               codes unpacked to 8-bit containers; for FC1 the gate and up
+//               halves in one 3-D box), TMA of both activation term planes in
+//               one 3-D box, the stage's weight scale atom (one bulk copy in the
+//               tiled layout, else 4-byte copies) and the activation scale atom
+//               (bulk copy; with the tokens on N 4-byte copies laid out for N,
+//               or, in the kScalesN kernels, one bulk copy of the atom the
+//               activations' producer wrote in that N layout);
 //   MMA         1 or 2 warps (alternate stages, own accumulators): tcgen05.cp of
 //               the stage's scale atoms to TMEM, then the block-scaled MMAs; one
 //               warp owns the TMEM allocation;
@@ -169,8 +171,6 @@ template <int kActRows, int kMmaW, int kWTiles, int kTm> struct Plan {
 };
 
 constexpr uint32_t kFmtE4M3 = 0, kFmtE2M1 = 5;
-
-
 
 template <int kStages> struct Bars {
     uint32_t base;
