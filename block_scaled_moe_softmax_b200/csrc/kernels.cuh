@@ -134,9 +134,11 @@ struct FcGemmArgs {
     // its row block's h only once all of them are counted.
     int32_t *rb_done;
     int fc2_tiles;               // FC2 with blocks of <= 16 rows: weight tiles per work unit (2 or 4)
-    // The activation scales also in the N layout (sf_n_byte) of blocks of n_rows rows, for units
-    // with their tokens on N: one 512-byte bulk copy per stage instead of 4-byte copies (nullptr:
-    // not written); FC1 writes h's scales in that layout too when hsf_n is set.
+    // Used by the kScalesN kernel instantiations only (launch_fc_gemm picks them when either is
+    // set): act_sf_n = the activation scales again in the N layout (sf_n_byte) of blocks of
+    // n_rows rows, which units with their tokens on N take with one 512-byte bulk copy per stage
+    // instead of 4-byte copies (nullptr: the 4-byte copies); hsf_n = where FC1 also writes h's
+    // scales in that layout (nullptr: not written).
     const uint8_t *act_sf_n;
     uint8_t *hsf_n;
     int n_rows;
