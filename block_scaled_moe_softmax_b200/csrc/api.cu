@@ -148,6 +148,7 @@ struct moe_mx_handle {
     int fuse_combine; // small batches: the combine in FC2's epilogue (MOE_MX_FUSE_COMBINE; off by default: slower)
     int two_phase;    // small batches: FC1 and FC2 in one launch (MOE_MX_TWO_PHASE, default 1)
     int two_phase_max_tokens; // ... up to this many tokens (at most 16)
+    int scales_n;             // N-layout activation scales up to 16 tokens (MOE_MX_SCALES_N, default 1)
     int fc2_tiles;            // FC2 of blocks of <= 16 rows: weight tiles per unit (MOE_MX_FC2_TILES: 0 = by
                               // token count, 2 or 4)
     int scale_layout; // MOE_MX_SCALES_ROW_MAJOR or MOE_MX_SCALES_TILED
@@ -263,6 +264,7 @@ int moe_mx_create_ex(moe_mx_handle **out, int hidden, int inter, int num_experts
     // (its FC2 units are one weight tile each, and short); MOE_MX_TWO_PHASE_TOKENS (<= 16) moves
     // the bound
     h->two_phase_max_tokens = env_int("MOE_MX_TWO_PHASE_TOKENS", 1);
+    h->scales_n = env_int("MOE_MX_SCALES_N", 1) != 0;
     h->fc2_tiles = env_int("MOE_MX_FC2_TILES", 0);
     if (h->fc2_tiles != 2 && h->fc2_tiles != 4)
         h->fc2_tiles = 0;
@@ -502,7 +504,8 @@ int forward_impl(moe_mx_handle *h, const void *x, const float *router_logits, co
         // 4-byte copies.  Measured: 1 token 0.0826 -> 0.0757 ms, 4 tokens 0.1739 ->
         // 0.1712, 16 tokens 0.4522 -> 0.4515; at 256 tokens slower (1.455 -> 1.48 ms), so the
         // 4-byte copies stay there.
-        const bool scales_n = tile_rows == 16 && T <= kScalesNTokens && grouped_rows_bound(E, pairs) <= h->n_rows_cap;
+        const bool scales_n = h->scales_n && tile_rows == 16 && T <= kScalesNTokens &&
+                              grouped_rows_bound(E, pairs) <= h->n_rows_cap;
         launch_gather(static_cast<const __nv_bfloat16 *>(x), (int)pairs, H, k, h->pos_of_pair, h->Aq, h->Asf,
                       (int)h->max_rows, mx8, scales_n ? h->AsfN : nullptr, tile_rows, h->num_sms, s, pdl);
 

@@ -210,6 +210,33 @@ def test_dependent_launch_gives_same_bits(name, act_mode, monkeypatch):
 
 
 
+# up to 16 tokens the activation scales also go through the N layout (one bulk copy per GEMM stage)
+N_LAYOUT_SHAPES = {
+    "tiny": workloads.WORKLOADS["tiny"],
+    "t16_e64": workloads.Workload("t16_e64", 16, 512, 256, 64, 8, "bf16", "none", 7),
+    "t4_e64": workloads.Workload("t4_e64", 4, 512, 256, 64, 8, "bf16", "none", 8),
+    "t1_e64": workloads.Workload("t1_e64", 1, 512, 256, 64, 8, "bf16", "none", 9),  # one launch, two phases
+}
+
+
+@pytest.mark.parametrize("name", list(N_LAYOUT_SHAPES))
+@pytest.mark.parametrize("act_mode", [0, 1], ids=["w4a16", "w4a8"])
+def test_n_layout_scales_give_same_bits(name, act_mode, monkeypatch):
+    """The activation scales taken from the N layout (the default up to 16 tokens) and through
+    4-byte copies from the row-block atoms (MOE_MX_SCALES_N=0) give bit-identical outputs."""
+    wl = N_LAYOUT_SHAPES[name]
+    inp = helpers.host_inputs(wl)
+    outs = []
+    for sn in ("1", "0"):
+        monkeypatch.setenv("MOE_MX_SCALES_N", sn)
+        layer, _, out = _run(wl, act_mode, monkeypatch, inp=inp)
+        outs.append(out.clone())
+        layer.close()
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    ref, _, _ = helpers.oracle_forward(inp, wl.top_k, act_mode)
+    helpers.check_output(outs[0], ref, f"{name} N-layout scales")
+
+
 def test_router_matches_hand_derived_cases():
     """The router on the hand-derived cases of tests/golden/routing_cases.txt (ties, -0 / +0, NaN
     and -inf logits, k = E), each padded to 8 experts with -inf logits and run as one token of a
