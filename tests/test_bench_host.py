@@ -1,5 +1,6 @@
 """Host-side logic of bench.py (CPU only): the algorithmic work it divides by, the reference
-arm's sampling, and the JSON line of the reference arm."""
+arm's sampling, the JSON line of the reference arm, and the use of the committed ncu traffic
+record (keyed on the FC GEMM's code)."""
 import json
 import os
 import subprocess
@@ -64,3 +65,40 @@ def test_reference_arm_json_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert d["config"]["pairs_per_token"] == 2.0
+
+
+def test_kernel_source_hash_ignores_comments_only():
+    """The traffic record is keyed on the FC GEMM's code: an edit of a comment or of whitespace
+    keeps the hash, an edit of the code changes it."""
+    csrc = os.path.join(ROOT, "block_scaled_moe_softmax_b200", "csrc")
+
+    def read(name):
+        with open(os.path.join(csrc, name)) as f:
+            return f.read()
+
+    base = bench.kernel_source_sha(read)
+    assert base == bench.kernel_source_sha()
+    commented = lambda n: read(n) + ("\n// a new remark\n/* and a block\n   comment */\n   \n" if n == "fc_gemm.cu" else "")
+    assert bench.kernel_source_sha(commented) == base
+    changed = lambda n: read(n) + ("\nconstexpr int kProbe = 1;\n" if n == "ptx.cuh" else "")
+    assert bench.kernel_source_sha(changed) != base
+
+
+def test_traffic_record_use(monkeypatch):
+    """A committed capture is used for its own workload and scaled by algorithmic bytes for the
+    workloads it lists under scales_to; nothing is reported once the kernel's code differs."""
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        rec = json.load(f)
+    caps = {c["workload"]: c for c in rec["fc1_captures"]}
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda read=None: rec["kernel_sha"])
+    for name, cap in caps.items():
+        dram = cap["dram_bytes_read"] + cap["dram_bytes_write"]
+        assert cap["dram_bytes_read"] > 0.9 * cap["algorithmic_bytes"]  # the weights are read
+        if name in workloads.WORKLOADS:
+            assert bench.traffic_record(workloads.WORKLOADS[name], 123) == dram
+        for target in cap.get("scales_to", []):
+            got = bench.traffic_record(workloads.WORKLOADS[target], 2 * cap["algorithmic_bytes"])
+            assert got == pytest.approx(2 * dram)
+    assert bench.traffic_record(workloads.WORKLOADS["prefill"], 1) is None  # tensor-bound: no scaling
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda read=None: "0" * 16)
+    assert bench.traffic_record(workloads.WORKLOADS["decode"], 1) is None
