@@ -336,6 +336,13 @@ def fc2_algorithmic_bytes(wl, counts):
     return hit * (wl.I * wl.H // 2 + wl.I * wl.H // 32) + P * wl.I * 2 + P * wl.H * 4
 
 
+def one_launch_gemms(stage):
+    """True when the forward ran FC1 and FC2 as one launch (two phases): its FC1 stage then
+    holds both GEMMs, and the FC2 stage no kernel, only the gap between two events (a few
+    microseconds), while a separate FC2 launch takes a large share of FC1's time."""
+    return stage["fc2"] < 0.2 * stage["fc1"]
+
+
 def layer_weight_bytes(wl, hit):
     return hit * (3 * wl.I * wl.H // 2 + 3 * wl.I * wl.H // 32)
 
@@ -533,9 +540,9 @@ def measure(args, wl, weights, world, rank, with_e2e=True):
 
     fc1_ms = stage["fc1"]
     kernel_name = "fc_gemm_kernel (FC1 + SwiGLU)"
-    if stage["fc2"] < 1e-3 <= fc1_ms:
-        # up to 16 tokens the library runs FC1 and FC2 as one launch (two phases): the roofline
-        # kernel is that launch, with both GEMMs' work
+    if one_launch_gemms(stage):
+        # at the smallest batches the library runs FC1 and FC2 as one launch (two phases): the
+        # roofline kernel is that launch, with both GEMMs' work
         kernel_name = "fc_gemm_kernel (FC1 + SwiGLU, then FC2, one launch)"
         fc1_bytes += fc2_algorithmic_bytes(wl, counts)
         fc1_flops *= 1.5

@@ -260,10 +260,10 @@ int moe_mx_create_ex(moe_mx_handle **out, int hidden, int inter, int num_experts
     h->wide = env_int("MOE_MX_WIDE", 1) != 0;
     h->fuse_combine = env_int("MOE_MX_FUSE_COMBINE", 0) != 0;
     h->two_phase = env_int("MOE_MX_TWO_PHASE", 1) != 0;
-    // measured: one launch gains at a single token (0.090 -> 0.083 ms) and loses from 2 tokens on
-    // (its FC2 units are one weight tile each, and short); MOE_MX_TWO_PHASE_TOKENS (<= 16) moves
-    // the bound
-    h->two_phase_max_tokens = env_int("MOE_MX_TWO_PHASE_TOKENS", 1);
+    // measured: one launch gains at 1 and 2 tokens (1 token 0.090 -> 0.083 ms; 2 tokens, with the
+    // N-layout scales, 0.1228 -> 0.1195 ms) and loses from 4 tokens on (0.172 -> 0.188 ms: its FC2
+    // units are one weight tile each, and short); MOE_MX_TWO_PHASE_TOKENS (<= 16) moves the bound
+    h->two_phase_max_tokens = env_int("MOE_MX_TWO_PHASE_TOKENS", 2);
     h->scales_n = env_int("MOE_MX_SCALES_N", 1) != 0;
     h->fc2_tiles = env_int("MOE_MX_FC2_TILES", 0);
     if (h->fc2_tiles != 2 && h->fc2_tiles != 4)

@@ -102,3 +102,14 @@ def test_traffic_record_use(monkeypatch):
     assert bench.traffic_record(workloads.WORKLOADS["prefill"], 1) is None  # tensor-bound: no scaling
     monkeypatch.setattr(bench, "kernel_source_sha", lambda read=None: "0" * 16)
     assert bench.traffic_record(workloads.WORKLOADS["decode"], 1) is None
+
+
+def test_one_launch_detection():
+    """The stage times of a forward whose GEMMs ran as one launch (measured at one token: FC1
+    stage 67 us, the empty FC2 stage 2.8 us) against separate launches (16 tokens: 293 and
+    146 us; prefill: 2.75 and 1.56 ms)."""
+    assert bench.one_launch_gemms({"fc1": 0.0670, "fc2": 0.0028})
+    assert bench.one_launch_gemms({"fc1": 0.1072, "fc2": 0.0027})
+    assert not bench.one_launch_gemms({"fc1": 0.2933, "fc2": 0.1465})
+    assert not bench.one_launch_gemms({"fc1": 2.75, "fc2": 1.56})
+    assert not bench.one_launch_gemms({"fc1": 0.0158, "fc2": 0.0134})  # tiny
